@@ -1,0 +1,350 @@
+"""Pins of the fp64 oracle against results the pages and the mathematics fix.
+
+Each pin returns (ok, detail).  The pins use small random inputs and
+independent textbook computations written with numpy matrices (not the
+oracle's loops) or torch's CPU attention in fp64.  ``run_all_pins`` is used
+both by the oracle tests and by the test that plants deliberate mistakes in
+the oracle and checks that some pin catches each one.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import wall_oracle as wo
+
+LN2 = np.log(2.0)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _inputs(seed, B=1, T=7, HQ=4, H=2, K=3, V=3, g_amp=0.3, decay=False, gs=False,
+            sink=False):
+    r = _rng(seed)
+    q = r.standard_normal((B, T, HQ, K))
+    k = r.standard_normal((B, T, H, K))
+    v = r.standard_normal((B, T, H, V))
+    g = r.standard_normal((B, T, HQ, K)) * g_amp
+    if decay:
+        g = -np.abs(g)
+    dO = r.standard_normal((B, T, HQ, V))
+    x = dict(q=q, k=k, v=v, g=g, dO=dO)
+    x["g_scalar"] = np.log(1.0 / (1.0 + np.exp(-(1.0 + r.standard_normal((B, T, HQ)))))) if gs else None
+    x["sink_bias"] = r.standard_normal(HQ) if sink else None
+    return x
+
+
+def textbook_attention(q, k, v, scale, bias=None, sink=None, window=0):
+    """Plain softmax attention of one sequence, numpy matrices.
+    q [T,HQ,K], k [T,H,K], v [T,H,V]; bias [HQ,T,T] added to the logits;
+    sink [HQ] an extra logit with a zero value row; causal, window W keeps
+    keys with 0 <= i-j < W.  Returns o [T,HQ,V], lse [T,HQ]."""
+    T, HQ, _ = q.shape
+    H = k.shape[1]
+    G = HQ // H
+    o = np.zeros((T, HQ, v.shape[2]))
+    lse = np.zeros((T, HQ))
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    vis = j <= i
+    if window and window > 0:
+        vis &= (i - j) < window
+    for h in range(HQ):
+        S = scale * q[:, h] @ k[:, h // G].T
+        if bias is not None:
+            S = S + bias[h]
+        S = np.where(vis, S, -np.inf)
+        if sink is not None:
+            S = np.concatenate([S, np.full((T, 1), sink[h])], axis=1)
+        m = S.max(axis=1, keepdims=True)
+        E = np.exp(S - m)
+        l = E.sum(axis=1, keepdims=True)
+        Pm = E / l
+        o[:, h] = Pm[:, :T] @ v[:, h // G]
+        lse[:, h] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def _err(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.max(np.abs(a - b))) if a.size else 0.0
+
+
+def _ok(name, err, tol):
+    return (err <= tol, f"{name}: err={err:.3e} tol={tol:.1e}")
+
+
+# ---------------------------------------------------------------------------
+# forward pins
+
+def pin_g_zero_textbook(seed=1):
+    """g = 0 is vanilla causal softmax attention (README introduction)."""
+    x = _inputs(seed, B=2, T=9, HQ=4, H=2, K=4, V=5)
+    g0 = np.zeros_like(x["g"])
+    worst = 0.0
+    for form in ("product", "prefix"):
+        o, lse = wo.forward(x["q"], x["k"], x["v"], g0, form=form)
+        for b in range(2):
+            ot, lt = textbook_attention(x["q"][b], x["k"][b], x["v"][b], 4 ** -0.5)
+            worst = max(worst, _err(o[b], ot), _err(lse[b], lt))
+    # and torch's own CPU attention (fp64, GQA by repeat_interleave)
+    o, _ = wo.forward(x["q"], x["k"], x["v"], g0)
+    qt = torch.from_numpy(x["q"]).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(x["k"]).permute(0, 2, 1, 3).repeat_interleave(2, dim=1)
+    vt = torch.from_numpy(x["v"]).permute(0, 2, 1, 3).repeat_interleave(2, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    worst = max(worst, _err(o, ref.permute(0, 2, 1, 3).numpy()))
+    return _ok("g=0 vs textbook/SDPA", worst, 1e-12)
+
+
+def pin_product_equals_prefix(seed=2):
+    """Product form (blog definition) == factorised prefix form, with every
+    option switched on."""
+    worst = 0.0
+    for decay in (False, True):
+        x = _inputs(seed, B=1, T=11, HQ=4, H=2, K=3, V=3, g_amp=0.4, decay=decay, gs=True,
+                    sink=True)
+        cu = np.array([0, 4, 11])
+        kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=3,
+                  cu_seqlens=cu)
+        o1, l1 = wo.forward(x["q"], x["k"], x["v"], x["g"], form="product", **kw)
+        o2, l2 = wo.forward(x["q"], x["k"], x["v"], x["g"], form="prefix", **kw)
+        worst = max(worst, _err(o1, o2), _err(l1, l2))
+        b1 = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], form="product", **kw)
+        b2 = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], form="prefix", **kw)
+        for key in ("dq", "dk", "dv", "dg", "dg_scalar", "dsink"):
+            worst = max(worst, _err(b1[key], b2[key]))
+    return _ok("product vs prefix form", worst, 1e-11)
+
+
+def pin_fox_scalar_gate(seed=3):
+    """g = 0 with g_scalar is the FoX formula softmax(scale q.k + log F_ij),
+    log F_ij = sum_{r=j+1..i} gs_r (blog, FoX formula)."""
+    x = _inputs(seed, B=1, T=8, HQ=2, H=1, K=4, V=3, gs=True)
+    g0 = np.zeros_like(x["g"])
+    o, lse = wo.forward(x["q"], x["k"], x["v"], g0, g_scalar=x["g_scalar"])
+    gs = x["g_scalar"][0]                      # [T,HQ]
+    cum = np.cumsum(gs, axis=0)                # inclusive
+    bias = np.stack([cum[:, h][:, None] - cum[:, h][None, :] for h in range(2)])
+    ot, lt = textbook_attention(x["q"][0], x["k"][0], x["v"][0], 4 ** -0.5, bias=bias)
+    return _ok("FoX additive bias", max(_err(o[0], ot), _err(lse[0], lt)), 1e-12)
+
+
+def pin_channel_constant_gate(seed=4):
+    """A gate equal across channels, g_{r,n} = c_r, multiplies the whole
+    logit: s_ij = scale * exp(C_i - C_j) * q_i . k_j (blog definition; the
+    gate acts on the input before the exponential kernel)."""
+    x = _inputs(seed, B=1, T=8, HQ=2, H=1, K=4, V=3)
+    c = _rng(seed + 100).standard_normal((1, 8, 2, 1)) * 0.5
+    g = np.repeat(c, 4, axis=3)
+    o, lse = wo.forward(x["q"], x["k"], x["v"], g)
+    C = np.cumsum(c[0, :, :, 0], axis=0)       # [T,HQ]
+    T = 8
+    o_t = np.zeros((T, 2, 3))
+    l_t = np.zeros((T, 2))
+    for h in range(2):
+        S = 0.5 * np.exp(C[:, h][:, None] - C[:, h][None, :]) * (x["q"][0, :, h] @ x["k"][0, :, 0].T)
+        S = np.where(np.tri(T, dtype=bool), S, -np.inf)
+        m = S.max(1, keepdims=True)
+        E = np.exp(S - m)
+        o_t[:, h] = (E / E.sum(1, keepdims=True)) @ x["v"][0, :, 0]
+        l_t[:, h] = (m + np.log(E.sum(1, keepdims=True)))[:, 0]
+    return _ok("channel-constant gate", max(_err(o[0], o_t), _err(lse[0], l_t)), 1e-12)
+
+
+def pin_window_sink_textbook(seed=5):
+    """g = 0 with a window and a sink: textbook windowed attention with one
+    extra logit in the softmax."""
+    x = _inputs(seed, B=1, T=10, HQ=4, H=2, K=3, V=3, sink=True)
+    g0 = np.zeros_like(x["g"])
+    o, lse = wo.forward(x["q"], x["k"], x["v"], g0, sink_bias=x["sink_bias"], window_size=4)
+    ot, lt = textbook_attention(x["q"][0], x["k"][0], x["v"][0], 3 ** -0.5,
+                                sink=x["sink_bias"], window=4)
+    return _ok("window + sink", max(_err(o[0], ot), _err(lse[0], lt)), 1e-12)
+
+
+def pin_gqa_repeat(seed=6):
+    """GQA equals repeating each kv head over its G query heads
+    (repeat_interleave), and dk/dv are the group sums."""
+    x = _inputs(seed, B=1, T=7, HQ=4, H=2, K=3, V=3, g_amp=0.3)
+    kr = np.repeat(x["k"], 2, axis=2)
+    vr = np.repeat(x["v"], 2, axis=2)
+    o1, l1 = wo.forward(x["q"], x["k"], x["v"], x["g"])
+    o2, l2 = wo.forward(x["q"], kr, vr, x["g"])
+    b1 = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"])
+    b2 = wo.backward(x["q"], kr, vr, x["g"], x["dO"])
+    worst = max(_err(o1, o2), _err(l1, l2), _err(b1["dq"], b2["dq"]), _err(b1["dg"], b2["dg"]),
+                _err(b1["dk"], b2["dk"].reshape(1, 7, 2, 2, 3).sum(3)),
+                _err(b1["dv"], b2["dv"].reshape(1, 7, 2, 2, 3).sum(3)))
+    return _ok("GQA = repeat_interleave", worst, 1e-12)
+
+
+def pin_varlen_independent(seed=7):
+    """Packed sequences behave as independent runs (no attention, prefix or
+    scalar-gate sum crosses a boundary)."""
+    x = _inputs(seed, B=1, T=12, HQ=2, H=1, K=3, V=3, gs=True, sink=True)
+    cu = np.array([0, 5, 5, 12])
+    kw = dict(sink_bias=x["sink_bias"], window_size=0)
+    o, lse = wo.forward(x["q"], x["k"], x["v"], x["g"], g_scalar=x["g_scalar"], cu_seqlens=cu, **kw)
+    bw = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], g_scalar=x["g_scalar"],
+                     cu_seqlens=cu, **kw)
+    worst = 0.0
+    dsink_sum = np.zeros(2)
+    for a, b in ((0, 5), (5, 12)):
+        sl = slice(a, b)
+        part = {n: x[n][:, sl] for n in ("q", "k", "v", "g", "dO")}
+        o2, l2 = wo.forward(part["q"], part["k"], part["v"], part["g"],
+                            g_scalar=x["g_scalar"][:, sl], **kw)
+        b2 = wo.backward(part["q"], part["k"], part["v"], part["g"], part["dO"],
+                         g_scalar=x["g_scalar"][:, sl], **kw)
+        worst = max(worst, _err(o[:, sl], o2), _err(lse[:, sl], l2))
+        for key in ("dq", "dk", "dv", "dg", "dg_scalar"):
+            worst = max(worst, _err(bw[key][:, sl], b2[key]))
+        dsink_sum += b2["dsink"]
+    worst = max(worst, _err(bw["dsink"], dsink_sum))
+    return _ok("varlen = independent runs", worst, 1e-12)
+
+
+def pin_decode_row(seed=8):
+    """The decode of the last row equals the forward's last row (README
+    Testing: decode reproduces the training forward token for token), and
+    decoding through the pre-rescaled cache k_tilde = k * 2^(R_c - P) with
+    the query scaled by 2^(p_curr - R_c) gives the same row (README
+    "Decode")."""
+    x = _inputs(seed, B=2, T=13, HQ=4, H=2, K=3, V=3, g_amp=0.3, decay=True)
+    o, lse = wo.forward(x["q"], x["k"], x["v"], x["g"])
+    o_r, l_r = wo.forward(x["q"], x["k"], x["v"], x["g"], rows=(12, 13))
+    worst = max(_err(o[:, 12], o_r[:, 12]), _err(lse[:, 12], l_r[:, 12]))
+    C = 4
+    kt, rc = wo.kv_cache(x["k"], x["g"], C)
+    P = wo.prefix_log2(x["g"])
+    scale = 3 ** -0.5
+    for b in range(2):
+        for h in range(4):
+            t = 12
+            qrow = x["q"][b, t, h]
+            s = np.array([scale * np.sum(qrow * 2.0 ** (P[b, t, h] - rc[b, j // C, h]) * kt[b, j, h])
+                          for j in range(t + 1)])
+            m = s.max()
+            e = np.exp(s - m)
+            od = (e / e.sum()) @ x["v"][b, :t + 1, h // 2]
+            worst = max(worst, _err(od, o[b, t, h]), _err(m + np.log(e.sum()), lse[b, t, h]))
+    return _ok("decode row", worst, 1e-12)
+
+
+def pin_prefix_closed_form(seed=9):
+    """2^P_t equals the product of the gates exp(g_u) over u <= t (blog:
+    P_t = sum_{u<=t} log g_u; README: base-2 prefix via scale 1/ln 2), per
+    sequence, with a carried-in prefix."""
+    r = _rng(seed)
+    g = r.standard_normal((1, 9, 2, 3)) * 0.3
+    cu = np.array([0, 4, 9])
+    carry = r.standard_normal((2, 2, 3))
+    P = wo.prefix_log2(g, cu_seqlens=cu, carry_in=carry)
+    worst = 0.0
+    for s, (a, b) in enumerate(((0, 4), (4, 9))):
+        for t in range(a, b):
+            prod = np.prod(np.exp(g[0, a:t + 1]), axis=0) * 2.0 ** carry[s]
+            worst = max(worst, _err(2.0 ** P[0, t], prod) / max(1.0, np.max(prod)))
+    return _ok("prefix = log2 of gate product", worst, 1e-12)
+
+
+def pin_prefix_magnitude_long_context():
+    """At T = 8192 with g = -0.05 |N(0,1)| the channel-mean |P_t| passes 160
+    near t = 2780 and reaches about 471 (blog, fast training: |P_t| exceeds
+    160 at sequence length 8192).  Closed form: E|N| = sqrt(2/pi), so the
+    mean slope is 0.05 * sqrt(2/pi) / ln 2 per row."""
+    r = _rng(10)
+    g = -0.05 * np.abs(r.standard_normal((1, 8192, 1, 128)))
+    P = wo.prefix_log2(g)
+    mean_abs = np.abs(P[0, :, 0, :]).mean(axis=1)
+    slope = 0.05 * np.sqrt(2 / np.pi) / LN2
+    t160 = int(np.argmax(mean_abs > 160))
+    ok = abs(mean_abs[-1] - slope * 8192) < 3.0 and abs(t160 - 160 / slope) < 40
+    return ok, f"|P_8192|={mean_abs[-1]:.1f} (expect {slope*8192:.1f}), t160={t160}"
+
+
+# ---------------------------------------------------------------------------
+# gradient pins
+
+def _fd_loss(x, kw, dO):
+    o, _ = wo.forward(x["q"], x["k"], x["v"], x["g"], **kw)
+    return float(np.sum(o * dO))
+
+
+def pin_gradients_fd(seed=11, h=1e-6):
+    """Every analytic gradient of the oracle matches central finite
+    differences with h = 1e-6 (README Testing: gradients checked against
+    central finite differences)."""
+    x = _inputs(seed, B=1, T=7, HQ=4, H=2, K=3, V=2, g_amp=0.4, gs=True, sink=True)
+    cu = np.array([0, 3, 7])
+    base = dict(window_size=3, cu_seqlens=cu)
+    names = ["q", "k", "v", "g", "g_scalar", "sink_bias"]
+    x = {n: x[n] for n in names + ["dO"]}
+
+    def kw_of(xx):
+        return dict(base, g_scalar=xx["g_scalar"], sink_bias=xx["sink_bias"])
+
+    an = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], **kw_of(x))
+    grads = dict(q=an["dq"], k=an["dk"], v=an["dv"], g=an["dg"], g_scalar=an["dg_scalar"],
+                 sink_bias=an["dsink"])
+    worst = 0.0
+    for n in names:
+        fd = np.zeros_like(x[n])
+        flat = x[n].reshape(-1)
+        for idx in range(flat.size):
+            keep = flat[idx]
+            flat[idx] = keep + h
+            lp = _fd_loss(x, kw_of(x), x["dO"])
+            flat[idx] = keep - h
+            lm = _fd_loss(x, kw_of(x), x["dO"])
+            flat[idx] = keep
+            fd.reshape(-1)[idx] = (lp - lm) / (2 * h)
+        rel = _err(grads[n], fd) / max(1e-3, float(np.max(np.abs(fd))))
+        worst = max(worst, rel)
+    return _ok("gradients vs central FD", worst, 1e-6)
+
+
+def pin_shift_invariance(seed=12):
+    """Adding a constant to g (or g_scalar) at a sequence's first position
+    leaves every logit unchanged, so their gradients there vanish."""
+    x = _inputs(seed, B=1, T=9, HQ=2, H=1, K=3, V=3, g_amp=0.4, gs=True)
+    cu = np.array([0, 4, 9])
+    bw = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], g_scalar=x["g_scalar"],
+                     cu_seqlens=cu)
+    scale = max(1.0, float(np.max(np.abs(bw["dg"]))))
+    worst = max(_err(bw["dg"][0, [0, 4]], 0.0), _err(bw["dg_scalar"][0, [0, 4]], 0.0)) / scale
+    return _ok("dg = 0 at sequence starts", worst, 1e-12)
+
+
+def pin_key_side_gate_grad(seed=13):
+    """The key-side part of the gate gradient is -K_j (.) dK_j per query
+    head (blog, fast training: dP_j = -ln2 K_j (.) dK_j with dP = ln2 dL),
+    and the query-side part is Q_i (.) dQ_i, so
+    dL_t = q_t (.) dq_t - k_t (.) dk^(h)_t and dg is its reverse cumsum."""
+    x = _inputs(seed, B=1, T=8, HQ=4, H=2, K=3, V=3, g_amp=0.3)
+    bw = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"])
+    kr = np.repeat(x["k"], 2, axis=2)
+    dL = x["q"] * bw["dq"] - kr * bw["dk_h"]
+    dg = np.flip(np.cumsum(np.flip(dL, axis=1), axis=1), axis=1)
+    return _ok("gate grad = q.dq - k.dk^(h), reverse cumsum", _err(dg, bw["dg"]), 1e-12)
+
+
+ALL_PINS = [pin_g_zero_textbook, pin_product_equals_prefix, pin_fox_scalar_gate,
+            pin_channel_constant_gate, pin_window_sink_textbook, pin_gqa_repeat,
+            pin_varlen_independent, pin_decode_row, pin_prefix_closed_form,
+            pin_prefix_magnitude_long_context, pin_gradients_fd, pin_shift_invariance,
+            pin_key_side_gate_grad]
+
+
+def run_all_pins():
+    out = {}
+    for p in ALL_PINS:
+        try:
+            out[p.__name__] = p()
+        except Exception as e:  # a planted mistake may also raise
+            out[p.__name__] = (False, f"raised {type(e).__name__}: {e}")
+    return out
