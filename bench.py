@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the Wall Attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (one JSON line on rank 0): fwd+bwd TFLOP/s of the training path at
+T = 8192 (B=1, HQ=16, H=4, K=V=128, bf16, decaying gate g = -0.05|N|), one
+step = prefix scan + forward + backward (dq, dk, dv, dg with the reverse
+scan), counting causal FLOPs: forward 2 * pairs * (K + V) per head,
+backward 2.5x that.  The same line carries the decode numbers (B=32,
+T_kv=32768, HQ=32, H=8, K=V=128, C=64): GB/s and tokens/s of one decode
+step, the cache build and prefix scan GB/s, and the 64-token streaming
+append loop.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
+the same workload on its own data (weak scaling, no collective on the data
+path); time is the max over ranks, value = all ranks' FLOPs / that time.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload, in the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from channel_decay_softmax_b200 import inputs as I  # noqa: E402
+
+METRIC = "fwd+bwd TFLOP/s & % of BF16 peak at T=8192; decode GB/s vs HBM peak"
+TRAIN_CFG = 3
+DECODE_CFG = 5
+SM_COUNT = 148
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+def train_flops(s: I.Spec, T=None):
+    """Algorithmic causal FLOPs of one forward and of forward+backward."""
+    T = s.T if T is None else T
+    pairs = I.causal_pairs(T, s.window) * s.B * s.HQ
+    fwd = 2.0 * pairs * (s.K + s.V)
+    return fwd, 3.5 * fwd
+
+
+def decode_bytes(s: I.Spec, T_kv: int):
+    """HBM bytes one decode step must move: k_tilde + v + r_cache + q +
+    p_curr + o (+ lse)."""
+    esz = 2 if s.dtype == torch.bfloat16 else 4
+    kt = s.B * T_kv * s.HQ * s.K * esz
+    v = s.B * T_kv * s.H * s.V * esz
+    rc = s.B * I.ceil_div(T_kv, s.chunk) * s.HQ * s.K * 4
+    small = s.B * s.HQ * (s.K * esz + s.K * 4 + s.V * esz + 4)
+    return kt + v + rc + small
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
+    timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], 0.0, set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = max(smax, float(r[2]))
+                for n, val in zip(names, r[5:9]):
+                    if "Active" in val and "Not" not in val:
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        busy = [x for x in sm if x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def bench_train(args, world, rank, peaks):
+    from channel_decay_softmax_b200 import api
+
+    s = I.spec(TRAIN_CFG, seed=I.CONFIGS[TRAIN_CFG].seed + 7919 * rank)
+    x = I.training_inputs(s, device="cuda")
+    q, k, v, g, dO = x["q"], x["k"], x["v"], x["g"], x["dO"]
+    fwd_flops, step_flops = train_flops(s)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        P = api.prefix_cumsum(g)
+        if ev is not None:
+            ev[0].record(stream)
+        o, lse = api.wall_attn_fwd(q, k, v, P, s.scale)
+        if ev is not None:
+            ev[1].record(stream)
+        out = api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale)
+        if ev is not None:
+            ev[2].record(stream)
+        return out
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()).start() if not args.no_clocks else None
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms = t0.elapsed_time(t1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # launches inside one step: prefix scan 1, forward 1, backward: dq 1,
+    # dk/dv 1, reduce 1, reverse scan 1
+    launches_per_step = 6
+    res = dict(ms=ms_max, value=world * step_flops / (ms_max * 1e-3) / 1e12,
+               fwd_ms=fwd_ms, bwd_ms=bwd_ms,
+               fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,
+               bwd_tflops=2.5 * fwd_flops / (bwd_ms * 1e-3) / 1e12,
+               launches=launches_per_step * args.steps, clocks=clk, spec=s,
+               step_flops=step_flops, fwd_flops=fwd_flops)
+    if not args.no_e2e:
+        res["e2e"] = bench_train_e2e(args, x, s, step_flops, world)
+    return res
+
+
+def bench_train_e2e(args, x, s, step_flops, world):
+    """The same step from pinned host buffers: H2D of q, k, v, g, dO and D2H
+    of dq, dk, dv, dg inside the timed region."""
+    from channel_decay_softmax_b200 import api
+
+    names_in = ("q", "k", "v", "g", "dO")
+    host_in = {n: x[n].cpu().pin_memory() for n in names_in}
+    dev_in = {n: torch.empty_like(x[n]) for n in names_in}
+    host_out = None
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nonlocal host_out
+        for n in names_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        P = api.prefix_cumsum(dev_in["g"])
+        o, lse = api.wall_attn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], P, s.scale)
+        dq, dk, dv, dg, _, _ = api.wall_attn_bwd(dev_in["dO"], dev_in["q"], dev_in["k"],
+                                                 dev_in["v"], P, o, lse, s.scale)
+        if host_out is None:
+            host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv, dg)]
+        for h, d in zip(host_out, (dq, dk, dv, dg)):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def bench_decode(args, rank, peaks):
+    from channel_decay_softmax_b200 import api
+
+    s = I.spec(DECODE_CFG, seed=I.CONFIGS[DECODE_CFG].seed + 7919 * rank)
+    d = I.decode_inputs(s, device="cuda", n_query_rows=64)
+    T = s.T
+    n_stream = 64
+    T0 = T - n_stream
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    out = {}
+    # prefix scan over the whole cache's gates (B*T*HQ*K elements)
+    a, b = ev(), ev()
+    a.record(stream)
+    P = api.prefix_cumsum(d["g"])
+    b.record(stream)
+    torch.cuda.synchronize()
+    n_el = d["g"].numel()
+    out["prefix_gbs"] = n_el * (2 + 4) / (a.elapsed_time(b) * 1e-3) / 1e9
+    # cache build over positions [0, T)
+    a, b = ev(), ev()
+    a.record(stream)
+    kt, rc = api.build_wall_kv_cache(d["k"], P, chunk_size=s.chunk)
+    b.record(stream)
+    torch.cuda.synchronize()
+    cb_bytes = d["k"].numel() * 2 + P.numel() * 4 + kt.numel() * 2 + rc.numel() * 4
+    out["cache_build_gbs"] = cb_bytes / (a.elapsed_time(b) * 1e-3) / 1e9
+    p_last = P[:, -1:].contiguous()
+    del P
+    q_last = d["q_tail"][:, -1:].contiguous()
+
+    def step():
+        return api.wall_attn_decode(q_last, d["v"], p_last, kt, rc, scale=s.scale,
+                                    cache_chunk_size=s.chunk)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    reps = max(10, args.steps)
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(reps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    nbytes = decode_bytes(s, T)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out.update(decode_ms=ms, decode_gbs=gbs, decode_frac_hbm=gbs / peaks["hbm_gbs"],
+               tokens_per_s=s.B / (ms * 1e-3), decode_bytes=nbytes,
+               decode_launches_per_step=2)
+    del kt, rc
+    torch.cuda.empty_cache()
+    # streaming append loop: cache of [0, T0) then 64 appended tokens
+    cache = api.WallDecodeCache(s.B, s.H, s.HQ, s.K, s.V, capacity=T, chunk_size=s.chunk,
+                                dtype=s.dtype, device="cuda", scale=s.scale)
+    cache.append(d["k"][:, :T0], d["v"][:, :T0], d["g"][:, :T0])
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record(stream)
+    for t in range(T0, T):
+        cache.step(d["q_tail"][:, t - T0:t - T0 + 1], d["k"][:, t:t + 1], d["v"][:, t:t + 1],
+                   d["g"][:, t:t + 1])
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_tok = a.elapsed_time(b) / n_stream
+    out.update(stream_ms_per_token=ms_tok, stream_tokens_per_s=s.B / (ms_tok * 1e-3))
+    del cache, d
+    torch.cuda.empty_cache()
+    out["workload"] = (f"decode B={s.B} T_kv={T} HQ={s.HQ} H={s.H} K=V={s.K} C={s.chunk} bf16, "
+                       f"g=-0.02|N|")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and the reference arm)
+
+def oracle_sample_tflops(T_sample: int):
+    """fp64 oracle forward+backward on the first T_sample rows of the
+    T=8192 workload (all 16 heads); returns (TFLOP/s in the bench's unit,
+    seconds, threads)."""
+    from oracle import wall_oracle as wo
+
+    s = I.spec(TRAIN_CFG, T=T_sample)
+    x = I.training_inputs(s)
+    threads = wo.default_threads()
+    t = time.perf_counter()
+    wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], scale=s.scale, nthreads=threads)
+    sec = time.perf_counter() - t
+    _, flops = train_flops(s)
+    return flops / sec / 1e12, sec, threads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    T_sample = int(os.environ.get("WALL_REF_T", "768"))
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample_tflops(T_sample)
+    for _ in range(args.steps):
+        vals.append(oracle_sample_tflops(T_sample))
+    v = statistics.mean(x[0] for x in vals)
+    sec = statistics.mean(x[1] for x in vals)
+    threads = vals[0][2]
+    sample = (f"fp64 oracle fwd+bwd on rows [0,{T_sample}) of the T=8192 workload, "
+              f"all 16 heads, per step")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(), "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_name():
+    s = I.spec(TRAIN_CFG)
+    return (f"wall_attn fwd+bwd B={s.B} T={s.T} HQ={s.HQ} H={s.H} K=V={s.K} bf16 causal, "
+            f"g=-0.05|N| (prefix scan + forward + backward incl. dg)")
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return 0
+
+    world, rank, local = dist_setup()
+    peaks = load_peaks()
+    tr = bench_train(args, world, rank, peaks)
+    dec = None
+    if not args.no_decode:
+        dec = bench_decode(args, rank, peaks)
+    barrier(world)
+    if rank == 0:
+        s = tr["spec"]
+        # dominant kernel: the backward (CUDA-core fp32 kernels on this path)
+        fma_peak = SM_COUNT * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        bwd_ach = tr["bwd_tflops"]
+        roof = {"kernel": "wall_attn_bwd", "bound": "alu", "achieved": bwd_ach,
+                "peak": fma_peak, "unit": "TFLOP/s", "frac": bwd_ach / fma_peak,
+                "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x sm_max_mhz",
+                "algorithmic": "2.5 x forward causal FLOPs per launch"}
+        line = {"metric": METRIC, "value": tr["value"], "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": tr["ms"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": workload_name(),
+                           "l2": "per-step working set ~0.45 GB > 126 MB L2 (no flush)",
+                           "parallelism": f"replicas x{world}"},
+                "frac_bf16_peak": tr["value"] / world / peaks["bf16_tflops_sustained"],
+                "fwd_tflops": tr["fwd_tflops"], "bwd_tflops": tr["bwd_tflops"],
+                "roofline": roof, "gpu_launches": tr["launches"],
+                "peaks": {k: peaks[k] for k in ("hbm_gbs", "bf16_tflops",
+                                                 "bf16_tflops_sustained", "source")}}
+        if tr.get("clocks"):
+            line["clocks"] = tr["clocks"]
+        if "e2e" in tr:
+            line["e2e"] = tr["e2e"]
+        if dec is not None:
+            line["decode"] = dec
+        if world == 1 and not args.no_cpu:
+            v, sec, threads = oracle_sample_tflops(int(os.environ.get("WALL_CPU_T", "1536")))
+            line["cpu_baseline"] = {
+                "value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "seconds": sec,
+                "sample": "fp64 oracle fwd+bwd on rows [0,%s) of the T=8192 workload, all 16 "
+                          "heads" % os.environ.get("WALL_CPU_T", "1536")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

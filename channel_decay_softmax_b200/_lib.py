@@ -1,0 +1,164 @@
+"""ctypes binding of libwall.so: one Python function per C-ABI entry point,
+same names, argument marshalling only (torch tensors in, device pointers
+out).  Every computation runs in the library's CUDA kernels; there is no
+fallback.  If the library or a CUDA device is missing, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwall.so")
+
+WALL_OK, WALL_ERR_INVALID_ARG, WALL_ERR_UNSUPPORTED, WALL_ERR_CUDA, WALL_ERR_TIMEOUT = range(5)
+WALL_BF16, WALL_FP32 = 0, 1
+
+EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn_fwd_workspace",
+           "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
+           "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status"]
+
+_lib = None
+
+
+class WallError(RuntimeError):
+    def __init__(self, call: str, code: int):
+        msg = lib().wall_error_string(code).decode() if _lib is not None else str(code)
+        super().__init__(f"{call} failed: {msg} (status {code})")
+        self.code = code
+
+
+def lib():
+    """Loads libwall.so (built by ``python -m channel_decay_softmax_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m channel_decay_softmax_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, ip, i, f, sz = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                ctypes.c_float, ctypes.c_size_t)
+        L.wall_version.restype = i
+        L.wall_error_string.restype = ctypes.c_char_p
+        L.wall_error_string.argtypes = [i]
+        L.wall_prefix_cumsum.restype = i
+        L.wall_prefix_cumsum.argtypes = [vp, i, fp, i, i, i, i, ip, i, fp, fp, vp]
+        L.wall_attn_fwd_workspace.restype = sz
+        L.wall_attn_fwd_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.wall_attn_fwd.restype = i
+        L.wall_attn_fwd.argtypes = [vp, vp, vp, fp, i, i, i, i, i, i, i, f, fp, fp, i, ip, i, vp,
+                                    fp, vp, sz, vp]
+        L.wall_attn_bwd_workspace.restype = sz
+        L.wall_attn_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.wall_attn_bwd.restype = i
+        L.wall_attn_bwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, i, i, f, fp, fp,
+                                    i, ip, i, vp, vp, vp, vp, fp, fp, vp, sz, vp]
+        L.wall_build_kv_cache.restype = i
+        L.wall_build_kv_cache.argtypes = [vp, fp, i, i, i, i, i, i, i, i, vp, fp, i, vp]
+        L.wall_attn_decode_workspace.restype = sz
+        L.wall_attn_decode_workspace.argtypes = [i, i, i, i, i, i]
+        L.wall_attn_decode.restype = i
+        L.wall_attn_decode.argtypes = [vp, vp, fp, vp, fp, fp, f, i, i, i, i, i, i, i, i, i, vp,
+                                       fp, vp, sz, vp]
+        L.wall_get_status.restype = i
+        L.wall_get_status.argtypes = [vp]
+        _lib = L
+    return _lib
+
+
+def _check(name, code):
+    if code != WALL_OK:
+        raise WallError(name, code)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return WALL_BF16
+    if t == torch.float32:
+        return WALL_FP32
+    raise TypeError(f"unsupported dtype {t}; use bfloat16 or float32")
+
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL); requires contiguous CUDA memory."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libwall takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libwall takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# one wrapper per entry point (argument order of include/wall.h)
+
+def wall_version() -> int:
+    return lib().wall_version()
+
+
+def wall_get_status(stream=None) -> int:
+    return lib().wall_get_status(_stream(stream))
+
+
+def wall_prefix_cumsum(g, P, B, T, HQ, K, cu_seqlens=None, n_seq=0, carry_in=None,
+                       carry_out=None, stream=None):
+    _check("wall_prefix_cumsum", lib().wall_prefix_cumsum(
+        _p(g), dtype_code(g.dtype), _p(P), B, T, HQ, K, _p(cu_seqlens), n_seq, _p(carry_in),
+        _p(carry_out), _stream(stream)))
+
+
+def wall_attn_fwd_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> int:
+    return lib().wall_attn_fwd_workspace(dtype_code(dtype), B, T, H, HQ, K, V,
+                                         int(bool(has_g_scalar)), n_seq)
+
+
+def wall_attn_fwd(q, k, v, P, B, T, H, HQ, K, V, scale, g_scalar, sink_bias, window_size,
+                  cu_seqlens, n_seq, o, lse, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_attn_fwd", lib().wall_attn_fwd(
+        _p(q), _p(k), _p(v), _p(P), dtype_code(q.dtype), B, T, H, HQ, K, V, float(scale),
+        _p(g_scalar), _p(sink_bias), int(window_size), _p(cu_seqlens), n_seq, _p(o), _p(lse),
+        _p(workspace), ws_bytes, _stream(stream)))
+
+
+def wall_attn_bwd_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> int:
+    return lib().wall_attn_bwd_workspace(dtype_code(dtype), B, T, H, HQ, K, V,
+                                         int(bool(has_g_scalar)), n_seq)
+
+
+def wall_attn_bwd(dO, q, k, v, P, o, lse, B, T, H, HQ, K, V, scale, g_scalar, sink_bias,
+                  window_size, cu_seqlens, n_seq, dq, dk, dv, dg, dg_scalar, dsink, workspace,
+                  stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_attn_bwd", lib().wall_attn_bwd(
+        _p(dO), _p(q), _p(k), _p(v), _p(P), _p(o), _p(lse), dtype_code(q.dtype), B, T, H, HQ, K,
+        V, float(scale), _p(g_scalar), _p(sink_bias), int(window_size), _p(cu_seqlens), n_seq,
+        _p(dq), _p(dk), _p(dv), _p(dg), _p(dg_scalar), _p(dsink), _p(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def wall_build_kv_cache(k, P, B, Tn, H, HQ, K, C, t0, k_tilde, r_cache, Tcap, stream=None):
+    _check("wall_build_kv_cache", lib().wall_build_kv_cache(
+        _p(k), _p(P), dtype_code(k.dtype), B, Tn, H, HQ, K, C, t0, _p(k_tilde), _p(r_cache),
+        Tcap, _stream(stream)))
+
+
+def wall_attn_decode_workspace(B, T_kv, H, HQ, V, C) -> int:
+    return lib().wall_attn_decode_workspace(B, T_kv, H, HQ, V, C)
+
+
+def wall_attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, scale, C, B, T_kv, Tcap, H, HQ,
+                     K, V, o, lse, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_attn_decode", lib().wall_attn_decode(
+        _p(q), _p(v), _p(p_curr), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
+        dtype_code(q.dtype), B, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _p(workspace), ws_bytes,
+        _stream(stream)))

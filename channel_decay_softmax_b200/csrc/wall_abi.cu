@@ -1,0 +1,306 @@
+// wall_abi.cu -- the extern "C" entry points of libwall.so: argument checks,
+// workspace layout and dispatch to the kernels.  See include/wall.h.
+#include <math.h>
+
+#include "wall_common.cuh"
+#include "wall_internal.h"
+
+namespace wall {
+
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr int kVersion = (0 << 16) | 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+bool ok_head_dim(int d) { return d >= 8 && d <= 128 && d % 8 == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int* status_ptr() {
+  static int* p = nullptr;
+  if (!p) {
+    int* q = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&q), g_status) != cudaSuccess)
+      return nullptr;
+    p = q;
+  }
+  return p;
+}
+
+// cu_seqlens must start at 0, never decrease and end at `rows`; a violation
+// is recorded in the status word (kernels clamp offsets, so none faults).
+__global__ void check_cu_kernel(const int32_t* cu, int n, long rows, int* status) {
+  for (int s = threadIdx.x; s <= n; s += blockDim.x) {
+    bool bad = false;
+    if (s == 0) bad = cu[0] != 0;
+    else bad = cu[s] < cu[s - 1];
+    if (s == n) bad = bad || cu[n] != rows;
+    if (bad) record_status(status, WALL_ERR_INVALID_ARG);
+  }
+}
+
+int check_cu(const int32_t* cu, int n, long rows, cudaStream_t stream) {
+  check_cu_kernel<<<1, 256, 0, stream>>>(cu, n, rows, status_ptr());
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+// Common shape checks of the training calls; fills `pb`.
+int make_problem(int dtype, int B, int T, int H, int HQ, int K, int V, float scale,
+                 int window_size, const int32_t* cu_seqlens, int n_seq, AttnProblem& pb) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || T < 0 || H < 1 || HQ < 1 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
+  if (!ok_head_dim(K) || !ok_head_dim(V)) return WALL_ERR_UNSUPPORTED;
+  if (cu_seqlens != nullptr) {
+    if (B != 1 || n_seq < 0 || n_seq > 65535 || !aligned16(cu_seqlens)) return WALL_ERR_INVALID_ARG;
+  }
+  if ((long)B * T * HQ * (long)(K > V ? K : V) >= (1L << 40)) return WALL_ERR_UNSUPPORTED;
+  pb.dtype = dtype;
+  pb.B = B; pb.T = T; pb.H = H; pb.HQ = HQ; pb.K = K; pb.V = V;
+  pb.scale = scale > 0.f ? scale : 1.f / sqrtf((float)K);
+  pb.window = window_size > 0 ? window_size : 0;
+  pb.rows = (long)B * T;
+  pb.seqs.cu = cu_seqlens;
+  pb.seqs.n = cu_seqlens ? n_seq : B;
+  pb.seqs.T = T;
+  pb.seqs.rows = pb.rows;
+  long nb = cu_seqlens ? (T + 63L) / 64 + n_seq : (long)B * ((T + 63L) / 64);
+  if (nb > 0x7fffffffL) return WALL_ERR_UNSUPPORTED;
+  pb.max_blocks64 = (int)nb;
+  if (HQ > 65535) return WALL_ERR_UNSUPPORTED;
+  return WALL_OK;
+}
+
+struct FwdWs {
+  size_t gs;  // inclusive prefix of g_scalar [rows, HQ]
+  size_t total;
+};
+FwdWs fwd_ws_layout(long rows, int HQ, int has_gs) {
+  FwdWs w;
+  w.gs = 0;
+  w.total = has_gs ? align256(sizeof(float) * rows * HQ) : 0;
+  return w;
+}
+
+struct BwdWs {
+  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, total;
+};
+BwdWs bwd_ws_layout(long rows, int HQ, int K, int V, int has_gs) {
+  BwdWs w;
+  size_t off = 0;
+  w.D = off;       off += align256(sizeof(float) * rows * HQ);
+  w.dq32 = off;    off += align256(sizeof(float) * rows * HQ * K);
+  w.dkh32 = off;   off += align256(sizeof(float) * rows * HQ * K);
+  w.dvh32 = off;   off += align256(sizeof(float) * rows * HQ * V);
+  w.dgs_row = off; off += align256(sizeof(float) * rows * HQ);
+  w.dgs_col = off; off += align256(sizeof(float) * rows * HQ);
+  w.gs = off;      off += has_gs ? align256(sizeof(float) * rows * HQ) : 0;
+  w.total = off;
+  return w;
+}
+
+inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+}  // namespace
+}  // namespace wall
+
+using namespace wall;
+
+extern "C" {
+
+int wall_version(void) { return kVersion; }
+
+const char* wall_error_string(int code) {
+  switch (code) {
+    case WALL_OK: return "ok";
+    case WALL_ERR_INVALID_ARG: return "invalid argument";
+    case WALL_ERR_UNSUPPORTED: return "unsupported dtype or size";
+    case WALL_ERR_CUDA: return "CUDA error";
+    case WALL_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int wall_get_status(wall_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WALL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return WALL_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return WALL_ERR_CUDA;
+  return v;
+}
+
+int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ, int K,
+                       const int32_t* cu_seqlens, int n_seq, const float* carry_in,
+                       float* carry_out, wall_stream_t stream) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || T < 0 || HQ < 1 || K < 1) return WALL_ERR_INVALID_ARG;
+  if (((long)HQ * K) % 8 != 0) return WALL_ERR_UNSUPPORTED;
+  if (cu_seqlens && (B != 1 || n_seq < 0 || !aligned16(cu_seqlens))) return WALL_ERR_INVALID_ARG;
+  const long rows = (long)B * T;
+  if (rows > 0 && (!ok_ptr(g) || !ok_ptr(P))) return WALL_ERR_INVALID_ARG;
+  if (!ok_opt(carry_in) || !ok_opt(carry_out)) return WALL_ERR_INVALID_ARG;
+  Seqs seqs;
+  seqs.cu = cu_seqlens;
+  seqs.n = cu_seqlens ? n_seq : B;
+  seqs.T = T;
+  seqs.rows = rows;
+  if (seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cu_seqlens) {
+    int rc = check_cu(cu_seqlens, n_seq, rows, s);
+    if (rc) return rc;
+  }
+  return scan_prefix_log2(g, dtype, P, (long)HQ * K, seqs, carry_in, carry_out, s);
+}
+
+size_t wall_attn_fwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                               int has_g_scalar, int n_seq) {
+  (void)n_seq;
+  AttnProblem pb;
+  if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
+  return fwd_ws_layout(pb.rows, HQ, has_g_scalar).total;
+}
+
+int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, int dtype, int B,
+                  int T, int H, int HQ, int K, int V, float scale, const float* g_scalar,
+                  const float* sink_bias, int window_size, const int32_t* cu_seqlens, int n_seq,
+                  void* o, float* lse, void* workspace, size_t workspace_bytes,
+                  wall_stream_t stream) {
+  AttnProblem pb;
+  int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
+  if (rc) return rc;
+  if (pb.rows == 0) return WALL_OK;
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o)) return WALL_ERR_INVALID_ARG;
+  if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(lse)) return WALL_ERR_INVALID_ARG;
+  FwdWs w = fwd_ws_layout(pb.rows, HQ, g_scalar != nullptr);
+  if (w.total > 0 && (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace)))
+    return WALL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cu_seqlens) {
+    rc = check_cu(cu_seqlens, n_seq, pb.rows, s);
+    if (rc) return rc;
+  }
+  FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.P = P; a.sink = sink_bias; a.o = o; a.lse = lse;
+  a.GS = nullptr;
+  if (g_scalar) {
+    float* gs = reinterpret_cast<float*>(at(workspace, w.gs));
+    rc = scan_prefix_plain(g_scalar, gs, HQ, pb.seqs, s);
+    if (rc) return rc;
+    a.GS = gs;
+  }
+  return attn_fwd_simt(pb, a, s);
+}
+
+size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                               int has_g_scalar, int n_seq) {
+  (void)n_seq;
+  AttnProblem pb;
+  if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
+  return bwd_ws_layout(pb.rows, HQ, K, V, has_g_scalar).total;
+}
+
+int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, const float* P,
+                  const void* o, const float* lse, int dtype, int B, int T, int H, int HQ,
+                  int K, int V, float scale, const float* g_scalar, const float* sink_bias,
+                  int window_size, const int32_t* cu_seqlens, int n_seq, void* dq, void* dk,
+                  void* dv, void* dg, float* dg_scalar, float* dsink, void* workspace,
+                  size_t workspace_bytes, wall_stream_t stream) {
+  AttnProblem pb;
+  int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
+  if (rc) return rc;
+  if ((g_scalar == nullptr) != (dg_scalar == nullptr)) return WALL_ERR_INVALID_ARG;
+  if (dsink != nullptr && sink_bias == nullptr) return WALL_ERR_INVALID_ARG;
+  if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(dg_scalar) || !ok_opt(dsink))
+    return WALL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dsink) {
+    if (cudaMemsetAsync(dsink, 0, sizeof(float) * HQ, s) != cudaSuccess) return WALL_ERR_CUDA;
+  }
+  if (pb.rows == 0) return WALL_OK;
+  if (!ok_ptr(dO) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o) ||
+      !ok_ptr(lse) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) || !ok_ptr(dg))
+    return WALL_ERR_INVALID_ARG;
+  BwdWs w = bwd_ws_layout(pb.rows, HQ, K, V, g_scalar != nullptr);
+  if (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace))
+    return WALL_ERR_INVALID_ARG;
+  if (cu_seqlens) {
+    rc = check_cu(cu_seqlens, n_seq, pb.rows, s);
+    if (rc) return rc;
+  }
+  BwdArgs a;
+  a.dO = dO; a.q = q; a.k = k; a.v = v; a.o = o; a.P = P; a.lse = lse;
+  a.sink = sink_bias;
+  a.dsink = dsink;
+  a.D = reinterpret_cast<float*>(at(workspace, w.D));
+  a.dq32 = reinterpret_cast<float*>(at(workspace, w.dq32));
+  a.dkh32 = reinterpret_cast<float*>(at(workspace, w.dkh32));
+  a.dvh32 = reinterpret_cast<float*>(at(workspace, w.dvh32));
+  a.dgs_row = reinterpret_cast<float*>(at(workspace, w.dgs_row));
+  a.dgs_col = reinterpret_cast<float*>(at(workspace, w.dgs_col));
+  a.GS = nullptr;
+  if (g_scalar) {
+    float* gs = reinterpret_cast<float*>(at(workspace, w.gs));
+    rc = scan_prefix_plain(g_scalar, gs, HQ, pb.seqs, s);
+    if (rc) return rc;
+    a.GS = gs;
+  }
+  rc = attn_bwd_simt(pb, a, s);
+  if (rc) return rc;
+  rc = attn_bwd_reduce(pb, a, dq, dk, dv, s);
+  if (rc) return rc;
+  // dg = reverse cumulative sum of dL (held in dq32 after the reduce)
+  rc = scan_reverse(a.dq32, dg, dtype, (long)HQ * K, pb.seqs, s);
+  if (rc) return rc;
+  if (g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, HQ, pb.seqs, s);
+  return rc;
+}
+
+int wall_build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ,
+                        int K, int C, int t0, void* k_tilde, float* r_cache, int Tcap,
+                        wall_stream_t stream) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || Tn < 0 || H < 1 || HQ < 1 || HQ % H != 0 || C < 1 || t0 < 0 || Tcap < 0)
+    return WALL_ERR_INVALID_ARG;
+  if ((long)t0 + Tn > Tcap) return WALL_ERR_INVALID_ARG;
+  if (K < 8 || K % 8 != 0) return WALL_ERR_UNSUPPORTED;
+  if ((long)B * Tn == 0) return WALL_OK;
+  if (!ok_ptr(k) || !ok_ptr(P) || !ok_ptr(k_tilde) || !ok_ptr(r_cache)) return WALL_ERR_INVALID_ARG;
+  return build_kv_cache(k, P, dtype, B, Tn, H, HQ, K, C, t0, k_tilde, r_cache, Tcap,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t wall_attn_decode_workspace(int B, int T_kv, int H, int HQ, int V, int C) {
+  if (B < 0 || T_kv < 1 || H < 1 || HQ < 1 || HQ % H != 0 || V < 1 || C < 1) return 0;
+  const int S = decode_splits(B, T_kv, H, C);
+  return align256(sizeof(float) * (size_t)B * HQ * S * (V + 2));
+}
+
+int wall_attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,
+                     const float* r_cache, const float* sink_bias, float scale, int C, int dtype,
+                     int B, int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
+                     void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || T_kv < 1 || Tcap < T_kv || H < 1 || HQ < 1 || HQ % H != 0 || C < 1)
+    return WALL_ERR_INVALID_ARG;
+  if (!ok_head_dim(K) || !ok_head_dim(V) || HQ / H > 32) return WALL_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return WALL_ERR_UNSUPPORTED;
+  if (B == 0) return WALL_OK;
+  if (!ok_ptr(q) || !ok_ptr(v) || !ok_ptr(p_curr) || !ok_ptr(k_tilde) || !ok_ptr(r_cache) ||
+      !ok_ptr(o) || !ok_opt(sink_bias) || !ok_opt(lse))
+    return WALL_ERR_INVALID_ARG;
+  const int S = decode_splits(B, T_kv, H, C);
+  const size_t need = align256(sizeof(float) * (size_t)B * HQ * S * (V + 2));
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    return WALL_ERR_INVALID_ARG;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)K);
+  return attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, sc, C, dtype, B, T_kv, Tcap, H,
+                     HQ, K, V, o, lse, static_cast<float*>(workspace), S,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// wall_internal.h -- launchers behind the C ABI (host side, namespace wall).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "wall.h"
+#include "wall_common.cuh"
+
+namespace wall {
+
+// ---- scans (wall_scan.cu) ----
+int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seqs,
+                     const float* carry_in, float* carry_out, cudaStream_t stream);
+int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream);
+int scan_reverse(const float* x, void* y, int out_dtype, long C, const Seqs& seqs,
+                 cudaStream_t stream);
+
+// ---- attention problem description shared by the fwd/bwd launchers ----
+struct AttnProblem {
+  int dtype;
+  int B, T, H, HQ, K, V;
+  float scale;
+  int window;        // <= 0: none
+  Seqs seqs;         // sequences over the B*T flattened rows
+  long rows;         // B*T
+  int max_blocks64;  // upper bound on 64-row blocks over all sequences
+};
+
+struct FwdArgs {
+  const void *q, *k, *v;
+  const float* P;
+  const float* GS;    // inclusive prefix of g_scalar [rows,HQ] or nullptr
+  const float* sink;  // [HQ] or nullptr
+  void* o;
+  float* lse;
+};
+
+struct BwdArgs {
+  const void *dO, *q, *k, *v, *o;
+  const float* P;
+  const float* lse;
+  const float* GS;
+  const float* sink;
+  // fp32 workspace
+  float* D;       // [rows,HQ]
+  float* dq32;    // [rows,HQ,K]  (becomes dL after the reduce)
+  float* dkh32;   // [rows,HQ,K]
+  float* dvh32;   // [rows,HQ,V]
+  float* dgs_row; // [rows,HQ]
+  float* dgs_col; // [rows,HQ]
+  float* dsink;   // [HQ] or nullptr (accumulated atomically, zeroed by the caller)
+};
+
+// ---- SIMT fp32 attention (wall_attn_simt.cu) ----
+int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);
+int attn_bwd_simt(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream);
+// dq, dk, dv outputs and dL (in place of dq32) from the per-head fp32 grads
+int attn_bwd_reduce(const AttnProblem& pb, const BwdArgs& a, void* dq, void* dk, void* dv,
+                    cudaStream_t stream);
+
+// ---- decode cache + decode (wall_decode.cu) ----
+int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ, int K,
+                   int C, int t0, void* k_tilde, float* r_cache, int Tcap, cudaStream_t stream);
+int decode_splits(int B, int T_kv, int H, int C);
+int attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,
+                const float* r_cache, const float* sink, float scale, int C, int dtype, int B,
+                int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
+                float* ws, int splits, cudaStream_t stream);
+
+}  // namespace wall

@@ -1,0 +1,199 @@
+/*
+ * wall.h -- C ABI of the B200 Wall Attention hot path (libwall.so).
+ *
+ * Wall Attention (Tilde blog "Wall Attention", "Definition: Wall Attention";
+ * wall-attention-release README, introduction) is causal softmax attention
+ * whose logit carries a per-channel decay accumulated between the two
+ * positions:
+ *
+ *     s_ij = scale * sum_n exp(sum_{r=j+1..i} g_{r,n}) q_{i,n} k_{j,n}
+ *            [+ sum_{r=j+1..i} g_scalar_r]                 (optional)
+ *     o_i  = sum_{j<=i} softmax_j(s_ij) v_j
+ *
+ * g is the natural-log gate per query head and channel, so g = 0 is vanilla
+ * softmax attention.  The kernels work with the base-2 prefix
+ * P_t = sum_{u<=t} g_u / ln 2 (README "Decode": cumulative sum of g with scale
+ * 1/ln 2; blog: P_t = sum_{u<=t} log g_u), and use exp2(P_i - P_j) =
+ * exp2(P_i - R) * exp2(R - P_j) with block anchors R (blog, fast training,
+ * per-block anchor).
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, row-major, in the README's BSHD layout:
+ *       q [B,T,HQ,K], k [B,T,H,K], v [B,T,H,V], g and P [B,T,HQ,K],
+ *       g_scalar [B,T,HQ], sink_bias [HQ], o [B,T,HQ,V], lse [B,T,HQ].
+ *     With cu_seqlens (varlen packing, README "Usage": requires B == 1) the
+ *     T rows hold n_seq sequences back to back; attention, P and the scalar
+ *     gate prefix never cross a sequence boundary.
+ *   - GQA: HQ % H == 0 and query head h reads kv head h / (HQ/H).
+ *   - dtype is WALL_BF16 or WALL_FP32 and applies to q, k, v, g, o, dO, dq,
+ *     dk, dv, dg, k_tilde.  P, lse, r_cache, g_scalar, sink_bias, dg_scalar,
+ *     dsink and carries are always fp32; cu_seqlens is int32 [n_seq+1],
+ *     starting at 0, non-decreasing and ending at T.
+ *   - Pointers are device pointers, 16-byte aligned.  The caller allocates
+ *     and owns every buffer, including workspaces whose sizes the *_workspace
+ *     calls return; the library allocates no device memory and keeps no
+ *     state between calls except one device status word (wall_get_status).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are checked on the host before any launch;
+ *     on a bad argument nothing is launched and the call returns an error.
+ *     Kernels never trap: a device-side failure (a bounded wait that timed
+ *     out) is recorded in the status word.
+ *   - scale <= 0 selects K^-0.5 (README "Usage": scale = K ** -0.5).
+ *     window_size <= 0 means no window; otherwise key j is visible from
+ *     query i iff 0 <= i - j < window_size.
+ *   - Empty problems (B == 0 or T == 0) are valid and launch nothing.
+ */
+#ifndef WALL_H
+#define WALL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* wall_stream_t; /* same type as cudaStream_t */
+
+/* status codes */
+#define WALL_OK 0
+#define WALL_ERR_INVALID_ARG 1 /* null pointer, bad shape, HQ % H != 0, misalignment, ... */
+#define WALL_ERR_UNSUPPORTED 2 /* dtype or head size not built */
+#define WALL_ERR_CUDA 3        /* a CUDA launch or copy failed */
+#define WALL_ERR_TIMEOUT 4     /* a kernel's bounded wait expired (from wall_get_status) */
+
+/* dtypes */
+#define WALL_BF16 0
+#define WALL_FP32 1
+
+/* Library version, (major << 16) | minor. */
+int wall_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* wall_error_string(int code);
+
+/*
+ * wall_prefix_cumsum -- base-2 inclusive prefix of the log-gate.
+ * README "Decode": P = cumulative sum of g with scale 1/ln 2; blog
+ * "Definition: Wall Attention": P_t = sum_{u<=t} log g_u.
+ *
+ *   P[b,t,h,n] = c[s,h,n] + (sum_{u = start(s) .. t} g[b,u,h,n]) / ln 2
+ *
+ * where s is the sequence holding row t (batch row b without cu_seqlens) and
+ * c = carry_in (NULL: zero).  g [B,T,HQ,K] in `dtype`; P [B,T,HQ,K] fp32.
+ * carry_in / carry_out: [n_s, HQ, K] fp32 with n_s = B (no cu_seqlens) or
+ * n_seq; carry_out receives each sequence's last P (carry_in when empty), so
+ * a stream of tokens can be scanned piece by piece.  Either may be NULL.
+ * Returns WALL_ERR_UNSUPPORTED for HQ*K not a multiple of 8.
+ */
+int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ, int K,
+                       const int32_t* cu_seqlens, int n_seq, const float* carry_in,
+                       float* carry_out, wall_stream_t stream);
+
+/*
+ * wall_attn_fwd_workspace -- bytes of workspace wall_attn_fwd needs for
+ * these sizes (0 is possible).  Returns 0 on bad sizes as well.
+ */
+size_t wall_attn_fwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                               int has_g_scalar, int n_seq);
+
+/*
+ * wall_attn_fwd -- Wall Attention forward (README "Usage": wall_attn; blog
+ * "Definition: Wall Attention").
+ *
+ * In:  q [B,T,HQ,K], k [B,T,H,K], v [B,T,H,V] in `dtype`; P [B,T,HQ,K] fp32
+ *      from wall_prefix_cumsum of g; optional g_scalar [B,T,HQ] fp32 (FoX-
+ *      style additive log-gate: the logit gains sum_{r=j+1..i} g_scalar_r,
+ *      added after `scale`), sink_bias [HQ] fp32 (one extra logit per head
+ *      with a zero value row, included in lse), window_size, cu_seqlens.
+ * Out: o [B,T,HQ,V] in `dtype`; lse [B,T,HQ] fp32, natural log of the
+ *      softmax denominator (sink included).  lse may be NULL.
+ * Supported: K, V in {16, 32, 64, 128} (multiples of 16 up to 128); the
+ * tensor-core path takes bf16 with K == V in {64, 128}, other cases use the
+ * fp32 SIMT path.  fp32 inputs are computed with fp32 products throughout.
+ */
+int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, int dtype, int B,
+                  int T, int H, int HQ, int K, int V, float scale, const float* g_scalar,
+                  const float* sink_bias, int window_size, const int32_t* cu_seqlens, int n_seq,
+                  void* o, float* lse, void* workspace, size_t workspace_bytes,
+                  wall_stream_t stream);
+
+/* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs. */
+size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                               int has_g_scalar, int n_seq);
+
+/*
+ * wall_attn_bwd -- gradients of a scalar loss through wall_attn_fwd (README
+ * "Usage": analytic gradients for q, k, v, g, and g_scalar).
+ *
+ * In:  dO [B,T,HQ,V], and the forward's q, k, v, P, options, o and lse.
+ * Out: dq [B,T,HQ,K], dk [B,T,H,K], dv [B,T,H,V], dg [B,T,HQ,K] in `dtype`;
+ *      dg_scalar [B,T,HQ] fp32 (must be NULL iff g_scalar is NULL);
+ *      dsink [HQ] fp32 (optional, may be NULL; requires sink_bias).
+ * The gate gradient follows the blog's fused gate gradient (fast training):
+ * per query head, dL_t = q_t (.) dq_t - k_t (.) dk^(h)_t with the key-side
+ * term -K_j (.) dK_j, then dg = the reverse cumulative sum of dL within each
+ * sequence.  dk^(h), dv^(h) are summed over each GQA group.
+ */
+int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, const float* P,
+                  const void* o, const float* lse, int dtype, int B, int T, int H, int HQ,
+                  int K, int V, float scale, const float* g_scalar, const float* sink_bias,
+                  int window_size, const int32_t* cu_seqlens, int n_seq, void* dq, void* dk,
+                  void* dv, void* dg, float* dg_scalar, float* dsink, void* workspace,
+                  size_t workspace_bytes, wall_stream_t stream);
+
+/*
+ * wall_build_kv_cache -- pre-rescaled decode cache (README "Decode":
+ * build_wall_kv_cache; k_tilde[j] = k[j] * exp2(R_c - P[j]) with a per-chunk
+ * anchor R_c).
+ *
+ * Writes cache positions t0 .. t0+Tn-1 of each batch row:
+ *   c = t / C;  R_c = r_cache[b,c,h,:] if c*C < t0 (chunk already started:
+ *   its anchor is kept), else R_c = P at position c*C (written to r_cache);
+ *   k_tilde[b,t,h,:] = k[b,t-t0,h/G,:] * exp2(R_c - P[b,t-t0,h,:]).
+ * In:  k [B,Tn,H,K] (`dtype`) and P [B,Tn,HQ,K] fp32 for positions t0..t0+Tn-1.
+ * Out: k_tilde [B,Tcap,HQ,K] (`dtype`), r_cache [B,ceil(Tcap/C),HQ,K] fp32.
+ * Requires t0 + Tn <= Tcap and C >= 1.  At chunk starts k_tilde equals k
+ * bit for bit (the factor is exp2(0) = 1).
+ */
+int wall_build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ,
+                        int K, int C, int t0, void* k_tilde, float* r_cache, int Tcap,
+                        wall_stream_t stream);
+
+/* wall_attn_decode_workspace -- bytes of workspace wall_attn_decode needs. */
+size_t wall_attn_decode_workspace(int B, int T_kv, int H, int HQ, int V, int C);
+
+/*
+ * wall_attn_decode -- one decode step against the pre-rescaled cache
+ * (README "Decode": wall_attn_decode; blog: the decode kernel folds the gate
+ * into the cached keys and needs no gate arithmetic in its inner loop).
+ *
+ * For each batch row b and query head h, with c(j) = j / C:
+ *   s_j = scale * sum_n q[b,h,n] exp2(p_curr[b,h,n] - r_cache[b,c(j),h,n])
+ *                  * k_tilde[b,j,h,n],      j = 0 .. T_kv-1
+ *   o = sum_j softmax(s, sink)_j v[b,j,h/G,:],   lse = log-sum-exp (natural)
+ * In:  q [B,1,HQ,K] (`dtype`), p_curr [B,1,HQ,K] fp32 (P at the current
+ *      position), k_tilde [B,Tcap,HQ,K] and v [B,Tcap,H,V] (`dtype`, the
+ *      first T_kv positions are read), r_cache [B,ceil(Tcap/C),HQ,K] fp32,
+ *      sink_bias [HQ] or NULL.  The current token's own key must already be
+ *      in the cache (position T_kv-1), so T_kv >= 1.
+ * Out: o [B,1,HQ,V] (`dtype`), lse [B,1,HQ] fp32 (may be NULL).
+ * Supported: bf16 or fp32, K and V multiples of 8 up to 128.
+ */
+int wall_attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,
+                     const float* r_cache, const float* sink_bias, float scale, int C, int dtype,
+                     int B, int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
+                     void* workspace, size_t workspace_bytes, wall_stream_t stream);
+
+/*
+ * wall_get_status -- synchronizes `stream`, returns the device status word
+ * (WALL_OK or WALL_ERR_TIMEOUT) and clears it.  Returns WALL_ERR_CUDA if the
+ * synchronization itself fails.
+ */
+int wall_get_status(wall_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WALL_H */

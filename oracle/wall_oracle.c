@@ -74,6 +74,8 @@ typedef struct {
     const int* units;      /* NULL: all nseq*HQ units */
     int n_units;
     long row_lo, row_hi;   /* rows relative to sequence start; hi < 0 = all */
+    long q_rows;           /* > 0: q holds only rows [row_lo, row_lo+q_rows) of
+                              each sequence, as [nseq, q_rows, HQ, K] */
     /* forward outputs */
     double *o, *lse;
     /* backward outputs (per query head; dk/dv before the GQA reduction) */
@@ -133,7 +135,8 @@ static void unit_tables(const job_t* J, unit_t* U) {
 static void row_logits(const job_t* J, const unit_t* U, long i, long jmin,
                        double* sc, double* F, double* Fmat) {
     const int K = J->K, HQ = J->HQ, H = J->H;
-    const double* qi = J->q + ((U->s0 + i) * HQ + U->h) * K;
+    const long qrow = J->q_rows > 0 ? (long)U->seq * J->q_rows + (i - J->row_lo) : U->s0 + i;
+    const double* qi = J->q + (qrow * HQ + U->h) * K;
     double bias = 0.0;
     for (int n = 0; n < K; ++n) F[n] = 1.0;
     for (long j = i; j >= jmin; --j) {
@@ -342,7 +345,7 @@ static int run(job_t* J, int nthreads) {
 int wo_forward(const double* q, const double* k, const double* v, const double* g,
                const double* gs, const double* sink, long TT, int H, int HQ, int K, int V,
                double scale, long window, const long* cu, int nseq, int form,
-               const int* units, int n_units, long row_lo, long row_hi,
+               const int* units, int n_units, long row_lo, long row_hi, long q_rows,
                double* o, double* lse, int nthreads) {
     job_t J;
     memset(&J, 0, sizeof(J));
@@ -350,6 +353,8 @@ int wo_forward(const double* q, const double* k, const double* v, const double* 
     J.TT = TT; J.H = H; J.HQ = HQ; J.K = K; J.V = V;
     J.scale = scale; J.window = window; J.cu = cu; J.nseq = nseq; J.form = form;
     J.units = units; J.n_units = n_units; J.row_lo = row_lo; J.row_hi = row_hi;
+    J.q_rows = q_rows;
+    if (q_rows > 0 && (row_lo < 0 || row_hi < 0 || row_hi - row_lo > q_rows)) return 1;
     J.o = o; J.lse = lse;
     return run(&J, nthreads);
 }

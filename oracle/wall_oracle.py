@@ -65,8 +65,8 @@ def _load():
         lib.wo_forward.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_long, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                    ctypes.c_long, _lp, ctypes.c_int, ctypes.c_int, _ip,
-                                   ctypes.c_int, ctypes.c_long, ctypes.c_long, _dp, _dp,
-                                   ctypes.c_int]
+                                   ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                   _dp, _dp, ctypes.c_int]
         lib.wo_backward.restype = ctypes.c_int
         lib.wo_backward.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_long,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -145,7 +145,8 @@ def prefix_log2(g, cu_seqlens=None, carry_in=None):
 
 
 def forward(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size=0,
-            cu_seqlens=None, form="product", units=None, rows=None, nthreads=None):
+            cu_seqlens=None, form="product", units=None, rows=None, nthreads=None,
+            q_rows_only=False):
     """Wall forward in fp64: returns (o [B,T,HQ,V], lse [B,T,HQ]).
 
     form="product" evaluates prod_{r=j+1..i} exp(g_r) directly (blog,
@@ -153,10 +154,19 @@ def forward(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size=0
     with L the natural-log prefix (blog, factorised form).  ``units`` lists
     (sequence * HQ + head) pairs to compute and ``rows`` = (lo, hi) limits
     the rows (relative to each sequence start); entries not computed are NaN.
+    With ``q_rows_only`` q holds only the queries of those rows,
+    [B, hi - lo, HQ, K] (dense batches only).
     """
     q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
-    B, T, HQ, K = q.shape
+    B, T, HQ, K = g.shape
     H, V = k.shape[2], v.shape[3]
+    q_rows = 0
+    if q_rows_only:
+        if rows is None or cu_seqlens is not None:
+            raise ValueError("q_rows_only needs rows=(lo, hi) and dense batches")
+        q_rows = rows[1] - rows[0]
+        if q.shape != (B, q_rows, HQ, K):
+            raise ValueError("q must be [B, hi - lo, HQ, K]")
     if scale is None:
         scale = K ** -0.5
     cu = _seqs(B, T, cu_seqlens)
@@ -169,7 +179,7 @@ def forward(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size=0
     rc = _load().wo_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gs), _ptr(sk), B * T, H,
                             HQ, K, V, float(scale), int(window_size or 0), _ptr(cu, _lp), nseq,
                             0 if form == "product" else 1, _ptr(u, _ip), nu, int(lo), int(hi),
-                            _ptr(o), _ptr(lse), int(nthreads or default_threads()))
+                            int(q_rows), _ptr(o), _ptr(lse), int(nthreads or default_threads()))
     if rc:
         raise ValueError("oracle forward: bad arguments")
     return o, lse

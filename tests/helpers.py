@@ -1,0 +1,62 @@
+"""Comparison helpers and tolerances shared by the parity tests.
+
+Tolerances (CUDA path vs the fp64 oracle on the same seeded inputs):
+  fp32 inputs: max-abs error <= 1e-5 on o, lse and every gradient;
+  bf16 inputs: max-abs error <= 2e-2 on o and lse, relative L2 error
+               <= 5e-2 on each gradient.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+TOL_FP32_MAXABS = 1e-5
+TOL_BF16_O_MAXABS = 2e-2
+TOL_BF16_GRAD_RELL2 = 5e-2
+
+
+def np64(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().double().numpy() if t.dtype == torch.bfloat16 \
+            else t.detach().cpu().double().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def max_abs(a, b, mask=None):
+    a, b = np64(a), np64(b)
+    d = np.abs(a - b)
+    if mask is not None:
+        d = d[mask]
+    return float(d.max()) if d.size else 0.0
+
+
+def rel_l2(a, b, mask=None):
+    a, b = np64(a), np64(b)
+    if mask is not None:
+        a, b = a[mask], b[mask]
+    den = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
+
+
+def assert_fwd(dtype, o_gpu, o_ref, lse_gpu=None, lse_ref=None, mask=None, what=""):
+    tol = TOL_FP32_MAXABS if dtype == torch.float32 else TOL_BF16_O_MAXABS
+    e = max_abs(o_gpu, o_ref, mask)
+    assert e <= tol, f"{what} o max-abs {e:.3e} > {tol}"
+    if lse_gpu is not None:
+        e = max_abs(lse_gpu, lse_ref, mask)
+        assert e <= tol, f"{what} lse max-abs {e:.3e} > {tol}"
+
+
+def assert_grad(dtype, name, g_gpu, g_ref, mask=None, what=""):
+    if dtype == torch.float32:
+        e = max_abs(g_gpu, g_ref, mask)
+        assert e <= TOL_FP32_MAXABS, f"{what} {name} max-abs {e:.3e} > {TOL_FP32_MAXABS}"
+    else:
+        e = rel_l2(g_gpu, g_ref, mask)
+        assert e <= TOL_BF16_GRAD_RELL2, f"{what} {name} rel-L2 {e:.3e} > {TOL_BF16_GRAD_RELL2}"
+
+
+def cuda_ok() -> bool:
+    return torch.cuda.is_available()

@@ -1,0 +1,141 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol that
+include/wall.h declares, and rejects bad arguments on the host before any
+launch (no GPU needed for any of these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from channel_decay_softmax_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wall.h")
+
+FAKE = 4096  # an aligned, never dereferenced address: every call below fails its checks first
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(wall_\w+)\s*\(", src,
+                                 flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from channel_decay_softmax_b200 import build
+    build.build()
+    return L.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.EXPORTS)
+
+
+def test_version_and_error_strings(lib):
+    assert lib.wall_version() >= 1
+    for code, word in ((0, b"ok"), (1, b"invalid"), (2, b"unsupported"), (3, b"CUDA"),
+                       (4, b"timed out")):
+        assert word in lib.wall_error_string(code)
+
+
+def _fwd(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, P=FAKE, dtype=0, B=1, T=16, H=2, HQ=4, K=64, V=64,
+             scale=0.0, gs=None, sink=None, window=0, cu=None, n_seq=0, o=FAKE, lse=FAKE,
+             ws=None, ws_bytes=0, stream=None)
+    a.update(over)
+    return lib.wall_attn_fwd(a["q"], a["k"], a["v"], a["P"], a["dtype"], a["B"], a["T"], a["H"],
+                             a["HQ"], a["K"], a["V"], a["scale"], a["gs"], a["sink"],
+                             a["window"], a["cu"], a["n_seq"], a["o"], a["lse"], a["ws"],
+                             a["ws_bytes"], a["stream"])
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert _fwd(lib, HQ=3) == L.WALL_ERR_INVALID_ARG            # HQ % H != 0
+    assert _fwd(lib, H=0) == L.WALL_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=5) == L.WALL_ERR_INVALID_ARG
+    assert _fwd(lib, K=100) == L.WALL_ERR_UNSUPPORTED           # not a multiple of 8
+    assert _fwd(lib, V=256) == L.WALL_ERR_UNSUPPORTED
+    assert _fwd(lib, q=None) == L.WALL_ERR_INVALID_ARG
+    assert _fwd(lib, q=FAKE + 4) == L.WALL_ERR_INVALID_ARG      # misaligned
+    assert _fwd(lib, B=2, cu=FAKE, n_seq=1) == L.WALL_ERR_INVALID_ARG  # varlen needs B == 1
+    # g_scalar needs workspace; none given
+    assert _fwd(lib, gs=FAKE) == L.WALL_ERR_INVALID_ARG
+    assert _fwd(lib, T=0) == L.WALL_OK                          # empty: nothing to do
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    def bwd(**over):
+        a = dict(dO=FAKE, gs=None, dgs=None, sink=None, dsink=None, ws=None, ws_bytes=0, T=16,
+                 HQ=4)
+        a.update(over)
+        return lib.wall_attn_bwd(a["dO"], FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, a["T"], 2,
+                                 a["HQ"], 64, 64, 0.0, a["gs"], a["sink"], 0, None, 0, FAKE,
+                                 FAKE, FAKE, FAKE, a["dgs"], a["dsink"], a["ws"], a["ws_bytes"],
+                                 None)
+    assert bwd(HQ=5) == L.WALL_ERR_INVALID_ARG
+    assert bwd(gs=FAKE) == L.WALL_ERR_INVALID_ARG               # dg_scalar missing
+    assert bwd(dgs=FAKE) == L.WALL_ERR_INVALID_ARG              # g_scalar missing
+    assert bwd(dO=None) == L.WALL_ERR_INVALID_ARG
+    assert bwd() == L.WALL_ERR_INVALID_ARG                      # no workspace
+    assert bwd(ws=FAKE, ws_bytes=16) == L.WALL_ERR_INVALID_ARG  # workspace too small
+
+
+def test_cache_and_decode_reject_bad_arguments(lib):
+    kc = lib.wall_build_kv_cache
+    assert kc(FAKE, FAKE, 0, 1, 10, 2, 4, 64, 64, 0, FAKE, FAKE, 9, None) == L.WALL_ERR_INVALID_ARG
+    assert kc(FAKE, FAKE, 0, 1, 10, 2, 4, 64, 0, 0, FAKE, FAKE, 10, None) == L.WALL_ERR_INVALID_ARG
+    assert kc(FAKE, FAKE, 0, 1, 10, 2, 4, 60, 64, 0, FAKE, FAKE, 10, None) == L.WALL_ERR_UNSUPPORTED
+    assert kc(FAKE, FAKE, 0, 1, 0, 2, 4, 64, 64, 0, FAKE, FAKE, 10, None) == L.WALL_OK
+    dec = lib.wall_attn_decode
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.0, 64, 0, 1]
+    # T_kv = 0 is invalid: the current token's key must be cached
+    assert dec(*args, 0, 10, 2, 4, 64, 64, FAKE, FAKE, FAKE, 1 << 20, None) == L.WALL_ERR_INVALID_ARG
+    # T_kv beyond capacity
+    assert dec(*args, 11, 10, 2, 4, 64, 64, FAKE, FAKE, FAKE, 1 << 20, None) == L.WALL_ERR_INVALID_ARG
+    # group of 64 query heads per kv head is beyond the decode kernel
+    assert dec(*args, 10, 10, 1, 64, 64, 64, FAKE, FAKE, FAKE, 1 << 20, None) == L.WALL_ERR_UNSUPPORTED
+    # workspace too small
+    assert dec(*args, 10, 10, 2, 4, 64, 64, FAKE, FAKE, FAKE, 8, None) == L.WALL_ERR_INVALID_ARG
+
+
+def test_prefix_rejects_bad_arguments(lib):
+    pc = lib.wall_prefix_cumsum
+    assert pc(FAKE, 3, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG
+    assert pc(None, 0, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG
+    assert pc(FAKE, 0, FAKE, 2, 8, 4, 64, FAKE, 1, None, None, None) == L.WALL_ERR_INVALID_ARG
+    assert pc(FAKE, 0, FAKE, 1, 8, 1, 3, None, 0, None, None, None) == L.WALL_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes(lib):
+    # backward: D, dq, dk^(h), dv^(h), two scalar-gate parts (+ its prefix)
+    rows, HQ, K, V = 2 * 100, 8, 64, 64
+    al = lambda x: (x + 255) // 256 * 256
+    want = al(4 * rows * HQ) + 2 * al(4 * rows * HQ * K) + al(4 * rows * HQ * V) + \
+        2 * al(4 * rows * HQ)
+    assert lib.wall_attn_bwd_workspace(0, 2, 100, 4, HQ, K, V, 0, 0) == want
+    assert lib.wall_attn_bwd_workspace(0, 2, 100, 4, HQ, K, V, 1, 0) == want + al(4 * rows * HQ)
+    assert lib.wall_attn_bwd_workspace(0, 2, 100, 3, HQ, K, V, 0, 0) == 0  # bad shape
+    assert lib.wall_attn_decode_workspace(32, 32768, 8, 32, 128, 64) > 0
+    assert lib.wall_attn_decode_workspace(1, 0, 1, 1, 64, 64) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "libwall.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(ImportError):
+        L.lib()
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "channel_decay_softmax_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "wall_oracle" not in src, f
