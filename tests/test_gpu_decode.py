@@ -53,7 +53,10 @@ def test_cache_layout_and_values():
 
 
 def test_cache_append_keeps_started_anchor():
-    """Appending rows inside a started chunk keeps that chunk's anchor."""
+    """Appending rows inside a started chunk keeps that chunk's anchor: after
+    appends that split chunks, r_cache holds the streamed P at each chunk's
+    first row bit for bit, and k_tilde matches the one-shot build (the
+    streamed prefix differs from the one-shot one only by fp32 rounding)."""
     s = _small_decode_spec(B=1, T=200)
     x = _stack(s)
     k, g = x["k"].to(DEV), x["g"].to(DEV)
@@ -62,10 +65,16 @@ def test_cache_append_keeps_started_anchor():
     cache = api.WallDecodeCache(s.B, s.H, s.HQ, s.K, s.V, capacity=200, chunk_size=64,
                                 dtype=s.dtype, device=DEV)
     v = x["v"].to(DEV)
+    parts = []
     for a, b in ((0, 70), (70, 71), (71, 128), (128, 200)):
-        cache.append(k[:, a:b], v[:, a:b], g[:, a:b])
+        parts.append(cache.append(k[:, a:b], v[:, a:b], g[:, a:b]))
     torch.cuda.synchronize()
-    assert torch.equal(cache.r_cache, rc_full)
+    P_stream = torch.cat(parts, 1)
+    assert torch.equal(cache.r_cache, P_stream[:, ::64])
+    assert max_abs(P_stream, P) <= 1e-5 * max(1.0, float(P.abs().max()))
+    assert torch.equal(cache.v, v)
+    kx = k.repeat_interleave(s.G, dim=2)
+    assert torch.equal(cache.k_tilde[:, ::64], kx[:, ::64])
     assert max_abs(cache.k_tilde, kt_full) <= 2 ** -6 * float(kt_full.float().abs().max())
 
 
