@@ -18,7 +18,8 @@ WALL_BF16, WALL_FP32 = 0, 1
 
 EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn_fwd_workspace",
            "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
-           "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status"]
+           "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
+           "wall_selftest_wait_timeout"]
 
 _lib = None
 
@@ -64,6 +65,8 @@ def lib():
                                        fp, vp, sz, vp]
         L.wall_get_status.restype = i
         L.wall_get_status.argtypes = [vp]
+        L.wall_selftest_wait_timeout.restype = i
+        L.wall_selftest_wait_timeout.argtypes = [i, vp]
         _lib = L
     return _lib
 
@@ -106,6 +109,11 @@ def wall_version() -> int:
 
 def wall_get_status(stream=None) -> int:
     return lib().wall_get_status(_stream(stream))
+
+
+def wall_selftest_wait_timeout(limit_us: int, stream=None):
+    _check("wall_selftest_wait_timeout", lib().wall_selftest_wait_timeout(int(limit_us),
+                                                                          _stream(stream)))
 
 
 def wall_prefix_cumsum(g, P, B, T, HQ, K, cu_seqlens=None, n_seq=0, carry_in=None,

@@ -2,6 +2,7 @@
 // workspace layout and dispatch to the kernels.  See include/wall.h.
 #include <math.h>
 
+#include "sm100_ptx.cuh"
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
@@ -42,6 +43,19 @@ __global__ void check_cu_kernel(const int32_t* cu, int n, long rows, int* status
   }
 }
 
+// A wait on an mbarrier that nothing ever arrives on: the bounded wait must
+// give up after limit_ns and record WALL_ERR_TIMEOUT.
+__global__ void selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  const uint32_t b = sm100::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(b, 0, status, limit_ns);
+}
+
 int check_cu(const int32_t* cu, int n, long rows, cudaStream_t stream) {
   check_cu_kernel<<<1, 256, 0, stream>>>(cu, n, rows, status_ptr());
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
@@ -66,6 +80,7 @@ int make_problem(int dtype, int B, int T, int H, int HQ, int K, int V, float sca
   pb.seqs.n = cu_seqlens ? n_seq : B;
   pb.seqs.T = T;
   pb.seqs.rows = pb.rows;
+  pb.extra_blocks = cu_seqlens ? n_seq : 0;
   long nb = cu_seqlens ? (T + 63L) / 64 + n_seq : (long)B * ((T + 63L) / 64);
   if (nb > 0x7fffffffL) return WALL_ERR_UNSUPPORTED;
   pb.max_blocks64 = (int)nb;
@@ -74,13 +89,31 @@ int make_problem(int dtype, int B, int T, int H, int HQ, int K, int V, float sca
 }
 
 struct FwdWs {
-  size_t gs;  // inclusive prefix of g_scalar [rows, HQ]
+  size_t gs;       // inclusive prefix of g_scalar [rows, HQ]
+  size_t qh, kh;   // anchored operands [rows, HQ, K] bf16 (tensor-core path)
+  size_t anchors;  // [n_blocks128, HQ, K] fp32
+  int n_blocks128;
   size_t total;
 };
-FwdWs fwd_ws_layout(long rows, int HQ, int has_gs) {
+int blocks128(const AttnProblem& pb) {
+  long nb = pb.extra_blocks > 0 ? (pb.T + 127L) / 128 + pb.extra_blocks
+                                : (long)pb.B * ((pb.T + 127L) / 128);
+  return (int)nb;
+}
+FwdWs fwd_ws_layout(const AttnProblem& pb, int has_gs) {
   FwdWs w;
-  w.gs = 0;
-  w.total = has_gs ? align256(sizeof(float) * rows * HQ) : 0;
+  size_t off = 0;
+  w.gs = off;
+  off += has_gs ? align256(sizeof(float) * pb.rows * pb.HQ) : 0;
+  w.qh = w.kh = w.anchors = off;
+  w.n_blocks128 = 0;
+  if (fwd_tc_supported(pb)) {
+    w.n_blocks128 = blocks128(pb);
+    w.qh = off;      off += align256((size_t)2 * pb.rows * pb.HQ * pb.K);
+    w.kh = off;      off += align256((size_t)2 * pb.rows * pb.HQ * pb.K);
+    w.anchors = off; off += align256(sizeof(float) * (size_t)w.n_blocks128 * pb.HQ * pb.K);
+  }
+  w.total = off;
   return w;
 }
 
@@ -133,6 +166,15 @@ int wall_get_status(wall_stream_t stream) {
   return v;
 }
 
+int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return WALL_ERR_INVALID_ARG;
+  int* st = status_ptr();
+  if (!st) return WALL_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      st, 1000ull * (unsigned long long)limit_us);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
 int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ, int K,
                        const int32_t* cu_seqlens, int n_seq, const float* carry_in,
                        float* carry_out, wall_stream_t stream) {
@@ -159,10 +201,11 @@ int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ,
 
 size_t wall_attn_fwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                int has_g_scalar, int n_seq) {
-  (void)n_seq;
   AttnProblem pb;
   if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
-  return fwd_ws_layout(pb.rows, HQ, has_g_scalar).total;
+  // with cu_seqlens (B == 1, n_seq > 0) each sequence may add one partial block
+  if (n_seq > 0 && B == 1) pb.extra_blocks = n_seq;
+  return fwd_ws_layout(pb, has_g_scalar).total;
 }
 
 int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, int dtype, int B,
@@ -176,7 +219,7 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
   if (pb.rows == 0) return WALL_OK;
   if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o)) return WALL_ERR_INVALID_ARG;
   if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(lse)) return WALL_ERR_INVALID_ARG;
-  FwdWs w = fwd_ws_layout(pb.rows, HQ, g_scalar != nullptr);
+  FwdWs w = fwd_ws_layout(pb, g_scalar != nullptr);
   if (w.total > 0 && (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace)))
     return WALL_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -192,6 +235,14 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
     rc = scan_prefix_plain(g_scalar, gs, HQ, pb.seqs, s);
     if (rc) return rc;
     a.GS = gs;
+  }
+  if (fwd_tc_supported(pb)) {
+    TcFwdWs tw;
+    tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
+    tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
+    tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+    tw.n_blocks128 = w.n_blocks128;
+    return attn_fwd_tc(pb, a, tw, status_ptr(), s);
   }
   return attn_fwd_simt(pb, a, s);
 }

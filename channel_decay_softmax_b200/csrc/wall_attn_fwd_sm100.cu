@@ -1,0 +1,595 @@
+// wall_attn_fwd_sm100.cu -- tensor-core (tcgen05 + TMEM + TMA) Wall
+// Attention forward for bf16 with K == V in {64, 128}.
+//
+// Math (Tilde blog "Wall Attention": definition and factorised form; fast
+// training section 1, per-block anchor):
+//   s_ij = scale * sum_n q_in k_jn 2^(P_in - P_jn)
+// Rows are cut into 128-row blocks per sequence; block I has anchor
+// R_I = P at its first row.  A preparation kernel writes
+//   Qh_i = q_i * 2^(P_i - R_I)   (i in block I)      bounded by one block
+//   Kh_j = k_j * 2^(R_J - P_j)   (j in block J)      bounded by one block
+// so that s_ij = scale * sum_n Qh_in * (Kh_jn * 2^(R_I,n - R_J,n)).  Inside
+// the kernel the per-tile, per-channel factor d = 2^(R_I - R_J) (128 exps per
+// tile, not 128*128) is applied to the key tile in shared memory, then
+//   S = Qh * Kt^T   and   O += P * V   run on tcgen05 with fp32 accumulators
+// in TMEM, and the online softmax (log2 domain) keeps one query row per
+// thread.  For decaying gates d only shrinks towards zero for distant tiles,
+// where the exact contribution is equally negligible; no exponent of a
+// global prefix ever reaches bf16 (the blog's reason for the anchors).
+//
+// CTA = one 128-row query block of one (sequence, head), 10 warps:
+//   warp 0      TMA producer: Qh once; Kh_J and V_J per tile (2-stage rings,
+//               the key stage is released after S, the value stage after PV)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2-5   key rescale: Kt_J = Kh_J (.) d in place (bf16 -> fp32 -> bf16),
+//               and the g_scalar key prefix of the tile
+//   warps 6-9   softmax: S from TMEM, mask, exp2, P -> swizzled SMEM (the A
+//               operand of PV), lazy O rescale in TMEM when the row max grows
+//               by more than 2^8, epilogue o = O / l, lse.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+V).
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
+#include "wall_common.cuh"
+#include "wall_internal.h"
+
+namespace wall {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kThreads = 320;
+constexpr float kRescaleThreshold = 8.f;  // log2 units: lazy O rescale
+
+struct FwdTcParams {
+  const float* anchors;  // [nblk, HQ, K]
+  const float* GS;       // [rows, HQ] or nullptr
+  const float* sink;     // [HQ] or nullptr
+  __nv_bfloat16* o;      // [rows, HQ, V]
+  float* lse;            // [rows, HQ] or nullptr
+  Seqs seqs;
+  int HQ, H, K, V;
+  float scale_log2;      // scale * log2(e)
+  int window;
+  int n_blocks;          // grid bound on 128-row blocks
+  int* status;
+};
+
+template <int KD>
+struct Smem {
+  static constexpr int kQ = BM * KD * 2;
+  static constexpr int kK = BN * KD * 2;
+  static constexpr int kV = BN * KD * 2;
+  static constexpr int kP = BM * BN * 2;
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + kQ;             // 2 stages
+  static constexpr int oV = oK + 2 * kK;         // 2 stages
+  static constexpr int oP = oV + 2 * kV;
+  static constexpr int oRI = oP + kP;            // float[KD]
+  static constexpr int oD = oRI + KD * 4;        // float[2 stages][4 warps][KD]
+  static constexpr int oGS = oD + 8 * KD * 4;    // float[4 warps][BN]
+  static constexpr int oBar = oGS + 4 * BN * 4;  // uint64 barriers
+  static constexpr int kBars = 16;
+  static constexpr int oMisc = oBar + kBars * 8; // tmem base, abort flag
+  static constexpr int kBytes = oMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;   // slack for 1 KB alignment
+};
+
+enum Bar {
+  B_QFULL = 0,
+  B_KFULL = 1,   // +stage
+  B_VFULL = 3,   // +stage
+  B_KREADY = 5,  // +stage
+  B_KEMPTY = 7,  // +stage
+  B_VEMPTY = 9,  // +stage
+  B_SFULL = 11,  // +stage
+  B_PFULL = 13,
+  B_PVDONE = 14,
+  B_MMADONE = 15,
+};
+
+__device__ __forceinline__ bool aborted(volatile int* flag) { return *flag != 0; }
+
+// bounded wait that also gives up once another role has given up
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
+                                         volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > 1000000000ull) {
+        record_status(status, WALL_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int KD>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, FwdTcParams p) {
+  using Lay = Smem<KD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
+  float* sD = reinterpret_cast<float*>(smem + Lay::oD);
+  float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.x;
+  const int HQ = p.HQ, K = KD, V = KD;
+  const int kh = h / (HQ / p.H);
+  // longest query blocks first (they have the most key tiles)
+  const int flat = p.n_blocks - 1 - (int)blockIdx.y;
+  int seq, blk;
+  if (!seq_block(p.seqs, BM, flat, seq, blk)) return;
+  const int blk_off = flat - blk;
+  const long s0 = p.seqs.start(seq);
+  const int L = p.seqs.len(seq);
+  const int i0 = blk * BM;
+  const int ni = min(BM, L - i0);
+  const int jb_hi = (i0 + ni - 1) / BN;
+  const int jb_lo = p.window > 0 ? max(0, i0 - p.window + 1) / BN : 0;
+  const int nT = jb_hi - jb_lo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_KREADY + s), 4);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+      mbar_init(bar(B_SFULL + s), 1);
+    }
+    mbar_init(bar(B_PFULL), 4);
+    mbar_init(bar(B_PVDONE), 1);
+    mbar_init(bar(B_MMADONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  for (int n = threadIdx.x; n < K; n += kThreads)
+    sRI[n] = p.anchors[((long)(blk_off + blk) * HQ + h) * K + n];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(bar(B_QFULL), Lay::kQ);
+      for (int b = 0; b < K / 64; ++b)
+        tma_load_3d(sbase + Lay::oQ + b * (BM * 128), &tm_q, bar(B_QFULL), b * 64, h,
+                    (int)(s0 + i0));
+      int k_issued = 0, v_issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t & 1;
+        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+        if (t >= 2 && !wait_bar(bar(B_KEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(B_KFULL + st), Lay::kK);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oK + st * Lay::kK + b * (BN * 128), &tm_k, bar(B_KFULL + st),
+                      b * 64, h, row);
+        k_issued = t + 1;
+        if (t >= 2 && !wait_bar(bar(B_VEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(B_VFULL + st), Lay::kV);
+        for (int b = 0; b < V / 64; ++b)
+          tma_load_3d(sbase + Lay::oV + st * Lay::kV + b * (BN * 128), &tm_v, bar(B_VFULL + st),
+                      b * 64, kh, row);
+        v_issued = t + 1;
+      }
+      // no bulk copy may still be landing in this CTA's shared memory at exit
+      for (int t = max(0, k_issued - 2); t < k_issued; ++t)
+        mbar_wait(bar(B_KFULL + (t & 1)), (t >> 1) & 1, p.status);
+      for (int t = max(0, v_issued - 2); t < v_issued; ++t)
+        mbar_wait(bar(B_VFULL + (t & 1)), (t >> 1) & 1, p.status);
+      mbar_wait(bar(B_QFULL), 0, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16(BM, BN, false, false);
+      const uint32_t idesc_pv = idesc_bf16(BM, V, false, true);
+      bool ok = wait_bar(bar(B_QFULL), 0, p.status, abort_flag);
+      auto issue_qk = [&](int t) -> bool {
+        const int st = t & 1;
+        if (!wait_bar(bar(B_KREADY + st), (t >> 1) & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + st * 128;
+#pragma unroll
+        for (int kk = 0; kk < KD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint64_t a = sdesc_sw128(sbase + Lay::oQ + off, 16, 1024);
+          const uint64_t b = sdesc_sw128(sbase + Lay::oK + st * Lay::kK + off, 16, 1024);
+          umma_bf16_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(B_SFULL + st));
+        umma_commit(bar(B_KEMPTY + st));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && nT > 1) ok = issue_qk(1);
+      for (int t = 0; ok && t < nT; ++t) {
+        const int st = t & 1;
+        if (!wait_bar(bar(B_VFULL + st), (t >> 1) & 1, p.status, abort_flag)) break;
+        if (!wait_bar(bar(B_PFULL), t & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // A = P [128 rows x 16 keys], K-major, two 64-key boxes
+          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint64_t a = sdesc_sw128(sbase + Lay::oP + aoff, 16, 1024);
+          // B = V [16 keys x V channels], MN-major: 8-key groups 1 KB apart,
+          // 64-channel boxes BN*128 bytes apart
+          const uint64_t b =
+              sdesc_sw128(sbase + Lay::oV + st * Lay::kV + kk * 16 * 128, BN * 128, 1024);
+          umma_bf16_ss(tmem + 256, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(B_PVDONE));
+        umma_commit(bar(B_VEMPTY + st));
+        if (t + 2 < nT) ok = issue_qk(t + 2);
+      }
+      // every MMA of this CTA has completed before TMEM is released
+      umma_commit(bar(B_MMADONE));
+      mbar_wait(bar(B_MMADONE), 0, p.status);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ key rescale
+    // Each warp computes the whole d vector it needs (no cross-warp barrier)
+    // and arrives on k_ready once its chunks are written and fenced.
+    const int wt = threadIdx.x - 64;  // 0..127
+    const int wq = warp - 2;          // 0..3
+    const float* anc = p.anchors + ((long)blk_off * HQ + h) * K;
+    for (int t = 0; t < nT; ++t) {
+      const int st = t & 1;
+      const int J = jb_lo + t;
+      float* d = sD + (st * 4 + wq) * KD;
+      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - anc[(long)J * HQ * K + n]);
+      const bool got = wait_bar(bar(B_KFULL + st), (t >> 1) & 1, p.status, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      __syncwarp();
+      uint8_t* kt = smem + Lay::oK + st * Lay::kK;
+      constexpr int nchunks = (KD / 64) * BN * 8;
+#pragma unroll 4
+      for (int c = wt; c < nchunks; c += 128) {
+        const int box = c / (BN * 8);
+        const int row = (c / 8) % BN;
+        const int pch = c % 8;
+        const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
+        uint4* ptr = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
+        uint4 u = *ptr;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+          float2 f = __bfloat1622float2(hv);
+          w[e] = pack_bf16x2(f.x * d[ch0 + 2 * e], f.y * d[ch0 + 2 * e + 1]);
+        }
+        *ptr = u;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_KREADY + st));
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;             // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;        // query row within the block
+    const int i = i0 + r;                     // row within the sequence
+    const bool row_ok = r < ni;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const float gs_i = (p.GS && row_ok) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+    float m_use = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nT; ++t) {
+      const int st = t & 1;
+      const int j0 = (jb_lo + t) * BN;
+      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix
+      if (p.GS) {
+        __syncwarp();
+        for (int c = lane; c < BN; c += 32) {
+          const int j = j0 + c;
+          gsk[c] = (j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
+        }
+        __syncwarp();
+      }
+      {
+        const bool got = wait_bar(bar(B_SFULL + st), (t >> 1) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + st * 128;
+      // logits (log2 domain) with the causal / window / sequence mask
+      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
+                        (p.window <= 0 || i - j0 < p.window);
+      auto logit = [&](uint32_t raw, int c) -> float {
+        float x = __uint_as_float(raw) * p.scale_log2;
+        if (p.GS) x += gs_i - gsk[c];
+        if (!full) {
+          const int j = j0 + c;
+          const bool vis = row_ok && j < L && j <= i && (p.window <= 0 || i - j < p.window);
+          x = vis ? x : -INFINITY;
+        }
+        return x;
+      };
+      // pass 1: row max
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t sv[32];
+        tmem_ld32(s_addr + c, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, logit(sv[e], c + e));
+      }
+      const bool resc = mx > m_use + kRescaleThreshold;
+      const float m_new = resc ? mx : m_use;
+      const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
+      if (t > 0) {
+        const bool got = wait_bar(bar(B_PVDONE), (t - 1) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          const float f = resc ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < V / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+            tmem_st32(tmem + lane_base + 256 + c * 32, ov);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (resc) l *= alpha;
+      m_use = m_new;
+      const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
+      // pass 2: p = exp2(s - m), row sum, bf16 P into the swizzled A tile
+      float rs = 0.f;
+      uint8_t* prow = smem + Lay::oP + r * 128;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t sv[32];
+        tmem_ld32(s_addr + c, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          float e8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            e8[e] = exp2f(logit(sv[g8 * 8 + e], c + g8 * 8 + e) - m_eff);
+            rs += e8[e];
+          }
+          uint4 u;
+          u.x = pack_bf16x2(e8[0], e8[1]);
+          u.y = pack_bf16x2(e8[2], e8[3]);
+          u.z = pack_bf16x2(e8[4], e8[5]);
+          u.w = pack_bf16x2(e8[6], e8[7]);
+          const int cc = c + g8 * 8;
+          const int box = cc / 64;
+          const int pch = ((cc % 64) / 8) ^ (r & 7);
+          *reinterpret_cast<uint4*>(prow + box * (BM * 128) + pch * 16) = u;
+        }
+      }
+      l += rs;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PFULL));
+    }
+    // ---- epilogue
+    if (ok) ok = __all_sync(0xffffffffu,
+                            wait_bar(bar(B_PVDONE), (nT - 1) & 1, p.status, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      float m_f = m_use, scale_o;
+      if (p.sink) {
+        const float s2 = p.sink[h] * kLog2e;
+        m_f = fmaxf(m_use, s2);
+        const float a = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_f);
+        l = l * a + exp2f(s2 - m_f);
+        scale_o = a / l;
+      } else {
+        scale_o = 1.f / l;
+      }
+      __nv_bfloat16* orow = p.o + ((s0 + i) * HQ + h) * (long)V;
+#pragma unroll
+      for (int c = 0; c < V / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * scale_o,
+                                __uint_as_float(ov[2 * e + 1]) * scale_o);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if (row_ok && p.lse) p.lse[(s0 + i) * HQ + h] = (m_f + log2f(l)) * kLn2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// preparation: anchored operands Qh, Kh (per query head) and block anchors
+
+__global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
+                                       const __nv_bfloat16* __restrict__ k,
+                                       const float* __restrict__ P, Seqs seqs, int HQ, int H,
+                                       int K, __nv_bfloat16* __restrict__ qh,
+                                       __nv_bfloat16* __restrict__ khat,
+                                       float* __restrict__ anchors) {
+  const int s = blockIdx.y;
+  __shared__ int s_blk_off;
+  if (threadIdx.x == 0) {
+    int off = 0;
+    if (seqs.cu) {
+      for (int x = 0; x < s; ++x) off += (seqs.len(x) + BM - 1) / BM;
+    } else {
+      off = s * ((seqs.T + BM - 1) / BM);
+    }
+    s_blk_off = off;
+  }
+  __syncthreads();
+  const long s0 = seqs.start(s);
+  const int L = seqs.len(s);
+  const int G = HQ / H;
+  const int kg = K / 8;
+  const long total = (long)L * HQ * kg;
+  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long)gridDim.x * blockDim.x) {
+    const int g8 = (int)(e % kg);
+    const int hh = (int)((e / kg) % HQ);
+    const int t = (int)(e / ((long)kg * HQ));
+    const int b = t / BM;
+    const long row = s0 + t;
+    const long arow = s0 + (long)b * BM;
+    float pv[8], rv[8], x[8], y[8];
+    load8(P + (row * HQ + hh) * K + g8 * 8, pv);
+    load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
+    load8(q + (row * HQ + hh) * K + g8 * 8, x);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(pv[c] - rv[c]);
+    store8(qh + (row * HQ + hh) * K + g8 * 8, y);
+    load8(k + (row * H + hh / G) * K + g8 * 8, x);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(rv[c] - pv[c]);
+    store8(khat + (row * HQ + hh) * K + g8 * 8, y);
+    if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, pv);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps and launch
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, heads, dim] bf16 viewed as a 3-D tensor (dim, heads, rows); box of
+// 64 elements (128 B, swizzled) x 1 head x 128 rows.
+bool make_map(CUtensorMap* m, const void* base, long rows, int heads, int dim) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * heads * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int KD>
+int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
+                  cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, ws.qh, pb.rows, pb.HQ, KD) || !make_map(&tk, ws.kh, pb.rows, pb.HQ, KD) ||
+      !make_map(&tv, a.v, pb.rows, pb.H, KD))
+    return WALL_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(fwd_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<KD>::kAlloc) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    attr = true;
+  }
+  FwdTcParams p;
+  p.anchors = ws.anchors;
+  p.GS = a.GS;
+  p.sink = a.sink;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.seqs = pb.seqs;
+  p.HQ = pb.HQ; p.H = pb.H; p.K = pb.K; p.V = pb.V;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.window = pb.window;
+  p.n_blocks = ws.n_blocks128;
+  p.status = status;
+  dim3 grid(pb.HQ, ws.n_blocks128);
+  fwd_tc_kernel<KD><<<grid, kThreads, Smem<KD>::kAlloc, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const AttnProblem& pb) {
+  return pb.dtype == WALL_BF16 && pb.K == pb.V && (pb.K == 64 || pb.K == 128);
+}
+
+int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
+                          const TcFwdWs& ws, cudaStream_t stream) {
+  if (pb.rows == 0 || pb.seqs.n == 0) return WALL_OK;
+  dim3 grid(64, pb.seqs.n);
+  anchor_operands_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), P, pb.seqs,
+      pb.HQ, pb.H, pb.K, ws.qh, ws.kh, ws.anchors);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
+                cudaStream_t stream) {
+  if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
+  int rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
+  if (rc) return rc;
+  return pb.K == 128 ? launch_fwd_tc<128>(pb, a, ws, status, stream)
+                     : launch_fwd_tc<64>(pb, a, ws, status, stream);
+}
+
+}  // namespace wall

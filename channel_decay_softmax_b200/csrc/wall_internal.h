@@ -26,6 +26,7 @@ struct AttnProblem {
   Seqs seqs;         // sequences over the B*T flattened rows
   long rows;         // B*T
   int max_blocks64;  // upper bound on 64-row blocks over all sequences
+  int extra_blocks;  // varlen: sequences (each may add one partial block), else 0
 };
 
 struct FwdArgs {
@@ -52,6 +53,19 @@ struct BwdArgs {
   float* dgs_col; // [rows,HQ]
   float* dsink;   // [HQ] or nullptr (accumulated atomically, zeroed by the caller)
 };
+
+// ---- tensor-core forward (wall_attn_fwd_sm100.cu) ----
+struct TcFwdWs {
+  __nv_bfloat16* qh;   // [rows, HQ, K]  q * 2^(P - R_block)
+  __nv_bfloat16* kh;   // [rows, HQ, K]  k * 2^(R_block - P)
+  float* anchors;      // [n_blocks128, HQ, K]  P at each 128-row block start
+  int n_blocks128;     // upper bound on 128-row blocks over all sequences
+};
+bool fwd_tc_supported(const AttnProblem& pb);
+int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
+                          const TcFwdWs& ws, cudaStream_t stream);
+int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
+                cudaStream_t stream);
 
 // ---- SIMT fp32 attention (wall_attn_simt.cu) ----
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);

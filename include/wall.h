@@ -108,7 +108,7 @@ size_t wall_attn_fwd_workspace(int dtype, int B, int T, int H, int HQ, int K, in
  *      with a zero value row, included in lse), window_size, cu_seqlens.
  * Out: o [B,T,HQ,V] in `dtype`; lse [B,T,HQ] fp32, natural log of the
  *      softmax denominator (sink included).  lse may be NULL.
- * Supported: K, V in {16, 32, 64, 128} (multiples of 16 up to 128); the
+ * Supported: K, V multiples of 8 up to 128; the
  * tensor-core path takes bf16 with K == V in {64, 128}, other cases use the
  * fp32 SIMT path.  fp32 inputs are computed with fp32 products throughout.
  */
@@ -191,6 +191,17 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
  * synchronization itself fails.
  */
 int wall_get_status(wall_stream_t stream);
+
+/*
+ * wall_selftest_wait_timeout -- failure-detection self test.  Launches one
+ * tiny kernel that waits on an mbarrier nothing ever arrives on, through the
+ * same bounded wait every kernel of the library uses (limit_us
+ * microseconds, 1 .. 2,000,000).  The wait gives up, records
+ * WALL_ERR_TIMEOUT in the status word and the kernel returns normally: the
+ * context stays usable.  The next wall_get_status returns WALL_ERR_TIMEOUT.
+ * No counterpart on the pages: it exercises this library's own error path.
+ */
+int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
 
 #ifdef __cplusplus
 }
