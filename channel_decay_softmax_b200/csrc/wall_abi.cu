@@ -118,9 +118,12 @@ FwdWs fwd_ws_layout(const AttnProblem& pb, int has_gs) {
 }
 
 struct BwdWs {
-  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, total;
+  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, qh, kh, anchors, total;
+  int n_blocks128;
 };
-BwdWs bwd_ws_layout(long rows, int HQ, int K, int V, int has_gs) {
+BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
+  const long rows = pb.rows;
+  const int HQ = pb.HQ, K = pb.K, V = pb.V;
   BwdWs w;
   size_t off = 0;
   w.D = off;       off += align256(sizeof(float) * rows * HQ);
@@ -130,6 +133,14 @@ BwdWs bwd_ws_layout(long rows, int HQ, int K, int V, int has_gs) {
   w.dgs_row = off; off += align256(sizeof(float) * rows * HQ);
   w.dgs_col = off; off += align256(sizeof(float) * rows * HQ);
   w.gs = off;      off += has_gs ? align256(sizeof(float) * rows * HQ) : 0;
+  w.qh = w.kh = w.anchors = off;
+  w.n_blocks128 = 0;
+  if (fwd_tc_supported(pb)) {
+    w.n_blocks128 = blocks128(pb);
+    w.qh = off;      off += align256((size_t)2 * rows * HQ * K);
+    w.kh = off;      off += align256((size_t)2 * rows * HQ * K);
+    w.anchors = off; off += align256(sizeof(float) * (size_t)w.n_blocks128 * HQ * K);
+  }
   w.total = off;
   return w;
 }
@@ -249,10 +260,10 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
 
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                int has_g_scalar, int n_seq) {
-  (void)n_seq;
   AttnProblem pb;
   if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
-  return bwd_ws_layout(pb.rows, HQ, K, V, has_g_scalar).total;
+  if (n_seq > 0 && B == 1) pb.extra_blocks = n_seq;
+  return bwd_ws_layout(pb, has_g_scalar).total;
 }
 
 int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, const float* P,
@@ -276,7 +287,7 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   if (!ok_ptr(dO) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o) ||
       !ok_ptr(lse) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) || !ok_ptr(dg))
     return WALL_ERR_INVALID_ARG;
-  BwdWs w = bwd_ws_layout(pb.rows, HQ, K, V, g_scalar != nullptr);
+  BwdWs w = bwd_ws_layout(pb, g_scalar != nullptr);
   if (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace))
     return WALL_ERR_INVALID_ARG;
   if (cu_seqlens) {
@@ -300,10 +311,20 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
     if (rc) return rc;
     a.GS = gs;
   }
-  rc = attn_bwd_simt(pb, a, s);
-  if (rc) return rc;
-  rc = attn_bwd_reduce(pb, a, dq, dk, dv, s);
-  if (rc) return rc;
+  if (fwd_tc_supported(pb)) {
+    TcFwdWs tw;
+    tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
+    tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
+    tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+    tw.n_blocks128 = w.n_blocks128;
+    rc = attn_bwd_tc(pb, a, tw, dq, dk, dv, status_ptr(), s);
+    if (rc) return rc;
+  } else {
+    rc = attn_bwd_simt(pb, a, s);
+    if (rc) return rc;
+    rc = attn_bwd_reduce(pb, a, dq, dk, dv, s);
+    if (rc) return rc;
+  }
   // dg = reverse cumulative sum of dL (held in dq32 after the reduce)
   rc = scan_reverse(a.dq32, dg, dtype, (long)HQ * K, pb.seqs, s);
   if (rc) return rc;

@@ -502,46 +502,13 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
 // ---------------------------------------------------------------------------
 // host: tensor maps and launch
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// [rows, heads, dim] bf16 viewed as a 3-D tensor (dim, heads, rows); box of
-// 64 elements (128 B, swizzled) x 1 head x 128 rows.
-bool make_map(CUtensorMap* m, const void* base, long rows, int heads, int dim) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t gstride[2] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * heads * 2};
-  cuuint32_t box[3] = {64, 1, 128};
-  cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride,
-                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int KD>
 int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
                   cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, ws.qh, pb.rows, pb.HQ, KD) || !make_map(&tk, ws.kh, pb.rows, pb.HQ, KD) ||
-      !make_map(&tv, a.v, pb.rows, pb.H, KD))
+  if (!make_tile_map(&tq, ws.qh, pb.rows, pb.HQ, KD, BM) ||
+      !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN) ||
+      !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BN))
     return WALL_ERR_CUDA;
   static bool attr = false;
   if (!attr) {

@@ -1,6 +1,7 @@
 // wall_internal.h -- launchers behind the C ABI (host side, namespace wall).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -66,6 +67,14 @@ int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, c
                           const TcFwdWs& ws, cudaStream_t stream);
 int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
                 cudaStream_t stream);
+
+// ---- tensor-core backward (wall_attn_bwd_sm100.cu) ----
+int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void* dq, void* dk,
+                void* dv, int* status, cudaStream_t stream);
+
+// ---- TMA tensor maps (wall_tma.cu) ----
+bool make_tile_map(CUtensorMap* m, const void* base, long rows, int heads, int dim,
+                   int box_rows);
 
 // ---- SIMT fp32 attention (wall_attn_simt.cu) ----
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);

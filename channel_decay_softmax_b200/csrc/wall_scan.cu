@@ -45,12 +45,12 @@ __global__ void __launch_bounds__(kCols * kParts)
   const long len = seqs.len(s);
 
   const float cin = (carry_in != nullptr && valid) ? carry_in[(long)s * C + col] : 0.f;
-  float run = 0.f;  // raw sum of the super-tiles already done
+  float run_hi = 0.f, run_lo = 0.f;  // compensated raw sum of the finished super-tiles
   int buf = 0;
   for (long base = 0; base < len; base += (long)kCS * kRowsPerCta, buf ^= 1) {
     const long row0 = base + (long)rank * kRowsPerCta + (long)part * kRowsPerThread;
     float vals[kRowsPerThread];
-    float sum = 0.f;
+    float sum = 0.f, sum_c = 0.f;  // compensated (Kahan) sum of this thread's rows
 #pragma unroll
     for (int r = 0; r < kRowsPerThread; ++r) {
       const long lr = row0 + r;
@@ -60,7 +60,10 @@ __global__ void __launch_bounds__(kCols * kParts)
         v = to_f32(x[pr * C + col]);
       }
       vals[r] = v;
-      sum += v;
+      const float yk = v - sum_c;
+      const float tk = sum + yk;
+      sum_c = (tk - sum) - yk;
+      sum = tk;
     }
     part_tot[part][c] = sum;
     __syncthreads();
@@ -80,20 +83,29 @@ __global__ void __launch_bounds__(kCols * kParts)
       if (r < rank) pre_cta += t;
       super_total += t;
     }
-    float acc = run + pre_cta + pre_part;
+    // running compensated sum: acc + acc_c carries the prefix of this row
+    float acc = run_hi + pre_cta + pre_part, acc_c = run_lo;
 #pragma unroll
     for (int r = 0; r < kRowsPerThread; ++r) {
       const long lr = row0 + r;
-      acc += vals[r];
+      const float yk = vals[r] - acc_c;
+      const float tk = acc + yk;
+      acc_c = (tk - acc) - yk;
+      acc = tk;
       if (valid && lr < len) {
         const long pr = kReverse ? start + len - 1 - lr : start + lr;
         y[pr * C + col] = from_f32<Tout>(cin + mul * acc);
       }
     }
-    run += super_total;
+    {  // run (two-float) += super_total
+      const float yk = super_total - run_lo;
+      const float tk = run_hi + yk;
+      run_lo = (tk - run_hi) - yk;
+      run_hi = tk;
+    }
   }
   if (carry_out != nullptr && valid && rank == 0 && part == 0)
-    carry_out[(long)s * C + col] = cin + mul * run;
+    carry_out[(long)s * C + col] = cin + mul * (run_hi - run_lo);
   // keep this CTA's shared memory alive until every peer finished reading it
   cluster.sync();
 }
