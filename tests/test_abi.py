@@ -112,14 +112,25 @@ def test_prefix_rejects_bad_arguments(lib):
 
 
 def test_workspace_sizes(lib):
-    # backward: D, dq, dk^(h), dv^(h), two scalar-gate parts (+ its prefix)
-    rows, HQ, K, V = 2 * 100, 8, 64, 64
+    # backward: D, dq, dk^(h), dv^(h), two scalar-gate parts (+ its prefix);
+    # the bf16 tensor-core path adds the anchored operands q^, k^ (bf16) and
+    # the 128-row block anchors (fp32)
+    B, T, HQ, K, V = 2, 100, 8, 64, 64
+    rows = B * T
     al = lambda x: (x + 255) // 256 * 256
-    want = al(4 * rows * HQ) + 2 * al(4 * rows * HQ * K) + al(4 * rows * HQ * V) + \
+    simt = al(4 * rows * HQ) + 2 * al(4 * rows * HQ * K) + al(4 * rows * HQ * V) + \
         2 * al(4 * rows * HQ)
-    assert lib.wall_attn_bwd_workspace(0, 2, 100, 4, HQ, K, V, 0, 0) == want
-    assert lib.wall_attn_bwd_workspace(0, 2, 100, 4, HQ, K, V, 1, 0) == want + al(4 * rows * HQ)
-    assert lib.wall_attn_bwd_workspace(0, 2, 100, 3, HQ, K, V, 0, 0) == 0  # bad shape
+    nblk = B * ((T + 127) // 128)
+    tc = 2 * al(2 * rows * HQ * K) + al(4 * nblk * HQ * K)
+    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 0, 0) == simt        # fp32
+    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 1, 0) == simt + al(4 * rows * HQ)
+    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc   # bf16
+    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, 32, 32, 0, 0) == \
+        al(4 * rows * HQ) + 2 * al(4 * rows * HQ * 32) + al(4 * rows * HQ * 32) + \
+        2 * al(4 * rows * HQ)                                                     # SIMT bf16
+    assert lib.wall_attn_bwd_workspace(0, B, T, 3, HQ, K, V, 0, 0) == 0           # bad shape
+    assert lib.wall_attn_fwd_workspace(1, B, T, 4, HQ, K, V, 0, 0) == 0           # fp32, no opts
+    assert lib.wall_attn_fwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == tc
     assert lib.wall_attn_decode_workspace(32, 32768, 8, 32, 128, 64) > 0
     assert lib.wall_attn_decode_workspace(1, 0, 1, 1, 64, 64) == 0
 
