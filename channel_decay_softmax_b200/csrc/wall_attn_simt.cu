@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
   float dqa[KD / 4];
 #pragma unroll
   for (int c = 0; c < KD / 4; ++c) dqa[c] = 0.f;
-  float rowsum = 0.f;
+  double rowsum = 0.0;  // fp64: the scalar-gate gradient sums many cancelling terms
   const float Di = Dv[row];
   const int jlast = i0 + ni - 1;
   const int jfirst = pb.window > 0 ? max(0, i0 - pb.window + 1) : 0;
@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
       for (int c = 0; c < KD / 4; ++c) dqa[c] += ds * kt[j * (KD + 1) + sub + 4 * c];
     }
   }
-  rowsum = warp4_sum(rowsum);
+  rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 1);
+  rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 2);
   if (row < ni) {
     const long qrow = (s0 + i0 + row) * HQ + h;
 #pragma unroll
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
         a.dq32[qrow * K + n] = pb.scale * f * dqa[c];
       }
     }
-    if (sub == 0) a.dgs_row[qrow] = rowsum;
+    if (sub == 0) a.dgs_row[qrow] = (float)rowsum;
   }
 }
 
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
   for (int c = 0; c < KD / 4; ++c) dka[c] = 0.f;
 #pragma unroll
   for (int c = 0; c < VD / 4; ++c) dva[c] = 0.f;
-  float colsum = 0.f;
+  double colsum = 0.0;  // fp64, as the row sums
 
   const int ilast = pb.window > 0 ? min(L - 1, j0 + nj - 1 + pb.window - 1) : L - 1;
   const float sl2 = pb.scale * kLog2e;
@@ -423,7 +424,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
       for (int c = 0; c < KD / 4; ++c) dka[c] += ds * qt[i * (KD + 1) + sub + 4 * c];
     }
   }
-  colsum = warp4_sum(colsum);
+  colsum += __shfl_xor_sync(0xffffffffu, colsum, 1);
+  colsum += __shfl_xor_sync(0xffffffffu, colsum, 2);
   if (jr < nj) {
     const long krow = (s0 + j0 + jr) * HQ + h;
 #pragma unroll
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
       if (cc < V) a.dvh32[krow * V + cc] = dva[c];
     }
     // the logit carries -GS_j for key j
-    if (sub == 0) a.dgs_col[krow] = -colsum;
+    if (sub == 0) a.dgs_col[krow] = (float)-colsum;
   }
 }
 
