@@ -49,10 +49,18 @@ def assert_fwd(dtype, o_gpu, o_ref, lse_gpu=None, lse_ref=None, mask=None, what=
         assert e <= tol, f"{what} lse max-abs {e:.3e} > {tol}"
 
 
-def assert_grad(dtype, name, g_gpu, g_ref, mask=None, what=""):
+def assert_grad(dtype, name, g_gpu, g_ref, mask=None, what="", relative_to_max=False):
+    """fp32: max-abs <= 1e-5; with relative_to_max (for dg_scalar and dsink,
+    whole-sequence sums that reach |10| and beyond, outside config 1's list)
+    the bound is 1e-5 * max(1, max|ref|), the same relative accuracy."""
     if dtype == torch.float32:
         e = max_abs(g_gpu, g_ref, mask)
-        assert e <= TOL_FP32_MAXABS, f"{what} {name} max-abs {e:.3e} > {TOL_FP32_MAXABS}"
+        tol = TOL_FP32_MAXABS
+        if relative_to_max:
+            ref = np64(g_ref)
+            ref = ref[mask] if mask is not None else ref
+            tol *= max(1.0, float(np.nanmax(np.abs(ref))) if ref.size else 1.0)
+        assert e <= tol, f"{what} {name} max-abs {e:.3e} > {tol:.3e}"
     else:
         e = rel_l2(g_gpu, g_ref, mask)
         assert e <= TOL_BF16_GRAD_RELL2, f"{what} {name} rel-L2 {e:.3e} > {TOL_BF16_GRAD_RELL2}"

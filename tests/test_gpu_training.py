@@ -57,9 +57,10 @@ def _check_all(s, x_cpu, units=None, what=""):
     assert_grad(s.dtype, "dv", dv, ref["dv"], kmask, what)
     assert_grad(s.dtype, "dg", dg, ref["dg"], mask, what)
     if dgs is not None:
-        assert_grad(s.dtype, "dg_scalar", dgs, ref["dg_scalar"], mask, what)
+        assert_grad(s.dtype, "dg_scalar", dgs, ref["dg_scalar"], mask, what,
+                    relative_to_max=True)
     if dsink is not None and units is None:
-        assert_grad(s.dtype, "dsink", dsink, ref["dsink"], None, what)
+        assert_grad(s.dtype, "dsink", dsink, ref["dsink"], None, what, relative_to_max=True)
     return P
 
 
