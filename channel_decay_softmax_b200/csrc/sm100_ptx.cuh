@@ -55,6 +55,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `hint_ns` inside the
+// instruction (it wakes as soon as the phase completes), so a waiting warp
+// does not take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns = 1000000u) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_ns` (about a second), records WALL_ERR_TIMEOUT and returns false,
 // so a kernel whose producer never arrives ends instead of hanging.
@@ -62,9 +78,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* st
                                           uint64_t limit_ns = 1000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
+  const uint32_t hint = limit_ns < 2000000ull ? (uint32_t)(limit_ns / 4 + 1) : 1000000u;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (global_timer_ns() - t0 > limit_ns) {
       record_status(status, WALL_ERR_TIMEOUT);
       return false;
     }

@@ -29,6 +29,8 @@
 // dQ^T double buffer [384,448), [448,512).
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 #include "wall_common.cuh"
 #include "wall_internal.h"
@@ -72,7 +74,7 @@ struct BSmem {
   static constexpr int oP = oO + 2 * kQ;
   static constexpr int oS = oP + kPS;
   static constexpr int oDw = oS + kPS;             // float[4 warps][KD]
-  static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][3][BQ]
+  static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][3][BQ] (2 used)
   static constexpr int oBar = oRow + 4 * 3 * BQ * 4;
   static constexpr int kBars = 20;
   static constexpr int oMisc = oBar + kBars * 8;
@@ -98,15 +100,14 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* sta
                                          volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > 1000000000ull) {
-        record_status(status, WALL_ERR_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
+  for (;;) {
+    // sleeps inside the instruction until the phase completes (or ~0.1 ms)
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      record_status(status, WALL_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -296,11 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
           uint4* ptr = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
           uint4 u = *ptr;
+          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+          const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
           uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * d[ch0 + 2 * e], f.y * d[ch0 + 2 * e + 1]);
+            w[e] = pack_bf16x2(f.x * dd[2 * e], f.y * dd[2 * e + 1]);
           }
           *ptr = u;
         }
@@ -342,18 +346,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool key_ok = r < nj;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const float gs_j = (p.GS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
-    float* rowv = sRow + (warp - 6) * 3 * BQ;  // this warp's lse2, D, GS of the tile's queries
+    float* rowv = sRow + (warp - 6) * 3 * BQ;  // this warp's copy of the tile's query terms
+    const int win = p.window > 0 ? p.window : 0x7fffffff;
     float colsum = 0.f;
     bool ok = true;
     for (int t = 0; t < nT; ++t) {
       const int i0 = (I0 + t) * BQ;
       __syncwarp();
+      // per query: c_i = GS_i*log2e - lse_i*log2e (logit offset), D_i
       for (int c = lane; c < BQ; c += 32) {
         const int i = i0 + c;
         const bool in = i < L;
-        rowv[c] = in ? p.lse[(s0 + i) * HQ + h] * kLog2e : 0.f;
+        const float gsi = (in && p.GS) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+        rowv[c] = in ? gsi - p.lse[(s0 + i) * HQ + h] * kLog2e : 0.f;
         rowv[BQ + c] = in ? p.D[(s0 + i) * HQ + h] : 0.f;
-        rowv[2 * BQ + c] = (in && p.GS) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
       }
       __syncwarp();
       {
@@ -361,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
+      // every query of the tile sees this key: no mask work in the loop
+      const bool full = key_ok && (i0 >= jj) && (i0 + BQ <= L) && (i0 + BQ - 1 - jj < win);
       uint8_t* prow = smem + Lay::oP + r * 128;
       uint8_t* srow = smem + Lay::oS + r * 128;
 #pragma unroll 1
@@ -369,23 +377,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + c, sv);
         tmem_ld32(tmem + lane_base + 64 + c, dv);
         tmem_wait_ld();
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
+        // 8 keys' worth of P and dS at a time: compute, pack, store
+        auto group = [&](int g8, auto masked) {
           float pe[8], de[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int q = c + g8 * 8 + e;
-            const int i = i0 + q;
-            const bool vis =
-                key_ok && i < L && jj <= i && (p.window <= 0 || i - jj < p.window);
-            const float s2 = __uint_as_float(sv[g8 * 8 + e]) * p.scale_log2 + rowv[2 * BQ + q] -
-                             gs_j - rowv[q];
-            const float pv = vis ? exp2f(s2) : 0.f;
-            const float ds = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
-            colsum += ds;
+            const float x = fmaf(__uint_as_float(sv[g8 * 8 + e]), p.scale_log2, rowv[q] - gs_j);
+            float pv;
+            if constexpr (decltype(masked)::value) {
+              const int i = i0 + q;
+              const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
+              pv = vis ? exp2f(x) : 0.f;
+            } else {
+              pv = exp2f(x);
+            }
             pe[e] = pv;
-            de[e] = ds;
+            de[e] = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
           }
+          colsum += ((de[0] + de[1]) + (de[2] + de[3])) + ((de[4] + de[5]) + (de[6] + de[7]));
           const int pch = ((c / 8) + g8) ^ (r & 7);
           *reinterpret_cast<uint4*>(prow + pch * 16) =
               make_uint4(pack_bf16x2(pe[0], pe[1]), pack_bf16x2(pe[2], pe[3]),
@@ -393,6 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(srow + pch * 16) =
               make_uint4(pack_bf16x2(de[0], de[1]), pack_bf16x2(de[2], de[3]),
                          pack_bf16x2(de[4], de[5]), pack_bf16x2(de[6], de[7]));
+        };
+        if (full) {
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) group(g8, std::false_type{});
+        } else {
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) group(g8, std::true_type{});
         }
       }
       fence_proxy_async_smem();

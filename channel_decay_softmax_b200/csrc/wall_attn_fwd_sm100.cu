@@ -90,22 +90,19 @@ enum Bar {
   B_MMADONE = 15,
 };
 
-__device__ __forceinline__ bool aborted(volatile int* flag) { return *flag != 0; }
-
 // bounded wait that also gives up once another role has given up
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
                                          volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > 1000000000ull) {
-        record_status(status, WALL_ERR_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
+  for (;;) {
+    // sleeps inside the instruction until the phase completes (or ~0.1 ms)
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      record_status(status, WALL_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -285,12 +282,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
         uint4* ptr = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
         uint4 u = *ptr;
+        const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+        const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+        const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
         uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
           float2 f = __bfloat1622float2(hv);
-          w[e] = pack_bf16x2(f.x * d[ch0 + 2 * e], f.y * d[ch0 + 2 * e + 1]);
+          w[e] = pack_bf16x2(f.x * dd[2 * e], f.y * dd[2 * e + 1]);
         }
         *ptr = u;
       }
@@ -305,18 +305,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = i0 + r;                     // row within the sequence
     const bool row_ok = r < ni;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const float gs_i = (p.GS && row_ok) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+    const bool has_gs = p.GS != nullptr;
+    const int win = p.window > 0 ? p.window : 0x7fffffff;
+    const float gs_i = (has_gs && row_ok) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < nT; ++t) {
       const int st = t & 1;
       const int j0 = (jb_lo + t) * BN;
-      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix
-      if (p.GS) {
+      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix (or zeros)
+      if (has_gs || t == 0) {
         __syncwarp();
         for (int c = lane; c < BN; c += 32) {
           const int j = j0 + c;
-          gsk[c] = (j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
+          gsk[c] = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
         }
         __syncwarp();
       }
@@ -326,29 +328,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + st * 128;
-      // logits (log2 domain) with the causal / window / sequence mask
-      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
-                        (p.window <= 0 || i - j0 < p.window);
-      auto logit = [&](uint32_t raw, int c) -> float {
-        float x = __uint_as_float(raw) * p.scale_log2;
-        if (p.GS) x += gs_i - gsk[c];
-        if (!full) {
-          const int j = j0 + c;
-          const bool vis = row_ok && j < L && j <= i && (p.window <= 0 || i - j < p.window);
-          x = vis ? x : -INFINITY;
-        }
-        return x;
-      };
+      // logits (log2 domain) with the causal / window / sequence mask.  The
+      // common case -- a fully visible tile without a scalar gate -- is a
+      // plain multiply; decisions are hoisted out of the element loops.
+      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) && (i - j0 < win);
+      const bool fast = full && !has_gs;
+      const float sl2 = p.scale_log2;
+      const float bias_i = has_gs ? gs_i : 0.f;
       // pass 1: row max
-      float mx = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t sv[32];
         tmem_ld32(s_addr + c, sv);
         tmem_wait_ld();
+        if (fast) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, logit(sv[e], c + e));
+          for (int e = 0; e < 32; e += 4) {
+            mx0 = fmaxf(mx0, __uint_as_float(sv[e]) * sl2);
+            mx1 = fmaxf(mx1, __uint_as_float(sv[e + 1]) * sl2);
+            mx2 = fmaxf(mx2, __uint_as_float(sv[e + 2]) * sl2);
+            mx3 = fmaxf(mx3, __uint_as_float(sv[e + 3]) * sl2);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = j0 + c + e;
+            const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
+            const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e]);
+            mx0 = fmaxf(mx0, vis ? x : -INFINITY);
+          }
+        }
       }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       const bool resc = mx > m_use + kRescaleThreshold;
       const float m_new = resc ? mx : m_use;
       const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
@@ -374,32 +386,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_use = m_new;
       const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
       // pass 2: p = exp2(s - m), row sum, bf16 P into the swizzled A tile
-      float rs = 0.f;
+      float rs0 = 0.f, rs1 = 0.f;
       uint8_t* prow = smem + Lay::oP + r * 128;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t sv[32];
         tmem_ld32(s_addr + c, sv);
         tmem_wait_ld();
+        float e32[32];
+        if (fast) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) e32[e] = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_eff));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = j0 + c + e;
+            const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
+            const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e] - m_eff);
+            e32[e] = vis ? exp2f(x) : 0.f;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          rs0 += e32[e];
+          rs1 += e32[e + 1];
+        }
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
-          float e8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            e8[e] = exp2f(logit(sv[g8 * 8 + e], c + g8 * 8 + e) - m_eff);
-            rs += e8[e];
-          }
           uint4 u;
-          u.x = pack_bf16x2(e8[0], e8[1]);
-          u.y = pack_bf16x2(e8[2], e8[3]);
-          u.z = pack_bf16x2(e8[4], e8[5]);
-          u.w = pack_bf16x2(e8[6], e8[7]);
+          u.x = pack_bf16x2(e32[g8 * 8 + 0], e32[g8 * 8 + 1]);
+          u.y = pack_bf16x2(e32[g8 * 8 + 2], e32[g8 * 8 + 3]);
+          u.z = pack_bf16x2(e32[g8 * 8 + 4], e32[g8 * 8 + 5]);
+          u.w = pack_bf16x2(e32[g8 * 8 + 6], e32[g8 * 8 + 7]);
           const int cc = c + g8 * 8;
           const int box = cc / 64;
           const int pch = ((cc % 64) / 8) ^ (r & 7);
           *reinterpret_cast<uint4*>(prow + box * (BM * 128) + pch * 16) = u;
         }
       }
+      const float rs = rs0 + rs1;
       l += rs;
       fence_proxy_async_smem();
       tc_fence_before();
