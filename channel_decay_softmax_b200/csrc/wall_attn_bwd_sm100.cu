@@ -73,9 +73,11 @@ struct BSmem {
   static constexpr int oO = oQ + 2 * kQ;    // 2 stages
   static constexpr int oP = oO + 2 * kQ;
   static constexpr int oS = oP + kPS;
-  static constexpr int oDw = oS + kPS;             // float[4 warps][KD]
-  static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][3][BQ] (2 used)
-  static constexpr int oBar = oRow + 4 * 3 * BQ * 4;
+  static constexpr int oDw = oS + kPS;             // float[2 stages][4 warps][KD]
+  static constexpr int oRow = oDw + 8 * KD * 4;    // float[4 warps][3][BQ] (2 used)
+  static constexpr int oRI = oRow + 4 * 3 * BQ * 4;  // float[2 stages][KD] query-block anchors
+  static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD] key-block anchor
+  static constexpr int oBar = oRJ + KD * 4;
   static constexpr int kBars = 20;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
@@ -172,6 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
+  {
+    float* rjs = reinterpret_cast<float*>(smem + Lay::oRJ);
+    for (int n = threadIdx.x; n < K; n += kThreads) rjs[n] = anc[(long)blk * HQ * K + n];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -197,8 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = (int)(s0 + (long)(I0 + t) * BQ);
         if (t >= 2 && !wait_bar(bar(QO_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(Q_FULL + st), Lay::kQ);
+        mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
         mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
+        bulk_load(sbase + Lay::oRI + st * K * 4,
+                  anc + (long)((I0 + t) / 2) * HQ * K, K * 4, bar(Q_FULL + st));
         for (int b = 0; b < K / 64; ++b) {
           tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
                       b * 64, h, row);
@@ -276,37 +284,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int n = quarter * 32 + lane;   // channel of this thread in the dQ^T epilogue
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    float* d = sDw + wq * KD;
-    const float RJn = anc[(long)blk * HQ * K + (n < K ? n : 0)];
+    const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
     for (int t = 0; t <= nT; ++t) {
       if (t < nT) {
         const int st = t & 1;
-        const int Ib = (I0 + t) / 2;  // 128-row block holding this query tile
-        for (int c = lane; c < K; c += 32)
-          d[c] = exp2f(anc[(long)Ib * HQ * K + c] - anc[(long)blk * HQ * K + c]);
+        // this warp's copy of d = 2^(R_I - R_J) for the tile, kept per stage
+        // so the dQ epilogue of the same tile (one iteration later) reads it
+        float* d = sDw + (st * 4 + wq) * KD;
         const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) break;
+        const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4);
+        for (int c = lane; c < K; c += 32) d[c] = exp2f(ri[c] - rjs[c]);
         __syncwarp();
         uint8_t* qt = smem + Lay::oQ + st * Lay::kQ;
-        constexpr int nchunks = (KD / 64) * BQ * 8;
-#pragma unroll 4
-        for (int c = wt; c < nchunks; c += 128) {
-          const int box = c / (BQ * 8);
-          const int row = (c / 8) % BQ;
-          const int pch = c % 8;
-          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-          uint4* ptr = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
-          uint4 u = *ptr;
-          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-          const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+        constexpr int kPer = (KD / 64) * BQ * 8 / 128;  // chunks per thread
+        constexpr int kBatch = kPer < 4 ? kPer : 4;
+#pragma unroll 1
+        for (int b0 = 0; b0 < kPer; b0 += kBatch) {
+          uint4 u[kBatch];
+          float dd[kBatch][8];
+          uint4* ptr[kBatch];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * dd[2 * e], f.y * dd[2 * e + 1]);
+          for (int x = 0; x < kBatch; ++x) {
+            const int c = wt + (b0 + x) * 128;
+            const int box = c / (BQ * 8);
+            const int row = (c / 8) % BQ;
+            const int pch = c % 8;
+            const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
+            ptr[x] = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
+            u[x] = *ptr[x];
+            const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+            const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+            dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
+            dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
           }
-          *ptr = u;
+#pragma unroll
+          for (int x = 0; x < kBatch; ++x) {
+            uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+              w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
+            }
+            *ptr[x] = u[x];
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -318,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool got = wait_bar(bar(DQ_FULL + su), (u >> 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) break;
         tc_fence_after();
-        const float dn = (n < K) ? exp2f(anc[(long)(Iu / 2) * HQ * K + n] - RJn) : 0.f;
+        const float dn = (n < K) ? sDw[(su * 4 + wq) * KD + n] : 0.f;
 #pragma unroll
         for (int c = 0; c < BQ; c += 32) {
           uint32_t v[32];

@@ -70,7 +70,8 @@ struct Smem {
   static constexpr int oRI = oP + kP;            // float[KD]
   static constexpr int oD = oRI + KD * 4;        // float[2 stages][4 warps][KD]
   static constexpr int oGS = oD + 8 * KD * 4;    // float[4 warps][BN]
-  static constexpr int oBar = oGS + 4 * BN * 4;  // uint64 barriers
+  static constexpr int oRJ = oGS + 4 * BN * 4;   // float[2 stages][KD] key-block anchors
+  static constexpr int oBar = oRJ + 2 * KD * 4;  // uint64 barriers
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8; // tmem base, abort flag
   static constexpr int kBytes = oMisc + 16;
@@ -189,10 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = (int)(s0 + (long)(jb_lo + t) * BN);
         if (t >= 2 && !wait_bar(bar(B_KEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(B_KFULL + st), Lay::kK);
+        mbar_expect_tx(bar(B_KFULL + st), Lay::kK + K * 4);
         for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oK + st * Lay::kK + b * (BN * 128), &tm_k, bar(B_KFULL + st),
                       b * 64, h, row);
+        bulk_load(sbase + Lay::oRJ + st * K * 4,
+                  p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
+                  bar(B_KFULL + st));
         k_issued = t + 1;
         if (t >= 2 && !wait_bar(bar(B_VEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
@@ -259,40 +263,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ key rescale
-    // Each warp computes the whole d vector it needs (no cross-warp barrier)
-    // and arrives on k_ready once its chunks are written and fenced.
+    // The key tile and its block anchors arrive together; each warp forms
+    // the whole factor vector d = 2^(R_I - R_J) it needs (no cross-warp
+    // barrier) and arrives on k_ready once its chunks are written and fenced.
     const int wt = threadIdx.x - 64;  // 0..127
     const int wq = warp - 2;          // 0..3
-    const float* anc = p.anchors + ((long)blk_off * HQ + h) * K;
     for (int t = 0; t < nT; ++t) {
       const int st = t & 1;
-      const int J = jb_lo + t;
       float* d = sD + (st * 4 + wq) * KD;
-      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - anc[(long)J * HQ * K + n]);
       const bool got = wait_bar(bar(B_KFULL + st), (t >> 1) & 1, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
+      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4);
+      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - rj[n]);
       __syncwarp();
       uint8_t* kt = smem + Lay::oK + st * Lay::kK;
-      constexpr int nchunks = (KD / 64) * BN * 8;
-#pragma unroll 4
-      for (int c = wt; c < nchunks; c += 128) {
-        const int box = c / (BN * 8);
-        const int row = (c / 8) % BN;
-        const int pch = c % 8;
-        const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-        uint4* ptr = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
-        uint4 u = *ptr;
-        const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-        const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-        const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+      constexpr int kPer = (KD / 64) * BN * 8 / 128;  // chunks per thread
+      constexpr int kBatch = 4;
+#pragma unroll 1
+      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
+        uint4 u[kBatch];
+        float dd[kBatch][8];
+        uint4* ptr[kBatch];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
-          float2 f = __bfloat1622float2(hv);
-          w[e] = pack_bf16x2(f.x * dd[2 * e], f.y * dd[2 * e + 1]);
+        for (int x = 0; x < kBatch; ++x) {
+          const int c = wt + (b0 + x) * 128;
+          const int box = c / (BN * 8);
+          const int row = (c / 8) % BN;
+          const int pch = c % 8;
+          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
+          ptr[x] = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
+          u[x] = *ptr[x];
+          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
+          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
         }
-        *ptr = u;
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
+          }
+          *ptr[x] = u[x];
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
