@@ -19,7 +19,7 @@ WALL_BF16, WALL_FP32 = 0, 1
 EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn_fwd_workspace",
            "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
            "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
-           "wall_selftest_wait_timeout"]
+           "wall_selftest_wait_timeout", "wall_attn_decode_noalloc"]
 
 _lib = None
 
@@ -67,6 +67,9 @@ def lib():
         L.wall_get_status.argtypes = [vp]
         L.wall_selftest_wait_timeout.restype = i
         L.wall_selftest_wait_timeout.argtypes = [i, vp]
+        L.wall_attn_decode_noalloc.restype = i
+        L.wall_attn_decode_noalloc.argtypes = [vp, vp, fp, vp, fp, fp, f, i, i, i, i, i, i, i, i,
+                                               i, vp, fp, vp]
         _lib = L
     return _lib
 
@@ -170,3 +173,11 @@ def wall_attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, scale, C, B, T_k
         _p(q), _p(v), _p(p_curr), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
         dtype_code(q.dtype), B, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _p(workspace), ws_bytes,
         _stream(stream)))
+
+
+def wall_attn_decode_noalloc(q, v, p_curr, k_tilde, r_cache, sink_bias, scale, C, B, T_kv, Tcap,
+                             H, HQ, K, V, o, lse, stream=None):
+    """wall_attn_decode without a workspace (fixed scratch inside the library)."""
+    _check("wall_attn_decode_noalloc", lib().wall_attn_decode_noalloc(
+        _p(q), _p(v), _p(p_curr), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
+        dtype_code(q.dtype), B, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _stream(stream)))

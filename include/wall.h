@@ -186,6 +186,29 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
                      void* workspace, size_t workspace_bytes, wall_stream_t stream);
 
 /*
+ * wall_attn_decode_noalloc -- wall_attn_decode for callers that cannot
+ * allocate device memory (code running during CUDA graph capture that must not
+ * allocate, serving loops whose memory is planned once, bindings without a
+ * device allocator).  The paper has no counterpart: it is a deployment variant.
+ *
+ * Same arguments, layout and results as wall_attn_decode, without the
+ * workspace: the split partials live in a fixed 4 MiB scratch array inside the
+ * library's device memory (every GPU that loads the library holds it until the
+ * process exits).  Problems needing more, B * HQ * splits * (V + 2) > 2^20
+ * floats with splits as wall_attn_decode chooses them, are rejected with
+ * WALL_ERR_UNSUPPORTED before anything runs; use wall_attn_decode for those.
+ * The entry point calls no allocator.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current, so
+ * make that first call before any stream capture.  All calls share the one
+ * array and each call overwrites every partial it reads, so nothing needs
+ * clearing; calls that overlap on the GPU (concurrent streams) race on it.
+ */
+int wall_attn_decode_noalloc(const void* q, const void* v, const float* p_curr,
+                             const void* k_tilde, const float* r_cache, const float* sink_bias,
+                             float scale, int C, int dtype, int B, int T_kv, int Tcap, int H,
+                             int HQ, int K, int V, void* o, float* lse, wall_stream_t stream);
+
+/*
  * wall_get_status -- synchronizes `stream`, returns the device status word
  * (WALL_OK or WALL_ERR_TIMEOUT) and clears it.  Returns WALL_ERR_CUDA if the
  * synchronization itself fails.
