@@ -18,13 +18,15 @@
 // reverse scan.  The row part of the scalar-gate gradient is analytic,
 // sum_j dS_ij = D_i * p_sink,i, and the column part is summed per key thread.
 //
-// CTA = one 128-row key block of one (sequence, head), 10 warps:
+// CTA = one 128-row key block of one (sequence, head), 14 warps:
 //   warp 0      TMA: Kh_J, V_J once; Qh_I and dO_I per tile (2-stage ring)
 //   warp 1      TMEM owner and MMA issuer
-//   warps 2-5   Qt_I = Qh_I (.) d in shared memory; dQ^T epilogue (one thread
-//               per channel: scale by d, coalesced fp32 atomic adds)
+//   warps 2-5   Qt_I = Qh_I (.) d in shared memory
 //   warps 6-9   one thread per key: P, dS -> swizzled SMEM (bf16), column
 //               sums; at the end dK, dV epilogue
+//   warps 10-13 dQ^T epilogue: one thread per channel, scale by d, coalesced
+//               fp32 atomic adds (own warps, so slow atomics never delay the
+//               next tile's rescale)
 // TMEM columns: S^T [0,64), dP^T [64,128), dV [128,256), dK [256,384),
 // dQ^T double buffer [384,448), [448,512).
 #include <cuda.h>
@@ -42,7 +44,7 @@ using namespace sm100;
 
 constexpr int BQ = 64;
 constexpr int BK = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 
 struct BwdTcParams {
   const float* anchors;  // [nblk128, HQ, K]
@@ -278,89 +280,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(MMA_DONE), 0, p.status);
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ Qt rescale, dQ epilogue
+    // ------------------------------------------------------------ Qt rescale
     const int wt = threadIdx.x - 64;
     const int wq = warp - 2;
+    const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
+    for (int t = 0; t < nT; ++t) {
+      const int st = t & 1;
+      // this warp's copy of d = 2^(R_I - R_J) for the tile, kept per stage so
+      // the dQ epilogue of the same tile reads it
+      float* d = sDw + (st * 4 + wq) * KD;
+      const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4);
+      for (int c = lane; c < K; c += 32) d[c] = exp2f(ri[c] - rjs[c]);
+      __syncwarp();
+      uint8_t* qt = smem + Lay::oQ + st * Lay::kQ;
+      constexpr int kPer = (KD / 64) * BQ * 8 / 128;  // chunks per thread
+      constexpr int kBatch = kPer < 4 ? kPer : 4;
+#pragma unroll 1
+      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
+        uint4 u[kBatch];
+        float dd[kBatch][8];
+        uint4* ptr[kBatch];
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int c = wt + (b0 + x) * 128;
+          const int box = c / (BQ * 8);
+          const int row = (c / 8) % BQ;
+          const int pch = c % 8;
+          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
+          ptr[x] = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
+          u[x] = *ptr[x];
+          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
+          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
+        }
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
+          }
+          *ptr[x] = u[x];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Q_READY + st));
+    }
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ dQ epilogue
     const int quarter = warp & 3;
-    const int n = quarter * 32 + lane;   // channel of this thread in the dQ^T epilogue
+    const int n = quarter * 32 + lane;   // channel of this thread
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
-    for (int t = 0; t <= nT; ++t) {
-      if (t < nT) {
-        const int st = t & 1;
-        // this warp's copy of d = 2^(R_I - R_J) for the tile, kept per stage
-        // so the dQ epilogue of the same tile (one iteration later) reads it
-        float* d = sDw + (st * 4 + wq) * KD;
-        const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) break;
-        const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4);
-        for (int c = lane; c < K; c += 32) d[c] = exp2f(ri[c] - rjs[c]);
-        __syncwarp();
-        uint8_t* qt = smem + Lay::oQ + st * Lay::kQ;
-        constexpr int kPer = (KD / 64) * BQ * 8 / 128;  // chunks per thread
-        constexpr int kBatch = kPer < 4 ? kPer : 4;
-#pragma unroll 1
-        for (int b0 = 0; b0 < kPer; b0 += kBatch) {
-          uint4 u[kBatch];
-          float dd[kBatch][8];
-          uint4* ptr[kBatch];
+    for (int u = 0; u < nT; ++u) {
+      const int su = u & 1;
+      const int Iu = I0 + u;
+      // d for this channel, from the anchors in global memory (the shared
+      // stage may already hold a later tile); loaded before the wait
+      const float ri_n = (n < K) ? anc[(long)(Iu / 2) * HQ * K + n] : 0.f;
+      const bool got = wait_bar(bar(DQ_FULL + su), (u >> 1) & 1, p.status, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const float dn = (n < K) ? exp2f(ri_n - rjs[n]) : 0.f;
 #pragma unroll
-          for (int x = 0; x < kBatch; ++x) {
-            const int c = wt + (b0 + x) * 128;
-            const int box = c / (BQ * 8);
-            const int row = (c / 8) % BQ;
-            const int pch = c % 8;
-            const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-            ptr[x] = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
-            u[x] = *ptr[x];
-            const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-            const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-            dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
-            dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
-          }
+      for (int c = 0; c < BQ; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + 384 + su * 64 + c, v);
+        tmem_wait_ld();
+        if (n < K) {
 #pragma unroll
-          for (int x = 0; x < kBatch; ++x) {
-            uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-              w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
-            }
-            *ptr[x] = u[x];
+          for (int e = 0; e < 32; ++e) {
+            const int i = Iu * BQ + c + e;
+            if (i < L) atomicAdd(p.dq32 + ((s0 + i) * HQ + h) * (long)K + n,
+                                 __uint_as_float(v[e]) * dn);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(Q_READY + st));
       }
-      if (t >= 1) {
-        const int u = t - 1, su = u & 1;
-        const int Iu = I0 + u;
-        const bool got = wait_bar(bar(DQ_FULL + su), (u >> 1) & 1, p.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) break;
-        tc_fence_after();
-        const float dn = (n < K) ? sDw[(su * 4 + wq) * KD + n] : 0.f;
-#pragma unroll
-        for (int c = 0; c < BQ; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + 384 + su * 64 + c, v);
-          tmem_wait_ld();
-          if (n < K) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int i = Iu * BQ + c + e;
-              if (i < L) atomicAdd(p.dq32 + ((s0 + i) * HQ + h) * (long)K + n,
-                                   __uint_as_float(v[e]) * dn);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(DQ_FREE + su));
-      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(DQ_FREE + su));
     }
   } else {
-    // ------------------------------------------------------------ P, dS per key
+    // ------------------------------------------------------------ P, dS per key (warps 6-9)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;   // key row within the block
     const int jj = j0 + r;               // key index within the sequence
@@ -649,7 +655,7 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void
   rc = pb.K == 128 ? launch_bwd_tc<128>(pb, a, ws, status, stream)
                    : launch_bwd_tc<64>(pb, a, ws, status, stream);
   if (rc) return rc;
-  dim3 grid(148 * 2 / (pb.seqs.n < 1 ? 1 : pb.seqs.n) + 1, pb.seqs.n);
+  dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
   bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.P,
       pb.seqs, pb.HQ, pb.H, pb.K, pb.V, pb.scale, a.dq32, a.dkh32, a.dvh32,

@@ -583,7 +583,9 @@ bool fwd_tc_supported(const AttnProblem& pb) {
 int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
                           const TcFwdWs& ws, cudaStream_t stream) {
   if (pb.rows == 0 || pb.seqs.n == 0) return WALL_OK;
-  dim3 grid(64, pb.seqs.n);
+  // enough CTAs to keep every SM streaming, split over the sequences
+  const int per_seq = (148 * 8 + pb.seqs.n - 1) / pb.seqs.n;
+  dim3 grid(per_seq < 1 ? 1 : per_seq, pb.seqs.n);
   anchor_operands_kernel<<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), P, pb.seqs,
       pb.HQ, pb.H, pb.K, ws.qh, ws.kh, ws.anchors);
