@@ -255,13 +255,13 @@ int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int 
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
-// Splits per (batch row, kv head): enough CTAs for several waves over the
-// 148 SMs, never more splits than chunks.  Non-decreasing in T_kv, so a
+// Splits per (batch row, kv head): about four waves of CTAs over the 148
+// SMs, never more splits than chunks.  Non-decreasing in T_kv, so a
 // workspace sized for the largest T_kv serves every shorter one.
 int decode_splits(int B, int T_kv, int H, int C) {
   const long units = (long)B * H;
   const long chunks = (T_kv + (long)C - 1) / C;
-  long s = (148L * 8 + units - 1) / units;
+  long s = (148L * 8 * 4 + units - 1) / units;
   if (s > chunks) s = chunks;
   if (s < 1) s = 1;
   return (int)s;
