@@ -23,9 +23,10 @@
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2-5   key rescale: Kt_J = Kh_J (.) d in place (bf16 -> fp32 -> bf16),
 //               and the g_scalar key prefix of the tile
-//   warps 6-9   softmax: S from TMEM, mask, exp2, P -> swizzled SMEM (the A
-//               operand of PV), lazy O rescale in TMEM when the row max grows
-//               by more than 2^8, epilogue o = O / l, lse.
+//   warps 6-9   softmax: S from TMEM, mask, exp2, P (bf16 pairs) written back
+//               over the consumed S columns as the TMEM A operand of PV, lazy
+//               O rescale in TMEM when the row max grows by more than 2^8,
+//               epilogue o = O / l, lse.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+V).
 #include <cuda.h>
 
@@ -62,12 +63,10 @@ struct Smem {
   static constexpr int kQ = BM * KD * 2;
   static constexpr int kK = BN * KD * 2;
   static constexpr int kV = BN * KD * 2;
-  static constexpr int kP = BM * BN * 2;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;             // 2 stages
   static constexpr int oV = oK + 2 * kK;         // 2 stages
-  static constexpr int oP = oV + 2 * kV;
-  static constexpr int oRI = oP + kP;            // float[KD]
+  static constexpr int oRI = oV + 2 * kV;        // float[KD]
   static constexpr int oD = oRI + KD * 4;        // float[2 stages][4 warps][KD]
   static constexpr int oGS = oD + 8 * KD * 4;    // float[4 warps][BN]
   static constexpr int oRJ = oGS + 4 * BN * 4;   // float[2 stages][KD] key-block anchors
@@ -244,14 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P [128 rows x 16 keys], K-major, two 64-key boxes
-          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          const uint64_t a = sdesc_sw128(sbase + Lay::oP + aoff, 16, 1024);
+          // A = P [128 rows x 16 keys] from TMEM: the softmax wrote bf16 pairs
+          // over the S buffer it had consumed, 8 columns per 16 keys
+          const uint32_t a = tmem + st * 128 + kk * 8;
           // B = V [16 keys x V channels], MN-major: 8-key groups 1 KB apart,
           // 64-channel boxes BN*128 bytes apart
           const uint64_t b =
               sdesc_sw128(sbase + Lay::oV + st * Lay::kV + kk * 16 * 128, BN * 128, 1024);
-          umma_bf16_ss(tmem + 256, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + 256, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(B_PVDONE));
         umma_commit(bar(B_VEMPTY + st));
@@ -402,7 +401,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
       // pass 2: p = exp2(s - m), row sum, bf16 P into the swizzled A tile
       float rs0 = 0.f, rs1 = 0.f;
-      uint8_t* prow = smem + Lay::oP + r * 128;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t sv[32];
@@ -421,27 +419,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             e32[e] = vis ? exp2f(x) : 0.f;
           }
         }
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           rs0 += e32[e];
           rs1 += e32[e + 1];
+          pk[e / 2] = pack_bf16x2(e32[e], e32[e + 1]);
         }
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          uint4 u;
-          u.x = pack_bf16x2(e32[g8 * 8 + 0], e32[g8 * 8 + 1]);
-          u.y = pack_bf16x2(e32[g8 * 8 + 2], e32[g8 * 8 + 3]);
-          u.z = pack_bf16x2(e32[g8 * 8 + 4], e32[g8 * 8 + 5]);
-          u.w = pack_bf16x2(e32[g8 * 8 + 6], e32[g8 * 8 + 7]);
-          const int cc = c + g8 * 8;
-          const int box = cc / 64;
-          const int pch = ((cc % 64) / 8) ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + box * (BM * 128) + pch * 16) = u;
-        }
+        // keys [c, c+32) -> columns [c/2, c/2+16) of this S buffer; every S
+        // column at or below them has been read already
+        tmem_st16(s_addr + c / 2, pk);
       }
+      tmem_wait_st();
       const float rs = rs0 + rs1;
       l += rs;
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_PFULL));
