@@ -2,33 +2,38 @@
 // Attention backward for bf16 with K == V in {64, 128}.
 //
 // Gradients of the anchored form used by the forward (Tilde blog "Wall
-// Attention", fast training sections 1 and 2).  For a 64-row query tile I
-// (anchor R_I of its 128-row block) and the CTA's 128-row key block J
-// (anchor R_J), with d = 2^(R_I - R_J) per channel and Qt_I = Qh_I (.) d:
+// Attention", fast training sections 1 and 2).  For a 128-row query tile I
+// (anchor R_I) and the CTA's 128-row key block J (anchor R_J), with
+// d = 2^(R_I - R_J) per channel and Qt_I = Qh_I (.) d:
 //   S^T  = Kh_J Qt_I^T              P_ij = 2^(S*scale*log2e + bias - lse2_i)
 //   dP^T = V_J dO_I^T               dS_ij = P_ij (dP_ij - D_i)
-//   dV_J  += P^T dO_I
-//   dKa_J += dS^T Qt_I              dk_j = scale * 2^(R_J - P_j) (.) dKa_j
-//   dQ^T_I = Kh_J^T dS^T            dq_i += (.)_n d_n * dQ_i   (fp32 atomics;
-//                                   the factor scale * 2^(P_i - R_I) is applied
-//                                   once per row by the finalize kernel)
+//   dV_J  += P^T dO_I               (P^T from TMEM)
+//   dKa_J += dS^T Qt_I              (dS^T from TMEM); dk_j = scale 2^(R_J - P_j) dKa_j
+//   dQ^T_I = Kh_J^T dS^T            dq_i += d_n * dQ_i   (fp32 atomics; the
+//                                   factor scale * 2^(P_i - R_I) is applied once
+//                                   per row by the finalize kernel)
 // The gate gradient needs dk per query head before the GQA sum; it is fused
 // into the finalize kernel as dL = q (.) dq - k (.) dk^(h) (blog, fast
 // training section 2: the key-side term is -K_j (.) dK_j), followed by the
 // reverse scan.  The row part of the scalar-gate gradient is analytic,
 // sum_j dS_ij = D_i * p_sink,i, and the column part is summed per key thread.
 //
+// Operands that the tensor core would otherwise read twice from shared memory
+// (P^T, dS^T) are written back into TMEM as bf16 pairs over the S^T / dP^T
+// columns they came from and fed as TMEM A operands; dQ^T then lands in the
+// two freed column halves.  All MMAs are M = 128 with N = 128 (N = 64 for the
+// dQ^T halves), which keeps shared-memory operand traffic below the tensor
+// rate.
+//
 // CTA = one 128-row key block of one (sequence, head), 14 warps:
-//   warp 0      TMA: Kh_J, V_J once; Qh_I and dO_I per tile (2-stage ring)
+//   warp 0      TMA: Kh_J, V_J once; Qh_I (2 stages) and dO_I (1 stage, freed
+//               by the first MMA that reads it last) per tile
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-5   Qt_I = Qh_I (.) d in shared memory
-//   warps 6-9   one thread per key: P, dS -> swizzled SMEM (bf16), column
-//               sums; at the end dK, dV epilogue
+//   warps 6-9   one thread per key: P, dS; P^T, dS^T -> TMEM, dS^T -> a
+//               swizzled shared tile; column sums; dK, dV epilogue at the end
 //   warps 10-13 dQ^T epilogue: one thread per channel, scale by d, coalesced
-//               fp32 atomic adds (own warps, so slow atomics never delay the
-//               next tile's rescale)
-// TMEM columns: S^T [0,64), dP^T [64,128), dV [128,256), dK [256,384),
-// dQ^T double buffer [384,448), [448,512).
+//               fp32 atomic adds after the TMEM columns are released
 #include <cuda.h>
 
 #include <type_traits>
@@ -42,8 +47,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BQ = 64;
-constexpr int BK = 128;
+constexpr int BQ = 128;  // query rows per tile
+constexpr int BK = 128;  // key rows per CTA
 constexpr int kThreads = 448;
 
 struct BwdTcParams {
@@ -68,19 +73,18 @@ template <int KD>
 struct BSmem {
   static constexpr int kKV = BK * KD * 2;   // key or value block
   static constexpr int kQ = BQ * KD * 2;    // query or dO tile
-  static constexpr int kPS = BK * BQ * 2;   // P^T or dS^T (bf16)
+  static constexpr int kS = BK * BQ * 2;    // dS^T (bf16), B operand of dQ^T
   static constexpr int oK = 0;
   static constexpr int oV = oK + kKV;
   static constexpr int oQ = oV + kKV;       // 2 stages
-  static constexpr int oO = oQ + 2 * kQ;    // 2 stages
-  static constexpr int oP = oO + 2 * kQ;
-  static constexpr int oS = oP + kPS;
-  static constexpr int oDw = oS + kPS;             // float[2 stages][4 warps][KD]
-  static constexpr int oRow = oDw + 8 * KD * 4;    // float[4 warps][3][BQ] (2 used)
-  static constexpr int oRI = oRow + 4 * 3 * BQ * 4;  // float[2 stages][KD] query-block anchors
-  static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD] key-block anchor
+  static constexpr int oO = oQ + 2 * kQ;    // 1 stage
+  static constexpr int oS = oO + kQ;
+  static constexpr int oDw = oS + kS;              // float[4 warps][KD]
+  static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][2][BQ]
+  static constexpr int oRI = oRow + 4 * 2 * BQ * 4;  // float[2 stages][KD]
+  static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD]
   static constexpr int oBar = oRJ + KD * 4;
-  static constexpr int kBars = 20;
+  static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -89,16 +93,25 @@ struct BSmem {
 enum BBar {
   KV_FULL = 0,
   Q_FULL = 1,     // +stage
-  O_FULL = 3,     // +stage
-  Q_READY = 5,    // +stage
-  QO_EMPTY = 7,   // +stage
+  O_FULL = 3,
+  Q_READY = 4,    // +stage
+  Q_EMPTY = 6,    // +stage
+  O_EMPTY = 8,
   S_FULL = 9,
   P_FULL = 10,
-  DQ_FULL = 11,   // +stage
-  DQ_FREE = 13,   // +stage
-  MM_DONE = 15,
-  MMA_DONE = 16,
+  DQ_FULL = 11,
+  DQ_FREE = 12,
+  MM_DONE = 13,
+  MMA_DONE = 14,
 };
+
+// TMEM columns: S^T [0,128) and dP^T [128,256) (lanes = keys, columns =
+// queries); the softmax writes P^T bf16 pairs over [0,64) and dS^T over
+// [128,192); dQ^T (lanes = channels) lands in the two freed halves
+// [64,128) (queries 0..63) and [192,256) (queries 64..127); dV [256,384),
+// dK [384,512).
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+constexpr uint32_t kColDQa = 64, kColDQb = 192;
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
                                          volatile int* abort_flag) {
@@ -151,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int j0 = blk * BK;
   const int nj = min(BK, L - j0);
   const int i_last = p.window > 0 ? min(L - 1, j0 + nj - 1 + p.window - 1) : L - 1;
-  const int I0 = j0 / BQ;
+  const int I0 = j0 / BQ;                 // first query tile (the diagonal one)
   const int nT = i_last / BQ - I0 + 1;
   const float* anc = p.anchors + ((long)blk_off * HQ + h) * K;  // + block * HQ * K
 
@@ -159,14 +172,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(KV_FULL), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Q_FULL + s), 1);
-      mbar_init(bar(O_FULL + s), 1);
       mbar_init(bar(Q_READY + s), 4);
-      mbar_init(bar(QO_EMPTY + s), 1);
-      mbar_init(bar(DQ_FULL + s), 1);
-      mbar_init(bar(DQ_FREE + s), 4);
+      mbar_init(bar(Q_EMPTY + s), 1);
     }
+    mbar_init(bar(O_FULL), 1);
+    mbar_init(bar(O_EMPTY), 1);
     mbar_init(bar(S_FULL), 1);
     mbar_init(bar(P_FULL), 4);
+    mbar_init(bar(DQ_FULL), 1);
+    mbar_init(bar(DQ_FREE), 4);
     mbar_init(bar(MM_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
     *abort_flag = 0;
@@ -199,81 +213,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + Lay::oV + b * (BK * 128), &tm_v, bar(KV_FULL), b * 64, kh,
                     (int)(s0 + j0));
       }
-      int issued = 0;
+      int q_issued = 0, o_issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t & 1;
         const int row = (int)(s0 + (long)(I0 + t) * BQ);
-        if (t >= 2 && !wait_bar(bar(QO_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+        if (t >= 2 && !wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
         mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
-        mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
-        bulk_load(sbase + Lay::oRI + st * K * 4,
-                  anc + (long)((I0 + t) / 2) * HQ * K, K * 4, bar(Q_FULL + st));
-        for (int b = 0; b < K / 64; ++b) {
+        for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
                       b * 64, h, row);
-          tma_load_3d(sbase + Lay::oO + st * Lay::kQ + b * (BQ * 128), &tm_o, bar(O_FULL + st),
-                      b * 64, h, row);
-        }
-        issued = t + 1;
+        bulk_load(sbase + Lay::oRI + st * K * 4, anc + (long)(I0 + t) * HQ * K, K * 4,
+                  bar(Q_FULL + st));
+        q_issued = t + 1;
+        if (t >= 1 && !wait_bar(bar(O_EMPTY), (t - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(bar(O_FULL), Lay::kQ);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oO + b * (BQ * 128), &tm_o, bar(O_FULL), b * 64, h, row);
+        o_issued = t + 1;
       }
-      for (int t = max(0, issued - 2); t < issued; ++t) {
+      for (int t = max(0, q_issued - 2); t < q_issued; ++t)
         mbar_wait(bar(Q_FULL + (t & 1)), (t >> 1) & 1, p.status);
-        mbar_wait(bar(O_FULL + (t & 1)), (t >> 1) & 1, p.status);
-      }
+      if (o_issued > 0) mbar_wait(bar(O_FULL), (o_issued - 1) & 1, p.status);
       mbar_wait(bar(KV_FULL), 0, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       const uint32_t id_sd = idesc_bf16(128, BQ, false, false);  // S^T, dP^T
-      const uint32_t id_acc = idesc_bf16(128, KD, false, true);  // dV, dK
-      const uint32_t id_dq = idesc_bf16(128, BQ, true, true);    // dQ^T
+      const uint32_t id_acc = idesc_bf16(128, KD, false, true);  // dV, dK (A from TMEM)
+      const uint32_t id_dq = idesc_bf16(128, 64, true, true);    // dQ^T halves
       bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
       for (int t = 0; ok && t < nT; ++t) {
         const int st = t & 1;
         if (!wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag)) break;
-        if (!wait_bar(bar(O_FULL + st), (t >> 1) & 1, p.status, abort_flag)) break;
+        if (!wait_bar(bar(O_FULL), t & 1, p.status, abort_flag)) break;
+        // the previous tile's dQ^T halves (in the S^T / dP^T columns) were read
+        if (t >= 1 && !wait_bar(bar(DQ_FREE), (t - 1) & 1, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ;
-        const uint32_t oa = sbase + Lay::oO + st * Lay::kQ;
-        // S^T = Kh Qt^T and dP^T = V dO^T: M = 128 keys, N = 64 queries, K = channels
+        const uint32_t oa = sbase + Lay::oO;
+        // S^T = Kh Qt^T and dP^T = V dO^T: M = 128 keys, N = 128 queries, K = channels
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t offA = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
           const uint32_t offB = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_bf16_ss(tmem + 0, sdesc_sw128(sbase + Lay::oK + offA, 16, 1024),
+          umma_bf16_ss(tmem + kColS, sdesc_sw128(sbase + Lay::oK + offA, 16, 1024),
                        sdesc_sw128(qa + offB, 16, 1024), id_sd, kk > 0);
-          umma_bf16_ss(tmem + 64, sdesc_sw128(sbase + Lay::oV + offA, 16, 1024),
+          umma_bf16_ss(tmem + kColDP, sdesc_sw128(sbase + Lay::oV + offA, 16, 1024),
                        sdesc_sw128(oa + offB, 16, 1024), id_sd, kk > 0);
         }
         umma_commit(bar(S_FULL));
         if (!wait_bar(bar(P_FULL), t & 1, p.status, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO and dK += dS^T Qt: M = 128 keys, N = channels, K = 64 queries
+        // dV += P^T dO: A = P^T from TMEM (8 columns per 16 queries), B = dO MN-major
+        const uint32_t acc0 = t > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t aP = sdesc_sw128(sbase + Lay::oP + kk * 32, 16, 1024);
-          const uint64_t aS = sdesc_sw128(sbase + Lay::oS + kk * 32, 16, 1024);
-          const uint64_t bO = sdesc_sw128(oa + kk * 16 * 128, BQ * 128, 1024);
-          const uint64_t bQ = sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024);
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16_ss(tmem + 128, aP, bO, id_acc, acc);
-          umma_bf16_ss(tmem + 256, aS, bQ, id_acc, acc);
-        }
-        umma_commit(bar(QO_EMPTY + st));
-        // dQ^T = Kh^T dS^T: M = 128 channels (for K = 64 the upper half is
-        // unused), N = 64 queries, K = 128 keys; both operands MN-major
-        if (t >= 2 && !wait_bar(bar(DQ_FREE + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
-          break;
-        tc_fence_after();
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          umma_bf16_ts(tmem + kColDV, tmem + kColS + kk * 8,
+                       sdesc_sw128(oa + kk * 16 * 128, BQ * 128, 1024), id_acc,
+                       (acc0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(O_EMPTY));
+        // dK += dS^T Qt: A = dS^T from TMEM, B = Qt MN-major
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t aK = sdesc_sw128(sbase + Lay::oK + kk * 16 * 128, BK * 128, 1024);
-          const uint64_t bS = sdesc_sw128(sbase + Lay::oS + kk * 16 * 128, 128, 1024);
-          umma_bf16_ss(tmem + 384 + st * 64, aK, bS, id_dq, kk > 0);
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          umma_bf16_ts(tmem + kColDK, tmem + kColDP + kk * 8,
+                       sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024), id_acc,
+                       (acc0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(Q_EMPTY + st));
+        // dQ^T = Kh^T dS^T in two 64-query halves: A = Kh MN-major (M =
+        // channels; for K = 64 the upper half is unused), B = the dS^T
+        // shared tile MN-major (one 64-query box per half), K = 128 keys
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t dcol = half ? kColDQb : kColDQa;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t aK = sdesc_sw128(sbase + Lay::oK + kk * 16 * 128, BK * 128, 1024);
+            const uint64_t bS =
+                sdesc_sw128(sbase + Lay::oS + half * (BK * 128) + kk * 16 * 128, 128, 1024);
+            umma_bf16_ss(tmem + dcol, aK, bS, id_dq, kk > 0);
+          }
         }
-        umma_commit(bar(DQ_FULL + st));
+        umma_commit(bar(DQ_FULL));
       }
       umma_commit(bar(MM_DONE));
       umma_commit(bar(MMA_DONE));
@@ -284,19 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wt = threadIdx.x - 64;
     const int wq = warp - 2;
     const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
+    float* d = sDw + wq * KD;
     for (int t = 0; t < nT; ++t) {
       const int st = t & 1;
-      // this warp's copy of d = 2^(R_I - R_J) for the tile, kept per stage so
-      // the dQ epilogue of the same tile reads it
-      float* d = sDw + (st * 4 + wq) * KD;
       const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4);
+      __syncwarp();
       for (int c = lane; c < K; c += 32) d[c] = exp2f(ri[c] - rjs[c]);
       __syncwarp();
       uint8_t* qt = smem + Lay::oQ + st * Lay::kQ;
       constexpr int kPer = (KD / 64) * BQ * 8 / 128;  // chunks per thread
-      constexpr int kBatch = kPer < 4 ? kPer : 4;
+      constexpr int kBatch = 4;
 #pragma unroll 1
       for (int b0 = 0; b0 < kPer; b0 += kBatch) {
         uint4 u[kBatch];
@@ -337,33 +358,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = quarter * 32 + lane;   // channel of this thread
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
-    for (int u = 0; u < nT; ++u) {
-      const int su = u & 1;
-      const int Iu = I0 + u;
+    for (int t = 0; t < nT; ++t) {
+      const int It = I0 + t;
       // d for this channel, from the anchors in global memory (the shared
       // stage may already hold a later tile); loaded before the wait
-      const float ri_n = (n < K) ? anc[(long)(Iu / 2) * HQ * K + n] : 0.f;
-      const bool got = wait_bar(bar(DQ_FULL + su), (u >> 1) & 1, p.status, abort_flag);
+      const float ri_n = (n < K) ? anc[(long)It * HQ * K + n] : 0.f;
+      const bool got = wait_bar(bar(DQ_FULL), t & 1, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const float dn = (n < K) ? exp2f(ri_n - rjs[n]) : 0.f;
-#pragma unroll
-      for (int c = 0; c < BQ; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + 384 + su * 64 + c, v);
+      float* dq_col = p.dq32 + ((s0 + (long)It * BQ) * HQ + h) * (long)K + n;
+      const long row_stride = (long)HQ * K;
+      // first half: read, add; second half: read, release the columns, add
+      const int rows_left = L - It * BQ;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t va[32], vb[32];
+        const uint32_t col = half ? kColDQb : kColDQa;
+        tmem_ld32(tmem + lane_base + col, va);
+        tmem_ld32(tmem + lane_base + col + 32, vb);
         tmem_wait_ld();
+        if (half == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(DQ_FREE));
+        }
         if (n < K) {
+          const int r0 = half * 64;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int i = Iu * BQ + c + e;
-            if (i < L) atomicAdd(p.dq32 + ((s0 + i) * HQ + h) * (long)K + n,
-                                 __uint_as_float(v[e]) * dn);
+            if (r0 + e < rows_left)
+              atomicAdd(dq_col + (r0 + e) * row_stride, __uint_as_float(va[e]) * dn);
+            if (r0 + e + 32 < rows_left)
+              atomicAdd(dq_col + (r0 + e + 32) * row_stride, __uint_as_float(vb[e]) * dn);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(DQ_FREE + su));
     }
   } else {
     // ------------------------------------------------------------ P, dS per key (warps 6-9)
@@ -373,10 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool key_ok = r < nj;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const float gs_j = (p.GS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
-    float* rowv = sRow + (warp - 6) * 3 * BQ;  // this warp's copy of the tile's query terms
+    float* rowv = sRow + (warp - 6) * 2 * BQ;  // this warp's copy of the tile's query terms
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     float colsum = 0.f;
     bool ok = true;
+    uint8_t* srow = smem + Lay::oS + r * 128;  // this key's row of the dS^T tile
     for (int t = 0; t < nT; ++t) {
       const int i0 = (I0 + t) * BQ;
       __syncwarp();
@@ -396,15 +427,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // every query of the tile sees this key: no mask work in the loop
       const bool full = key_ok && (i0 >= jj) && (i0 + BQ <= L) && (i0 + BQ - 1 - jj < win);
-      uint8_t* prow = smem + Lay::oP + r * 128;
-      uint8_t* srow = smem + Lay::oS + r * 128;
 #pragma unroll 1
       for (int c = 0; c < BQ; c += 32) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_base + c, sv);
-        tmem_ld32(tmem + lane_base + 64 + c, dv);
+        tmem_ld32(tmem + lane_base + kColS + c, sv);
+        tmem_ld32(tmem + lane_base + kColDP + c, dv);
         tmem_wait_ld();
-        // 8 keys' worth of P and dS at a time: compute, pack, store
+        uint32_t pp[16], dd[16];
         auto group = [&](int g8, auto masked) {
           float pe[8], de[8];
 #pragma unroll
@@ -423,13 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             de[e] = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
           }
           colsum += ((de[0] + de[1]) + (de[2] + de[3])) + ((de[4] + de[5]) + (de[6] + de[7]));
-          const int pch = ((c / 8) + g8) ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + pch * 16) =
-              make_uint4(pack_bf16x2(pe[0], pe[1]), pack_bf16x2(pe[2], pe[3]),
-                         pack_bf16x2(pe[4], pe[5]), pack_bf16x2(pe[6], pe[7]));
-          *reinterpret_cast<uint4*>(srow + pch * 16) =
-              make_uint4(pack_bf16x2(de[0], de[1]), pack_bf16x2(de[2], de[3]),
-                         pack_bf16x2(de[4], de[5]), pack_bf16x2(de[6], de[7]));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pp[g8 * 4 + e] = pack_bf16x2(pe[2 * e], pe[2 * e + 1]);
+            dd[g8 * 4 + e] = pack_bf16x2(de[2 * e], de[2 * e + 1]);
+          }
         };
         if (full) {
 #pragma unroll
@@ -438,7 +465,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int g8 = 0; g8 < 4; ++g8) group(g8, std::true_type{});
         }
+        // P^T, dS^T as bf16 pairs over the consumed S^T / dP^T columns
+        tmem_st16(tmem + lane_base + kColS + c / 2, pp);
+        tmem_st16(tmem + lane_base + kColDP + c / 2, dd);
+        // dS^T also into the swizzled shared tile (B operand of dQ^T):
+        // queries [c, c+32) -> box c/64, 16-byte chunks (c%64)/8 .. +3
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          const int q0 = c + g8 * 8;
+          const int pch = ((q0 % 64) / 8) ^ (r & 7);
+          *reinterpret_cast<uint4*>(srow + (q0 / 64) * (BK * 128) + pch * 16) =
+              make_uint4(dd[g8 * 4], dd[g8 * 4 + 1], dd[g8 * 4 + 2], dd[g8 * 4 + 3]);
+        }
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -452,8 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < KD; c += 32) {
         uint32_t kv[32], vv[32];
-        tmem_ld32(tmem + lane_base + 256 + c, kv);
-        tmem_ld32(tmem + lane_base + 128 + c, vv);
+        tmem_ld32(tmem + lane_base + kColDK + c, kv);
+        tmem_ld32(tmem + lane_base + kColDV + c, vv);
         tmem_wait_ld();
         if (key_ok) {
           const float* Pj = p.P + krow * K + c;
