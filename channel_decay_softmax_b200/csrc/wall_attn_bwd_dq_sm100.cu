@@ -1,0 +1,459 @@
+// wall_attn_bwd_dq_sm100.cu -- tensor-core dq of the Wall Attention backward
+// (bf16, K == V in {64, 128}), one CTA per 128-row query block, no atomics.
+//
+// Same anchored form as the forward (Tilde blog "Wall Attention", fast
+// training section 1): for the CTA's query block I and key tile J,
+// Kt_J = Kh_J (.) 2^(R_I - R_J) per channel, and
+//   S  = Qh_I Kt_J^T           P_ij = 2^(S*scale*log2e + bias - lse2_i)
+//   dP = dO_I V_J^T            dS_ij = P_ij (dP_ij - D_i)
+//   dQa += dS Kt_J             (dS from TMEM, Kt MN-major from shared memory)
+// so that dq_i = scale * 2^(P_i - R_I) (.) dQa_i; the factor is applied per row
+// by the finalize kernel, which also forms the gate-gradient summand.  dq is
+// written once per row: deterministic, and no fp32 atomics through L2.
+//
+// CTA = 10 warps:
+//   warp 0      TMA: Qh_I, dO_I once; Kh_J (+ block anchors, 3 stages) and V_J
+//               (1 stage: it is read by one MMA only) per key tile
+//   warp 1      TMEM owner and MMA issuer: S two tiles ahead, dP one ahead
+//   warps 2-5   key rescale Kt_J = Kh_J (.) d in shared memory
+//   warps 6-9   one thread per query row: P, dS -> bf16 pairs over the
+//               consumed S columns; epilogue dQa -> fp32 workspace
+// TMEM columns: S0 [0,128), S1 [128,256), dP [256,384), dQa [384,512).
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
+#include "wall_common.cuh"
+#include "wall_internal.h"
+
+namespace wall {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kKS = 3;  // key stages
+constexpr int kThreads = 320;
+
+struct DqParams {
+  const float* anchors;  // [nblk, HQ, K]
+  const float* lse;      // [rows, HQ]
+  const float* D;        // [rows, HQ]
+  const float* GS;       // [rows, HQ] or nullptr
+  float* dq32;           // [rows, HQ, K]  raw dQa (without scale * 2^(P - R_I))
+  Seqs seqs;
+  int HQ, H;
+  float scale_log2;
+  int window;
+  int n_blocks;
+  int* status;
+};
+
+template <int KD>
+struct DSmem {
+  static constexpr int kT = BM * KD * 2;  // one 128-row bf16 tile
+  static constexpr int oQ = 0;
+  static constexpr int oO = oQ + kT;
+  static constexpr int oK = oO + kT;           // kKS stages
+  static constexpr int oV = oK + kKS * kT;     // 1 stage
+  static constexpr int oRI = oV + kT;          // float[KD]
+  static constexpr int oRJ = oRI + KD * 4;     // float[kKS][KD]
+  static constexpr int oD = oRJ + kKS * KD * 4;  // float[4 warps][KD]
+  static constexpr int oGS = oD + 4 * KD * 4;    // float[4 warps][BN]
+  static constexpr int oBar = oGS + 4 * BN * 4;
+  static constexpr int kBars = 16;
+  static constexpr int oMisc = oBar + kBars * 8;
+  static constexpr int kBytes = oMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+enum DBar {
+  QO_FULL = 0,
+  K_FULL = 1,    // + stage (3)
+  K_READY = 4,   // + stage (3)
+  K_EMPTY = 7,   // + stage (3)
+  V_FULL = 10,
+  V_EMPTY = 11,
+  SD_FULL = 12,
+  P_FULL = 13,
+  DQ_DONE = 14,
+  MMA_DONE = 15,
+};
+
+constexpr uint32_t kColS = 0, kColDP = 256, kColDQ = 384;
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
+                                         volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      record_status(status, WALL_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int KD>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  DqParams p) {
+  using Lay = DSmem<KD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
+  float* sD = reinterpret_cast<float*>(smem + Lay::oD);
+  float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.x;
+  const int HQ = p.HQ, K = KD;
+  const int kh = h / (HQ / p.H);
+  // longest query blocks first
+  const int flat = p.n_blocks - 1 - (int)blockIdx.y;
+  int seq, blk;
+  if (!seq_block(p.seqs, BM, flat, seq, blk)) return;
+  const int blk_off = flat - blk;
+  const long s0 = p.seqs.start(seq);
+  const int L = p.seqs.len(seq);
+  const int i0 = blk * BM;
+  const int ni = min(BM, L - i0);
+  const int jb_hi = (i0 + ni - 1) / BN;
+  const int jb_lo = p.window > 0 ? max(0, i0 - p.window + 1) / BN : 0;
+  const int nT = jb_hi - jb_lo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(QO_FULL), 1);
+    for (int s = 0; s < kKS; ++s) {
+      mbar_init(bar(K_FULL + s), 1);
+      mbar_init(bar(K_READY + s), 4);
+      mbar_init(bar(K_EMPTY + s), 1);
+    }
+    mbar_init(bar(V_FULL), 1);
+    mbar_init(bar(V_EMPTY), 1);
+    mbar_init(bar(SD_FULL), 1);
+    mbar_init(bar(P_FULL), 4);
+    mbar_init(bar(DQ_DONE), 1);
+    mbar_init(bar(MMA_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  for (int n = threadIdx.x; n < K; n += kThreads)
+    sRI[n] = p.anchors[((long)(blk_off + blk) * HQ + h) * K + n];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_o);
+      mbar_expect_tx(bar(QO_FULL), 2 * Lay::kT);
+      for (int b = 0; b < K / 64; ++b) {
+        tma_load_3d(sbase + Lay::oQ + b * (BM * 128), &tm_q, bar(QO_FULL), b * 64, h,
+                    (int)(s0 + i0));
+        tma_load_3d(sbase + Lay::oO + b * (BM * 128), &tm_o, bar(QO_FULL), b * 64, h,
+                    (int)(s0 + i0));
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kKS;
+        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+        if (t >= kKS &&
+            !wait_bar(bar(K_EMPTY + st), ((t / kKS) - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(K_FULL + st), Lay::kT + K * 4);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k, bar(K_FULL + st),
+                      b * 64, h, row);
+        bulk_load(sbase + Lay::oRJ + st * K * 4,
+                  p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
+                  bar(K_FULL + st));
+        k_issued = t + 1;
+        if (t >= 1 && !wait_bar(bar(V_EMPTY), (t - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(bar(V_FULL), Lay::kT);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oV + b * (BN * 128), &tm_v, bar(V_FULL), b * 64, kh, row);
+        v_issued = t + 1;
+      }
+      for (int t = max(0, k_issued - kKS); t < k_issued; ++t)
+        mbar_wait(bar(K_FULL + t % kKS), (t / kKS) & 1, p.status);
+      if (v_issued > 0) mbar_wait(bar(V_FULL), (v_issued - 1) & 1, p.status);
+      mbar_wait(bar(QO_FULL), 0, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(BM, BN, false, false);   // S, dP
+      const uint32_t id_dq = idesc_bf16(BM, KD, false, true);   // dQa (A from TMEM)
+      bool ok = wait_bar(bar(QO_FULL), 0, p.status, abort_flag);
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % kKS;
+        if (!wait_bar(bar(K_READY + st), (t / kKS) & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + kColS + (t & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < KD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_bf16_ss(d_tmem, sdesc_sw128(sbase + Lay::oQ + off, 16, 1024),
+                       sdesc_sw128(sbase + Lay::oK + st * Lay::kT + off, 16, 1024), id_s,
+                       kk > 0 ? 1u : 0u);
+        }
+        return true;
+      };
+      auto issue_dp = [&](int t) -> bool {
+        if (!wait_bar(bar(V_FULL), t & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < KD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_bf16_ss(tmem + kColDP, sdesc_sw128(sbase + Lay::oO + off, 16, 1024),
+                       sdesc_sw128(sbase + Lay::oV + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(V_EMPTY));
+        umma_commit(bar(SD_FULL));  // S(t) was issued earlier: both are ready
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok) ok = issue_dp(0);
+      if (ok && nT > 1) ok = issue_s(1);
+      for (int t = 0; ok && t < nT; ++t) {
+        const int st = t % kKS;
+        if (!wait_bar(bar(P_FULL), t & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        // dQa += dS Kt: A = dS (bf16 pairs over the S buffer, 8 columns per 16
+        // keys), B = Kt [keys x channels] MN-major: 8-key groups 1 KB apart,
+        // 64-channel boxes BN*128 bytes apart
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(tmem + kColDQ, tmem + kColS + (t & 1) * 128 + kk * 8,
+                       sdesc_sw128(sbase + Lay::oK + st * Lay::kT + kk * 16 * 128, BN * 128,
+                                   1024),
+                       id_dq, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(K_EMPTY + st));
+        if (t + 1 < nT) ok = issue_dp(t + 1);
+        if (ok && t + 2 < nT) ok = issue_s(t + 2);
+      }
+      umma_commit(bar(DQ_DONE));
+      umma_commit(bar(MMA_DONE));
+      mbar_wait(bar(MMA_DONE), 0, p.status);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ key rescale
+    const int wt = threadIdx.x - 64;
+    const int wq = warp - 2;
+    float* d = sD + wq * KD;
+    for (int t = 0; t < nT; ++t) {
+      const int st = t % kKS;
+      const bool got = wait_bar(bar(K_FULL + st), (t / kKS) & 1, p.status, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4);
+      __syncwarp();
+      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - rj[n]);
+      __syncwarp();
+      uint8_t* kt = smem + Lay::oK + st * Lay::kT;
+      constexpr int kPer = (KD / 64) * BN * 8 / 128;
+      constexpr int kBatch = 4;
+#pragma unroll 1
+      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
+        uint4 u[kBatch];
+        float dd[kBatch][8];
+        uint4* ptr[kBatch];
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int c = wt + (b0 + x) * 128;
+          const int box = c / (BN * 8);
+          const int row = (c / 8) % BN;
+          const int pch = c % 8;
+          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
+          ptr[x] = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
+          u[x] = *ptr[x];
+          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
+          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
+          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
+          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
+        }
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
+          }
+          *ptr[x] = u[x];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(K_READY + st));
+    }
+  } else {
+    // ------------------------------------------------------------ dS per query row
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int i = i0 + r;
+    const bool row_ok = r < ni;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const bool has_gs = p.GS != nullptr;
+    const int win = p.window > 0 ? p.window : 0x7fffffff;
+    const long grow = (s0 + i) * HQ + h;
+    const float lse2 = row_ok ? p.lse[grow] * kLog2e : 0.f;
+    const float Di = row_ok ? p.D[grow] : 0.f;
+    const float gs_i = (has_gs && row_ok) ? p.GS[grow] * kLog2e : 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < nT; ++t) {
+      const int j0 = (jb_lo + t) * BN;
+      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix (or zeros)
+      if (has_gs || t == 0) {
+        __syncwarp();
+        for (int c = lane; c < BN; c += 32) {
+          const int j = j0 + c;
+          gsk[c] = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
+        }
+        __syncwarp();
+      }
+      {
+        const bool got = wait_bar(bar(SD_FULL), t & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + kColS + (t & 1) * 128;
+      const uint32_t dp_addr = tmem + lane_base + kColDP;
+      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) && (i - j0 < win);
+      const bool fast = full && !has_gs;
+      const float off_i = (has_gs ? gs_i : 0.f) - lse2;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(s_addr + c, sv);
+        tmem_ld32(dp_addr + c, dv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+        if (fast) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = exp2f(fmaf(__uint_as_float(sv[e]), sl2, off_i));
+            const float p1 = exp2f(fmaf(__uint_as_float(sv[e + 1]), sl2, off_i));
+            pk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - Di),
+                                    p1 * (__uint_as_float(dv[e + 1]) - Di));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float ds[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int j = j0 + c + e + x;
+              const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
+              const float a = fmaf(__uint_as_float(sv[e + x]), sl2, off_i - gsk[c + e + x]);
+              const float pv = vis ? exp2f(a) : 0.f;
+              ds[x] = pv * (__uint_as_float(dv[e + x]) - Di);
+            }
+            pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+          }
+        }
+        // keys [c, c+32) -> columns [c/2, c/2+16) of this S buffer (already read)
+        tmem_st16(s_addr + c / 2, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(P_FULL));
+    }
+    // ---- epilogue: the raw dQa row
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(DQ_DONE), 0, p.status, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      float* out = p.dq32 + grow * K;
+#pragma unroll 1
+      for (int c = 0; c < KD; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + kColDQ + c, v);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(out + c + e) =
+                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int KD>
+int launch_dq(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
+              cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tile_map(&tq, ws.qh, pb.rows, pb.HQ, KD, BM) ||
+      !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN) ||
+      !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BN) ||
+      !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BM))
+    return WALL_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(bwd_dq_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DSmem<KD>::kAlloc) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    attr = true;
+  }
+  DqParams p;
+  p.anchors = ws.anchors;
+  p.lse = a.lse;
+  p.D = a.D;
+  p.GS = a.GS;
+  p.dq32 = a.dq32;
+  p.seqs = pb.seqs;
+  p.HQ = pb.HQ;
+  p.H = pb.H;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.window = pb.window;
+  p.n_blocks = ws.n_blocks128;
+  p.status = status;
+  dim3 grid(pb.HQ, ws.n_blocks128);
+  bwd_dq_kernel<KD><<<grid, kThreads, DSmem<KD>::kAlloc, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+}  // namespace
+
+int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
+                   cudaStream_t stream) {
+  if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
+  return pb.K == 128 ? launch_dq<128>(pb, a, ws, status, stream)
+                     : launch_dq<64>(pb, a, ws, status, stream);
+}
+
+}  // namespace wall

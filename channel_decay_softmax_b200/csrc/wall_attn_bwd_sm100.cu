@@ -9,9 +9,8 @@
 //   dP^T = V_J dO_I^T               dS_ij = P_ij (dP_ij - D_i)
 //   dV_J  += P^T dO_I               (P^T from TMEM)
 //   dKa_J += dS^T Qt_I              (dS^T from TMEM); dk_j = scale 2^(R_J - P_j) dKa_j
-//   dQ^T_I = Kh_J^T dS^T            dq_i += d_n * dQ_i   (fp32 atomics; the
-//                                   factor scale * 2^(P_i - R_I) is applied once
-//                                   per row by the finalize kernel)
+// dq comes from a separate query-block kernel (wall_attn_bwd_dq_sm100.cu), so
+// no fp32 atomics are needed.
 // The gate gradient needs dk per query head before the GQA sum; it is fused
 // into the finalize kernel as dL = q (.) dq - k (.) dk^(h) (blog, fast
 // training section 2: the key-side term is -K_j (.) dK_j), followed by the
@@ -20,20 +19,16 @@
 //
 // Operands that the tensor core would otherwise read twice from shared memory
 // (P^T, dS^T) are written back into TMEM as bf16 pairs over the S^T / dP^T
-// columns they came from and fed as TMEM A operands; dQ^T then lands in the
-// two freed column halves.  All MMAs are M = 128 with N = 128 (N = 64 for the
-// dQ^T halves), which keeps shared-memory operand traffic below the tensor
-// rate.
+// columns they came from and fed as TMEM A operands.  All MMAs are M = 128,
+// N = 128.
 //
-// CTA = one 128-row key block of one (sequence, head), 14 warps:
+// CTA = one 128-row key block of one (sequence, head), 10 warps:
 //   warp 0      TMA: Kh_J, V_J once; Qh_I (2 stages) and dO_I (1 stage, freed
 //               by the first MMA that reads it last) per tile
 //   warp 1      TMEM owner and MMA issuer
 //   warps 2-5   Qt_I = Qh_I (.) d in shared memory
-//   warps 6-9   one thread per key: P, dS; P^T, dS^T -> TMEM, dS^T -> a
-//               swizzled shared tile; column sums; dK, dV epilogue at the end
-//   warps 10-13 dQ^T epilogue: one thread per channel, scale by d, coalesced
-//               fp32 atomic adds after the TMEM columns are released
+//   warps 6-9   one thread per key: P, dS; P^T, dS^T -> TMEM; column sums;
+//               dK, dV epilogue at the end
 #include <cuda.h>
 
 #include <type_traits>
@@ -49,7 +44,7 @@ using namespace sm100;
 
 constexpr int BQ = 128;  // query rows per tile
 constexpr int BK = 128;  // key rows per CTA
-constexpr int kThreads = 448;
+constexpr int kThreads = 320;
 
 struct BwdTcParams {
   const float* anchors;  // [nblk128, HQ, K]
@@ -57,7 +52,6 @@ struct BwdTcParams {
   const float* lse;      // [rows, HQ]
   const float* D;        // [rows, HQ]
   const float* GS;       // [rows, HQ] or nullptr
-  float* dq32;           // [rows, HQ, K], zeroed, accumulated atomically
   float* dkh32;          // [rows, HQ, K]
   float* dvh32;          // [rows, HQ, V]
   float* dgs_col;        // [rows, HQ] or nullptr
@@ -73,13 +67,11 @@ template <int KD>
 struct BSmem {
   static constexpr int kKV = BK * KD * 2;   // key or value block
   static constexpr int kQ = BQ * KD * 2;    // query or dO tile
-  static constexpr int kS = BK * BQ * 2;    // dS^T (bf16), B operand of dQ^T
   static constexpr int oK = 0;
   static constexpr int oV = oK + kKV;
   static constexpr int oQ = oV + kKV;       // 2 stages
   static constexpr int oO = oQ + 2 * kQ;    // 1 stage
-  static constexpr int oS = oO + kQ;
-  static constexpr int oDw = oS + kS;              // float[4 warps][KD]
+  static constexpr int oDw = oO + kQ;              // float[4 warps][KD]
   static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][2][BQ]
   static constexpr int oRI = oRow + 4 * 2 * BQ * 4;  // float[2 stages][KD]
   static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD]
@@ -99,19 +91,14 @@ enum BBar {
   O_EMPTY = 8,
   S_FULL = 9,
   P_FULL = 10,
-  DQ_FULL = 11,
-  DQ_FREE = 12,
-  MM_DONE = 13,
-  MMA_DONE = 14,
+  MM_DONE = 11,
+  MMA_DONE = 12,
 };
 
 // TMEM columns: S^T [0,128) and dP^T [128,256) (lanes = keys, columns =
 // queries); the softmax writes P^T bf16 pairs over [0,64) and dS^T over
-// [128,192); dQ^T (lanes = channels) lands in the two freed halves
-// [64,128) (queries 0..63) and [192,256) (queries 64..127); dV [256,384),
-// dK [384,512).
+// [128,192); dV [256,384), dK [384,512).
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
-constexpr uint32_t kColDQa = 64, kColDQb = 192;
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
                                          volatile int* abort_flag) {
@@ -179,8 +166,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(O_EMPTY), 1);
     mbar_init(bar(S_FULL), 1);
     mbar_init(bar(P_FULL), 4);
-    mbar_init(bar(DQ_FULL), 1);
-    mbar_init(bar(DQ_FREE), 4);
     mbar_init(bar(MM_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
     *abort_flag = 0;
@@ -242,14 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_sd = idesc_bf16(128, BQ, false, false);  // S^T, dP^T
       const uint32_t id_acc = idesc_bf16(128, KD, false, true);  // dV, dK (A from TMEM)
-      const uint32_t id_dq = idesc_bf16(128, 64, true, true);    // dQ^T halves
       bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
       for (int t = 0; ok && t < nT; ++t) {
         const int st = t & 1;
         if (!wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag)) break;
         if (!wait_bar(bar(O_FULL), t & 1, p.status, abort_flag)) break;
-        // the previous tile's dQ^T halves (in the S^T / dP^T columns) were read
-        if (t >= 1 && !wait_bar(bar(DQ_FREE), (t - 1) & 1, p.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ;
         const uint32_t oa = sbase + Lay::oO;
@@ -281,21 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024), id_acc,
                        (acc0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(Q_EMPTY + st));
-        // dQ^T = Kh^T dS^T in two 64-query halves: A = Kh MN-major (M =
-        // channels; for K = 64 the upper half is unused), B = the dS^T
-        // shared tile MN-major (one 64-query box per half), K = 128 keys
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t dcol = half ? kColDQb : kColDQa;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t aK = sdesc_sw128(sbase + Lay::oK + kk * 16 * 128, BK * 128, 1024);
-            const uint64_t bS =
-                sdesc_sw128(sbase + Lay::oS + half * (BK * 128) + kk * 16 * 128, 128, 1024);
-            umma_bf16_ss(tmem + dcol, aK, bS, id_dq, kk > 0);
-          }
-        }
-        umma_commit(bar(DQ_FULL));
       }
       umma_commit(bar(MM_DONE));
       umma_commit(bar(MMA_DONE));
@@ -352,49 +319,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(Q_READY + st));
     }
-  } else if (warp >= 10) {
-    // ------------------------------------------------------------ dQ epilogue
-    const int quarter = warp & 3;
-    const int n = quarter * 32 + lane;   // channel of this thread
-    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
-    for (int t = 0; t < nT; ++t) {
-      const int It = I0 + t;
-      // d for this channel, from the anchors in global memory (the shared
-      // stage may already hold a later tile); loaded before the wait
-      const float ri_n = (n < K) ? anc[(long)It * HQ * K + n] : 0.f;
-      const bool got = wait_bar(bar(DQ_FULL), t & 1, p.status, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      const float dn = (n < K) ? exp2f(ri_n - rjs[n]) : 0.f;
-      float* dq_col = p.dq32 + ((s0 + (long)It * BQ) * HQ + h) * (long)K + n;
-      const long row_stride = (long)HQ * K;
-      // first half: read, add; second half: read, release the columns, add
-      const int rows_left = L - It * BQ;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t va[32], vb[32];
-        const uint32_t col = half ? kColDQb : kColDQa;
-        tmem_ld32(tmem + lane_base + col, va);
-        tmem_ld32(tmem + lane_base + col + 32, vb);
-        tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(DQ_FREE));
-        }
-        if (n < K) {
-          const int r0 = half * 64;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (r0 + e < rows_left)
-              atomicAdd(dq_col + (r0 + e) * row_stride, __uint_as_float(va[e]) * dn);
-            if (r0 + e + 32 < rows_left)
-              atomicAdd(dq_col + (r0 + e + 32) * row_stride, __uint_as_float(vb[e]) * dn);
-          }
-        }
-      }
-    }
   } else {
     // ------------------------------------------------------------ P, dS per key (warps 6-9)
     const int quarter = warp & 3;
@@ -407,7 +331,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     float colsum = 0.f;
     bool ok = true;
-    uint8_t* srow = smem + Lay::oS + r * 128;  // this key's row of the dS^T tile
     for (int t = 0; t < nT; ++t) {
       const int i0 = (I0 + t) * BQ;
       __syncwarp();
@@ -468,18 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P^T, dS^T as bf16 pairs over the consumed S^T / dP^T columns
         tmem_st16(tmem + lane_base + kColS + c / 2, pp);
         tmem_st16(tmem + lane_base + kColDP + c / 2, dd);
-        // dS^T also into the swizzled shared tile (B operand of dQ^T):
-        // queries [c, c+32) -> box c/64, 16-byte chunks (c%64)/8 .. +3
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          const int q0 = c + g8 * 8;
-          const int pch = ((q0 % 64) / 8) ^ (r & 7);
-          *reinterpret_cast<uint4*>(srow + (q0 / 64) * (BK * 128) + pch * 16) =
-              make_uint4(dd[g8 * 4], dd[g8 * 4 + 1], dd[g8 * 4 + 2], dd[g8 * 4 + 3]);
-        }
       }
       tmem_wait_st();
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(P_FULL));
@@ -658,7 +571,6 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.lse = a.lse;
   p.D = a.D;
   p.GS = a.GS;
-  p.dq32 = a.dq32;
   p.dkh32 = a.dkh32;
   p.dvh32 = a.dvh32;
   p.dgs_col = a.GS ? a.dgs_col : nullptr;
@@ -690,10 +602,10 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void
         a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr, a.dsink);
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
   }
-  if (cudaMemsetAsync(a.dq32, 0, sizeof(float) * pb.rows * pb.HQ * pb.K, stream) != cudaSuccess)
-    return WALL_ERR_CUDA;
   rc = pb.K == 128 ? launch_bwd_tc<128>(pb, a, ws, status, stream)
                    : launch_bwd_tc<64>(pb, a, ws, status, stream);
+  if (rc) return rc;
+  rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
   if (rc) return rc;
   dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
   bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(

@@ -71,6 +71,9 @@ int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int*
 // ---- tensor-core backward (wall_attn_bwd_sm100.cu) ----
 int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void* dq, void* dk,
                 void* dv, int* status, cudaStream_t stream);
+// raw dq (without the per-row anchor factor) into a.dq32 (wall_attn_bwd_dq_sm100.cu)
+int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
+                   cudaStream_t stream);
 
 // ---- TMA tensor maps (wall_tma.cu) ----
 bool make_tile_map(CUtensorMap* m, const void* base, long rows, int heads, int dim,
