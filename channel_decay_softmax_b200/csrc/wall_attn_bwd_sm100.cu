@@ -70,8 +70,8 @@ struct BSmem {
   static constexpr int oK = 0;
   static constexpr int oV = oK + kKV;
   static constexpr int oQ = oV + kKV;       // 2 stages
-  static constexpr int oO = oQ + 2 * kQ;    // 1 stage
-  static constexpr int oDw = oO + kQ;              // float[4 warps][KD]
+  static constexpr int oO = oQ + 2 * kQ;    // 2 stages
+  static constexpr int oDw = oO + 2 * kQ;          // float[4 warps][KD]
   static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][2][BQ]
   static constexpr int oRI = oRow + 4 * 2 * BQ * 4;  // float[2 stages][KD]
   static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD]
@@ -85,19 +85,20 @@ struct BSmem {
 enum BBar {
   KV_FULL = 0,
   Q_FULL = 1,     // +stage
-  O_FULL = 3,
-  Q_READY = 4,    // +stage
-  Q_EMPTY = 6,    // +stage
-  O_EMPTY = 8,
-  S_FULL = 9,
-  P_FULL = 10,
-  MM_DONE = 11,
-  MMA_DONE = 12,
+  O_FULL = 3,     // +stage
+  Q_READY = 5,    // +stage
+  QO_EMPTY = 7,   // +stage
+  SD_FULL = 9,    // +half
+  P_FULL = 11,    // +half
+  MM_DONE = 13,
+  MMA_DONE = 14,
 };
 
-// TMEM columns: S^T [0,128) and dP^T [128,256) (lanes = keys, columns =
-// queries); the softmax writes P^T bf16 pairs over [0,64) and dS^T over
-// [128,192); dV [256,384), dK [384,512).
+// TMEM columns (lanes = keys): S^T of the two 64-query halves [0,64),
+// [64,128); dP^T halves [128,192), [192,256); the softmax writes P^T (dS^T)
+// bf16 pairs over the first 32 columns of each S^T (dP^T) half; dV
+// [256,384), dK [384,512).  While one half is in the softmax, the tensor core
+// works on the other.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
@@ -159,13 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(KV_FULL), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Q_FULL + s), 1);
+      mbar_init(bar(O_FULL + s), 1);
       mbar_init(bar(Q_READY + s), 4);
-      mbar_init(bar(Q_EMPTY + s), 1);
+      mbar_init(bar(QO_EMPTY + s), 1);
+      mbar_init(bar(SD_FULL + s), 1);
+      mbar_init(bar(P_FULL + s), 4);
     }
-    mbar_init(bar(O_FULL), 1);
-    mbar_init(bar(O_EMPTY), 1);
-    mbar_init(bar(S_FULL), 1);
-    mbar_init(bar(P_FULL), 4);
     mbar_init(bar(MM_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
     *abort_flag = 0;
@@ -198,71 +198,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + Lay::oV + b * (BK * 128), &tm_v, bar(KV_FULL), b * 64, kh,
                     (int)(s0 + j0));
       }
-      int q_issued = 0, o_issued = 0;
+      int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t & 1;
         const int row = (int)(s0 + (long)(I0 + t) * BQ);
-        if (t >= 2 && !wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+        if (t >= 2 && !wait_bar(bar(QO_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
         mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
-        for (int b = 0; b < K / 64; ++b)
+        mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
+        for (int b = 0; b < K / 64; ++b) {
           tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
                       b * 64, h, row);
+          tma_load_3d(sbase + Lay::oO + st * Lay::kQ + b * (BQ * 128), &tm_o, bar(O_FULL + st),
+                      b * 64, h, row);
+        }
         bulk_load(sbase + Lay::oRI + st * K * 4, anc + (long)(I0 + t) * HQ * K, K * 4,
                   bar(Q_FULL + st));
-        q_issued = t + 1;
-        if (t >= 1 && !wait_bar(bar(O_EMPTY), (t - 1) & 1, p.status, abort_flag)) break;
-        mbar_expect_tx(bar(O_FULL), Lay::kQ);
-        for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oO + b * (BQ * 128), &tm_o, bar(O_FULL), b * 64, h, row);
-        o_issued = t + 1;
+        issued = t + 1;
       }
-      for (int t = max(0, q_issued - 2); t < q_issued; ++t)
+      for (int t = max(0, issued - 2); t < issued; ++t) {
         mbar_wait(bar(Q_FULL + (t & 1)), (t >> 1) & 1, p.status);
-      if (o_issued > 0) mbar_wait(bar(O_FULL), (o_issued - 1) & 1, p.status);
+        mbar_wait(bar(O_FULL + (t & 1)), (t >> 1) & 1, p.status);
+      }
       mbar_wait(bar(KV_FULL), 0, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
-      const uint32_t id_sd = idesc_bf16(128, BQ, false, false);  // S^T, dP^T
+      const uint32_t id_sd = idesc_bf16(128, 64, false, false);  // S^T, dP^T halves
       const uint32_t id_acc = idesc_bf16(128, KD, false, true);  // dV, dK (A from TMEM)
       bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
-      for (int t = 0; ok && t < nT; ++t) {
+      // S^T and dP^T of one 64-query half: M = 128 keys, N = 64, K = channels
+      auto issue_sd = [&](int t, int hf) {
         const int st = t & 1;
-        if (!wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag)) break;
-        if (!wait_bar(bar(O_FULL), t & 1, p.status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ;
-        const uint32_t oa = sbase + Lay::oO;
-        // S^T = Kh Qt^T and dP^T = V dO^T: M = 128 keys, N = 128 queries, K = channels
+        const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ + hf * 64 * 128;
+        const uint32_t oa = sbase + Lay::oO + st * Lay::kQ + hf * 64 * 128;
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t offA = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
           const uint32_t offB = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_bf16_ss(tmem + kColS, sdesc_sw128(sbase + Lay::oK + offA, 16, 1024),
+          umma_bf16_ss(tmem + kColS + hf * 64, sdesc_sw128(sbase + Lay::oK + offA, 16, 1024),
                        sdesc_sw128(qa + offB, 16, 1024), id_sd, kk > 0);
-          umma_bf16_ss(tmem + kColDP, sdesc_sw128(sbase + Lay::oV + offA, 16, 1024),
+          umma_bf16_ss(tmem + kColDP + hf * 64, sdesc_sw128(sbase + Lay::oV + offA, 16, 1024),
                        sdesc_sw128(oa + offB, 16, 1024), id_sd, kk > 0);
         }
-        umma_commit(bar(S_FULL));
-        if (!wait_bar(bar(P_FULL), t & 1, p.status, abort_flag)) break;
+        umma_commit(bar(SD_FULL + hf));
+      };
+      // dV += P^T dO and dK += dS^T Qt over one half: A from TMEM (8 columns
+      // per 16 queries), B = dO / Qt rows of the half, MN-major
+      auto issue_acc = [&](int t, int hf) {
+        const int st = t & 1;
+        const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ + hf * 64 * 128;
+        const uint32_t oa = sbase + Lay::oO + st * Lay::kQ + hf * 64 * 128;
+#pragma unroll
+        for (int kk = 0; kk < 64 / 16; ++kk) {
+          const uint32_t acc = (t > 0 || hf > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16_ts(tmem + kColDV, tmem + kColS + hf * 64 + kk * 8,
+                       sdesc_sw128(oa + kk * 16 * 128, BQ * 128, 1024), id_acc, acc);
+          umma_bf16_ts(tmem + kColDK, tmem + kColDP + hf * 64 + kk * 8,
+                       sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024), id_acc, acc);
+        }
+      };
+      auto tile_ready = [&](int t) -> bool {
+        const int st = t & 1;
+        if (!wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag)) return false;
+        if (!wait_bar(bar(O_FULL + st), (t >> 1) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
-        // dV += P^T dO: A = P^T from TMEM (8 columns per 16 queries), B = dO MN-major
-        const uint32_t acc0 = t > 0 ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          umma_bf16_ts(tmem + kColDV, tmem + kColS + kk * 8,
-                       sdesc_sw128(oa + kk * 16 * 128, BQ * 128, 1024), id_acc,
-                       (acc0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(O_EMPTY));
-        // dK += dS^T Qt: A = dS^T from TMEM, B = Qt MN-major
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          umma_bf16_ts(tmem + kColDK, tmem + kColDP + kk * 8,
-                       sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024), id_acc,
-                       (acc0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(Q_EMPTY + st));
+        return true;
+      };
+      if (ok) ok = tile_ready(0);
+      if (ok) {
+        issue_sd(0, 0);
+        issue_sd(0, 1);
+      }
+      for (int t = 0; ok && t < nT; ++t) {
+        const int st = t & 1;
+        if (!wait_bar(bar(P_FULL + 0), t & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        issue_acc(t, 0);
+        const bool next = t + 1 < nT;
+        if (next) {
+          if (!tile_ready(t + 1)) break;
+          issue_sd(t + 1, 0);  // overwrites half a: in order after its dV/dK
+        }
+        if (!wait_bar(bar(P_FULL + 1), t & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        issue_acc(t, 1);
+        umma_commit(bar(QO_EMPTY + st));
+        if (next) issue_sd(t + 1, 1);
       }
       umma_commit(bar(MM_DONE));
       umma_commit(bar(MMA_DONE));
@@ -331,71 +354,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     float colsum = 0.f;
     bool ok = true;
-    for (int t = 0; t < nT; ++t) {
-      const int i0 = (I0 + t) * BQ;
-      __syncwarp();
-      // per query: c_i = GS_i*log2e - lse_i*log2e (logit offset), D_i
-      for (int c = lane; c < BQ; c += 32) {
-        const int i = i0 + c;
-        const bool in = i < L;
-        const float gsi = (in && p.GS) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
-        rowv[c] = in ? gsi - p.lse[(s0 + i) * HQ + h] * kLog2e : 0.f;
-        rowv[BQ + c] = in ? p.D[(s0 + i) * HQ + h] : 0.f;
-      }
-      __syncwarp();
-      {
-        const bool got = wait_bar(bar(S_FULL), t & 1, p.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      }
-      tc_fence_after();
-      // every query of the tile sees this key: no mask work in the loop
-      const bool full = key_ok && (i0 >= jj) && (i0 + BQ <= L) && (i0 + BQ - 1 - jj < win);
-#pragma unroll 1
-      for (int c = 0; c < BQ; c += 32) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_base + kColS + c, sv);
-        tmem_ld32(tmem + lane_base + kColDP + c, dv);
-        tmem_wait_ld();
-        uint32_t pp[16], dd[16];
-        auto group = [&](int g8, auto masked) {
-          float pe[8], de[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int q = c + g8 * 8 + e;
-            const float x = fmaf(__uint_as_float(sv[g8 * 8 + e]), p.scale_log2, rowv[q] - gs_j);
-            float pv;
-            if constexpr (decltype(masked)::value) {
-              const int i = i0 + q;
-              const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
-              pv = vis ? exp2f(x) : 0.f;
-            } else {
-              pv = exp2f(x);
-            }
-            pe[e] = pv;
-            de[e] = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
-          }
-          colsum += ((de[0] + de[1]) + (de[2] + de[3])) + ((de[4] + de[5]) + (de[6] + de[7]));
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            pp[g8 * 4 + e] = pack_bf16x2(pe[2 * e], pe[2 * e + 1]);
-            dd[g8 * 4 + e] = pack_bf16x2(de[2 * e], de[2 * e + 1]);
-          }
-        };
-        if (full) {
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) group(g8, std::false_type{});
-        } else {
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) group(g8, std::true_type{});
+    for (int t = 0; t < nT && ok; ++t) {
+      for (int hf = 0; hf < 2; ++hf) {
+        const int i0 = (I0 + t) * BQ + hf * 64;  // first query of this half
+        __syncwarp();
+        // per query: c_i = GS_i*log2e - lse_i*log2e (logit offset), D_i
+        for (int c = lane; c < 64; c += 32) {
+          const int i = i0 + c;
+          const bool in = i < L;
+          const float gsi = (in && p.GS) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+          rowv[c] = in ? gsi - p.lse[(s0 + i) * HQ + h] * kLog2e : 0.f;
+          rowv[BQ + c] = in ? p.D[(s0 + i) * HQ + h] : 0.f;
         }
-        // P^T, dS^T as bf16 pairs over the consumed S^T / dP^T columns
-        tmem_st16(tmem + lane_base + kColS + c / 2, pp);
-        tmem_st16(tmem + lane_base + kColDP + c / 2, dd);
+        __syncwarp();
+        {
+          const bool got = wait_bar(bar(SD_FULL + hf), t & 1, p.status, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        }
+        tc_fence_after();
+        // every query of the half sees this key: no mask work in the loop
+        const bool full = key_ok && (i0 >= jj) && (i0 + 64 <= L) && (i0 + 63 - jj < win);
+        const uint32_t scol = kColS + hf * 64, dcol = kColDP + hf * 64;
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tmem + lane_base + scol + c, sv);
+          tmem_ld32(tmem + lane_base + dcol + c, dv);
+          tmem_wait_ld();
+          uint32_t pp[16], dd[16];
+          auto group = [&](int g8, auto masked) {
+            float pe[8], de[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int q = c + g8 * 8 + e;
+              const float x =
+                  fmaf(__uint_as_float(sv[g8 * 8 + e]), p.scale_log2, rowv[q] - gs_j);
+              float pv;
+              if constexpr (decltype(masked)::value) {
+                const int i = i0 + q;
+                const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
+                pv = vis ? exp2f(x) : 0.f;
+              } else {
+                pv = exp2f(x);
+              }
+              pe[e] = pv;
+              de[e] = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
+            }
+            colsum += ((de[0] + de[1]) + (de[2] + de[3])) + ((de[4] + de[5]) + (de[6] + de[7]));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              pp[g8 * 4 + e] = pack_bf16x2(pe[2 * e], pe[2 * e + 1]);
+              dd[g8 * 4 + e] = pack_bf16x2(de[2 * e], de[2 * e + 1]);
+            }
+          };
+          if (full) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) group(g8, std::false_type{});
+          } else {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) group(g8, std::true_type{});
+          }
+          // P^T, dS^T as bf16 pairs over the consumed S^T / dP^T columns
+          tmem_st16(tmem + lane_base + scol + c / 2, pp);
+          tmem_st16(tmem + lane_base + dcol + c / 2, dd);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(P_FULL + hf));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(P_FULL));
     }
     // ---- dK, dV epilogue for this key block
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(MM_DONE), 0, p.status, abort_flag));
