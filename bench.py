@@ -207,8 +207,9 @@ def bench_train(args, world, rank, peaks):
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     # launches of this library inside one step: prefix scan 1; forward:
     # operand preparation 1 + tcgen05 forward 1; backward: operand preparation
-    # 1, D/sink pre-pass 1, tcgen05 backward 1, finalize 1, reverse scan 1
-    launches_per_step = 8
+    # 1, D/sink pre-pass 1, tcgen05 key-block (dK, dV) 1, tcgen05 query-block
+    # (dq) 1, finalize 1, reverse scan 1
+    launches_per_step = 9
     res = dict(ms=ms_max, value=world * step_flops / (ms_max * 1e-3) / 1e12,
                fwd_ms=fwd_ms, bwd_ms=bwd_ms,
                fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,

@@ -1,5 +1,6 @@
 // wall_attn_bwd_sm100.cu -- tensor-core (tcgen05 + TMEM + TMA) Wall
-// Attention backward for bf16 with K == V in {64, 128}.
+// Attention backward for bf16 with K == V in {64, 128}: the key-block kernel
+// (dK, dV) plus the D / sink pre-pass and the finalize kernel.
 //
 // Gradients of the anchored form used by the forward (Tilde blog "Wall
 // Attention", fast training sections 1 and 2).  For a 128-row query tile I
@@ -17,18 +18,25 @@
 // reverse scan.  The row part of the scalar-gate gradient is analytic,
 // sum_j dS_ij = D_i * p_sink,i, and the column part is summed per key thread.
 //
-// Operands that the tensor core would otherwise read twice from shared memory
-// (P^T, dS^T) are written back into TMEM as bf16 pairs over the S^T / dP^T
-// columns they came from and fed as TMEM A operands.  All MMAs are M = 128,
-// N = 128.
+// Shared memory is the scarce resource on sm_100: an M = N = 128 SS MMA
+// already reads 128 B/clk.  So the per-tile factor d is applied while the
+// query tile travels from global memory to shared memory (registers in
+// between, one pass of stores), P^T and dS^T go back into TMEM as bf16 pairs
+// and are read from there by the dV / dK MMAs, and S^T, dP^T are single
+// M = N = 128 MMAs.
 //
-// CTA = one 128-row key block of one (sequence, head), 10 warps:
-//   warp 0      TMA: Kh_J, V_J once; Qh_I (2 stages) and dO_I (1 stage, freed
-//               by the first MMA that reads it last) per tile
-//   warp 1      TMEM owner and MMA issuer
-//   warps 2-5   Qt_I = Qh_I (.) d in shared memory
-//   warps 6-9   one thread per key: P, dS; P^T, dS^T -> TMEM; column sums;
-//               dK, dV epilogue at the end
+// CTA = one 128-row key block of one (sequence, head), 12 warps (3 per SM
+// sub-partition, 168 registers each):
+//   warp 0      TMA: Kh_J, V_J once; dO_I per tile (2 stages)
+//   warp 1      TMEM owner and MMA issuer.  Order per tile t:
+//               dV(t), S(t+1), dK(t), dP(t+1), so that the tensor core works
+//               on the next tile while the softmax computes dS(t)
+//   warps 2-3   Qt_I = Qh_I (.) d into shared memory (2 stages); the whole
+//               next tile is loaded into registers while the MMAs read the
+//               current one; per-query terms (lse, D, gate) of the tile
+//   warps 4-11  P, dS: one thread per (key, 64-query half of the tile); the
+//               two warps of a TMEM lane quarter take the two halves.  dK, dV
+//               epilogue at the end
 #include <cuda.h>
 
 #include <type_traits>
@@ -44,17 +52,18 @@ using namespace sm100;
 
 constexpr int BQ = 128;  // query rows per tile
 constexpr int BK = 128;  // key rows per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 
 struct BwdTcParams {
-  const float* anchors;  // [nblk128, HQ, K]
-  const float* P;        // [rows, HQ, K]
-  const float* lse;      // [rows, HQ]
-  const float* D;        // [rows, HQ]
-  const float* GS;       // [rows, HQ] or nullptr
-  float* dkh32;          // [rows, HQ, K]
-  float* dvh32;          // [rows, HQ, V]
-  float* dgs_col;        // [rows, HQ] or nullptr
+  const __nv_bfloat16* qh;  // [rows, HQ, K] anchored queries
+  const float* anchors;     // [nblk128, HQ, K]
+  const float* P;           // [rows, HQ, K]
+  const float* lse;         // [rows, HQ]
+  const float* D;           // [rows, HQ]
+  const float* GS;          // [rows, HQ] or nullptr
+  float* dkh32;             // [rows, HQ, K]
+  float* dvh32;             // [rows, HQ, V]
+  float* dgs_col;           // [rows, HQ] or nullptr
   Seqs seqs;
   int HQ, H;
   float scale, scale_log2;
@@ -69,13 +78,11 @@ struct BSmem {
   static constexpr int kQ = BQ * KD * 2;    // query or dO tile
   static constexpr int oK = 0;
   static constexpr int oV = oK + kKV;
-  static constexpr int oQ = oV + kKV;       // 2 stages
-  static constexpr int oO = oQ + 2 * kQ;    // 2 stages
-  static constexpr int oDw = oO + 2 * kQ;          // float[4 warps][KD]
-  static constexpr int oRow = oDw + 4 * KD * 4;    // float[4 warps][2][BQ]
-  static constexpr int oRI = oRow + 4 * 2 * BQ * 4;  // float[2 stages][KD]
-  static constexpr int oRJ = oRI + 2 * KD * 4;       // float[KD]
-  static constexpr int oBar = oRJ + KD * 4;
+  static constexpr int oQ = oV + kKV;       // 2 stages of Qt
+  static constexpr int oO = oQ + 2 * kQ;    // 2 stages of dO
+  static constexpr int oRow = oO + 2 * kQ;  // float[2 stages][2][BQ]: c_i, D_i
+  static constexpr int oCol = oRow + 2 * 2 * BQ * 4;  // float[BK]: column sums of the second half
+  static constexpr int oBar = oCol + BK * 4;
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
@@ -84,21 +91,22 @@ struct BSmem {
 
 enum BBar {
   KV_FULL = 0,
-  Q_FULL = 1,     // +stage
-  O_FULL = 3,     // +stage
-  Q_READY = 5,    // +stage
-  QO_EMPTY = 7,   // +stage
-  SD_FULL = 9,    // +half
-  P_FULL = 11,    // +half
+  Q_READY = 1,   // +stage, 2 producer warps
+  Q_EMPTY = 3,   // +stage, tcgen05.commit after dK(t)
+  O_FULL = 5,    // +stage, TMA
+  O_EMPTY = 7,   // +stage, tcgen05.commit after dV(t)
+  S_FULL = 9,
+  DP_FULL = 10,
+  P_READY = 11,  // 8 softmax warps
+  DS_READY = 12, // 8 softmax warps
   MM_DONE = 13,
   MMA_DONE = 14,
+  COL_READY = 15,  // 4 warps of the second half: column sums in shared memory
 };
 
-// TMEM columns (lanes = keys): S^T of the two 64-query halves [0,64),
-// [64,128); dP^T halves [128,192), [192,256); the softmax writes P^T (dS^T)
-// bf16 pairs over the first 32 columns of each S^T (dP^T) half; dV
-// [256,384), dK [384,512).  While one half is in the softmax, the tensor core
-// works on the other.
+// TMEM columns (lanes = keys): S^T [0,128), dP^T [128,256), dV [256,384),
+// dK [384,512).  The softmax half h (queries 64h..64h+63) writes its P^T
+// (dS^T) bf16 pairs over the first 32 of its own 64 S^T (dP^T) columns.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
@@ -122,18 +130,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int KD>
+// 8 bf16 scaled by 8 per-channel factors, rounded back to bf16
+__device__ __forceinline__ uint4 scale8(uint4 u, const float (&d)[8]) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+    w[e] = pack_bf16x2(f.x * d[2 * e], f.y * d[2 * e + 1]);
+  }
+  return u;
+}
+
+template <int KD, bool kGS>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  BwdTcParams p) {
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_o, BwdTcParams p) {
   using Lay = BSmem<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* sDw = reinterpret_cast<float*>(smem + Lay::oDw);
   float* sRow = reinterpret_cast<float*>(smem + Lay::oRow);
+  float* sCol = reinterpret_cast<float*>(smem + Lay::oCol);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
@@ -159,25 +177,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(KV_FULL), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(Q_FULL + s), 1);
+      mbar_init(bar(Q_READY + s), 2);
+      mbar_init(bar(Q_EMPTY + s), 1);
       mbar_init(bar(O_FULL + s), 1);
-      mbar_init(bar(Q_READY + s), 4);
-      mbar_init(bar(QO_EMPTY + s), 1);
-      mbar_init(bar(SD_FULL + s), 1);
-      mbar_init(bar(P_FULL + s), 4);
+      mbar_init(bar(O_EMPTY + s), 1);
     }
+    mbar_init(bar(S_FULL), 1);
+    mbar_init(bar(DP_FULL), 1);
+    mbar_init(bar(P_READY), 8);
+    mbar_init(bar(DS_READY), 8);
     mbar_init(bar(MM_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
+    mbar_init(bar(COL_READY), 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
-  }
-  {
-    float* rjs = reinterpret_cast<float*>(smem + Lay::oRJ);
-    for (int n = threadIdx.x; n < K; n += kThreads) rjs[n] = anc[(long)blk * HQ * K + n];
   }
   tc_fence_before();
   __syncthreads();
@@ -187,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
@@ -201,236 +217,248 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t & 1;
-        const int row = (int)(s0 + (long)(I0 + t) * BQ);
-        if (t >= 2 && !wait_bar(bar(QO_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+        if (t >= 2 && !wait_bar(bar(O_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
         mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
-        for (int b = 0; b < K / 64; ++b) {
-          tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
-                      b * 64, h, row);
+        const int row = (int)(s0 + (long)(I0 + t) * BQ);
+        for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oO + st * Lay::kQ + b * (BQ * 128), &tm_o, bar(O_FULL + st),
                       b * 64, h, row);
-        }
-        bulk_load(sbase + Lay::oRI + st * K * 4, anc + (long)(I0 + t) * HQ * K, K * 4,
-                  bar(Q_FULL + st));
         issued = t + 1;
       }
-      for (int t = max(0, issued - 2); t < issued; ++t) {
-        mbar_wait(bar(Q_FULL + (t & 1)), (t >> 1) & 1, p.status);
+      // no copy may still be in flight when the CTA exits
+      for (int t = max(0, issued - 2); t < issued; ++t)
         mbar_wait(bar(O_FULL + (t & 1)), (t >> 1) & 1, p.status);
-      }
       mbar_wait(bar(KV_FULL), 0, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
-      const uint32_t id_sd = idesc_bf16(128, 64, false, false);  // S^T, dP^T halves
-      const uint32_t id_acc = idesc_bf16(128, KD, false, true);  // dV, dK (A from TMEM)
-      bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
-      // S^T and dP^T of one 64-query half: M = 128 keys, N = 64, K = channels
-      auto issue_sd = [&](int t, int hf) {
-        const int st = t & 1;
-        const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ + hf * 64 * 128;
-        const uint32_t oa = sbase + Lay::oO + st * Lay::kQ + hf * 64 * 128;
+      const uint32_t id_sd = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+      const uint32_t id_acc = idesc_bf16(128, KD, false, true);   // dV, dK (A from TMEM)
+      // S^T (dP^T) of the whole tile: M = 128 keys, N = 128 queries, K = channels
+      auto issue_sd = [&](uint32_t a_off, uint32_t b_off, uint32_t col) {
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t offA = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
           const uint32_t offB = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_bf16_ss(tmem + kColS + hf * 64, sdesc_sw128(sbase + Lay::oK + offA, 16, 1024),
-                       sdesc_sw128(qa + offB, 16, 1024), id_sd, kk > 0);
-          umma_bf16_ss(tmem + kColDP + hf * 64, sdesc_sw128(sbase + Lay::oV + offA, 16, 1024),
-                       sdesc_sw128(oa + offB, 16, 1024), id_sd, kk > 0);
+          umma_bf16_ss(tmem + col, sdesc_sw128(sbase + a_off + offA, 16, 1024),
+                       sdesc_sw128(sbase + b_off + offB, 16, 1024), id_sd, kk > 0);
         }
-        umma_commit(bar(SD_FULL + hf));
       };
-      // dV += P^T dO and dK += dS^T Qt over one half: A from TMEM (8 columns
-      // per 16 queries), B = dO / Qt rows of the half, MN-major
-      auto issue_acc = [&](int t, int hf) {
-        const int st = t & 1;
-        const uint32_t qa = sbase + Lay::oQ + st * Lay::kQ + hf * 64 * 128;
-        const uint32_t oa = sbase + Lay::oO + st * Lay::kQ + hf * 64 * 128;
+      // dV += P^T dO (dK += dS^T Qt): A from TMEM, 8 columns per 16 queries,
+      // the two 64-query halves 64 columns apart; B = rows of the tile, MN-major
+      auto issue_acc = [&](uint32_t a_col, uint32_t b_off, uint32_t d_col, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < 64 / 16; ++kk) {
-          const uint32_t acc = (t > 0 || hf > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16_ts(tmem + kColDV, tmem + kColS + hf * 64 + kk * 8,
-                       sdesc_sw128(oa + kk * 16 * 128, BQ * 128, 1024), id_acc, acc);
-          umma_bf16_ts(tmem + kColDK, tmem + kColDP + hf * 64 + kk * 8,
-                       sdesc_sw128(qa + kk * 16 * 128, BQ * 128, 1024), id_acc, acc);
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          umma_bf16_ts(tmem + d_col, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
+                       sdesc_sw128(sbase + b_off + kk * 16 * 128, BQ * 128, 1024), id_acc,
+                       (first && kk == 0) ? 0u : 1u);
         }
       };
-      auto tile_ready = [&](int t) -> bool {
-        const int st = t & 1;
-        if (!wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag)) return false;
-        if (!wait_bar(bar(O_FULL + st), (t >> 1) & 1, p.status, abort_flag)) return false;
-        tc_fence_after();
-        return true;
-      };
-      if (ok) ok = tile_ready(0);
+      auto q_off = [&](int t) { return (uint32_t)(Lay::oQ + (t & 1) * Lay::kQ); };
+      auto o_off = [&](int t) { return (uint32_t)(Lay::oO + (t & 1) * Lay::kQ); };
+      bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
+      if (ok) ok = wait_bar(bar(Q_READY), 0, p.status, abort_flag);
+      if (ok) ok = wait_bar(bar(O_FULL), 0, p.status, abort_flag);
       if (ok) {
-        issue_sd(0, 0);
-        issue_sd(0, 1);
+        tc_fence_after();
+        issue_sd(Lay::oK, q_off(0), kColS);
+        umma_commit(bar(S_FULL));
+        issue_sd(Lay::oV, o_off(0), kColDP);
+        umma_commit(bar(DP_FULL));
       }
       for (int t = 0; ok && t < nT; ++t) {
         const int st = t & 1;
-        if (!wait_bar(bar(P_FULL + 0), t & 1, p.status, abort_flag)) break;
-        tc_fence_after();
-        issue_acc(t, 0);
         const bool next = t + 1 < nT;
-        if (next) {
-          if (!tile_ready(t + 1)) break;
-          issue_sd(t + 1, 0);  // overwrites half a: in order after its dV/dK
-        }
-        if (!wait_bar(bar(P_FULL + 1), t & 1, p.status, abort_flag)) break;
+        if (!wait_bar(bar(P_READY), t & 1, p.status, abort_flag)) break;
         tc_fence_after();
-        issue_acc(t, 1);
-        umma_commit(bar(QO_EMPTY + st));
-        if (next) issue_sd(t + 1, 1);
+        issue_acc(kColS, o_off(t), kColDV, t == 0);
+        umma_commit(bar(O_EMPTY + st));
+        if (next) {
+          if (!wait_bar(bar(Q_READY + (st ^ 1)), ((t + 1) >> 1) & 1, p.status, abort_flag)) break;
+          tc_fence_after();
+          issue_sd(Lay::oK, q_off(t + 1), kColS);  // in order after dV(t) read P^T
+          umma_commit(bar(S_FULL));
+        }
+        if (!wait_bar(bar(DS_READY), t & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        issue_acc(kColDP, q_off(t), kColDK, t == 0);
+        umma_commit(bar(Q_EMPTY + st));
+        if (next) {
+          if (!wait_bar(bar(O_FULL + (st ^ 1)), ((t + 1) >> 1) & 1, p.status, abort_flag)) break;
+          tc_fence_after();
+          issue_sd(Lay::oV, o_off(t + 1), kColDP);  // in order after dK(t) read dS^T
+          umma_commit(bar(DP_FULL));
+        }
       }
       umma_commit(bar(MM_DONE));
       umma_commit(bar(MMA_DONE));
       mbar_wait(bar(MMA_DONE), 0, p.status);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ Qt rescale
-    const int wt = threadIdx.x - 64;
-    const int wq = warp - 2;
-    const float* rjs = reinterpret_cast<const float*>(smem + Lay::oRJ);
-    float* d = sDw + wq * KD;
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ Qt producer
+    constexpr int kChunks = KD / 8;          // 16-byte chunks per row
+    constexpr int kRowStep = 64 / kChunks;   // rows covered by one pass of 64 threads
+    constexpr int kRows = BQ / kRowStep;     // rows per thread
+    const int tid = threadIdx.x - 64;
+    const int ch = tid % kChunks;
+    const int rs = tid / kChunks;
+    const float* rj = anc + (long)blk * HQ * K + ch * 8;  // R_J of this thread's channels
+    const __nv_bfloat16* qsrc = p.qh + (long)h * K + ch * 8;
+    const long rstride = (long)HQ * K;
+    uint4 u[kRows];
+    float ri[8], ci[2], di[2];
+    auto prefetch = [&](int t) {
+      const int i0 = (I0 + t) * BQ;
+#pragma unroll
+      for (int m = 0; m < kRows; ++m) {
+        const int i = i0 + rs + m * kRowStep;
+        u[m] = i < L ? __ldg(reinterpret_cast<const uint4*>(qsrc + (s0 + i) * rstride))
+                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+      const float* a = anc + (long)(I0 + t) * HQ * K + ch * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ri[e] = __ldg(a + e);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int i = i0 + tid + 64 * x;
+        const long e = (s0 + i) * HQ + h;
+        ci[x] = i < L ? ((kGS ? __ldg(p.GS + e) : 0.f) - __ldg(p.lse + e)) * kLog2e : 0.f;
+        di[x] = i < L ? __ldg(p.D + e) : 0.f;
+      }
+    };
+    prefetch(0);
     for (int t = 0; t < nT; ++t) {
       const int st = t & 1;
-      const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4);
-      __syncwarp();
-      for (int c = lane; c < K; c += 32) d[c] = exp2f(ri[c] - rjs[c]);
-      __syncwarp();
-      uint8_t* qt = smem + Lay::oQ + st * Lay::kQ;
-      constexpr int kPer = (KD / 64) * BQ * 8 / 128;  // chunks per thread
-      constexpr int kBatch = 4;
-#pragma unroll 1
-      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
-        uint4 u[kBatch];
-        float dd[kBatch][8];
-        uint4* ptr[kBatch];
+      if (t >= 2) {
+        const bool got = wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) break;
+      }
+      float d[8];
 #pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          const int c = wt + (b0 + x) * 128;
-          const int box = c / (BQ * 8);
-          const int row = (c / 8) % BQ;
-          const int pch = c % 8;
-          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-          ptr[x] = reinterpret_cast<uint4*>(qt + box * (BQ * 128) + row * 128 + pch * 16);
-          u[x] = *ptr[x];
-          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
-          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
-        }
+      for (int e = 0; e < 8; ++e) d[e] = exp2f(ri[e] - __ldg(rj + e));
+      uint8_t* qt = smem + Lay::oQ + st * Lay::kQ + (ch / 8) * (BQ * 128);
 #pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+      for (int m = 0; m < kRows; ++m) {
+        const int r = rs + m * kRowStep;
+        *reinterpret_cast<uint4*>(qt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = scale8(u[m], d);
+      }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
-          }
-          *ptr[x] = u[x];
-        }
+      for (int x = 0; x < 2; ++x) {
+        sRow[st * 2 * BQ + tid + 64 * x] = ci[x];
+        sRow[st * 2 * BQ + BQ + tid + 64 * x] = di[x];
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(Q_READY + st));
+      if (t + 1 < nT) prefetch(t + 1);
     }
   } else {
-    // ------------------------------------------------------------ P, dS per key (warps 6-9)
+    // ------------------------------------------------------------ P, dS (warps 4-11)
     const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;    // queries 64*half .. 64*half+63 of each tile
     const int r = quarter * 32 + lane;   // key row within the block
     const int jj = j0 + r;               // key index within the sequence
     const bool key_ok = r < nj;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const float gs_j = (p.GS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
-    float* rowv = sRow + (warp - 6) * 2 * BQ;  // this warp's copy of the tile's query terms
+    const float gs_j = (kGS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
+    const uint32_t scol = kColS + half * 64, dcol = kColDP + half * 64;
     float colsum = 0.f;
     bool ok = true;
     for (int t = 0; t < nT && ok; ++t) {
-      for (int hf = 0; hf < 2; ++hf) {
-        const int i0 = (I0 + t) * BQ + hf * 64;  // first query of this half
-        __syncwarp();
-        // per query: c_i = GS_i*log2e - lse_i*log2e (logit offset), D_i
-        for (int c = lane; c < 64; c += 32) {
-          const int i = i0 + c;
-          const bool in = i < L;
-          const float gsi = (in && p.GS) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
-          rowv[c] = in ? gsi - p.lse[(s0 + i) * HQ + h] * kLog2e : 0.f;
-          rowv[BQ + c] = in ? p.D[(s0 + i) * HQ + h] : 0.f;
-        }
-        __syncwarp();
-        {
-          const bool got = wait_bar(bar(SD_FULL + hf), t & 1, p.status, abort_flag);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        }
-        tc_fence_after();
-        // every query of the half sees this key: no mask work in the loop
-        const bool full = key_ok && (i0 >= jj) && (i0 + 64 <= L) && (i0 + 63 - jj < win);
-        const uint32_t scol = kColS + hf * 64, dcol = kColDP + hf * 64;
-#pragma unroll 1
-        for (int c = 0; c < 64; c += 32) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32(tmem + lane_base + scol + c, sv);
-          tmem_ld32(tmem + lane_base + dcol + c, dv);
-          tmem_wait_ld();
-          uint32_t pp[16], dd[16];
-          auto group = [&](int g8, auto masked) {
-            float pe[8], de[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int q = c + g8 * 8 + e;
-              const float x =
-                  fmaf(__uint_as_float(sv[g8 * 8 + e]), p.scale_log2, rowv[q] - gs_j);
-              float pv;
-              if constexpr (decltype(masked)::value) {
-                const int i = i0 + q;
-                const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
-                pv = vis ? exp2f(x) : 0.f;
-              } else {
-                pv = exp2f(x);
-              }
-              pe[e] = pv;
-              de[e] = pv * (__uint_as_float(dv[g8 * 8 + e]) - rowv[BQ + q]);
-            }
-            colsum += ((de[0] + de[1]) + (de[2] + de[3])) + ((de[4] + de[5]) + (de[6] + de[7]));
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              pp[g8 * 4 + e] = pack_bf16x2(pe[2 * e], pe[2 * e + 1]);
-              dd[g8 * 4 + e] = pack_bf16x2(de[2 * e], de[2 * e + 1]);
-            }
-          };
-          if (full) {
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) group(g8, std::false_type{});
-          } else {
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) group(g8, std::true_type{});
-          }
-          // P^T, dS^T as bf16 pairs over the consumed S^T / dP^T columns
-          tmem_st16(tmem + lane_base + scol + c / 2, pp);
-          tmem_st16(tmem + lane_base + dcol + c / 2, dd);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(P_FULL + hf));
+      const int st = t & 1;
+      const int i0 = (I0 + t) * BQ + half * 64;  // first query of this half
+      {
+        bool got = wait_bar(bar(S_FULL), t & 1, p.status, abort_flag);
+        // acquire the producers' per-query terms (that phase has completed)
+        got = got && wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
+      tc_fence_after();
+      const float* cv = sRow + st * 2 * BQ + half * 64;
+      const float* dvv = cv + BQ;
+      // every query of the half sees every key of the warp: no mask work in the
+      // loop.  Warp-uniform, since the branch holds the warp-wide TMEM loads
+      const bool full = __all_sync(
+          0xffffffffu, key_ok && (i0 >= jj) && (i0 + 64 <= L) && (i0 + 63 - jj < win));
+      float pv[64];
+      auto p_part = [&](auto masked) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t sv[32];
+          tmem_ld32(tmem + lane_base + scol + c, sv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(cv + c + e);
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const float arg = fmaf(__uint_as_float(sv[e + x]), p.scale_log2,
+                                     kGS ? cc[x] - gs_j : cc[x]);
+              if constexpr (decltype(masked)::value) {
+                const int i = i0 + c + e + x;
+                const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
+                pv[c + e + x] = vis ? exp2f(arg) : 0.f;
+              } else {
+                pv[c + e + x] = exp2f(arg);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[c + 2 * e], pv[c + 2 * e + 1]);
+          tmem_st16(tmem + lane_base + scol + c / 2, pk);
+        }
+      };
+      if (full)
+        p_part(std::false_type{});
+      else
+        p_part(std::true_type{});
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(P_READY));
+      {
+        const bool got = wait_bar(bar(DP_FULL), t & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 64; c += 32) {
+        uint32_t dv[32];
+        tmem_ld32(tmem + lane_base + dcol + c, dv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dvv + c + e);
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float ds = pv[c + e + x] * (__uint_as_float(dv[e + x]) - dd[x]);
+            if (kGS) colsum += ds;
+            pv[c + e + x] = ds;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[c + 2 * e], pv[c + 2 * e + 1]);
+        tmem_st16(tmem + lane_base + dcol + c / 2, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(DS_READY));
     }
-    // ---- dK, dV epilogue for this key block
+    // ---- dK, dV epilogue for this key block: each half takes half the channels
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(MM_DONE), 0, p.status, abort_flag));
     if (ok) {
       tc_fence_after();
       const long krow = (s0 + jj) * HQ + h;
 #pragma unroll 1
-      for (int c = 0; c < KD; c += 32) {
+      for (int c = half * (KD / 2); c < (half + 1) * (KD / 2); c += 32) {
         uint32_t kv[32], vv[32];
         tmem_ld32(tmem + lane_base + kColDK + c, kv);
         tmem_ld32(tmem + lane_base + kColDV + c, vv);
@@ -456,8 +484,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // the logit carries -GS_j for key j
-      if (key_ok && p.dgs_col) p.dgs_col[krow] = -colsum;
+    }
+    if (kGS) {
+      // column sums of the two halves meet in shared memory; the logit
+      // carries -GS_j for key j
+      if (half == 1) {
+        sCol[r] = colsum;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(COL_READY));
+      } else {
+        const bool got = wait_bar(bar(COL_READY), 0, p.status, abort_flag);
+        if (ok && got && key_ok && p.dgs_col) p.dgs_col[(s0 + jj) * HQ + h] = -(colsum + sCol[r]);
+      }
     }
   }
   tc_fence_before();
@@ -576,23 +614,23 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict
   }
 }
 
-template <int KD>
+template <int KD, bool kGS>
 int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                   cudaStream_t stream) {
-  CUtensorMap tq, tk, tv, to;
-  if (!make_tile_map(&tq, ws.qh, pb.rows, pb.HQ, KD, BQ) ||
-      !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BK) ||
+  CUtensorMap tk, tv, to;
+  if (!make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BK) ||
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BK) ||
       !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BQ))
     return WALL_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(bwd_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(bwd_tc_kernel<KD, kGS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              BSmem<KD>::kAlloc) != cudaSuccess)
       return WALL_ERR_CUDA;
     attr = true;
   }
   BwdTcParams p;
+  p.qh = static_cast<const __nv_bfloat16*>(ws.qh);
   p.anchors = ws.anchors;
   p.P = a.P;
   p.lse = a.lse;
@@ -610,8 +648,15 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.n_blocks = ws.n_blocks128;
   p.status = status;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  bwd_tc_kernel<KD><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tq, tk, tv, to, p);
+  bwd_tc_kernel<KD, kGS><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+template <int KD>
+int launch_bwd_tc_gs(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
+                     cudaStream_t stream) {
+  return a.GS ? launch_bwd_tc<KD, true>(pb, a, ws, status, stream)
+              : launch_bwd_tc<KD, false>(pb, a, ws, status, stream);
 }
 
 }  // namespace
@@ -629,8 +674,8 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void
         a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr, a.dsink);
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
   }
-  rc = pb.K == 128 ? launch_bwd_tc<128>(pb, a, ws, status, stream)
-                   : launch_bwd_tc<64>(pb, a, ws, status, stream);
+  rc = pb.K == 128 ? launch_bwd_tc_gs<128>(pb, a, ws, status, stream)
+                   : launch_bwd_tc_gs<64>(pb, a, ws, status, stream);
   if (rc) return rc;
   rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
   if (rc) return rc;
