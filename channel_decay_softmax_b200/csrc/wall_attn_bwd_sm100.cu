@@ -19,21 +19,20 @@
 // sum_j dS_ij = D_i * p_sink,i, and the column part is summed per key thread.
 //
 // Shared memory is the scarce resource on sm_100: an M = N = 128 SS MMA
-// already reads 128 B/clk.  So the per-tile factor d is applied while the
-// query tile travels from global memory to shared memory (registers in
-// between, one pass of stores), P^T and dS^T go back into TMEM as bf16 pairs
-// and are read from there by the dV / dK MMAs, and S^T, dP^T are single
-// M = N = 128 MMAs.
+// already reads 128 B/clk.  So P^T and dS^T go back into TMEM as bf16 pairs
+// and are read from there by the dV / dK MMAs, S^T and dP^T are single
+// M = N = 128 MMAs, and the per-tile factor d is applied in place, one
+// 16-byte chunk per load and store, to the query tile TMA brought in.
 //
 // CTA = one 128-row key block of one (sequence, head), 12 warps (3 per SM
 // sub-partition, 168 registers each):
-//   warp 0      TMA: Kh_J, V_J once; dO_I per tile (2 stages)
+//   warp 0      TMA: Kh_J, V_J once; Qh_I with its anchors R_I, and dO_I per
+//               tile (2 stages each)
 //   warp 1      TMEM owner and MMA issuer.  Order per tile t:
 //               dV(t), S(t+1), dK(t), dP(t+1), so that the tensor core works
 //               on the next tile while the softmax computes dS(t)
-//   warps 2-3   Qt_I = Qh_I (.) d into shared memory (2 stages); the whole
-//               next tile is loaded into registers while the MMAs read the
-//               current one; per-query terms (lse, D, gate) of the tile
+//   warps 2-3   Qt_I = Qh_I (.) d in place; per-query terms (lse, D, gate)
+//               of the tile, loaded two tiles ahead
 //   warps 4-11  P, dS: one thread per (key, 64-query half of the tile); the
 //               two warps of a TMEM lane quarter take the two halves.  dK, dV
 //               epilogue at the end
@@ -82,8 +81,10 @@ struct BSmem {
   static constexpr int oO = oQ + 2 * kQ;    // 2 stages of dO
   static constexpr int oRow = oO + 2 * kQ;  // float[2 stages][2][BQ]: c_i, D_i
   static constexpr int oCol = oRow + 2 * 2 * BQ * 4;  // float[BK]: column sums of the second half
-  static constexpr int oBar = oCol + BK * 4;
-  static constexpr int kBars = 16;
+  static constexpr int oRJ = oCol + BK * 4;           // float[KD]: R_J
+  static constexpr int oRI = oRJ + KD * 4;            // float[2 stages][KD]: R_I
+  static constexpr int oBar = oRI + 2 * KD * 4;
+  static constexpr int kBars = 18;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -102,6 +103,7 @@ enum BBar {
   MM_DONE = 13,
   MMA_DONE = 14,
   COL_READY = 15,  // 4 warps of the second half: column sums in shared memory
+  Q_FULL = 16,     // +stage, TMA
 };
 
 // TMEM columns (lanes = keys): S^T [0,128), dP^T [128,256), dV [256,384),
@@ -130,21 +132,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// 8 bf16 scaled by 8 per-channel factors, rounded back to bf16
-__device__ __forceinline__ uint4 scale8(uint4 u, const float (&d)[8]) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+// 2^k as bf16 bits for an integer k (the anchors are integers): exact in
+// the normal range, 0 below it (a factor under 2^-126 scales an operand that
+// decays to nothing) and +inf above it, as the fp32 product would overflow.
+__device__ __forceinline__ uint32_t pow2_bf16(float k) {
+  const int e = (int)k;
+  return e < -126 ? 0u : e > 127 ? 0x7F80u : uint32_t(e + 127) << 7;
+}
+
+// 8 bf16 times 8 per-channel powers of two (bf16x2 pairs): exact
+__device__ __forceinline__ uint4 scale8(uint4 u, const __nv_bfloat162 (&d)[4]) {
+  __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-    w[e] = pack_bf16x2(f.x * d[2 * e], f.y * d[2 * e + 1]);
-  }
+  for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
   return u;
 }
 
 template <int KD, bool kGS>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const __grid_constant__ CUtensorMap tm_o, BwdTcParams p) {
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  BwdTcParams p) {
   using Lay = BSmem<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -178,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(KV_FULL), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Q_READY + s), 2);
+      mbar_init(bar(Q_FULL + s), 1);
       mbar_init(bar(Q_EMPTY + s), 1);
       mbar_init(bar(O_FULL + s), 1);
       mbar_init(bar(O_EMPTY + s), 1);
@@ -204,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
@@ -214,21 +224,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + Lay::oV + b * (BK * 128), &tm_v, bar(KV_FULL), b * 64, kh,
                     (int)(s0 + j0));
       }
-      int issued = 0;
+      int issued_o = 0, issued_q = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t & 1;
+        const int row = (int)(s0 + (long)(I0 + t) * BQ);
+        // dO(t - 2) is released by dV(t - 2), before Qt(t - 2) by dK(t - 2)
         if (t >= 2 && !wait_bar(bar(O_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
           break;
         mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
-        const int row = (int)(s0 + (long)(I0 + t) * BQ);
         for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oO + st * Lay::kQ + b * (BQ * 128), &tm_o, bar(O_FULL + st),
                       b * 64, h, row);
-        issued = t + 1;
+        issued_o = t + 1;
+        if (t >= 2 && !wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
+                      b * 64, h, row);
+        bulk_load(sbase + Lay::oRI + st * K * 4, anc + (long)(I0 + t) * HQ * K, K * 4,
+                  bar(Q_FULL + st));
+        issued_q = t + 1;
       }
       // no copy may still be in flight when the CTA exits
-      for (int t = max(0, issued - 2); t < issued; ++t)
+      for (int t = max(0, issued_o - 2); t < issued_o; ++t)
         mbar_wait(bar(O_FULL + (t & 1)), (t >> 1) & 1, p.status);
+      for (int t = max(0, issued_q - 2); t < issued_q; ++t)
+        mbar_wait(bar(Q_FULL + (t & 1)), (t >> 1) & 1, p.status);
       mbar_wait(bar(KV_FULL), 0, p.status);
     }
   } else if (warp == 1) {
@@ -275,16 +297,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_acc(kColS, o_off(t), kColDV, t == 0);
         umma_commit(bar(O_EMPTY + st));
-        if (next) {
-          if (!wait_bar(bar(Q_READY + (st ^ 1)), ((t + 1) >> 1) & 1, p.status, abort_flag)) break;
+        // S(t+1) may go before dK(t) (the tensor core then works while the
+        // softmax finishes dS(t)), but only if its query tile is ready:
+        // dK(t) frees the stage the tile after next is written to
+        const uint32_t q_next = bar(Q_READY + (st ^ 1));
+        const uint32_t q_par = ((t + 1) >> 1) & 1;
+        bool s_done = false;
+        if (next && mbar_try_wait(q_next, q_par)) {
           tc_fence_after();
           issue_sd(Lay::oK, q_off(t + 1), kColS);  // in order after dV(t) read P^T
           umma_commit(bar(S_FULL));
+          s_done = true;
         }
         if (!wait_bar(bar(DS_READY), t & 1, p.status, abort_flag)) break;
         tc_fence_after();
         issue_acc(kColDP, q_off(t), kColDK, t == 0);
         umma_commit(bar(Q_EMPTY + st));
+        if (next && !s_done) {
+          if (!wait_bar(q_next, q_par, p.status, abort_flag)) break;
+          tc_fence_after();
+          issue_sd(Lay::oK, q_off(t + 1), kColS);
+          umma_commit(bar(S_FULL));
+        }
         if (next) {
           if (!wait_bar(bar(O_FULL + (st ^ 1)), ((t + 1) >> 1) & 1, p.status, abort_flag)) break;
           tc_fence_after();
@@ -304,55 +338,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x - 64;
     const int ch = tid % kChunks;
     const int rs = tid / kChunks;
-    const float* rj = anc + (long)blk * HQ * K + ch * 8;  // R_J of this thread's channels
-    const __nv_bfloat16* qsrc = p.qh + (long)h * K + ch * 8;
-    const long rstride = (long)HQ * K;
-    uint4 u[kRows];
-    float ri[8], ci[2], di[2];
-    auto prefetch = [&](int t) {
-      const int i0 = (I0 + t) * BQ;
+    float rj[8];
 #pragma unroll
-      for (int m = 0; m < kRows; ++m) {
-        const int i = i0 + rs + m * kRowStep;
-        u[m] = i < L ? __ldg(reinterpret_cast<const uint4*>(qsrc + (s0 + i) * rstride))
-                     : make_uint4(0u, 0u, 0u, 0u);
-      }
-      const float* a = anc + (long)(I0 + t) * HQ * K + ch * 8;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ri[e] = __ldg(a + e);
+    for (int e = 0; e < 8; ++e) rj[e] = __ldg(anc + (long)blk * HQ * K + ch * 8 + e);
+    // per-query terms two tiles ahead: plain loads take a few microseconds
+    // while the tensor core streams
+    float cc[2], dc[2], cn[2], dn[2];  // tiles t and t + 1
+    auto rows_of = [&](int t, float (&c)[2], float (&dd)[2]) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const int i = i0 + tid + 64 * x;
+        const int i = (I0 + t) * BQ + tid + 64 * x;
         const long e = (s0 + i) * HQ + h;
-        ci[x] = i < L ? ((kGS ? __ldg(p.GS + e) : 0.f) - __ldg(p.lse + e)) * kLog2e : 0.f;
-        di[x] = i < L ? __ldg(p.D + e) : 0.f;
+        const bool in = t < nT && i < L;
+        c[x] = in ? ((kGS ? __ldg(p.GS + e) : 0.f) - __ldg(p.lse + e)) * kLog2e : 0.f;
+        dd[x] = in ? __ldg(p.D + e) : 0.f;
       }
     };
-    prefetch(0);
+    rows_of(0, cc, dc);
+    rows_of(1, cn, dn);
     for (int t = 0; t < nT; ++t) {
       const int st = t & 1;
-      if (t >= 2) {
-        const bool got = wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag);
+      {
+        const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) break;
       }
-      float d[8];
+      const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4) + ch * 8;
+      __nv_bfloat162 d[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) d[e] = exp2f(ri[e] - __ldg(rj + e));
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+      }
       uint8_t* qt = smem + Lay::oQ + st * Lay::kQ + (ch / 8) * (BQ * 128);
+      constexpr int kBatch = 8;
 #pragma unroll
-      for (int m = 0; m < kRows; ++m) {
-        const int r = rs + m * kRowStep;
-        *reinterpret_cast<uint4*>(qt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = scale8(u[m], d);
+      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int r = rs + (m0 + x) * kRowStep;
+          v[x] = *reinterpret_cast<const uint4*>(qt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+        }
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int r = rs + (m0 + x) * kRowStep;
+          *reinterpret_cast<uint4*>(qt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = scale8(v[x], d);
+        }
       }
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        sRow[st * 2 * BQ + tid + 64 * x] = ci[x];
-        sRow[st * 2 * BQ + BQ + tid + 64 * x] = di[x];
+        sRow[st * 2 * BQ + tid + 64 * x] = cc[x];
+        sRow[st * 2 * BQ + BQ + tid + 64 * x] = dc[x];
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(Q_READY + st));
-      if (t + 1 < nT) prefetch(t + 1);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        cc[x] = cn[x];
+        dc[x] = dn[x];
+      }
+      rows_of(t + 2, cn, dn);
     }
   } else {
     // ------------------------------------------------------------ P, dS (warps 4-11)
@@ -385,11 +432,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           0xffffffffu, key_ok && (i0 >= jj) && (i0 + 64 <= L) && (i0 + 63 - jj < win));
       float pv[64];
       auto p_part = [&](auto masked) {
+        uint32_t sv[64];  // both loads in flight before the one wait
+        tmem_ld32(tmem + lane_base + scol, sv);
+        tmem_ld32(tmem + lane_base + scol + 32, sv + 32);
+        tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 64; c += 32) {
-          uint32_t sv[32];
-          tmem_ld32(tmem + lane_base + scol + c, sv);
-          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
@@ -397,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-              const float arg = fmaf(__uint_as_float(sv[e + x]), p.scale_log2,
+              const float arg = fmaf(__uint_as_float(sv[c + e + x]), p.scale_log2,
                                      kGS ? cc[x] - gs_j : cc[x]);
               if constexpr (decltype(masked)::value) {
                 const int i = i0 + c + e + x;
@@ -426,11 +474,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
+      uint32_t dv[64];
+      tmem_ld32(tmem + lane_base + dcol, dv);
+      tmem_ld32(tmem + lane_base + dcol + 32, dv + 32);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
-        uint32_t dv[32];
-        tmem_ld32(tmem + lane_base + dcol + c, dv);
-        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -438,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
-            const float ds = pv[c + e + x] * (__uint_as_float(dv[e + x]) - dd[x]);
+            const float ds = pv[c + e + x] * (__uint_as_float(dv[c + e + x]) - dd[x]);
             if (kGS) colsum += ds;
             pv[c + e + x] = ds;
           }
@@ -539,8 +588,8 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-// dq = scale * 2^(P - R_I) (.) dq32 for the tensor-core path (R_I = P at the
-// row's 128-row block start), then dL = q (.) dq - k (.) dk^(h) over dq32;
+// dq = scale * 2^(P - R_I) (.) dq32 for the tensor-core path (R_I = floor of P
+// at the row's 128-row block start), then dL = q (.) dq - k (.) dk^(h) over dq32;
 // dk, dv = group sums; dGS = row + column parts.
 template <typename T>
 __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict__ k,
@@ -568,6 +617,8 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict
     float pv[8], rv[8], a[8], qq[8], kk[8], dkv[8], out[8];
     load8(P + off, pv);
     load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) rv[x] = floorf(rv[x]);
     load8(dq32 + off, a);
     load8(q + off, qq);
     load8(k + (row * H + hh / G) * K + g8 * 8, kk);
@@ -617,8 +668,9 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict
 template <int KD, bool kGS>
 int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                   cudaStream_t stream) {
-  CUtensorMap tk, tv, to;
-  if (!make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BK) ||
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tile_map(&tq, ws.qh, pb.rows, pb.HQ, KD, BQ) ||
+      !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BK) ||
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BK) ||
       !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BQ))
     return WALL_ERR_CUDA;
@@ -648,7 +700,7 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.n_blocks = ws.n_blocks128;
   p.status = status;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  bwd_tc_kernel<KD, kGS><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tk, tv, to, p);
+  bwd_tc_kernel<KD, kGS><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

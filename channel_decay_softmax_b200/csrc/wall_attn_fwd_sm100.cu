@@ -5,7 +5,9 @@
 // training section 1, per-block anchor):
 //   s_ij = scale * sum_n q_in k_jn 2^(P_in - P_jn)
 // Rows are cut into 128-row blocks per sequence; block I has anchor
-// R_I = P at its first row.  A preparation kernel writes
+// R_I = floor(P at its first row), per channel.  Integer anchors make every
+// per-tile factor 2^(R_I - R_J) an exact power of two, so scaling a bf16
+// operand by it is exact.  A preparation kernel writes
 //   Qh_i = q_i * 2^(P_i - R_I)   (i in block I)      bounded by one block
 //   Kh_j = k_j * 2^(R_J - P_j)   (j in block J)      bounded by one block
 // so that s_ij = scale * sum_n Qh_in * (Kh_jn * 2^(R_I,n - R_J,n)).  Inside
@@ -518,6 +520,8 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
     float pv[8], rv[8], x[8], y[8];
     load8(P + (row * HQ + hh) * K + g8 * 8, pv);
     load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) rv[c] = floorf(rv[c]);
     load8(q + (row * HQ + hh) * K + g8 * 8, x);
 #pragma unroll
     for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(pv[c] - rv[c]);
@@ -526,7 +530,7 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
 #pragma unroll
     for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(rv[c] - pv[c]);
     store8(khat + (row * HQ + hh) * K + g8 * 8, y);
-    if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, pv);
+    if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, rv);
   }
 }
 
