@@ -26,8 +26,9 @@
 //
 // CTA = one 128-row key block of one (sequence, head), 12 warps (3 per SM
 // sub-partition, 168 registers each):
-//   warp 0      TMA: Kh_J, V_J once; Qh_I with its anchors R_I, and dO_I per
-//               tile (2 stages each)
+//   warp 0      TMA: Kh_J, V_J once; Qh_I with its anchors R_I (3 stages) and
+//               dO_I (1 stage: dP(t+1) is the last MMA of a tile, so its load
+//               overlaps the softmax of P(t+1)) per tile
 //   warp 1      TMEM owner and MMA issuer.  Order per tile t:
 //               dV(t), S(t+1), dK(t), dP(t+1), so that the tensor core works
 //               on the next tile while the softmax computes dS(t)
@@ -77,14 +78,14 @@ struct BSmem {
   static constexpr int kQ = BQ * KD * 2;    // query or dO tile
   static constexpr int oK = 0;
   static constexpr int oV = oK + kKV;
-  static constexpr int oQ = oV + kKV;       // 2 stages of Qt
-  static constexpr int oO = oQ + 2 * kQ;    // 2 stages of dO
-  static constexpr int oRow = oO + 2 * kQ;  // float[2 stages][2][BQ]: c_i, D_i
-  static constexpr int oCol = oRow + 2 * 2 * BQ * 4;  // float[BK]: column sums of the second half
-  static constexpr int oRJ = oCol + BK * 4;           // float[KD]: R_J
-  static constexpr int oRI = oRJ + KD * 4;            // float[2 stages][KD]: R_I
-  static constexpr int oBar = oRI + 2 * KD * 4;
-  static constexpr int kBars = 18;
+  static constexpr int kStages = 3;         // query tiles in flight
+  static constexpr int oQ = oV + kKV;       // kStages stages of Qt
+  static constexpr int oO = oQ + kStages * kQ;  // dO, one stage
+  static constexpr int oRow = oO + kQ;      // float[kStages][2][BQ]: c_i, D_i
+  static constexpr int oCol = oRow + kStages * 2 * BQ * 4;  // float[BK]: column sums of the second half
+  static constexpr int oRI = oCol + BK * 4;                 // float[kStages][KD]: R_I
+  static constexpr int oBar = oRI + kStages * KD * 4;
+  static constexpr int kBars = 20;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -92,18 +93,18 @@ struct BSmem {
 
 enum BBar {
   KV_FULL = 0,
-  Q_READY = 1,   // +stage, 2 producer warps
-  Q_EMPTY = 3,   // +stage, tcgen05.commit after dK(t)
-  O_FULL = 5,    // +stage, TMA
-  O_EMPTY = 7,   // +stage, tcgen05.commit after dV(t)
-  S_FULL = 9,
-  DP_FULL = 10,
-  P_READY = 11,  // 8 softmax warps
-  DS_READY = 12, // 8 softmax warps
-  MM_DONE = 13,
-  MMA_DONE = 14,
-  COL_READY = 15,  // 4 warps of the second half: column sums in shared memory
-  Q_FULL = 16,     // +stage, TMA
+  Q_FULL = 1,     // +stage (3), TMA
+  Q_READY = 4,    // +stage (3), 2 producer warps
+  Q_EMPTY = 7,    // +stage (3), tcgen05.commit after dK(t)
+  O_FULL = 10,    // TMA
+  O_EMPTY = 11,   // tcgen05.commit after dV(t)
+  S_FULL = 12,
+  DP_FULL = 13,
+  P_READY = 14,   // 8 softmax warps
+  DS_READY = 15,  // 8 softmax warps
+  MM_DONE = 16,
+  MMA_DONE = 17,
+  COL_READY = 18,  // 4 warps of the second half: column sums in shared memory
 };
 
 // TMEM columns (lanes = keys): S^T [0,128), dP^T [128,256), dV [256,384),
@@ -184,13 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(KV_FULL), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Lay::kStages; ++s) {
       mbar_init(bar(Q_READY + s), 2);
       mbar_init(bar(Q_FULL + s), 1);
       mbar_init(bar(Q_EMPTY + s), 1);
-      mbar_init(bar(O_FULL + s), 1);
-      mbar_init(bar(O_EMPTY + s), 1);
     }
+    mbar_init(bar(O_FULL), 1);
+    mbar_init(bar(O_EMPTY), 1);
     mbar_init(bar(S_FULL), 1);
     mbar_init(bar(DP_FULL), 1);
     mbar_init(bar(P_READY), 8);
@@ -212,11 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
+    // lane 0: Kh_J, V_J and the query ring; lane 1: dO (one stage).  The two
+    // lanes wait on different barriers and progress independently.
+    constexpr int NS = Lay::kStages;
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_o);
       mbar_expect_tx(bar(KV_FULL), 2 * Lay::kKV);
       for (int b = 0; b < K / 64; ++b) {
         tma_load_3d(sbase + Lay::oK + b * (BK * 128), &tm_k, bar(KV_FULL), b * 64, h,
@@ -224,34 +227,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + Lay::oV + b * (BK * 128), &tm_v, bar(KV_FULL), b * 64, kh,
                     (int)(s0 + j0));
       }
-      int issued_o = 0, issued_q = 0;
+      int issued = 0;
       for (int t = 0; t < nT; ++t) {
-        const int st = t & 1;
-        const int row = (int)(s0 + (long)(I0 + t) * BQ);
-        // dO(t - 2) is released by dV(t - 2), before Qt(t - 2) by dK(t - 2)
-        if (t >= 2 && !wait_bar(bar(O_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
-          break;
-        mbar_expect_tx(bar(O_FULL + st), Lay::kQ);
-        for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oO + st * Lay::kQ + b * (BQ * 128), &tm_o, bar(O_FULL + st),
-                      b * 64, h, row);
-        issued_o = t + 1;
-        if (t >= 2 && !wait_bar(bar(Q_EMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+        const int st = t % NS;
+        if (t >= NS && !wait_bar(bar(Q_EMPTY + st), (t / NS - 1) & 1, p.status, abort_flag))
           break;
         mbar_expect_tx(bar(Q_FULL + st), Lay::kQ + K * 4);
+        const int row = (int)(s0 + (long)(I0 + t) * BQ);
         for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oQ + st * Lay::kQ + b * (BQ * 128), &tm_q, bar(Q_FULL + st),
                       b * 64, h, row);
         bulk_load(sbase + Lay::oRI + st * K * 4, anc + (long)(I0 + t) * HQ * K, K * 4,
                   bar(Q_FULL + st));
-        issued_q = t + 1;
+        issued = t + 1;
       }
       // no copy may still be in flight when the CTA exits
-      for (int t = max(0, issued_o - 2); t < issued_o; ++t)
-        mbar_wait(bar(O_FULL + (t & 1)), (t >> 1) & 1, p.status);
-      for (int t = max(0, issued_q - 2); t < issued_q; ++t)
-        mbar_wait(bar(Q_FULL + (t & 1)), (t >> 1) & 1, p.status);
+      for (int t = max(0, issued - NS); t < issued; ++t)
+        mbar_wait(bar(Q_FULL + t % NS), (t / NS) & 1, p.status);
       mbar_wait(bar(KV_FULL), 0, p.status);
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tm_o);
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        // dO(t) goes into the stage once dV(t - 1) has read dO(t - 1)
+        if (t >= 1 && !wait_bar(bar(O_EMPTY), (t - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(bar(O_FULL), Lay::kQ);
+        const int row = (int)(s0 + (long)(I0 + t) * BQ);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oO + b * (BQ * 128), &tm_o, bar(O_FULL), b * 64, h, row);
+        issued = t + 1;
+      }
+      if (issued > 0) mbar_wait(bar(O_FULL), (issued - 1) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
@@ -278,8 +284,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                        (first && kk == 0) ? 0u : 1u);
         }
       };
-      auto q_off = [&](int t) { return (uint32_t)(Lay::oQ + (t & 1) * Lay::kQ); };
-      auto o_off = [&](int t) { return (uint32_t)(Lay::oO + (t & 1) * Lay::kQ); };
+      constexpr int NS = Lay::kStages;
+      auto q_off = [&](int t) { return (uint32_t)(Lay::oQ + (t % NS) * Lay::kQ); };
+      const uint32_t o_off = Lay::oO;
       bool ok = wait_bar(bar(KV_FULL), 0, p.status, abort_flag);
       if (ok) ok = wait_bar(bar(Q_READY), 0, p.status, abort_flag);
       if (ok) ok = wait_bar(bar(O_FULL), 0, p.status, abort_flag);
@@ -287,21 +294,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_sd(Lay::oK, q_off(0), kColS);
         umma_commit(bar(S_FULL));
-        issue_sd(Lay::oV, o_off(0), kColDP);
+        issue_sd(Lay::oV, o_off, kColDP);
         umma_commit(bar(DP_FULL));
       }
       for (int t = 0; ok && t < nT; ++t) {
-        const int st = t & 1;
+        const int st = t % NS;
         const bool next = t + 1 < nT;
         if (!wait_bar(bar(P_READY), t & 1, p.status, abort_flag)) break;
         tc_fence_after();
-        issue_acc(kColS, o_off(t), kColDV, t == 0);
-        umma_commit(bar(O_EMPTY + st));
+        issue_acc(kColS, o_off, kColDV, t == 0);
+        umma_commit(bar(O_EMPTY));
         // S(t+1) may go before dK(t) (the tensor core then works while the
         // softmax finishes dS(t)), but only if its query tile is ready:
         // dK(t) frees the stage the tile after next is written to
-        const uint32_t q_next = bar(Q_READY + (st ^ 1));
-        const uint32_t q_par = ((t + 1) >> 1) & 1;
+        const uint32_t q_next = bar(Q_READY + (t + 1) % NS);
+        const uint32_t q_par = ((t + 1) / NS) & 1;
         bool s_done = false;
         if (next && mbar_try_wait(q_next, q_par)) {
           tc_fence_after();
@@ -320,9 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(bar(S_FULL));
         }
         if (next) {
-          if (!wait_bar(bar(O_FULL + (st ^ 1)), ((t + 1) >> 1) & 1, p.status, abort_flag)) break;
+          if (!wait_bar(bar(O_FULL), (t + 1) & 1, p.status, abort_flag)) break;
           tc_fence_after();
-          issue_sd(Lay::oV, o_off(t + 1), kColDP);  // in order after dK(t) read dS^T
+          issue_sd(Lay::oV, o_off, kColDP);  // in order after dK(t) read dS^T
           umma_commit(bar(DP_FULL));
         }
       }
@@ -357,9 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     rows_of(0, cc, dc);
     rows_of(1, cn, dn);
     for (int t = 0; t < nT; ++t) {
-      const int st = t & 1;
+      const int st = t % Lay::kStages;
       {
-        const bool got = wait_bar(bar(Q_FULL + st), (t >> 1) & 1, p.status, abort_flag);
+        const bool got = wait_bar(bar(Q_FULL + st), (t / Lay::kStages) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) break;
       }
       const float* ri = reinterpret_cast<const float*>(smem + Lay::oRI + st * K * 4) + ch * 8;
@@ -415,17 +422,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     float colsum = 0.f;
     bool ok = true;
     for (int t = 0; t < nT && ok; ++t) {
-      const int st = t & 1;
+      const int st = t % Lay::kStages;
       const int i0 = (I0 + t) * BQ + half * 64;  // first query of this half
+      const float* cv = sRow + st * 2 * BQ + half * 64;
+      const float* dvv = cv + BQ;
+      // The logit offsets of the half's queries are read before the wait for
+      // S: while the tensor core streams operands, a shared-memory load takes
+      // hundreds of cycles, and here that latency overlaps the wait.
+      float cr[64];
       {
-        bool got = wait_bar(bar(S_FULL), t & 1, p.status, abort_flag);
         // acquire the producers' per-query terms (that phase has completed)
-        got = got && wait_bar(bar(Q_READY + st), (t >> 1) & 1, p.status, abort_flag);
+        const bool got =
+            wait_bar(bar(Q_READY + st), (t / Lay::kStages) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int e = 0; e < 64; e += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(cv + e);
+        cr[e] = c4.x;
+        cr[e + 1] = c4.y;
+        cr[e + 2] = c4.z;
+        cr[e + 3] = c4.w;
+      }
+      {
+        const bool got = wait_bar(bar(S_FULL), t & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
-      const float* cv = sRow + st * 2 * BQ + half * 64;
-      const float* dvv = cv + BQ;
       // every query of the half sees every key of the warp: no mask work in the
       // loop.  Warp-uniform, since the branch holds the warp-wide TMEM loads
       const bool full = __all_sync(
@@ -441,18 +464,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(cv + c + e);
-            const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
+              const float cx = cr[c + e + x];
               const float arg = fmaf(__uint_as_float(sv[c + e + x]), p.scale_log2,
-                                     kGS ? cc[x] - gs_j : cc[x]);
+                                     kGS ? cx - gs_j : cx);
+              // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
+              const float ev = ((e + x) & 7) >= 5 ? exp2_fma(arg) : exp2f(arg);
               if constexpr (decltype(masked)::value) {
                 const int i = i0 + c + e + x;
                 const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);
-                pv[c + e + x] = vis ? exp2f(arg) : 0.f;
+                pv[c + e + x] = vis ? ev : 0.f;
               } else {
-                pv[c + e + x] = exp2f(arg);
+                pv[c + e + x] = ev;
               }
             }
           }

@@ -10,6 +10,25 @@
 namespace wall {
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the FMA and integer pipes, for softmax exponents (x <= ~0), so that
+// part of a tile's exponentials can bypass the 16-per-clock MUFU unit.
+// Cody-Waite style range reduction x = n + f with n = round(x) (added to and
+// subtracted from 1.5 * 2^23, which leaves n in the low mantissa bits) and
+// |f| <= 1/2, then a degree-3 polynomial for 2^f whose coefficients are our
+// own relative-error minimax fit on [-1/2, 1/2] (max relative error 7.6e-5,
+// well under the 2^-9 step of the bf16 P it feeds), and n added to the
+// exponent field.  x is clamped at -126, where 2^x no longer matters next to
+// the row's leading terms; the result there is 0 or a tiny subnormal.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float y = x + 12582912.f;
+  const float f = x - (y - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05517049878835678f, f, 0.24260851740837097f), f,
+                            0.6932609677314758f),
+                       f, 0.9999282360076904f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kInvLn2 = 1.4426950408889634f;
 
