@@ -11,13 +11,20 @@
 // by the finalize kernel, which also forms the gate-gradient summand.  dq is
 // written once per row: deterministic, and no fp32 atomics through L2.
 //
-// CTA = 10 warps:
+// The block anchors are integers, so d = 2^(R_I - R_J) is an exact power of
+// two and Kt_J = Kh_J (.) d is an exact packed bf16 multiply, done in place.
+//
+// CTA = 12 warps (3 per SM sub-partition, 168 registers each):
 //   warp 0      TMA: Qh_I, dO_I once; Kh_J (+ block anchors, 3 stages) and V_J
 //               (1 stage: it is read by one MMA only) per key tile
-//   warp 1      TMEM owner and MMA issuer: S two tiles ahead, dP one ahead
-//   warps 2-5   key rescale Kt_J = Kh_J (.) d in shared memory
-//   warps 6-9   one thread per query row: P, dS -> bf16 pairs over the
-//               consumed S columns; epilogue dQa -> fp32 workspace
+//   warp 1      TMEM owner and MMA issuer.  Per tile: dP(t+1) as soon as the
+//               softmax has read dP(t), then dQa(t), then S(t+2)
+//   warps 2-3   key rescale Kt_J = Kh_J (.) d in place; each thread keeps one
+//               16-byte channel chunk, so its 8 factors stay in registers
+//   warps 4-11  one thread per (query row, 64-key half of the tile): P, dS ->
+//               bf16 pairs over the first 32 of the half's S columns; the two
+//               warps of a TMEM lane quarter take the two halves; epilogue
+//               dQa -> fp32 workspace
 // TMEM columns: S0 [0,128), S1 [128,256), dP [256,384), dQa [384,512).
 #include <cuda.h>
 
@@ -33,7 +40,7 @@ using namespace sm100;
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int kKS = 3;  // key stages
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 
 struct DqParams {
   const float* anchors;  // [nblk, HQ, K]
@@ -58,9 +65,8 @@ struct DSmem {
   static constexpr int oV = oK + kKS * kT;     // 1 stage
   static constexpr int oRI = oV + kT;          // float[KD]
   static constexpr int oRJ = oRI + KD * 4;     // float[kKS][KD]
-  static constexpr int oD = oRJ + kKS * KD * 4;  // float[4 warps][KD]
-  static constexpr int oGS = oD + 4 * KD * 4;    // float[4 warps][BN]
-  static constexpr int oBar = oGS + 4 * BN * 4;
+  static constexpr int oGS = oRJ + kKS * KD * 4;  // float[8 warps][64]: key prefix
+  static constexpr int oBar = oGS + 8 * 64 * 4;
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
@@ -79,6 +85,14 @@ enum DBar {
   DQ_DONE = 14,
   MMA_DONE = 15,
 };
+
+// 2^k as bf16 bits for an integer k (the anchors are integers): exact in
+// the normal range, 0 below it (a factor under 2^-126 scales a key that
+// decays to nothing) and +inf above it, as the fp32 product would overflow.
+__device__ __forceinline__ uint32_t pow2_bf16(float k) {
+  const int e = (int)k;
+  return e < -126 ? 0u : e > 127 ? 0x7F80u : uint32_t(e + 127) << 7;
+}
 
 constexpr uint32_t kColS = 0, kColDP = 256, kColDQ = 384;
 
@@ -113,7 +127,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
-  float* sD = reinterpret_cast<float*>(smem + Lay::oD);
   float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
@@ -141,13 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(QO_FULL), 1);
     for (int s = 0; s < kKS; ++s) {
       mbar_init(bar(K_FULL + s), 1);
-      mbar_init(bar(K_READY + s), 4);
+      mbar_init(bar(K_READY + s), 2);
       mbar_init(bar(K_EMPTY + s), 1);
     }
     mbar_init(bar(V_FULL), 1);
     mbar_init(bar(V_EMPTY), 1);
     mbar_init(bar(SD_FULL), 1);
-    mbar_init(bar(P_FULL), 4);
+    mbar_init(bar(P_FULL), 8);
     mbar_init(bar(DQ_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
     *abort_flag = 0;
@@ -244,67 +257,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = t % kKS;
         if (!wait_bar(bar(P_FULL), t & 1, p.status, abort_flag)) break;
         tc_fence_after();
+        // the softmax has read dP(t): dP(t+1) first, so that the softmax of
+        // tile t+1 can start while the tensor core accumulates dQa(t)
+        if (t + 1 < nT) ok = issue_dp(t + 1);
         // dQa += dS Kt: A = dS (bf16 pairs over the S buffer, 8 columns per 16
-        // keys), B = Kt [keys x channels] MN-major: 8-key groups 1 KB apart,
-        // 64-channel boxes BN*128 bytes apart
+        // keys, the two 64-key halves 64 columns apart), B = Kt [keys x
+        // channels] MN-major: 8-key groups 1 KB apart, 64-channel boxes BN*128
+        // bytes apart
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts(tmem + kColDQ, tmem + kColS + (t & 1) * 128 + kk * 8,
+          umma_bf16_ts(tmem + kColDQ, tmem + kColS + (t & 1) * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
                        sdesc_sw128(sbase + Lay::oK + st * Lay::kT + kk * 16 * 128, BN * 128,
                                    1024),
                        id_dq, (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(K_EMPTY + st));
-        if (t + 1 < nT) ok = issue_dp(t + 1);
-        if (ok && t + 2 < nT) ok = issue_s(t + 2);
+        if (ok && t + 2 < nT) ok = issue_s(t + 2);  // in order after dQa(t) read dS(t)
       }
       umma_commit(bar(DQ_DONE));
       umma_commit(bar(MMA_DONE));
       mbar_wait(bar(MMA_DONE), 0, p.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ key rescale
-    const int wt = threadIdx.x - 64;
-    const int wq = warp - 2;
-    float* d = sD + wq * KD;
+    constexpr int kChunks = KD / 8;          // 16-byte chunks per row
+    constexpr int kRowStep = 64 / kChunks;   // rows covered by one pass of 64 threads
+    constexpr int kRows = BN / kRowStep;     // rows per thread
+    const int tid = threadIdx.x - 64;
+    const int ch = tid % kChunks;
+    const int rs = tid / kChunks;
+    float ri[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ri[e] = sRI[ch * 8 + e];
     for (int t = 0; t < nT; ++t) {
       const int st = t % kKS;
-      const bool got = wait_bar(bar(K_FULL + st), (t / kKS) & 1, p.status, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4);
-      __syncwarp();
-      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - rj[n]);
-      __syncwarp();
-      uint8_t* kt = smem + Lay::oK + st * Lay::kT;
-      constexpr int kPer = (KD / 64) * BN * 8 / 128;
-      constexpr int kBatch = 4;
-#pragma unroll 1
-      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
-        uint4 u[kBatch];
-        float dd[kBatch][8];
-        uint4* ptr[kBatch];
+      {
+        const bool got = wait_bar(bar(K_FULL + st), (t / kKS) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) break;
+      }
+      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
+      __nv_bfloat162 d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+      }
+      uint8_t* kt = smem + Lay::oK + st * Lay::kT + (ch / 8) * (BN * 128);
+      constexpr int kBatch = 8;
+#pragma unroll
+      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+        uint4 v[kBatch];
 #pragma unroll
         for (int x = 0; x < kBatch; ++x) {
-          const int c = wt + (b0 + x) * 128;
-          const int box = c / (BN * 8);
-          const int row = (c / 8) % BN;
-          const int pch = c % 8;
-          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-          ptr[x] = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
-          u[x] = *ptr[x];
-          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
-          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
+          const int r = rs + (m0 + x) * kRowStep;
+          v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
         }
 #pragma unroll
         for (int x = 0; x < kBatch; ++x) {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+          const int r = rs + (m0 + x) * kRowStep;
+          __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
-          }
-          *ptr[x] = u[x];
+          for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
+          *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
         }
       }
       fence_proxy_async_smem();
@@ -312,8 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(K_READY + st));
     }
   } else {
-    // ------------------------------------------------------------ dS per query row
+    // ------------------------------------------------------------ dS per (query row, key half)
     const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;  // keys 64*half .. 64*half+63 of each tile
     const int r = quarter * 32 + lane;
     const int i = i0 + r;
     const bool row_ok = r < ni;
@@ -325,13 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float Di = row_ok ? p.D[grow] : 0.f;
     const float gs_i = (has_gs && row_ok) ? p.GS[grow] * kLog2e : 0.f;
     const float sl2 = p.scale_log2;
+    const float off_i = (has_gs ? gs_i : 0.f) - lse2;
+    float* gsk = sGS + (warp - 4) * 64;  // this warp's copy of the key prefix (or zeros)
     bool ok = true;
     for (int t = 0; t < nT; ++t) {
-      const int j0 = (jb_lo + t) * BN;
-      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix (or zeros)
+      const int j0 = (jb_lo + t) * BN + half * 64;  // first key of this half
       if (has_gs || t == 0) {
         __syncwarp();
-        for (int c = lane; c < BN; c += 32) {
+        for (int c = lane; c < 64; c += 32) {
           const int j = j0 + c;
           gsk[c] = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
         }
@@ -342,13 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + kColS + (t & 1) * 128;
-      const uint32_t dp_addr = tmem + lane_base + kColDP;
-      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) && (i - j0 < win);
-      const bool fast = full && !has_gs;
-      const float off_i = (has_gs ? gs_i : 0.f) - lse2;
+      const uint32_t s_addr = tmem + lane_base + kColS + (t & 1) * 128 + half * 64;
+      const uint32_t dp_addr = tmem + lane_base + kColDP + half * 64;
+      const bool fast = __all_sync(0xffffffffu, row_ok && (j0 + 63 <= i) && (j0 + 64 <= L) &&
+                                                    (i - j0 < win) && !has_gs);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         uint32_t sv[32], dv[32];
         tmem_ld32(s_addr + c, sv);
         tmem_ld32(dp_addr + c, dv);
@@ -357,10 +372,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (fast) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = exp2f(fmaf(__uint_as_float(sv[e]), sl2, off_i));
-            const float p1 = exp2f(fmaf(__uint_as_float(sv[e + 1]), sl2, off_i));
-            pk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - Di),
-                                    p1 * (__uint_as_float(dv[e + 1]) - Di));
+            float ds[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const float a = fmaf(__uint_as_float(sv[e + x]), sl2, off_i);
+              // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
+              const float pv = ((e + x) & 7) >= 5 ? exp2_fma(a) : exp2f(a);
+              ds[x] = pv * (__uint_as_float(dv[e + x]) - Di);
+            }
+            pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
           }
         } else {
 #pragma unroll
@@ -377,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
           }
         }
-        // keys [c, c+32) -> columns [c/2, c/2+16) of this S buffer (already read)
+        // keys [c, c+32) of the half -> its columns [c/2, c/2+16) (already read)
         tmem_st16(s_addr + c / 2, pk);
       }
       tmem_wait_st();
@@ -385,13 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(P_FULL));
     }
-    // ---- epilogue: the raw dQa row
+    // ---- epilogue: the raw dQa row, each half writes half of the channels
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(DQ_DONE), 0, p.status, abort_flag));
     if (ok) {
       tc_fence_after();
       float* out = p.dq32 + grow * K;
 #pragma unroll 1
-      for (int c = 0; c < KD; c += 32) {
+      for (int c = half * (KD / 2); c < (half + 1) * (KD / 2); c += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + kColDQ + c, v);
         tmem_wait_ld();
