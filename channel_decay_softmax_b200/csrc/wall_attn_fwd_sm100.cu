@@ -11,25 +11,34 @@
 //   Qh_i = q_i * 2^(P_i - R_I)   (i in block I)      bounded by one block
 //   Kh_j = k_j * 2^(R_J - P_j)   (j in block J)      bounded by one block
 // so that s_ij = scale * sum_n Qh_in * (Kh_jn * 2^(R_I,n - R_J,n)).  Inside
-// the kernel the per-tile, per-channel factor d = 2^(R_I - R_J) (128 exps per
-// tile, not 128*128) is applied to the key tile in shared memory, then
+// the kernel the per-tile, per-channel factor d = 2^(R_I - R_J) is applied to
+// the key tile in shared memory (packed bf16 multiplies, exact), then
 //   S = Qh * Kt^T   and   O += P * V   run on tcgen05 with fp32 accumulators
 // in TMEM, and the online softmax (log2 domain) keeps one query row per
 // thread.  For decaying gates d only shrinks towards zero for distant tiles,
 // where the exact contribution is equally negligible; no exponent of a
 // global prefix ever reaches bf16 (the blog's reason for the anchors).
 //
-// CTA = one 128-row query block of one (sequence, head), 10 warps:
-//   warp 0      TMA producer: Qh once; Kh_J and V_J per tile (2-stage rings,
-//               the key stage is released after S, the value stage after PV)
+// The key tiles of a query block are split between two softmax groups, even
+// and odd tiles, each with its own running max, sum and O accumulator, so
+// two tiles are in the softmax at once; the two partial results are merged
+// once at the end, as a split-KV decode merges its splits.
+//
+// CTA = one 128-row query block of one (sequence, head), 12 warps (3 per SM
+// sub-partition, 168 registers each):
+//   warp 0      TMA producer, lane 0: Qh once and the key ring (3 stages,
+//               released after S); lane 1: the value ring (2 stages,
+//               released after PV)
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2-5   key rescale: Kt_J = Kh_J (.) d in place (bf16 -> fp32 -> bf16),
-//               and the g_scalar key prefix of the tile
-//   warps 6-9   softmax: S from TMEM, mask, exp2, P (bf16 pairs) written back
-//               over the consumed S columns as the TMEM A operand of PV, lazy
-//               O rescale in TMEM when the row max grows by more than 2^8,
-//               epilogue o = O / l, lse.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+V).
+//   warps 2-3   key rescale: Kt_J = Kh_J (.) d in place; each thread keeps one
+//               16-byte channel chunk, so its 8 factors stay in registers
+//   warps 4-7   softmax of the even tiles, warps 8-11 of the odd tiles: S from
+//               TMEM, mask, exp2, P (bf16 pairs) written back over the consumed
+//               S columns as the TMEM A operand of PV, lazy O rescale in TMEM
+//               when the row max grows by more than 2^8; epilogue merges the
+//               two groups, o = O / l, lse.
+// TMEM columns: S0 [0,128), S1 [128,256), O_even [256, 256+V),
+// O_odd [256+V, 256+2V).
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -43,7 +52,9 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kKS = 3;                    // key stages
+constexpr int kVS = 2;                    // value stages
 constexpr float kRescaleThreshold = 8.f;  // log2 units: lazy O rescale
 
 struct FwdTcParams {
@@ -62,34 +73,33 @@ struct FwdTcParams {
 
 template <int KD>
 struct Smem {
-  static constexpr int kQ = BM * KD * 2;
-  static constexpr int kK = BN * KD * 2;
-  static constexpr int kV = BN * KD * 2;
+  static constexpr int kT = BN * KD * 2;          // one 128-row bf16 tile
   static constexpr int oQ = 0;
-  static constexpr int oK = oQ + kQ;             // 2 stages
-  static constexpr int oV = oK + 2 * kK;         // 2 stages
-  static constexpr int oRI = oV + 2 * kV;        // float[KD]
-  static constexpr int oD = oRI + KD * 4;        // float[2 stages][4 warps][KD]
-  static constexpr int oGS = oD + 8 * KD * 4;    // float[4 warps][BN]
-  static constexpr int oRJ = oGS + 4 * BN * 4;   // float[2 stages][KD] key-block anchors
-  static constexpr int oBar = oRJ + 2 * KD * 4;  // uint64 barriers
-  static constexpr int kBars = 16;
-  static constexpr int oMisc = oBar + kBars * 8; // tmem base, abort flag
+  static constexpr int oK = oQ + kT;              // kKS stages
+  static constexpr int oV = oK + kKS * kT;        // kVS stages
+  static constexpr int oRI = oV + kVS * kT;       // float[KD]
+  static constexpr int oRJ = oRI + KD * 4;        // float[kKS][KD] key-block anchors
+  static constexpr int oGS = oRJ + kKS * KD * 4;  // float[8 warps][BN] key prefix
+  static constexpr int oX = oGS + 8 * BN * 4;     // float[2 groups][2][BM]: m, l
+  static constexpr int oBar = oX + 2 * 2 * BM * 4;
+  static constexpr int kBars = 22;
+  static constexpr int oMisc = oBar + kBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = oMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;   // slack for 1 KB alignment
+  static constexpr int kAlloc = kBytes + 1024;    // slack for 1 KB alignment
 };
 
 enum Bar {
   B_QFULL = 0,
-  B_KFULL = 1,   // +stage
-  B_VFULL = 3,   // +stage
-  B_KREADY = 5,  // +stage
-  B_KEMPTY = 7,  // +stage
-  B_VEMPTY = 9,  // +stage
-  B_SFULL = 11,  // +stage
-  B_PFULL = 13,
-  B_PVDONE = 14,
-  B_MMADONE = 15,
+  B_KFULL = 1,    // +stage (3)
+  B_KREADY = 4,   // +stage (3), 2 rescale warps
+  B_KEMPTY = 7,   // +stage (3)
+  B_VFULL = 10,   // +stage (2)
+  B_VEMPTY = 12,  // +stage (2)
+  B_SFULL = 14,   // +S buffer (2)
+  B_PFULL = 16,   // +group (2), 4 warps each
+  B_PVDONE = 18,  // +group (2): O_group holds every PV issued so far
+  B_XCHG = 20,    // epilogue exchange of m, l between the groups (8 warps)
+  B_MMADONE = 21,
 };
 
 // bounded wait that also gives up once another role has given up
@@ -114,6 +124,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 2^k as bf16 bits for an integer k (the anchors are integers): exact in
+// the normal range, 0 below it (a factor under 2^-126 scales a key that
+// decays to nothing) and +inf above it, as the fp32 product would overflow.
+__device__ __forceinline__ uint32_t pow2_bf16(float k) {
+  const int e = (int)k;
+  return e < -126 ? 0u : e > 127 ? 0x7F80u : uint32_t(e + 127) << 7;
+}
+
 template <int KD>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -124,8 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
-  float* sD = reinterpret_cast<float*>(smem + Lay::oD);
   float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
+  float* sX = reinterpret_cast<float*>(smem + Lay::oX);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
@@ -150,16 +168,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKS; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_KREADY + s), 4);
+      mbar_init(bar(B_KREADY + s), 2);
       mbar_init(bar(B_KEMPTY + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
-      mbar_init(bar(B_SFULL + s), 1);
     }
-    mbar_init(bar(B_PFULL), 4);
-    mbar_init(bar(B_PVDONE), 1);
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar(B_SFULL + g), 1);
+      mbar_init(bar(B_PFULL + g), 4);
+      mbar_init(bar(B_PVDONE + g), 1);
+    }
+    mbar_init(bar(B_XCHG), 8);
     mbar_init(bar(B_MMADONE), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -177,42 +200,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
+    // lane 0: Qh and the key ring; lane 1: the value ring.  The two lanes
+    // wait on different barriers and progress independently.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_expect_tx(bar(B_QFULL), Lay::kQ);
+      mbar_expect_tx(bar(B_QFULL), Lay::kT);
       for (int b = 0; b < K / 64; ++b)
         tma_load_3d(sbase + Lay::oQ + b * (BM * 128), &tm_q, bar(B_QFULL), b * 64, h,
                     (int)(s0 + i0));
-      int k_issued = 0, v_issued = 0;
+      int issued = 0;
       for (int t = 0; t < nT; ++t) {
-        const int st = t & 1;
-        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
-        if (t >= 2 && !wait_bar(bar(B_KEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
+        const int st = t % kKS;
+        if (t >= kKS && !wait_bar(bar(B_KEMPTY + st), (t / kKS - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(B_KFULL + st), Lay::kK + K * 4);
+        mbar_expect_tx(bar(B_KFULL + st), Lay::kT + K * 4);
+        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
         for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oK + st * Lay::kK + b * (BN * 128), &tm_k, bar(B_KFULL + st),
+          tma_load_3d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k, bar(B_KFULL + st),
                       b * 64, h, row);
         bulk_load(sbase + Lay::oRJ + st * K * 4,
                   p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
                   bar(B_KFULL + st));
-        k_issued = t + 1;
-        if (t >= 2 && !wait_bar(bar(B_VEMPTY + st), ((t >> 1) - 1) & 1, p.status, abort_flag))
-          break;
-        mbar_expect_tx(bar(B_VFULL + st), Lay::kV);
-        for (int b = 0; b < V / 64; ++b)
-          tma_load_3d(sbase + Lay::oV + st * Lay::kV + b * (BN * 128), &tm_v, bar(B_VFULL + st),
-                      b * 64, kh, row);
-        v_issued = t + 1;
+        issued = t + 1;
       }
       // no bulk copy may still be landing in this CTA's shared memory at exit
-      for (int t = max(0, k_issued - 2); t < k_issued; ++t)
-        mbar_wait(bar(B_KFULL + (t & 1)), (t >> 1) & 1, p.status);
-      for (int t = max(0, v_issued - 2); t < v_issued; ++t)
-        mbar_wait(bar(B_VFULL + (t & 1)), (t >> 1) & 1, p.status);
+      for (int t = max(0, issued - kKS); t < issued; ++t)
+        mbar_wait(bar(B_KFULL + t % kKS), (t / kKS) & 1, p.status);
       mbar_wait(bar(B_QFULL), 0, p.status);
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kVS;
+        if (t >= kVS && !wait_bar(bar(B_VEMPTY + st), (t / kVS - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(B_VFULL + st), Lay::kT);
+        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+        for (int b = 0; b < V / 64; ++b)
+          tma_load_3d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v, bar(B_VFULL + st),
+                      b * 64, kh, row);
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - kVS); t < issued; ++t)
+        mbar_wait(bar(B_VFULL + t % kVS), (t / kVS) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
@@ -220,94 +251,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_qk = idesc_bf16(BM, BN, false, false);
       const uint32_t idesc_pv = idesc_bf16(BM, V, false, true);
       bool ok = wait_bar(bar(B_QFULL), 0, p.status, abort_flag);
+      // S(t) into buffer t & 1; it is free once PV(t - 2) has read P(t - 2)
       auto issue_qk = [&](int t) -> bool {
-        const int st = t & 1;
-        if (!wait_bar(bar(B_KREADY + st), (t >> 1) & 1, p.status, abort_flag)) return false;
+        const int st = t % kKS;
+        if (!wait_bar(bar(B_KREADY + st), (t / kKS) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + st * 128;
+        const uint32_t d_tmem = tmem + (t & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           const uint64_t a = sdesc_sw128(sbase + Lay::oQ + off, 16, 1024);
-          const uint64_t b = sdesc_sw128(sbase + Lay::oK + st * Lay::kK + off, 16, 1024);
+          const uint64_t b = sdesc_sw128(sbase + Lay::oK + st * Lay::kT + off, 16, 1024);
           umma_bf16_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(B_SFULL + st));
+        umma_commit(bar(B_SFULL + (t & 1)));
         umma_commit(bar(B_KEMPTY + st));
         return true;
       };
       if (ok) ok = issue_qk(0);
       if (ok && nT > 1) ok = issue_qk(1);
       for (int t = 0; ok && t < nT; ++t) {
-        const int st = t & 1;
-        if (!wait_bar(bar(B_VFULL + st), (t >> 1) & 1, p.status, abort_flag)) break;
-        if (!wait_bar(bar(B_PFULL), t & 1, p.status, abort_flag)) break;
+        const int g = t & 1;  // softmax group and S / O buffers of this tile
+        const int vs = t % kVS;
+        if (!wait_bar(bar(B_VFULL + vs), (t / kVS) & 1, p.status, abort_flag)) break;
+        if (!wait_bar(bar(B_PFULL + g), (t >> 1) & 1, p.status, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // A = P [128 rows x 16 keys] from TMEM: the softmax wrote bf16 pairs
           // over the S buffer it had consumed, 8 columns per 16 keys
-          const uint32_t a = tmem + st * 128 + kk * 8;
+          const uint32_t a = tmem + g * 128 + kk * 8;
           // B = V [16 keys x V channels], MN-major: 8-key groups 1 KB apart,
           // 64-channel boxes BN*128 bytes apart
           const uint64_t b =
-              sdesc_sw128(sbase + Lay::oV + st * Lay::kV + kk * 16 * 128, BN * 128, 1024);
-          umma_bf16_ts(tmem + 256, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+              sdesc_sw128(sbase + Lay::oV + vs * Lay::kT + kk * 16 * 128, BN * 128, 1024);
+          umma_bf16_ts(tmem + 256 + g * V, a, b, idesc_pv, (t >= 2 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar(B_PVDONE));
-        umma_commit(bar(B_VEMPTY + st));
+        umma_commit(bar(B_PVDONE + g));
+        umma_commit(bar(B_VEMPTY + vs));
         if (t + 2 < nT) ok = issue_qk(t + 2);
       }
       // every MMA of this CTA has completed before TMEM is released
       umma_commit(bar(B_MMADONE));
       mbar_wait(bar(B_MMADONE), 0, p.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ key rescale
-    // The key tile and its block anchors arrive together; each warp forms
-    // the whole factor vector d = 2^(R_I - R_J) it needs (no cross-warp
-    // barrier) and arrives on k_ready once its chunks are written and fenced.
-    const int wt = threadIdx.x - 64;  // 0..127
-    const int wq = warp - 2;          // 0..3
+    constexpr int kChunks = KD / 8;          // 16-byte chunks per row
+    constexpr int kRowStep = 64 / kChunks;   // rows covered by one pass of 64 threads
+    constexpr int kRows = BN / kRowStep;     // rows per thread
+    const int tid = threadIdx.x - 64;
+    const int ch = tid % kChunks;
+    const int rs = tid / kChunks;
+    float ri[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ri[e] = sRI[ch * 8 + e];
     for (int t = 0; t < nT; ++t) {
-      const int st = t & 1;
-      float* d = sD + (st * 4 + wq) * KD;
-      const bool got = wait_bar(bar(B_KFULL + st), (t >> 1) & 1, p.status, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4);
-      for (int n = lane; n < K; n += 32) d[n] = exp2f(sRI[n] - rj[n]);
-      __syncwarp();
-      uint8_t* kt = smem + Lay::oK + st * Lay::kK;
-      constexpr int kPer = (KD / 64) * BN * 8 / 128;  // chunks per thread
-      constexpr int kBatch = 4;
-#pragma unroll 1
-      for (int b0 = 0; b0 < kPer; b0 += kBatch) {
-        uint4 u[kBatch];
-        float dd[kBatch][8];
-        uint4* ptr[kBatch];
+      const int st = t % kKS;
+      {
+        const bool got = wait_bar(bar(B_KFULL + st), (t / kKS) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) break;
+      }
+      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
+      __nv_bfloat162 d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+      }
+      uint8_t* kt = smem + Lay::oK + st * Lay::kT + (ch / 8) * (BN * 128);
+      constexpr int kBatch = 8;
+#pragma unroll
+      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+        uint4 v[kBatch];
 #pragma unroll
         for (int x = 0; x < kBatch; ++x) {
-          const int c = wt + (b0 + x) * 128;
-          const int box = c / (BN * 8);
-          const int row = (c / 8) % BN;
-          const int pch = c % 8;
-          const int ch0 = box * 64 + ((pch ^ (row & 7)) * 8);
-          ptr[x] = reinterpret_cast<uint4*>(kt + box * (BN * 128) + row * 128 + pch * 16);
-          u[x] = *ptr[x];
-          const float4 da = *reinterpret_cast<const float4*>(d + ch0);
-          const float4 db = *reinterpret_cast<const float4*>(d + ch0 + 4);
-          dd[x][0] = da.x; dd[x][1] = da.y; dd[x][2] = da.z; dd[x][3] = da.w;
-          dd[x][4] = db.x; dd[x][5] = db.y; dd[x][6] = db.z; dd[x][7] = db.w;
+          const int r = rs + (m0 + x) * kRowStep;
+          v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
         }
 #pragma unroll
         for (int x = 0; x < kBatch; ++x) {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u[x]);
+          const int r = rs + (m0 + x) * kRowStep;
+          __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * dd[x][2 * e], f.y * dd[x][2 * e + 1]);
-          }
-          *ptr[x] = u[x];
+          for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
+          *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
         }
       }
       fence_proxy_async_smem();
@@ -316,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int grp = (warp - 4) >> 2;          // 0: even key tiles, 1: odd ones
     const int quarter = warp & 3;             // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;        // query row within the block
     const int i = i0 + r;                     // row within the sequence
@@ -324,13 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_gs = p.GS != nullptr;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     const float gs_i = (has_gs && row_ok) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+    const uint32_t s_addr = tmem + lane_base + grp * 128;
+    const uint32_t o_addr = tmem + lane_base + 256 + grp * V;
+    float* gsk = sGS + (warp - 4) * BN;  // this warp's copy of the key prefix (or zeros)
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < nT; ++t) {
-      const int st = t & 1;
+    for (int t = grp; t < nT; t += 2) {
       const int j0 = (jb_lo + t) * BN;
-      float* gsk = sGS + (warp - 6) * BN;  // this warp's copy of the key prefix (or zeros)
-      if (has_gs || t == 0) {
+      if (has_gs || t == grp) {
         __syncwarp();
         for (int c = lane; c < BN; c += 32) {
           const int j = j0 + c;
@@ -339,28 +370,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       {
-        const bool got = wait_bar(bar(B_SFULL + st), (t >> 1) & 1, p.status, abort_flag);
+        const bool got = wait_bar(bar(B_SFULL + grp), (t >> 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + st * 128;
       // logits (log2 domain) with the causal / window / sequence mask.  The
       // common case -- a fully visible tile without a scalar gate -- is a
-      // plain multiply; decisions are hoisted out of the element loops.
-      const bool full = row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) && (i - j0 < win);
-      const bool fast = full && !has_gs;
+      // plain multiply; the decision is warp-uniform and hoisted out of the
+      // element loops.
+      const bool fast = __all_sync(0xffffffffu, row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
+                                                    (i - j0 < win) && !has_gs);
       const float sl2 = p.scale_log2;
       const float bias_i = has_gs ? gs_i : 0.f;
       // pass 1: row max
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t sv[32];
+      for (int c = 0; c < BN; c += 64) {
+        uint32_t sv[64];
         tmem_ld32(s_addr + c, sv);
+        tmem_ld32(s_addr + c + 32, sv + 32);
         tmem_wait_ld();
         if (fast) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
+          for (int e = 0; e < 64; e += 4) {
             mx0 = fmaxf(mx0, __uint_as_float(sv[e]) * sl2);
             mx1 = fmaxf(mx1, __uint_as_float(sv[e + 1]) * sl2);
             mx2 = fmaxf(mx2, __uint_as_float(sv[e + 2]) * sl2);
@@ -368,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 64; ++e) {
             const int j = j0 + c + e;
             const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
             const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e]);
@@ -380,8 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool resc = mx > m_use + kRescaleThreshold;
       const float m_new = resc ? mx : m_use;
       const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
-      if (t > 0) {
-        const bool got = wait_bar(bar(B_PVDONE), (t - 1) & 1, p.status, abort_flag);
+      if (t >= 2) {
+        // this group's previous PV has landed in its O before O is rescaled
+        const bool got = wait_bar(bar(B_PVDONE + grp), ((t >> 1) - 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
@@ -389,11 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < V / 32; ++c) {
             uint32_t ov[32];
-            tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
+            tmem_ld32(o_addr + c * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(tmem + lane_base + 256 + c * 32, ov);
+            tmem_st32(o_addr + c * 32, ov);
           }
           tmem_wait_st();
         }
@@ -401,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (resc) l *= alpha;
       m_use = m_new;
       const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-      // pass 2: p = exp2(s - m), row sum, bf16 P into the swizzled A tile
+      // pass 2: p = exp2(s - m), row sum, bf16 P over the consumed S columns
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
@@ -411,7 +444,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float e32[32];
         if (fast) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) e32[e] = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_eff));
+          for (int e = 0; e < 32; ++e) {
+            const float x = fmaf(__uint_as_float(sv[e]), sl2, -m_eff);
+            // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
+            e32[e] = (e & 7) >= 5 ? exp2_fma(x) : exp2f(x);
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -433,46 +470,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(s_addr + c / 2, pk);
       }
       tmem_wait_st();
-      const float rs = rs0 + rs1;
-      l += rs;
+      l += rs0 + rs1;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_PFULL));
+      if (lane == 0) mbar_arrive(bar(B_PFULL + grp));
     }
-    // ---- epilogue
-    if (ok) ok = __all_sync(0xffffffffu,
-                            wait_bar(bar(B_PVDONE), (nT - 1) & 1, p.status, abort_flag));
+    // ---- epilogue: merge the two groups' (m, l, O), as split-KV partials
+    const int n0 = (nT + 1) / 2, n1 = nT / 2;  // tiles per group
+    const int nmine = grp == 0 ? n0 : n1;
+    if (ok && nmine > 0)
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(bar(B_PVDONE + grp), (nmine - 1) & 1, p.status, abort_flag));
+    sX[(grp * 2) * BM + r] = m_use;
+    sX[(grp * 2 + 1) * BM + r] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(B_XCHG));  // every warp arrives, even after an abort
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(B_XCHG), 0, p.status, abort_flag));
     if (ok) {
       tc_fence_after();
-      float m_f = m_use, scale_o;
-      if (p.sink) {
-        const float s2 = p.sink[h] * kLog2e;
-        m_f = fmaxf(m_use, s2);
-        const float a = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_f);
-        l = l * a + exp2f(s2 - m_f);
-        scale_o = a / l;
-      } else {
-        scale_o = 1.f / l;
-      }
+      const float m0 = sX[0 * BM + r], l0 = sX[1 * BM + r];
+      const float m1 = sX[2 * BM + r], l1 = sX[3 * BM + r];
+      float m_f = fmaxf(m0, m1);
+      if (p.sink) m_f = fmaxf(m_f, p.sink[h] * kLog2e);
+      const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - m_f);
+      const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - m_f);
+      float lt = l0 * a0 + l1 * a1;
+      if (p.sink) lt += exp2f(p.sink[h] * kLog2e - m_f);
+      const float inv = 1.f / lt;
+      const float f0 = a0 * inv, f1 = a1 * inv;
       __nv_bfloat16* orow = p.o + ((s0 + i) * HQ + h) * (long)V;
-#pragma unroll
-      for (int c = 0; c < V / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
+      // each group writes half of the channels; O_odd exists only if the odd
+      // group had tiles (warp-uniform)
+#pragma unroll 1
+      for (int c = grp * (V / 2); c < (grp + 1) * (V / 2); c += 32) {
+        uint32_t ov0[32], ov1[32];
+        tmem_ld32(tmem + lane_base + 256 + c, ov0);
+        if (n1 > 0) tmem_ld32(tmem + lane_base + 256 + V + c, ov1);
         tmem_wait_ld();
         if (row_ok) {
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * scale_o,
-                                __uint_as_float(ov[2 * e + 1]) * scale_o);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          for (int e = 0; e < 16; ++e) {
+            float x0 = __uint_as_float(ov0[2 * e]) * f0;
+            float x1 = __uint_as_float(ov0[2 * e + 1]) * f0;
+            if (n1 > 0) {
+              x0 = fmaf(__uint_as_float(ov1[2 * e]), f1, x0);
+              x1 = fmaf(__uint_as_float(ov1[2 * e + 1]), f1, x1);
+            }
+            pk[e] = pack_bf16x2(x0, x1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (row_ok && p.lse) p.lse[(s0 + i) * HQ + h] = (m_f + log2f(l)) * kLn2;
+      if (grp == 0 && row_ok && p.lse) p.lse[(s0 + i) * HQ + h] = (m_f + log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
