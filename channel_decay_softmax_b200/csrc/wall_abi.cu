@@ -326,9 +326,10 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
     if (rc) return rc;
   }
   // dg = reverse cumulative sum of dL (held in dq32 after the reduce)
-  rc = scan_reverse(a.dq32, dg, dtype, (long)HQ * K, pb.seqs, s);
+  // the per-head dk buffer is dead after the finalize: chunk scratch
+  rc = scan_reverse(a.dq32, dg, dtype, a.dkh32, (long)HQ * K, pb.seqs, s);
   if (rc) return rc;
-  if (g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, HQ, pb.seqs, s);
+  if (g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, a.dgs_col, HQ, pb.seqs, s);
   return rc;
 }
 

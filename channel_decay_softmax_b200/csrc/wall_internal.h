@@ -15,8 +15,8 @@ namespace wall {
 int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seqs,
                      const float* carry_in, float* carry_out, cudaStream_t stream);
 int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream);
-int scan_reverse(const float* x, void* y, int out_dtype, long C, const Seqs& seqs,
-                 cudaStream_t stream);
+int scan_reverse(const float* x, void* y, int out_dtype, float* scratch, long C,
+                 const Seqs& seqs, cudaStream_t stream);
 
 // ---- attention problem description shared by the fwd/bwd launchers ----
 struct AttnProblem {
