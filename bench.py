@@ -27,6 +27,7 @@ import os
 import statistics
 import subprocess
 import sys
+import datetime
 import tempfile
 import time
 
@@ -38,9 +39,15 @@ import torch  # noqa: E402
 from channel_decay_softmax_b200 import inputs as I  # noqa: E402
 
 METRIC = "fwd+bwd TFLOP/s & % of BF16 peak at T=8192; decode GB/s vs HBM peak"
-# DRAM bytes (read + write) of one bwd_tc_kernel launch at T=8192 from the ncu
-# capture summarized in profiles/; None once the kernel changed since.
-BWD_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) of one launch of the key-block backward kernel
+# (bwd_tc_kernel) on the T=8192 workload, from the ncu capture summarized in
+# profiles/; None once the kernel changed since that capture.
+BWD_KEY_TRAFFIC_BYTES = 267359488 + 94179072
+# algorithmic FLOPs of each tensor-core stage per launch, as multiples of the
+# forward's 2*N*(K+V): the backward's five contractions are QK^T, dO V^T, dV,
+# dK (the key-block kernel) and dq (the query-block kernel, which also
+# recomputes S and dP; recomputation is not algorithmic work)
+STAGE_FWD_MULT = {"fwd_tc": 1.0, "bwd_keyblock": 2.0, "bwd_dq": 0.5}
 TRAIN_CFG = 3
 DECODE_CFG = 5
 SM_COUNT = 148
@@ -78,10 +85,11 @@ def decode_bytes(s: I.Spec, T_kv: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
-    timed region runs."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms; start()
+    returns once the first sample is in, mark() brackets the timed region and
+    only samples stamped inside it (plus one interval after) are kept."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -89,17 +97,28 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.file = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        deadline = time.time() + 5.0
+        while time.time() < deadline and os.path.getsize(self.file.name) == 0:
+            time.sleep(0.02)
         return self
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
@@ -117,9 +136,12 @@ class ClockSampler:
         sm, smax, reasons = [], 0.0, set()
         for r in rows:
             try:
-                sm.append(float(r[1]))
-                smax = max(smax, float(r[2]))
-                for n, val in zip(names, r[5:9]):
+                stamp = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.t0 is not None and not (self.t0 <= stamp <= (self.t1 or stamp) + 0.06):
+                    continue
+                sm.append(float(r[2]))
+                smax = max(smax, float(r[3]))
+                for n, val in zip(names, r[6:10]):
                     if "Active" in val and "Not" not in val:
                         reasons.add(n)
             except (ValueError, IndexError):
@@ -128,7 +150,8 @@ class ClockSampler:
             return None
         busy = [x for x in sm if x > 0.5 * smax] or sm
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window_ms": (self.t1 - self.t0) * 1e3 if self.t0 and self.t1 else None}
 
 
 # ---------------------------------------------------------------------------
@@ -188,33 +211,41 @@ def bench_train(args, world, rank, peaks):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # the library's own per-stage events, recorded on the launch stream
+    api.timing_enable(True)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device()).start() if not args.no_clocks else None
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.mark(True)
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(False)
     barrier(world)
+    stages = api.timing_read()
+    api.timing_enable(False)
     clk = clocks.stop() if clocks else None
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, world)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    # launches of this library inside one step: prefix scan 1; forward:
-    # operand preparation 1 + tcgen05 forward 1; backward: operand preparation
-    # 1, D/sink pre-pass 1, tcgen05 key-block (dK, dV) 1, tcgen05 query-block
-    # (dq) 1, finalize 1, reverse scan 1
-    launches_per_step = 9
+    # launches of this library inside one step: prefix scan 3 (chunk sums,
+    # carries, chunk scans); forward: operand preparation 1 + tcgen05 forward
+    # 1; backward: operand preparation 1, D/sink pre-pass 1, tcgen05 key-block
+    # (dK, dV) 1, tcgen05 query-block (dq) 1, finalize 1, reverse scan 3
+    launches_per_step = 13
     res = dict(ms=ms_max, value=world * step_flops / (ms_max * 1e-3) / 1e12,
                fwd_ms=fwd_ms, bwd_ms=bwd_ms,
                fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,
                bwd_tflops=2.5 * fwd_flops / (bwd_ms * 1e-3) / 1e12,
-               launches=launches_per_step * args.steps, clocks=clk, spec=s,
+               launches=launches_per_step * args.steps, clocks=clk, spec=s, stages=stages,
                step_flops=step_flops, fwd_flops=fwd_flops)
     if not args.no_e2e:
         res["e2e"] = bench_train_e2e(args, x, s, step_flops, world)
@@ -392,7 +423,7 @@ def workload_name():
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
@@ -417,17 +448,34 @@ def main(argv=None):
     barrier(world)
     if rank == 0:
         s = tr["spec"]
-        # dominant call: the backward (tcgen05 kernel plus its preparation,
-        # finalize and reverse-scan kernels; the tcgen05 kernel is ~80% of the
-        # call in the committed ncu launch list), against the sustained bf16
-        # peak since it is timed inside a long step
+        # per-stage device time from the library's events over the timed
+        # steps; the dominant stage's roofline uses its algorithmic FLOPs per
+        # launch over its average launch time, against the sustained bf16
+        # peak since it runs inside a long step
         peak = peaks["bf16_tflops_sustained"]
-        bwd_ach = tr["bwd_tflops"]
-        roof = {"kernel": "wall_attn_bwd (bwd_tc_kernel + prep/finalize/scan)",
-                "bound": "tensor", "achieved": bwd_ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": bwd_ach / peak, "traffic": BWD_TRAFFIC_BYTES,
+        stage_rows = {}
+        for name, (n, ms) in tr["stages"].items():
+            if n == 0:
+                continue
+            row = {"launches": n, "ms_per_launch": ms / n}
+            if name in STAGE_FWD_MULT:
+                fl = STAGE_FWD_MULT[name] * tr["fwd_flops"]
+                row["algorithmic_tflop"] = fl / 1e12
+                row["tflops"] = fl / (ms / n * 1e-3) / 1e12
+            stage_rows[name] = row
+        dom = max(STAGE_FWD_MULT, key=lambda k: stage_rows.get(k, {}).get("ms_per_launch", 0.0))
+        d = stage_rows[dom]
+        roof = {"kernel": {"bwd_keyblock": "bwd_tc_kernel (key-block dK, dV)",
+                           "bwd_dq": "bwd_dq_kernel (query-block dq)",
+                           "fwd_tc": "fwd_tc_kernel"}[dom],
+                "bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
+                "frac": d["tflops"] / peak,
+                "traffic": BWD_KEY_TRAFFIC_BYTES if dom == "bwd_keyblock" else None,
                 "peak_source": f"bf16_tflops_sustained of {peaks['source']} peaks",
-                "algorithmic": "2.5 x forward causal FLOPs per launch (6.87e11 at T=8192)"}
+                "ms_per_launch": d["ms_per_launch"],
+                "algorithmic": "%.3g FLOP per launch = %g x the forward's 2*N*(K+V) summed "
+                               "over (b,h)" % (d["algorithmic_tflop"] * 1e12,
+                                               STAGE_FWD_MULT[dom])}
         line = {"metric": METRIC, "value": tr["value"], "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": tr["ms"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -437,7 +485,7 @@ def main(argv=None):
                            "parallelism": f"replicas x{world}"},
                 "frac_bf16_peak": tr["value"] / world / peaks["bf16_tflops_sustained"],
                 "fwd_tflops": tr["fwd_tflops"], "bwd_tflops": tr["bwd_tflops"],
-                "roofline": roof, "gpu_launches": tr["launches"],
+                "roofline": roof, "stages": stage_rows, "gpu_launches": tr["launches"],
                 "peaks": {k: peaks[k] for k in ("hbm_gbs", "bf16_tflops",
                                                  "bf16_tflops_sustained", "source")}}
         if tr.get("clocks"):

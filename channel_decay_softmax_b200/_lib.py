@@ -19,7 +19,8 @@ WALL_BF16, WALL_FP32 = 0, 1
 EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn_fwd_workspace",
            "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
            "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
-           "wall_selftest_wait_timeout", "wall_attn_decode_noalloc"]
+           "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
+           "wall_timing_read"]
 
 _lib = None
 
@@ -70,6 +71,11 @@ def lib():
         L.wall_attn_decode_noalloc.restype = i
         L.wall_attn_decode_noalloc.argtypes = [vp, vp, fp, vp, fp, fp, f, i, i, i, i, i, i, i, i,
                                                i, vp, fp, vp]
+        L.wall_timing_enable.restype = i
+        L.wall_timing_enable.argtypes = [i]
+        L.wall_timing_read.restype = i
+        L.wall_timing_read.argtypes = [i, ctypes.POINTER(ctypes.c_char_p),
+                                       ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
         _lib = L
     return _lib
 

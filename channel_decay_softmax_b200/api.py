@@ -207,3 +207,22 @@ class WallDecodeCache:
         """Appends one token and decodes its query; returns (o, lse)."""
         P = self.append(k, v, g)
         return self.decode(q, P[:, -1:])
+
+
+def timing_enable(on=True):
+    """Starts (clears) or stops the library's per-stage device timing: each
+    timed stage records CUDA events on the stream it runs on (wall.h,
+    wall_timing_enable)."""
+    L._check("wall_timing_enable", L.lib().wall_timing_enable(1 if on else 0))
+
+
+def timing_read():
+    """Per-stage {name: (launches, total_ms)} since the last read or enable;
+    synchronizes on the recorded events and clears the totals."""
+    import ctypes
+    n = 10
+    names = (ctypes.c_char_p * n)()
+    launches = (ctypes.c_int * n)()
+    ms = (ctypes.c_double * n)()
+    L._check("wall_timing_read", L.lib().wall_timing_read(n, names, launches, ms))
+    return {names[i].decode(): (launches[i], ms[i]) for i in range(n)}

@@ -207,7 +207,10 @@ int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ,
     int rc = check_cu(cu_seqlens, n_seq, rows, s);
     if (rc) return rc;
   }
-  return scan_prefix_log2(g, dtype, P, (long)HQ * K, seqs, carry_in, carry_out, s);
+  timing_mark(T_PREFIX, s);
+  const int rc = scan_prefix_log2(g, dtype, P, (long)HQ * K, seqs, carry_in, carry_out, s);
+  timing_mark(T_PREFIX, s);
+  return rc;
 }
 
 size_t wall_attn_fwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
@@ -327,9 +330,10 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   }
   // dg = reverse cumulative sum of dL (held in dq32 after the reduce)
   // the per-head dk buffer is dead after the finalize: chunk scratch
+  timing_mark(T_REV_SCAN, s);
   rc = scan_reverse(a.dq32, dg, dtype, a.dkh32, (long)HQ * K, pb.seqs, s);
-  if (rc) return rc;
-  if (g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, a.dgs_col, HQ, pb.seqs, s);
+  if (!rc && g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, a.dgs_col, HQ, pb.seqs, s);
+  timing_mark(T_REV_SCAN, s);
   return rc;
 }
 
@@ -343,8 +347,11 @@ int wall_build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn,
   if (K < 8 || K % 8 != 0) return WALL_ERR_UNSUPPORTED;
   if ((long)B * Tn == 0) return WALL_OK;
   if (!ok_ptr(k) || !ok_ptr(P) || !ok_ptr(k_tilde) || !ok_ptr(r_cache)) return WALL_ERR_INVALID_ARG;
-  return build_kv_cache(k, P, dtype, B, Tn, H, HQ, K, C, t0, k_tilde, r_cache, Tcap,
-                        reinterpret_cast<cudaStream_t>(stream));
+  timing_mark(T_CACHE, reinterpret_cast<cudaStream_t>(stream));
+  const int rc = build_kv_cache(k, P, dtype, B, Tn, H, HQ, K, C, t0, k_tilde, r_cache, Tcap,
+                                reinterpret_cast<cudaStream_t>(stream));
+  timing_mark(T_CACHE, reinterpret_cast<cudaStream_t>(stream));
+  return rc;
 }
 
 size_t wall_attn_decode_workspace(int B, int T_kv, int H, int HQ, int V, int C) {
@@ -371,9 +378,12 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
     return WALL_ERR_INVALID_ARG;
   const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)K);
-  return attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, sc, C, dtype, B, T_kv, Tcap, H,
-                     HQ, K, V, o, lse, static_cast<float*>(workspace), S,
-                     reinterpret_cast<cudaStream_t>(stream));
+  timing_mark(T_DECODE, reinterpret_cast<cudaStream_t>(stream));
+  const int rc = attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, sc, C, dtype, B, T_kv,
+                             Tcap, H, HQ, K, V, o, lse, static_cast<float*>(workspace), S,
+                             reinterpret_cast<cudaStream_t>(stream));
+  timing_mark(T_DECODE, reinterpret_cast<cudaStream_t>(stream));
+  return rc;
 }
 
 }  // extern "C"

@@ -740,8 +740,11 @@ int launch_bwd_tc_gs(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws,
 int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void* dq, void* dk,
                 void* dv, int* status, cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
+  timing_mark(T_OPERANDS, stream);
   int rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
+  timing_mark(T_OPERANDS, stream);
   if (rc) return rc;
+  timing_mark(T_BWD_PRE, stream);
   {
     const long threads = pb.rows * pb.HQ * 8;
     const int blocks = (int)((threads + 255) / 256);
@@ -750,17 +753,24 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void
         a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr, a.dsink);
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
   }
+  timing_mark(T_BWD_PRE, stream);
+  timing_mark(T_BWD_KEY, stream);
   rc = pb.K == 128 ? launch_bwd_tc_gs<128>(pb, a, ws, status, stream)
                    : launch_bwd_tc_gs<64>(pb, a, ws, status, stream);
+  timing_mark(T_BWD_KEY, stream);
   if (rc) return rc;
+  timing_mark(T_BWD_DQ, stream);
   rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
+  timing_mark(T_BWD_DQ, stream);
   if (rc) return rc;
+  timing_mark(T_BWD_FIN, stream);
   dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
   bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.P,
       pb.seqs, pb.HQ, pb.H, pb.K, pb.V, pb.scale, a.dq32, a.dkh32, a.dvh32,
       a.GS ? a.dgs_row : nullptr, a.GS ? a.dgs_col : nullptr, static_cast<__nv_bfloat16*>(dq),
       static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+  timing_mark(T_BWD_FIN, stream);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

@@ -643,10 +643,15 @@ int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, c
 int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
                 cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
+  timing_mark(T_OPERANDS, stream);
   int rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
+  timing_mark(T_OPERANDS, stream);
   if (rc) return rc;
-  return pb.K == 128 ? launch_fwd_tc<128>(pb, a, ws, status, stream)
-                     : launch_fwd_tc<64>(pb, a, ws, status, stream);
+  timing_mark(T_FWD, stream);
+  rc = pb.K == 128 ? launch_fwd_tc<128>(pb, a, ws, status, stream)
+                   : launch_fwd_tc<64>(pb, a, ws, status, stream);
+  timing_mark(T_FWD, stream);
+  return rc;
 }
 
 }  // namespace wall

@@ -11,6 +11,14 @@
 
 namespace wall {
 
+// ---- per-stage timing (wall_timing.cu): records an event on `stream` for
+// `slot` while timing is enabled; calls come in begin / end pairs ----
+void timing_mark(int slot, cudaStream_t stream);
+enum TimingSlot {
+  T_PREFIX = 0, T_OPERANDS = 1, T_FWD = 2, T_BWD_PRE = 3, T_BWD_KEY = 4, T_BWD_DQ = 5,
+  T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9,
+};
+
 // ---- scans (wall_scan.cu) ----
 int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seqs,
                      const float* carry_in, float* carry_out, cudaStream_t stream);

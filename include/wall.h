@@ -226,6 +226,37 @@ int wall_get_status(wall_stream_t stream);
  */
 int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
 
+/*
+ * Per-stage device timing, for measurement (a profiling aid with no
+ * counterpart on the pages).  While enabled, every launch of a timed stage
+ * is bracketed by two CUDA events recorded on the stream the stage runs on;
+ * the events are the library's own and are reused.  Stages (slot: name):
+ *   0 prefix_scan     the three kernels of wall_prefix_cumsum
+ *   1 operands        anchored-operand preparation (fwd and bwd each)
+ *   2 fwd_tc          tensor-core forward
+ *   3 bwd_pre         D / sink pre-pass
+ *   4 bwd_keyblock    tensor-core key-block backward (dK, dV)
+ *   5 bwd_dq          tensor-core query-block backward (dq)
+ *   6 bwd_finalize    dq scaling, gate-gradient summand, GQA sums
+ *   7 reverse_scan    the reverse scan(s) of wall_attn_bwd
+ *   8 decode          wall_attn_decode (split and merge kernels)
+ *   9 cache_build     wall_build_kv_cache
+ * wall_timing_enable(1) starts recording (and clears the totals);
+ * wall_timing_enable(0) stops.  Not thread-safe: one host thread at a time.
+ */
+#define WALL_TIMING_SLOTS 10
+int wall_timing_enable(int on);
+
+/*
+ * wall_timing_read -- for slots [0, n) (n <= WALL_TIMING_SLOTS) writes the
+ * number of timed launches since the last read (or enable) and their total
+ * device time in milliseconds, then clears them.  Synchronizes on the
+ * recorded events.  `launches` and `ms` are host arrays of n entries; `names`
+ * may be NULL, else it receives n static strings.  Returns WALL_ERR_CUDA if
+ * an event query fails, WALL_ERR_INVALID_ARG for a bad n or null array.
+ */
+int wall_timing_read(int n, const char** names, int* launches, double* ms);
+
 #ifdef __cplusplus
 }
 #endif
