@@ -15,8 +15,8 @@
 // two and Kt_J = Kh_J (.) d is an exact packed bf16 multiply, done in place.
 //
 // CTA = 12 warps (3 per SM sub-partition, 168 registers each):
-//   warp 0      TMA: Qh_I, dO_I once; Kh_J (+ block anchors, 3 stages) and V_J
-//               (1 stage: it is read by one MMA only) per key tile
+//   warp 0      TMA, lane 0: Qh_I, dO_I once and the key ring (Kh_J with its
+//               block anchors, 4 stages); lane 1: the value ring (1 stage)
 //   warp 1      TMEM owner and MMA issuer.  Per tile: dP(t+1) as soon as the
 //               softmax has read dP(t), then dQa(t), then S(t+2)
 //   warps 2-3   key rescale Kt_J = Kh_J (.) d in place; each thread keeps one
@@ -39,7 +39,8 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kKS = 3;  // key stages
+constexpr int kKS = 4;  // key stages: the refill (TMA + in-place scaling) spans a tile
+constexpr int kVS = 1;  // value stages
 constexpr int kThreads = 384;
 
 struct DqParams {
@@ -62,29 +63,33 @@ struct DSmem {
   static constexpr int oQ = 0;
   static constexpr int oO = oQ + kT;
   static constexpr int oK = oO + kT;           // kKS stages
-  static constexpr int oV = oK + kKS * kT;     // 1 stage
-  static constexpr int oRI = oV + kT;          // float[KD]
+  static constexpr int oV = oK + kKS * kT;     // kVS stages
+  static constexpr int oRI = oV + kVS * kT;    // float[KD]
   static constexpr int oRJ = oRI + KD * 4;     // float[kKS][KD]
-  static constexpr int oGS = oRJ + kKS * KD * 4;  // float[8 warps][64]: key prefix
-  static constexpr int oBar = oGS + 8 * 64 * 4;
-  static constexpr int kBars = 16;
+  static constexpr int oBar = oRJ + kKS * KD * 4;
+  static constexpr int kBars = 20;  // >= kNumBars
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;
+  // no alignment slack: the shared window is used from its start, which the
+  // kernel checks is 1 KB aligned (the 128-byte swizzle atoms need it)
+  static constexpr int kAlloc = kBytes;
 };
 
 enum DBar {
   QO_FULL = 0,
-  K_FULL = 1,    // + stage (3)
-  K_READY = 4,   // + stage (3)
-  K_EMPTY = 7,   // + stage (3)
-  V_FULL = 10,
-  V_EMPTY = 11,
-  SD_FULL = 12,
-  P_FULL = 13,
-  DQ_DONE = 14,
-  MMA_DONE = 15,
+  K_FULL = 1,                    // + stage (kKS)
+  K_READY = K_FULL + kKS,        // + stage
+  K_EMPTY = K_READY + kKS,       // + stage
+  V_FULL = K_EMPTY + kKS,        // + stage (kVS)
+  V_EMPTY = V_FULL + kVS,        // + stage
+  SD_FULL = V_EMPTY + kVS,
+  P_FULL = SD_FULL + 1,
+  DQ_DONE = P_FULL + 1,
+  MMA_DONE = DQ_DONE + 1,
+  kNumBars = MMA_DONE + 1,
 };
+static_assert(kNumBars <= DSmem<128>::kBars, "barrier slots");
+static_assert(DSmem<128>::kAlloc <= 227 * 1024, "shared memory");
 
 // 2^k as bf16 bits for an integer k (the anchors are integers): exact in
 // the normal range, 0 below it (a factor under 2^-126 scales a key that
@@ -123,11 +128,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                   DqParams p) {
   using Lay = DSmem<KD>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // uniform: every thread returns before any barrier
+    if (threadIdx.x == 0) record_status(p.status, WALL_ERR_UNSUPPORTED);
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
-  float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
@@ -157,8 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(K_READY + s), 2);
       mbar_init(bar(K_EMPTY + s), 1);
     }
-    mbar_init(bar(V_FULL), 1);
-    mbar_init(bar(V_EMPTY), 1);
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(bar(V_FULL + s), 1);
+      mbar_init(bar(V_EMPTY + s), 1);
+    }
     mbar_init(bar(SD_FULL), 1);
     mbar_init(bar(P_FULL), 8);
     mbar_init(bar(DQ_DONE), 1);
@@ -179,10 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
+    // lane 0: Qh, dO and the key ring; lane 1: the value ring.  The two lanes
+    // wait on different barriers and progress independently.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
       mbar_expect_tx(bar(QO_FULL), 2 * Lay::kT);
       for (int b = 0; b < K / 64; ++b) {
@@ -191,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sbase + Lay::oO + b * (BM * 128), &tm_o, bar(QO_FULL), b * 64, h,
                     (int)(s0 + i0));
       }
-      int k_issued = 0, v_issued = 0;
+      int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t % kKS;
         const int row = (int)(s0 + (long)(jb_lo + t) * BN);
@@ -205,17 +215,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(sbase + Lay::oRJ + st * K * 4,
                   p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
                   bar(K_FULL + st));
-        k_issued = t + 1;
-        if (t >= 1 && !wait_bar(bar(V_EMPTY), (t - 1) & 1, p.status, abort_flag)) break;
-        mbar_expect_tx(bar(V_FULL), Lay::kT);
-        for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oV + b * (BN * 128), &tm_v, bar(V_FULL), b * 64, kh, row);
-        v_issued = t + 1;
+        issued = t + 1;
       }
-      for (int t = max(0, k_issued - kKS); t < k_issued; ++t)
+      for (int t = max(0, issued - kKS); t < issued; ++t)
         mbar_wait(bar(K_FULL + t % kKS), (t / kKS) & 1, p.status);
-      if (v_issued > 0) mbar_wait(bar(V_FULL), (v_issued - 1) & 1, p.status);
       mbar_wait(bar(QO_FULL), 0, p.status);
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kVS;
+        if (t >= kVS && !wait_bar(bar(V_EMPTY + st), (t / kVS - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(V_FULL + st), Lay::kT);
+        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v, bar(V_FULL + st),
+                      b * 64, kh, row);
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - kVS); t < issued; ++t)
+        mbar_wait(bar(V_FULL + t % kVS), (t / kVS) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
@@ -238,15 +258,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_dp = [&](int t) -> bool {
-        if (!wait_bar(bar(V_FULL), t & 1, p.status, abort_flag)) return false;
+        const int vs = t % kVS;
+        if (!wait_bar(bar(V_FULL + vs), (t / kVS) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
           umma_bf16_ss(tmem + kColDP, sdesc_sw128(sbase + Lay::oO + off, 16, 1024),
-                       sdesc_sw128(sbase + Lay::oV + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                       sdesc_sw128(sbase + Lay::oV + vs * Lay::kT + off, 16, 1024), id_s,
+                       kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(V_EMPTY));
+        umma_commit(bar(V_EMPTY + vs));
         umma_commit(bar(SD_FULL));  // S(t) was issued earlier: both are ready
         return true;
       };
@@ -341,18 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gs_i = (has_gs && row_ok) ? p.GS[grow] * kLog2e : 0.f;
     const float sl2 = p.scale_log2;
     const float off_i = (has_gs ? gs_i : 0.f) - lse2;
-    float* gsk = sGS + (warp - 4) * 64;  // this warp's copy of the key prefix (or zeros)
     bool ok = true;
     for (int t = 0; t < nT; ++t) {
       const int j0 = (jb_lo + t) * BN + half * 64;  // first key of this half
-      if (has_gs || t == 0) {
-        __syncwarp();
-        for (int c = lane; c < 64; c += 32) {
-          const int j = j0 + c;
-          gsk[c] = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
-        }
-        __syncwarp();
-      }
       {
         const bool got = wait_bar(bar(SD_FULL), t & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -390,7 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < 2; ++x) {
               const int j = j0 + c + e + x;
               const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
-              const float a = fmaf(__uint_as_float(sv[e + x]), sl2, off_i - gsk[c + e + x]);
+              // the key prefix of the scalar gate, straight from global
+              // memory (L1-resident across the warp; this path is rare)
+              const float gk = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
+              const float a = fmaf(__uint_as_float(sv[e + x]), sl2, off_i - gk);
               const float pv = vis ? exp2f(a) : 0.f;
               ds[x] = pv * (__uint_as_float(dv[e + x]) - Di);
             }
