@@ -148,6 +148,9 @@ BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
 inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
 }  // namespace
+
+int* device_status() { return status_ptr(); }
+
 }  // namespace wall
 
 using namespace wall;

@@ -14,11 +14,19 @@
 // lane scores one key per 32-key step with 16-byte loads, keeps an online
 // softmax in the log2 domain, and accumulates o with warp shuffles of p.
 // Splits are merged by their (max, sum) pairs in a second small kernel.
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "sm100_ptx.cuh"
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
 namespace wall {
 namespace {
+
+using namespace sm100;
+using T_bf16 = __nv_bfloat16;
 
 template <typename T>
 __global__ void cache_kernel(const T* __restrict__ k, const float* __restrict__ P, int B, int Tn,
@@ -191,6 +199,256 @@ __global__ void decode_split_kernel(DecodeArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming decode (bf16, K, V in {64, 128}, G <= 8, C a multiple of 32): a
+// persistent grid, one CTA per SM, walks (batch row, kv head, key range)
+// work items.  The last warp's lane 0 keeps a ring of TMA stages full: per
+// 32-key tile the G heads' k_tilde boxes, the value box and the chunk's
+// anchors, about 40 KB in flight per stage, so HBM sees long bulk reads
+// instead of per-lane gathers.  Each query head has WPH warps that take
+// alternate tiles with their own online-softmax state, merged at the end of
+// the item through shared memory: lane = key for the scores (the 128-byte
+// swizzle makes the 32 rows conflict-free, four independent accumulators),
+// then lane = VD/32 value channels for P V.  Partials go to the same
+// workspace as the split kernel above and are merged the same way.
+constexpr int kDecTile = 32;
+
+template <int KD, int VD, int WPH>
+__global__ void __launch_bounds__(32 * 9, 1)
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, DecodeArgs a, int G,
+                         int n_items, int stages, int stage_bytes, int* status) {
+  constexpr int VPL = VD / 32;  // value channels per lane
+  constexpr int QPL = KD / 32;  // query channels per lane (for the scaled query)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  constexpr int kKBox = kDecTile * 128;             // one 64-channel box of 32 rows
+  const int oV = G * (KD / 64) * kKBox;             // within a stage
+  const int oR = oV + (VD / 64) * kKBox;            // anchors [G][KD] fp32
+  const int nw = G * WPH;                           // consumer warps
+  float* qts = reinterpret_cast<float*>(smem + stages * stage_bytes);  // [nw][KD]
+  float* xch = qts + nw * KD;                       // [G][32][VPL + 2]: second warp's state
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xch + G * 32 * (VPL + 2));
+  auto full = [&](int st) { return smem_u32(&bars[st]); };
+  auto empty = [&](int st) { return smem_u32(&bars[stages + st]); };
+  auto xfull = [&](int g) { return smem_u32(&bars[2 * stages + g]); };
+  auto xempty = [&](int g) { return smem_u32(&bars[2 * stages + G + g]); };
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int NC = (a.Tcap + a.C - 1) / a.C;
+  const int kps = a.keys_per_split;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), G);  // the G warps (one per head) that take the tile
+    }
+    for (int g = 0; g < G; ++g) {
+      mbar_init(xfull(g), 1);
+      mbar_init(xempty(g), 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto item_of = [&](int it, int& b, int& kh, int& s) {
+    s = it % a.splits;
+    kh = (it / a.splits) % a.H;
+    b = it / (a.splits * a.H);
+  };
+  if (warp == nw) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint32_t bytes = (uint32_t)(oR + G * KD * 4);
+      long seq = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        int b, kh, s;
+        item_of(it, b, kh, s);
+        const long k0 = (long)s * kps, k1 = min((long)a.T_kv, k0 + kps);
+        for (long j0 = k0; j0 < k1; j0 += kDecTile, ++seq) {
+          const int st = (int)(seq % stages);
+          if (seq >= stages && !mbar_wait(empty(st), (uint32_t)((seq / stages - 1) & 1), status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(full(st), bytes);
+          const uint32_t sb = sbase + st * stage_bytes;
+          const int row = (int)((long)b * a.Tcap + j0);
+          for (int g = 0; g < G; ++g)
+            for (int bx = 0; bx < KD / 64; ++bx)
+              tma_load_3d(sb + (g * (KD / 64) + bx) * kKBox, &tm_k, full(st), bx * 64,
+                          kh * G + g, row);
+          for (int bx = 0; bx < VD / 64; ++bx)
+            tma_load_3d(sb + oV + bx * kKBox, &tm_v, full(st), bx * 64, kh, row);
+          const long c = j0 / a.C;
+          bulk_load(sb + oR, a.rc + (((long)b * NC + c) * a.HQ + (long)kh * G) * KD, G * KD * 4,
+                    full(st));
+        }
+      }
+      // no copy may still be landing when the CTA exits
+      for (long q = seq > stages ? seq - stages : 0; q < seq; ++q)
+        mbar_wait(full((int)(q % stages)), (uint32_t)((q / stages) & 1), status);
+    }
+  } else if (warp < nw) {
+    // ------------------------------------------------------------ query heads
+    const int g = warp % G, par = warp / G;  // head of the group; which tiles
+    const T_bf16* q = static_cast<const T_bf16*>(a.q);
+    const float sl2 = a.scale * kLog2e;
+    float* qt = qts + warp * KD;
+    float* xs = xch + (g * 32 + lane) * (VPL + 2);
+    long seq = 0;
+    int n_it = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++n_it) {
+      int b, kh, s;
+      item_of(it, b, kh, s);
+      const int h = kh * G + g;
+      const long k0 = (long)s * kps, k1 = min((long)a.T_kv, k0 + kps);
+      const long qoff = ((long)b * a.HQ + h) * KD;
+      float qv[QPL], pv[QPL];
+#pragma unroll
+      for (int i = 0; i < QPL; ++i) {
+        qv[i] = to_f32(q[qoff + lane * QPL + i]);
+        pv[i] = a.pc[qoff + lane * QPL + i];
+      }
+      float m = -INFINITY, l = 0.f, acc[VPL];
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+      long c_last = -1;
+      for (long j0 = k0; ok && j0 < k1; j0 += kDecTile, ++seq) {
+        if ((((j0 - k0) / kDecTile) % WPH) != par) continue;  // the other warp's tile
+        const int st = (int)(seq % stages);
+        {
+          const bool got = mbar_wait(full(st), (uint32_t)((seq / stages) & 1), status);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        }
+        const uint8_t* sb = smem + st * stage_bytes;
+        const long c = j0 / a.C;
+        if (c != c_last) {
+          // the query scaled for this chunk: scale*log2e * q * 2^(p_curr - R_c)
+          const float* R = reinterpret_cast<const float*>(sb + oR) + g * KD;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < QPL; ++i)
+            qt[lane * QPL + i] = sl2 * qv[i] * exp2f(pv[i] - R[lane * QPL + i]);
+          __syncwarp();
+          c_last = c;
+        }
+        // scores: lane = key of the tile, four independent partial sums
+        const int r = lane;
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int bx = 0; bx < KD / 64; ++bx) {
+          const uint8_t* krow = sb + (g * (KD / 64) + bx) * kKBox + r * 128;
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(krow + ((c8 ^ (r & 7)) << 4));
+            const float4 qa = *reinterpret_cast<const float4*>(qt + bx * 64 + c8 * 8);
+            const float4 qb = *reinterpret_cast<const float4*>(qt + bx * 64 + c8 * 8 + 4);
+            const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+            const float2 f0 = __bfloat1622float2(hv[0]), f1 = __bfloat1622float2(hv[1]);
+            const float2 f2 = __bfloat1622float2(hv[2]), f3 = __bfloat1622float2(hv[3]);
+            d4[0] = fmaf(f0.x, qa.x, d4[0]); d4[1] = fmaf(f0.y, qa.y, d4[1]);
+            d4[2] = fmaf(f1.x, qa.z, d4[2]); d4[3] = fmaf(f1.y, qa.w, d4[3]);
+            d4[0] = fmaf(f2.x, qb.x, d4[0]); d4[1] = fmaf(f2.y, qb.y, d4[1]);
+            d4[2] = fmaf(f3.x, qb.z, d4[2]); d4[3] = fmaf(f3.y, qb.w, d4[3]);
+          }
+        }
+        const bool valid = j0 + r < k1;
+        const float sc = valid ? (d4[0] + d4[1]) + (d4[2] + d4[3]) : -INFINITY;
+        float mt = sc;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float m_new = fmaxf(m, mt);
+        const float alpha = exp2f(m - m_new);
+        const float p = valid ? exp2f(sc - m_new) : 0.f;
+        float ps = p;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l = l * alpha + ps;
+        m = m_new;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) acc[i] *= alpha;
+        // P V: lane = VPL value channels; keys past the range are skipped (their
+        // rows may hold anything)
+        const int nk = (int)min((long)kDecTile, k1 - j0);
+        const int vbx = (lane * VPL) / 64, vch = (lane * VPL) % 64;
+        const uint8_t* vbase = sb + oV + vbx * kKBox + (vch % 8) * 2;
+        if (nk == kDecTile) {
+#pragma unroll
+          for (int jj = 0; jj < kDecTile; ++jj) {
+            const float pj = __shfl_sync(0xffffffffu, p, jj);
+            const uint8_t* vp = vbase + jj * 128 + (((vch / 8) ^ (jj & 7)) << 4);
+            float x[VPL];
+            if constexpr (VPL == 4) {
+              const uint2 u = *reinterpret_cast<const uint2*>(vp);
+              const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+              const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+              x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+            } else {
+              const uint32_t u = *reinterpret_cast<const uint32_t*>(vp);
+              const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+              x[0] = f0.x; x[1] = f0.y;
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) acc[i] = fmaf(pj, x[i], acc[i]);
+          }
+        } else {
+          for (int jj = 0; jj < nk; ++jj) {
+            const float pj = __shfl_sync(0xffffffffu, p, jj);
+            const uint8_t* vp = vbase + jj * 128 + (((vch / 8) ^ (jj & 7)) << 4);
+            const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(vp);
+#pragma unroll
+            for (int i = 0; i < VPL; i += 2) {
+              const float2 f = __bfloat1622float2(hv[i / 2]);
+              acc[i] = fmaf(pj, f.x, acc[i]);
+              acc[i + 1] = fmaf(pj, f.y, acc[i + 1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(st));
+      }
+      if (!__all_sync(0xffffffffu, ok)) ok = false;
+      // the head's warps meet: the second hands its state to the first
+      if (WPH == 2 && par == 1) {
+        const bool got = n_it == 0 || mbar_wait(xempty(g), (uint32_t)((n_it - 1) & 1), status);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) xs[i] = acc[i];
+        xs[VPL] = m;
+        xs[VPL + 1] = l;
+        __syncwarp();
+        if (lane == 0 && got) mbar_arrive(xfull(g));
+        continue;
+      }
+      if (WPH == 2) {
+        const bool got = mbar_wait(xfull(g), (uint32_t)(n_it & 1), status);
+        if (got) {
+          const float m1 = xs[VPL], l1 = xs[VPL + 1];
+          const float mt = fmaxf(m, m1);
+          const float a0 = (m == -INFINITY) ? 0.f : exp2f(m - mt);
+          const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mt);
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) acc[i] = acc[i] * a0 + xs[i] * a1;
+          l = l * a0 + l1 * a1;
+          m = mt;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xempty(g));
+      }
+      const long part = ((long)b * a.HQ + h) * a.splits + s;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) a.ws_o[part * VD + lane * VPL + i] = acc[i];
+      if (lane == 0) {
+        a.ws_ml[part * 2] = m;
+        a.ws_ml[part * 2 + 1] = l;
+      }
+    }
+  }
+}
+
 template <typename T>
 __global__ void decode_merge_kernel(DecodeArgs a, T* __restrict__ o, float* __restrict__ lse) {
   const int h = blockIdx.x, b = blockIdx.y;
@@ -224,9 +482,67 @@ int launch_decode(const DecodeArgs& a, T* o, float* lse, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
+// the streaming kernel's shared memory: stages of (G heads' key boxes, the
+// value box, anchors), the scaled queries and the barriers
+template <int KD, int VD, int WPH>
+int launch_decode_stream(const DecodeArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
+  const int G = a.HQ / a.H;
+  CUtensorMap tk, tv;
+  if (!make_tile_map(&tk, a.kt, (long)a.B * a.Tcap, a.HQ, KD, kDecTile) ||
+      !make_tile_map(&tv, a.v, (long)a.B * a.Tcap, a.H, VD, kDecTile))
+    return WALL_ERR_CUDA;
+  const int oR = G * (KD / 64) * kDecTile * 128 + (VD / 64) * kDecTile * 128;
+  const int stage_bytes = (oR + G * KD * 4 + 1023) & ~1023;
+  const int tail = G * WPH * KD * 4 + G * 32 * (VD / 32 + 2) * 4 + (2 * 4 + 2 * G) * 8;
+  const int budget = 227 * 1024 - 1024 - tail;
+  int stages = budget / stage_bytes;
+  if (stages > 4) stages = 4;
+  if (stages < 2) return WALL_ERR_UNSUPPORTED;
+  const int smem = stages * stage_bytes + tail + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(decode_stream_kernel<KD, VD, WPH>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    attr = true;
+  }
+  const int n_items = a.B * a.H * a.splits;
+  const int grid = n_items < 148 ? n_items : 148;
+  decode_stream_kernel<KD, VD, WPH><<<grid, 32 * (G * WPH + 1), smem, stream>>>(
+      tk, tv, a, G, n_items, stages, stage_bytes, device_status());
+  if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+  decode_merge_kernel<__nv_bfloat16><<<dim3(a.HQ, a.B), 128, 0, stream>>>(a, o, lse);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
 template <typename T>
 int decode_dispatch(const DecodeArgs& a, void* o, float* lse, cudaStream_t s) {
   T* out = static_cast<T*>(o);
+  const int G = a.H > 0 ? a.HQ / a.H : 0;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // the streaming kernel: bf16, K and V in {64, 128}, up to 8 query heads
+    // per kv head, tiles of 32 keys that never straddle a cache chunk, and
+    // 16-byte aligned operands for the bulk copies
+    const bool aligned = ((reinterpret_cast<uintptr_t>(a.kt) | reinterpret_cast<uintptr_t>(a.v) |
+                           reinterpret_cast<uintptr_t>(a.rc)) & 15) == 0;
+    if ((a.K == 64 || a.K == 128) && (a.V == 64 || a.V == 128) && G >= 1 && G <= 8 &&
+        a.C % kDecTile == 0 && aligned) {
+      // two warps per query head while they fit in the 9-warp CTA
+      int rc;
+      if (G <= 4) {
+        if (a.K == 128 && a.V == 128) rc = launch_decode_stream<128, 128, 2>(a, out, lse, s);
+        else if (a.K == 128) rc = launch_decode_stream<128, 64, 2>(a, out, lse, s);
+        else if (a.V == 128) rc = launch_decode_stream<64, 128, 2>(a, out, lse, s);
+        else rc = launch_decode_stream<64, 64, 2>(a, out, lse, s);
+      } else {
+        if (a.K == 128 && a.V == 128) rc = launch_decode_stream<128, 128, 1>(a, out, lse, s);
+        else if (a.K == 128) rc = launch_decode_stream<128, 64, 1>(a, out, lse, s);
+        else if (a.V == 128) rc = launch_decode_stream<64, 128, 1>(a, out, lse, s);
+        else rc = launch_decode_stream<64, 64, 1>(a, out, lse, s);
+      }
+      if (rc != WALL_ERR_UNSUPPORTED) return rc;
+    }
+  }
   const bool k64 = a.K <= 64, v64 = a.V <= 64;
   if (k64 && v64) return launch_decode<T, 64, 64>(a, out, lse, s);
   if (k64) return launch_decode<T, 64, 128>(a, out, lse, s);

@@ -98,6 +98,9 @@ int attn_bwd_reduce(const AttnProblem& pb, const BwdArgs& a, void* dq, void* dk,
 int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ, int K,
                    int C, int t0, void* k_tilde, float* r_cache, int Tcap, cudaStream_t stream);
 int decode_splits(int B, int T_kv, int H, int C);
+// the device status word kernels record bounded-wait timeouts in (wall_abi.cu)
+int* device_status();
+
 int attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,
                 const float* r_cache, const float* sink, float scale, int C, int dtype, int B,
                 int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
