@@ -298,7 +298,8 @@ def bench_train_e2e(args, x, s, step_flops, world):
 def bench_decode(args, rank, peaks):
     from channel_decay_softmax_b200 import api
 
-    s = I.spec(DECODE_CFG, seed=I.CONFIGS[DECODE_CFG].seed + 7919 * rank)
+    over = {"B": args.decode_batch} if args.decode_batch else {}
+    s = I.spec(DECODE_CFG, seed=I.CONFIGS[DECODE_CFG].seed + 7919 * rank, **over)
     d = I.decode_inputs(s, device="cuda", n_query_rows=64)
     T = s.T
     n_stream = 64
@@ -427,6 +428,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
+    # a smaller decode batch, for profiler captures (the reported decode line
+    # is the full workload only without this flag)
+    ap.add_argument("--decode-batch", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
