@@ -105,6 +105,7 @@ enum BBar {
   MM_DONE = 16,
   MMA_DONE = 17,
   COL_READY = 18,  // 4 warps of the second half: column sums in shared memory
+  EPI_STAGED = 19, // 8 softmax warps: dK, dV staged in shared memory
 };
 
 // TMEM columns (lanes = keys): S^T [0,128), dP^T [128,256), dV [256,384),
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(MM_DONE), 1);
     mbar_init(bar(MMA_DONE), 1);
     mbar_init(bar(COL_READY), 4);
+    mbar_init(bar(EPI_STAGED), 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -525,36 +527,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(DS_READY));
     }
-    // ---- dK, dV epilogue for this key block: each half takes half the channels
+    // ---- dK, dV epilogue.  Thread = key row in TMEM, but a row per thread
+    // makes every global access of a warp touch 32 rows: the accumulators go
+    // through shared memory (free once every MMA has completed), then each
+    // warp writes whole rows.  Staging layout: fp32 [2][BK][KD], 16-byte group
+    // g of row r at group g ^ (r & 7), so both the row-wise writes and the
+    // column-wise reads spread over all banks.
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(MM_DONE), 0, p.status, abort_flag));
+    float* stage = reinterpret_cast<float*>(smem);  // the K, V, query and dO buffers
     if (ok) {
       tc_fence_after();
-      const long krow = (s0 + jj) * HQ + h;
 #pragma unroll 1
       for (int c = half * (KD / 2); c < (half + 1) * (KD / 2); c += 32) {
         uint32_t kv[32], vv[32];
         tmem_ld32(tmem + lane_base + kColDK + c, kv);
         tmem_ld32(tmem + lane_base + kColDV + c, vv);
         tmem_wait_ld();
-        if (key_ok) {
-          const float* Pj = p.P + krow * K + c;
-          const float* Rj = anc + (long)blk * HQ * K + c;
-          float* dk = p.dkh32 + krow * K + c;
-          float* dvp = p.dvh32 + krow * V + c;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 pj = *reinterpret_cast<const float4*>(Pj + e);
-            const float4 rj = *reinterpret_cast<const float4*>(Rj + e);
-            float4 o;
-            o.x = p.scale * exp2f(rj.x - pj.x) * __uint_as_float(kv[e]);
-            o.y = p.scale * exp2f(rj.y - pj.y) * __uint_as_float(kv[e + 1]);
-            o.z = p.scale * exp2f(rj.z - pj.z) * __uint_as_float(kv[e + 2]);
-            o.w = p.scale * exp2f(rj.w - pj.w) * __uint_as_float(kv[e + 3]);
-            *reinterpret_cast<float4*>(dk + e) = o;
-            *reinterpret_cast<float4*>(dvp + e) =
-                make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
-                            __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]));
-          }
+        for (int e = 0; e < 32; e += 4) {
+          const int pos = r * KD + ((((c + e) >> 2) ^ (r & 7)) << 2);
+          *reinterpret_cast<float4*>(stage + pos) =
+              make_float4(__uint_as_float(kv[e]), __uint_as_float(kv[e + 1]),
+                          __uint_as_float(kv[e + 2]), __uint_as_float(kv[e + 3]));
+          *reinterpret_cast<float4*>(stage + BK * KD + pos) =
+              make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
+                          __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]));
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(EPI_STAGED));  // every warp arrives, even after an abort
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(EPI_STAGED), 0, p.status, abort_flag));
+    if (ok) {
+      // warp w takes rows w, w + 8, ...; lane = KD/32 consecutive channels;
+      // dk_j = scale 2^(R_J - P_j) dKa_j
+      constexpr int CPL = KD / 32;
+      const int c0 = lane * CPL;
+      float rjv[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) rjv[i] = anc[(long)blk * HQ * K + c0 + i];
+      // every P load of the warp's 16 rows in flight before the first use
+      constexpr int kRowsPerWarp = BK / 8;
+      float pj[kRowsPerWarp][CPL];
+#pragma unroll
+      for (int x = 0; x < kRowsPerWarp; ++x) {
+        const int rr = (warp - 4) + 8 * x;
+        const long krow = (s0 + j0 + (rr < nj ? rr : 0)) * HQ + h;
+        if constexpr (CPL == 4) {
+          const float4 a = *reinterpret_cast<const float4*>(p.P + krow * K + c0);
+          pj[x][0] = a.x; pj[x][1] = a.y; pj[x][2 % CPL] = a.z; pj[x][3 % CPL] = a.w;
+        } else {
+          const float2 a = *reinterpret_cast<const float2*>(p.P + krow * K + c0);
+          pj[x][0] = a.x; pj[x][1 % CPL] = a.y;
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < kRowsPerWarp; ++x) {
+        const int rr = (warp - 4) + 8 * x;
+        if (rr >= nj) break;
+        const long krow = (s0 + j0 + rr) * HQ + h;
+        const int pos = rr * KD + (((c0 >> 2) ^ (rr & 7)) << 2) + (c0 & 3);
+        float ka[CPL], va[CPL], ko[CPL];
+        if constexpr (CPL == 4) {
+          const float4 b = *reinterpret_cast<const float4*>(stage + pos);
+          const float4 d = *reinterpret_cast<const float4*>(stage + BK * KD + pos);
+          ka[0] = b.x; ka[1] = b.y; ka[2 % CPL] = b.z; ka[3 % CPL] = b.w;
+          va[0] = d.x; va[1] = d.y; va[2 % CPL] = d.z; va[3 % CPL] = d.w;
+        } else {
+          const float2 b = *reinterpret_cast<const float2*>(stage + pos);
+          const float2 d = *reinterpret_cast<const float2*>(stage + BK * KD + pos);
+          ka[0] = b.x; ka[1 % CPL] = b.y;
+          va[0] = d.x; va[1 % CPL] = d.y;
+        }
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) ko[i] = p.scale * exp2f(rjv[i] - pj[x][i]) * ka[i];
+        float* dk = p.dkh32 + krow * K + c0;
+        float* dvp = p.dvh32 + krow * V + c0;
+        if constexpr (CPL == 4) {
+          *reinterpret_cast<float4*>(dk) = make_float4(ko[0], ko[1], ko[2 % CPL], ko[3 % CPL]);
+          *reinterpret_cast<float4*>(dvp) = make_float4(va[0], va[1], va[2 % CPL], va[3 % CPL]);
+        } else {
+          *reinterpret_cast<float2*>(dk) = make_float2(ko[0], ko[1 % CPL]);
+          *reinterpret_cast<float2*>(dvp) = make_float2(va[0], va[1 % CPL]);
         }
       }
     }
