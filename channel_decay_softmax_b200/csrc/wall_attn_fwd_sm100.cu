@@ -382,95 +382,133 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                     (i - j0 < win) && !has_gs);
       const float sl2 = p.scale_log2;
       const float bias_i = has_gs ? gs_i : 0.f;
-      // pass 1: row max
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 64) {
-        uint32_t sv[64];
-        tmem_ld32(s_addr + c, sv);
-        tmem_ld32(s_addr + c + 32, sv + 32);
-        tmem_wait_ld();
-        if (fast) {
+      bool done = false;
+      // One pass when every row's running max is set: exponentials against
+      // it, P held packed in registers and stored only if no row's max grew
+      // past the lazy threshold; otherwise S, still intact in TMEM, goes
+      // through the two passes below (max, O rescale, exponentials).
+      if (fast && __all_sync(0xffffffffu, m_use != -INFINITY)) {
+        uint32_t pk1[64];
+        float r0 = 0.f, r1 = 0.f, mxx = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 64; e += 4) {
-            mx0 = fmaxf(mx0, __uint_as_float(sv[e]) * sl2);
-            mx1 = fmaxf(mx1, __uint_as_float(sv[e + 1]) * sl2);
-            mx2 = fmaxf(mx2, __uint_as_float(sv[e + 2]) * sl2);
-            mx3 = fmaxf(mx3, __uint_as_float(sv[e + 3]) * sl2);
-          }
-        } else {
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t sv[64];
+          tmem_ld32(s_addr + c, sv);
+          tmem_ld32(s_addr + c + 32, sv + 32);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int j = j0 + c + e;
-            const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
-            const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e]);
-            mx0 = fmaxf(mx0, vis ? x : -INFINITY);
-          }
-        }
-      }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      const bool resc = mx > m_use + kRescaleThreshold;
-      const float m_new = resc ? mx : m_use;
-      const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
-      if (t >= 2) {
-        // this group's previous PV has landed in its O before O is rescaled
-        const bool got = wait_bar(bar(B_PVDONE + grp), ((t >> 1) - 1) & 1, p.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const float f = resc ? alpha : 1.f;
-#pragma unroll 1
-          for (int c = 0; c < V / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(o_addr + c * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(o_addr + c * 32, ov);
-          }
-          tmem_wait_st();
-        }
-      }
-      if (resc) l *= alpha;
-      m_use = m_new;
-      const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
-      // pass 2: p = exp2(s - m), row sum, bf16 P over the consumed S columns
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t sv[32];
-        tmem_ld32(s_addr + c, sv);
-        tmem_wait_ld();
-        float e32[32];
-        if (fast) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = fmaf(__uint_as_float(sv[e]), sl2, -m_eff);
+          for (int e = 0; e < 64; e += 2) {
+            const float x0 = fmaf(__uint_as_float(sv[e]), sl2, -m_use);
+            const float x1 = fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use);
+            mxx = fmaxf(mxx, fmaxf(x0, x1));
             // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
-            e32[e] = (e & 7) >= 5 ? exp2_fma(x) : exp2f(x);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = j0 + c + e;
-            const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
-            const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e] - m_eff);
-            e32[e] = vis ? exp2f(x) : 0.f;
+            const float p0 = (e & 7) >= 5 ? exp2_fma(x0) : exp2f(x0);
+            const float p1 = ((e + 1) & 7) >= 5 ? exp2_fma(x1) : exp2f(x1);
+            r0 += p0;
+            r1 += p1;
+            pk1[(c + e) / 2] = pack_bf16x2(p0, p1);
           }
         }
-        uint32_t pk[16];
+        if (!__any_sync(0xffffffffu, mxx > kRescaleThreshold)) {
+          // keys [32c, 32c+32) -> columns [16c, 16c+16): all of S was read
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          rs0 += e32[e];
-          rs1 += e32[e + 1];
-          pk[e / 2] = pack_bf16x2(e32[e], e32[e + 1]);
+          for (int c = 0; c < 4; ++c) tmem_st16(s_addr + c * 16, pk1 + c * 16);
+          tmem_wait_st();
+          l += r0 + r1;
+          done = true;
         }
-        // keys [c, c+32) -> columns [c/2, c/2+16) of this S buffer; every S
-        // column at or below them has been read already
-        tmem_st16(s_addr + c / 2, pk);
       }
-      tmem_wait_st();
-      l += rs0 + rs1;
+      if (!done) {
+        // pass 1: row max
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t sv[64];
+          tmem_ld32(s_addr + c, sv);
+          tmem_ld32(s_addr + c + 32, sv + 32);
+          tmem_wait_ld();
+          if (fast) {
+#pragma unroll
+            for (int e = 0; e < 64; e += 4) {
+              mx0 = fmaxf(mx0, __uint_as_float(sv[e]) * sl2);
+              mx1 = fmaxf(mx1, __uint_as_float(sv[e + 1]) * sl2);
+              mx2 = fmaxf(mx2, __uint_as_float(sv[e + 2]) * sl2);
+              mx3 = fmaxf(mx3, __uint_as_float(sv[e + 3]) * sl2);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              const int j = j0 + c + e;
+              const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
+              const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e]);
+              mx0 = fmaxf(mx0, vis ? x : -INFINITY);
+            }
+          }
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const bool resc = mx > m_use + kRescaleThreshold;
+        const float m_new = resc ? mx : m_use;
+        const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - m_new);
+        if (t >= 2) {
+          // this group's previous PV has landed in its O before O is rescaled
+          const bool got = wait_bar(bar(B_PVDONE + grp), ((t >> 1) - 1) & 1, p.status, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, resc)) {
+            const float f = resc ? alpha : 1.f;
+#pragma unroll 1
+            for (int c = 0; c < V / 32; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(o_addr + c * 32, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+              tmem_st32(o_addr + c * 32, ov);
+            }
+            tmem_wait_st();
+          }
+        }
+        if (resc) l *= alpha;
+        m_use = m_new;
+        const float m_eff = (m_use == -INFINITY) ? 0.f : m_use;
+        // pass 2: p = exp2(s - m), row sum, bf16 P over the consumed S columns
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t sv[32];
+          tmem_ld32(s_addr + c, sv);
+          tmem_wait_ld();
+          float e32[32];
+          if (fast) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x = fmaf(__uint_as_float(sv[e]), sl2, -m_eff);
+              // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
+              e32[e] = (e & 7) >= 5 ? exp2_fma(x) : exp2f(x);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int j = j0 + c + e;
+              const bool vis = row_ok & (j < L) & (j <= i) & (i - j < win);
+              const float x = fmaf(__uint_as_float(sv[e]), sl2, bias_i - gsk[c + e] - m_eff);
+              e32[e] = vis ? exp2f(x) : 0.f;
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            rs0 += e32[e];
+            rs1 += e32[e + 1];
+            pk[e / 2] = pack_bf16x2(e32[e], e32[e + 1]);
+          }
+          // keys [c, c+32) -> columns [c/2, c/2+16) of this S buffer; every S
+          // column at or below them has been read already
+          tmem_st16(s_addr + c / 2, pk);
+        }
+        tmem_wait_st();
+        l += rs0 + rs1;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_PFULL + grp));
