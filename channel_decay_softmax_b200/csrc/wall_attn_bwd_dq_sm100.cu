@@ -64,8 +64,7 @@ struct DSmem {
   static constexpr int oO = oQ + kT;
   static constexpr int oK = oO + kT;           // kKS stages
   static constexpr int oV = oK + kKS * kT;     // kVS stages
-  static constexpr int oRI = oV + kVS * kT;    // float[KD]
-  static constexpr int oRJ = oRI + KD * 4;     // float[kKS][KD]
+  static constexpr int oRJ = oV + kVS * kT;     // float[kKS][KD]
   static constexpr int oBar = oRJ + kKS * KD * 4;
   static constexpr int kBars = 20;  // >= kNumBars
   static constexpr int oMisc = oBar + kBars * 8;
@@ -134,7 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   const uint32_t sbase = smem_u32(smem);
-  float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
@@ -179,8 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
-  for (int n = threadIdx.x; n < K; n += kThreads)
-    sRI[n] = p.anchors[((long)(blk_off + blk) * HQ + h) * K + n];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -307,9 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x - 64;
     const int ch = tid % kChunks;
     const int rs = tid / kChunks;
+    // the query block's anchors: only these warps need them, so they load
+    // them here rather than everyone before the setup barrier
     float ri[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ri[e] = sRI[ch * 8 + e];
+    for (int e = 0; e < 8; ++e) ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
     for (int t = 0; t < nT; ++t) {
       const int st = t % kKS;
       {

@@ -77,8 +77,7 @@ struct Smem {
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kT;              // kKS stages
   static constexpr int oV = oK + kKS * kT;        // kVS stages
-  static constexpr int oRI = oV + kVS * kT;       // float[KD]
-  static constexpr int oRJ = oRI + KD * 4;        // float[kKS][KD] key-block anchors
+  static constexpr int oRJ = oV + kVS * kT;        // float[kKS][KD] key-block anchors
   static constexpr int oGS = oRJ + kKS * KD * 4;  // float[8 warps][BN] key prefix
   static constexpr int oX = oGS + 8 * BN * 4;     // float[2 groups][2][BM]: m, l
   static constexpr int oBar = oX + 2 * 2 * BM * 4;
@@ -141,7 +140,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float* sRI = reinterpret_cast<float*>(smem + Lay::oRI);
   float* sGS = reinterpret_cast<float*>(smem + Lay::oGS);
   float* sX = reinterpret_cast<float*>(smem + Lay::oX);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
@@ -191,8 +189,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
-  for (int n = threadIdx.x; n < K; n += kThreads)
-    sRI[n] = p.anchors[((long)(blk_off + blk) * HQ + h) * K + n];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -303,9 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x - 64;
     const int ch = tid % kChunks;
     const int rs = tid / kChunks;
+    // the query block's anchors: only these warps need them, so they load
+    // them here rather than everyone before the setup barrier
     float ri[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ri[e] = sRI[ch * 8 + e];
+    for (int e = 0; e < 8; ++e) ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
     for (int t = 0; t < nT; ++t) {
       const int st = t % kKS;
       {
