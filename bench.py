@@ -200,10 +200,11 @@ def bench_train(args, world, rank, peaks):
         P = api.prefix_cumsum(g)
         if ev is not None:
             ev[0].record(stream)
-        o, lse = api.wall_attn_fwd(q, k, v, P, s.scale)
+        # the forward's anchored operands are reused by the backward
+        o, lse, fws = api.wall_attn_fwd(q, k, v, P, s.scale, return_workspace=True)
         if ev is not None:
             ev[1].record(stream)
-        out = api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale)
+        out = api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, fwd_workspace=fws)
         if ev is not None:
             ev[2].record(stream)
         return out
@@ -238,9 +239,10 @@ def bench_train(args, world, rank, peaks):
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     # launches of this library inside one step: prefix scan 3 (chunk sums,
     # carries, chunk scans); forward: operand preparation 1 + tcgen05 forward
-    # 1; backward: operand preparation 1, D/sink pre-pass 1, tcgen05 key-block
-    # (dK, dV) 1, tcgen05 query-block (dq) 1, finalize 1, reverse scan 3
-    launches_per_step = 13
+    # 1; backward (reusing the forward's operands): D/sink pre-pass 1, tcgen05
+    # key-block (dK, dV) 1, tcgen05 query-block (dq) 1, finalize 1, reverse
+    # scan 3
+    launches_per_step = 12
     res = dict(ms=ms_max, value=world * step_flops / (ms_max * 1e-3) / 1e12,
                fwd_ms=fwd_ms, bwd_ms=bwd_ms,
                fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,
@@ -268,9 +270,11 @@ def bench_train_e2e(args, x, s, step_flops, world):
         for n in names_in:
             dev_in[n].copy_(host_in[n], non_blocking=True)
         P = api.prefix_cumsum(dev_in["g"])
-        o, lse = api.wall_attn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], P, s.scale)
+        o, lse, fws = api.wall_attn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], P, s.scale,
+                                        return_workspace=True)
         dq, dk, dv, dg, _, _ = api.wall_attn_bwd(dev_in["dO"], dev_in["q"], dev_in["k"],
-                                                 dev_in["v"], P, o, lse, s.scale)
+                                                 dev_in["v"], P, o, lse, s.scale,
+                                                 fwd_workspace=fws)
         if host_out is None:
             host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv, dg)]
         for h, d in zip(host_out, (dq, dk, dv, dg)):

@@ -56,7 +56,7 @@ def lib():
         L.wall_attn_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
         L.wall_attn_bwd.restype = i
         L.wall_attn_bwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, i, i, f, fp, fp,
-                                    i, ip, i, vp, vp, vp, vp, fp, fp, vp, sz, vp]
+                                    i, ip, i, vp, vp, vp, vp, fp, fp, vp, sz, vp, vp]
         L.wall_build_kv_cache.restype = i
         L.wall_build_kv_cache.argtypes = [vp, fp, i, i, i, i, i, i, i, i, vp, fp, i, vp]
         L.wall_attn_decode_workspace.restype = sz
@@ -153,13 +153,13 @@ def wall_attn_bwd_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> 
 
 def wall_attn_bwd(dO, q, k, v, P, o, lse, B, T, H, HQ, K, V, scale, g_scalar, sink_bias,
                   window_size, cu_seqlens, n_seq, dq, dk, dv, dg, dg_scalar, dsink, workspace,
-                  stream=None):
+                  fwd_workspace=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("wall_attn_bwd", lib().wall_attn_bwd(
         _p(dO), _p(q), _p(k), _p(v), _p(P), _p(o), _p(lse), dtype_code(q.dtype), B, T, H, HQ, K,
         V, float(scale), _p(g_scalar), _p(sink_bias), int(window_size), _p(cu_seqlens), n_seq,
         _p(dq), _p(dk), _p(dv), _p(dg), _p(dg_scalar), _p(dsink), _p(workspace), ws_bytes,
-        _stream(stream)))
+        _p(fwd_workspace), _stream(stream)))
 
 
 def wall_build_kv_cache(k, P, B, Tn, H, HQ, K, C, t0, k_tilde, r_cache, Tcap, stream=None):

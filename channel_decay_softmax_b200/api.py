@@ -54,8 +54,10 @@ def prefix_cumsum(g, cu_seqlens=None, carry_in=None, return_carry=False):
 
 
 def wall_attn_fwd(q, k, v, P, scale=None, g_scalar=None, sink_bias=None, window_size=None,
-                  cu_seqlens=None):
-    """Forward from a precomputed prefix P; returns (o, lse)."""
+                  cu_seqlens=None, return_workspace=False):
+    """Forward from a precomputed prefix P; returns (o, lse), or (o, lse,
+    workspace) with return_workspace: the workspace holds the anchored
+    operands, which wall_attn_bwd can reuse (its fwd_workspace)."""
     B, T, H, HQ, K, V = _shape_checks(q, k, v, P)
     nseq = _n_seq(cu_seqlens, B)
     o = torch.empty((B, T, HQ, V), dtype=q.dtype, device=q.device)
@@ -64,12 +66,14 @@ def wall_attn_fwd(q, k, v, P, scale=None, g_scalar=None, sink_bias=None, window_
              q.device)
     L.wall_attn_fwd(q, k, v, P, B, T, H, HQ, K, V, scale or 0.0, g_scalar, sink_bias,
                     window_size or 0, cu_seqlens, nseq, o, lse, ws)
-    return o, lse
+    return (o, lse, ws) if return_workspace else (o, lse)
 
 
 def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=None,
-                  window_size=None, cu_seqlens=None, want_dsink=False):
-    """Backward; returns dq, dk, dv, dg, dg_scalar (or None), dsink (or None)."""
+                  window_size=None, cu_seqlens=None, want_dsink=False, fwd_workspace=None):
+    """Backward; returns dq, dk, dv, dg, dg_scalar (or None), dsink (or None).
+    fwd_workspace: the workspace returned by wall_attn_fwd(..., return_workspace=True)
+    for the same inputs, whose anchored operands are then reused."""
     B, T, H, HQ, K, V = _shape_checks(q, k, v, P)
     nseq = _n_seq(cu_seqlens, B)
     dq = torch.empty_like(q)
@@ -83,7 +87,7 @@ def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=N
              q.device)
     L.wall_attn_bwd(dO.contiguous(), q, k, v, P, o, lse, B, T, H, HQ, K, V, scale or 0.0,
                     g_scalar, sink_bias, window_size or 0, cu_seqlens, nseq, dq, dk, dv, dg, dgs,
-                    dsink, ws)
+                    dsink, ws, fwd_workspace)
     return dq, dk, dv, dg, dgs, dsink
 
 
@@ -96,8 +100,9 @@ class WallAttnFunction(torch.autograd.Function):
         gs = g_scalar.contiguous().float() if g_scalar is not None else None
         sk = sink_bias.contiguous().float() if sink_bias is not None else None
         P = prefix_cumsum(g, cu_seqlens)
-        o, lse = wall_attn_fwd(q, k, v, P, scale, gs, sk, window_size, cu_seqlens)
-        ctx.save_for_backward(q, k, v, P, o, lse, gs, sk, cu_seqlens)
+        o, lse, fws = wall_attn_fwd(q, k, v, P, scale, gs, sk, window_size, cu_seqlens,
+                                    return_workspace=True)
+        ctx.save_for_backward(q, k, v, P, o, lse, gs, sk, cu_seqlens, fws)
         ctx.scale, ctx.window_size = scale, window_size
         ctx.gs_dtype = g_scalar.dtype if g_scalar is not None else None
         ctx.sk_dtype = sink_bias.dtype if sink_bias is not None else None
@@ -105,10 +110,10 @@ class WallAttnFunction(torch.autograd.Function):
 
     @staticmethod
     def backward(ctx, dO):
-        q, k, v, P, o, lse, gs, sk, cu = ctx.saved_tensors
+        q, k, v, P, o, lse, gs, sk, cu, fws = ctx.saved_tensors
         want_dsink = sk is not None and ctx.needs_input_grad[6]
         dq, dk, dv, dg, dgs, dsink = wall_attn_bwd(dO, q, k, v, P, o, lse, ctx.scale, gs, sk,
-                                                   ctx.window_size, cu, want_dsink)
+                                                   ctx.window_size, cu, want_dsink, fws)
         if dgs is not None and ctx.gs_dtype is not None:
             dgs = dgs.to(ctx.gs_dtype)
         if dsink is not None:

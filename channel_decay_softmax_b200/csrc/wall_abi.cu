@@ -277,11 +277,12 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
                   int K, int V, float scale, const float* g_scalar, const float* sink_bias,
                   int window_size, const int32_t* cu_seqlens, int n_seq, void* dq, void* dk,
                   void* dv, void* dg, float* dg_scalar, float* dsink, void* workspace,
-                  size_t workspace_bytes, wall_stream_t stream) {
+                  size_t workspace_bytes, const void* fwd_workspace, wall_stream_t stream) {
   AttnProblem pb;
   int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
   if (rc) return rc;
   if ((g_scalar == nullptr) != (dg_scalar == nullptr)) return WALL_ERR_INVALID_ARG;
+  if (!ok_opt(fwd_workspace)) return WALL_ERR_INVALID_ARG;
   if (dsink != nullptr && sink_bias == nullptr) return WALL_ERR_INVALID_ARG;
   if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(dg_scalar) || !ok_opt(dsink))
     return WALL_ERR_INVALID_ARG;
@@ -323,7 +324,16 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
     tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
     tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
     tw.n_blocks128 = w.n_blocks128;
-    rc = attn_bwd_tc(pb, a, tw, dq, dk, dv, status_ptr(), s);
+    const bool reuse = fwd_workspace != nullptr;
+    if (reuse) {
+      // the forward's anchored operands, in its own workspace layout
+      const FwdWs fw = fwd_ws_layout(pb, g_scalar != nullptr);
+      void* fws = const_cast<void*>(fwd_workspace);
+      tw.qh = reinterpret_cast<__nv_bfloat16*>(at(fws, fw.qh));
+      tw.kh = reinterpret_cast<__nv_bfloat16*>(at(fws, fw.kh));
+      tw.anchors = reinterpret_cast<float*>(at(fws, fw.anchors));
+    }
+    rc = attn_bwd_tc(pb, a, tw, !reuse, dq, dk, dv, status_ptr(), s);
     if (rc) return rc;
   } else {
     rc = attn_bwd_simt(pb, a, s);

@@ -791,13 +791,16 @@ int launch_bwd_tc_gs(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws,
 
 }  // namespace
 
-int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void* dq, void* dk,
-                void* dv, int* status, cudaStream_t stream) {
+int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool prepare, void* dq,
+                void* dk, void* dv, int* status, cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
-  timing_mark(T_OPERANDS, stream);
-  int rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
-  timing_mark(T_OPERANDS, stream);
-  if (rc) return rc;
+  int rc = WALL_OK;
+  if (prepare) {  // else the forward's operands are reused
+    timing_mark(T_OPERANDS, stream);
+    rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
+    timing_mark(T_OPERANDS, stream);
+    if (rc) return rc;
+  }
   timing_mark(T_BWD_PRE, stream);
   {
     const long threads = pb.rows * pb.HQ * 8;

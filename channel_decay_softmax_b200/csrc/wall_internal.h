@@ -77,8 +77,9 @@ int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int*
                 cudaStream_t stream);
 
 // ---- tensor-core backward (wall_attn_bwd_sm100.cu) ----
-int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, void* dq, void* dk,
-                void* dv, int* status, cudaStream_t stream);
+// prepare: false when ws already holds the forward's anchored operands
+int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool prepare,
+                void* dq, void* dk, void* dv, int* status, cudaStream_t stream);
 // raw dq (without the per-row anchor factor) into a.dq32 (wall_attn_bwd_dq_sm100.cu)
 int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                    cudaStream_t stream);

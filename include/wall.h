@@ -134,13 +134,18 @@ size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, in
  * per query head, dL_t = q_t (.) dq_t - k_t (.) dk^(h)_t with the key-side
  * term -K_j (.) dK_j, then dg = the reverse cumulative sum of dL within each
  * sequence.  dk^(h), dv^(h) are summed over each GQA group.
+ * fwd_workspace: NULL, or the workspace of the wall_attn_fwd call that
+ * produced o and lse, with the same q, k, P, shapes and options and left
+ * unchanged since.  On the bf16 tensor-core path the anchored operands that
+ * call prepared in it are then read instead of recomputed; it is only read.
+ * Elsewhere it is ignored.
  */
 int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, const float* P,
                   const void* o, const float* lse, int dtype, int B, int T, int H, int HQ,
                   int K, int V, float scale, const float* g_scalar, const float* sink_bias,
                   int window_size, const int32_t* cu_seqlens, int n_seq, void* dq, void* dk,
                   void* dv, void* dg, float* dg_scalar, float* dsink, void* workspace,
-                  size_t workspace_bytes, wall_stream_t stream);
+                  size_t workspace_bytes, const void* fwd_workspace, wall_stream_t stream);
 
 /*
  * wall_build_kv_cache -- pre-rescaled decode cache (README "Decode":

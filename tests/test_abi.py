@@ -71,18 +71,19 @@ def test_fwd_rejects_bad_arguments(lib):
 def test_bwd_rejects_bad_arguments(lib):
     def bwd(**over):
         a = dict(dO=FAKE, gs=None, dgs=None, sink=None, dsink=None, ws=None, ws_bytes=0, T=16,
-                 HQ=4)
+                 HQ=4, fws=None)
         a.update(over)
         return lib.wall_attn_bwd(a["dO"], FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, a["T"], 2,
                                  a["HQ"], 64, 64, 0.0, a["gs"], a["sink"], 0, None, 0, FAKE,
                                  FAKE, FAKE, FAKE, a["dgs"], a["dsink"], a["ws"], a["ws_bytes"],
-                                 None)
+                                 a["fws"], None)
     assert bwd(HQ=5) == L.WALL_ERR_INVALID_ARG
     assert bwd(gs=FAKE) == L.WALL_ERR_INVALID_ARG               # dg_scalar missing
     assert bwd(dgs=FAKE) == L.WALL_ERR_INVALID_ARG              # g_scalar missing
     assert bwd(dO=None) == L.WALL_ERR_INVALID_ARG
     assert bwd() == L.WALL_ERR_INVALID_ARG                      # no workspace
     assert bwd(ws=FAKE, ws_bytes=16) == L.WALL_ERR_INVALID_ARG  # workspace too small
+    assert bwd(fws=FAKE + 4) == L.WALL_ERR_INVALID_ARG          # misaligned forward workspace
 
 
 def test_cache_and_decode_reject_bad_arguments(lib):

@@ -187,3 +187,20 @@ def test_empty_and_single_row():
             # one visible key: o = v of the same row, dq = dk = dg = 0
             assert max_abs(o[0, 0], x["v"][0, 0].repeat_interleave(s.G, 0)) == 0.0
             assert float(grads[0].float().abs().max()) < 1e-5
+
+
+def test_backward_reuses_forward_operands_bit_exactly():
+    """wall_attn_bwd with the forward's workspace reads the anchored operands
+    that call prepared instead of recomputing them: the same deterministic
+    values, so every gradient must match the recomputing call bit for bit
+    (config 2 shape, no sink: no atomics on the path)."""
+    s = I.spec(2)
+    x = _to(I.training_inputs(s))
+    q, k, v = x["q"], x["k"], x["v"]
+    P = api.prefix_cumsum(x["g"])
+    o, lse, fws = api.wall_attn_fwd(q, k, v, P, x["scale"], return_workspace=True)
+    a = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"])
+    b = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], fwd_workspace=fws)
+    torch.cuda.synchronize()
+    for name, ta, tb in zip(("dq", "dk", "dv", "dg"), a[:4], b[:4]):
+        assert torch.equal(ta, tb), name
