@@ -255,48 +255,72 @@ def bench_train(args, world, rank, peaks):
 
 
 def bench_train_e2e(args, x, s, step_flops, world):
-    """The same step from pinned host buffers: H2D of q, k, v, g, dO and D2H
-    of dq, dk, dv, dg inside the timed region."""
+    """The same step from pinned host buffers: every step uploads its inputs
+    (q, k, v, g, dO) and downloads its gradients (dq, dk, dv, dg) inside the
+    timed region, as a training input pipeline does: on three streams, the
+    upload of step i+1 and the download of step i-1 overlap the compute of
+    step i (device inputs and pinned host outputs double-buffered, events
+    order each buffer's reuse)."""
     from channel_decay_softmax_b200 import api
 
     names_in = ("q", "k", "v", "g", "dO")
     host_in = {n: x[n].cpu().pin_memory() for n in names_in}
-    dev_in = {n: torch.empty_like(x[n]) for n in names_in}
-    host_out = None
-    stream = torch.cuda.current_stream()
+    dev_in = [{n: torch.empty_like(x[n]) for n in names_in} for _ in range(2)]
+    host_out = [None, None]
+    s_comp = torch.cuda.current_stream()
+    s_h2d = torch.cuda.Stream()
+    s_d2h = torch.cuda.Stream()
+    inputs_free = [torch.cuda.Event(), torch.cuda.Event()]   # compute done with dev_in[b]
+    inputs_ready = [torch.cuda.Event(), torch.cuda.Event()]  # upload into dev_in[b] done
+    outputs_ready = [torch.cuda.Event(), torch.cuda.Event()]
+    for e in inputs_free:
+        e.record(s_comp)
 
-    def step():
-        nonlocal host_out
-        for n in names_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        P = api.prefix_cumsum(dev_in["g"])
-        o, lse, fws = api.wall_attn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], P, s.scale,
-                                        return_workspace=True)
-        dq, dk, dv, dg, _, _ = api.wall_attn_bwd(dev_in["dO"], dev_in["q"], dev_in["k"],
-                                                 dev_in["v"], P, o, lse, s.scale,
-                                                 fwd_workspace=fws)
-        if host_out is None:
-            host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv, dg)]
-        for h, d in zip(host_out, (dq, dk, dv, dg)):
-            h.copy_(d, non_blocking=True)
+    def step(i):
+        b = i % 2
+        d = dev_in[b]
+        with torch.cuda.stream(s_h2d):
+            s_h2d.wait_event(inputs_free[b])
+            for n in names_in:
+                d[n].copy_(host_in[n], non_blocking=True)
+            inputs_ready[b].record(s_h2d)
+        s_comp.wait_event(inputs_ready[b])
+        P = api.prefix_cumsum(d["g"])
+        o, lse, fws = api.wall_attn_fwd(d["q"], d["k"], d["v"], P, s.scale, return_workspace=True)
+        dq, dk, dv, dg, _, _ = api.wall_attn_bwd(d["dO"], d["q"], d["k"], d["v"], P, o, lse,
+                                                 s.scale, fwd_workspace=fws)
+        inputs_free[b].record(s_comp)
+        outputs_ready[b].record(s_comp)
+        outs = (dq, dk, dv, dg)
+        if host_out[b] is None:
+            host_out[b] = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(outputs_ready[b])
+            for h, t in zip(host_out[b], outs):
+                t.record_stream(s_d2h)  # the allocator keeps it until the copy is done
+                h.copy_(t, non_blocking=True)
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize()
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step()
-    t1.record(stream)
+    t0.record(s_h2d)
+    s_comp.wait_stream(s_h2d)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    s_d2h.wait_stream(s_comp)
+    t1.record(s_d2h)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
     return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "3 streams: upload of step i+1 and download of step i-1 overlap "
+                         "step i; every step moves its own inputs and gradients"}
 
 
 def bench_decode(args, rank, peaks):
