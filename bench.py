@@ -377,20 +377,37 @@ def bench_decode(args, rank, peaks):
                decode_launches_per_step=2)
     del kt, rc
     torch.cuda.empty_cache()
-    # streaming append loop: cache of [0, T0) then 64 appended tokens
+    # streaming append loop: cache of [0, T0) then 64 appended tokens, once
+    # with the one-launch fused step and once with the three-call path
+    # (prefix scan, cache build + value copy, decode) from the same prefill
     cache = api.WallDecodeCache(s.B, s.H, s.HQ, s.K, s.V, capacity=T, chunk_size=s.chunk,
                                 dtype=s.dtype, device="cuda", scale=s.scale)
     cache.append(d["k"][:, :T0], d["v"][:, :T0], d["g"][:, :T0])
+    carry0 = cache.carry.clone()
     torch.cuda.synchronize()
-    a, b = ev(), ev()
-    a.record(stream)
-    for t in range(T0, T):
-        cache.step(d["q_tail"][:, t - T0:t - T0 + 1], d["k"][:, t:t + 1], d["v"][:, t:t + 1],
-                   d["g"][:, t:t + 1])
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms_tok = a.elapsed_time(b) / n_stream
-    out.update(stream_ms_per_token=ms_tok, stream_tokens_per_s=s.B / (ms_tok * 1e-3))
+
+    def stream_loop(fused):
+        cache.length = T0
+        cache.carry = carry0.clone()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for t in range(T0, T):
+            cache.step(d["q_tail"][:, t - T0:t - T0 + 1], d["k"][:, t:t + 1],
+                       d["v"][:, t:t + 1], d["g"][:, t:t + 1], fused=fused)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n_stream
+
+    stream_loop(True)  # warm-up of both paths
+    stream_loop(False)
+    ms_tok = stream_loop(True)
+    ms_tok3 = stream_loop(False)
+    stream_bytes = sum(decode_bytes(s, t + 1) for t in range(T0, T)) / n_stream
+    out.update(stream_ms_per_token=ms_tok, stream_tokens_per_s=s.B / (ms_tok * 1e-3),
+               stream_gbs=stream_bytes / (ms_tok * 1e-3) / 1e9, stream_launches_per_token=1,
+               stream_three_call_ms_per_token=ms_tok3,
+               stream_three_call_launches_per_token=7)
     del cache, d
     torch.cuda.empty_cache()
     out["workload"] = (f"decode B={s.B} T_kv={T} HQ={s.HQ} H={s.H} K=V={s.K} C={s.chunk} bf16, "

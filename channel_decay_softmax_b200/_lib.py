@@ -20,7 +20,7 @@ EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn
            "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
            "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
            "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
-           "wall_timing_read"]
+           "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step"]
 
 _lib = None
 
@@ -76,6 +76,11 @@ def lib():
         L.wall_timing_read.restype = i
         L.wall_timing_read.argtypes = [i, ctypes.POINTER(ctypes.c_char_p),
                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
+        L.wall_decode_step_workspace.restype = sz
+        L.wall_decode_step_workspace.argtypes = [i, i, i, i, i, i]
+        L.wall_decode_step.restype = i
+        L.wall_decode_step.argtypes = [vp, vp, vp, vp, i, fp, vp, vp, fp, fp, f, i, i, i, i, i,
+                                       i, i, i, vp, fp, vp, sz, vp]
         _lib = L
     return _lib
 
@@ -187,3 +192,17 @@ def wall_attn_decode_noalloc(q, v, p_curr, k_tilde, r_cache, sink_bias, scale, C
     _check("wall_attn_decode_noalloc", lib().wall_attn_decode_noalloc(
         _p(q), _p(v), _p(p_curr), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
         dtype_code(q.dtype), B, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _stream(stream)))
+
+
+def wall_decode_step_workspace(B, Tcap, H, HQ, V, C) -> int:
+    return lib().wall_decode_step_workspace(B, Tcap, H, HQ, V, C)
+
+
+def wall_decode_step(q, k, v, g, carry, k_tilde, v_cache, r_cache, sink_bias, scale, C, t, B,
+                     Tcap, H, HQ, K, V, o, lse, workspace, stream=None):
+    """One streaming token: prefix update, cache append and decode in one launch."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_decode_step", lib().wall_decode_step(
+        _p(q), _p(k), _p(v), _p(g), dtype_code(q.dtype), _p(carry), _p(k_tilde), _p(v_cache),
+        _p(r_cache), _p(sink_bias), float(scale), C, t, B, Tcap, H, HQ, K, V, _p(o), _p(lse),
+        _p(workspace), ws_bytes, _stream(stream)))

@@ -167,9 +167,12 @@ class WallDecodeCache:
     """Append-as-you-go decode state (README "Decode": the streaming serving
     loop): cache buffers of a fixed capacity plus the running prefix.
 
-    ``prefill(k, v, g)`` fills the first T positions; each ``step(q, k, v,
-    g)`` appends one token (prefix update, new chunk anchor when a chunk
-    starts, k_tilde and v rows) and decodes it.
+    ``append(k, v, g)`` fills the next positions (prefill); each ``step(q,
+    k, v, g)`` appends one token (prefix update, new chunk anchor when a
+    chunk starts, k_tilde and v rows) and decodes it.  Inside the fused
+    step's domain (bf16, K and V in {64, 128}, HQ/H <= 8, chunk a multiple
+    of 32) a step is one launch of wall_decode_step; elsewhere it is the
+    prefix scan, the cache build and wall_attn_decode in turn.
     """
 
     def __init__(self, B, H, HQ, K, V, capacity, chunk_size=64, dtype=torch.bfloat16,
@@ -184,7 +187,13 @@ class WallDecodeCache:
         self.sink = sink_bias.contiguous().float() if sink_bias is not None else None
         self.length = 0
         self.ws = _ws(L.wall_attn_decode_workspace(B, capacity, H, HQ, V, chunk_size), device)
-        self.P_step = torch.empty((B, 1, HQ, K), dtype=torch.float32, device=device)
+        self.fused = (dtype == torch.bfloat16 and K in (64, 128) and V in (64, 128)
+                      and HQ // H <= 8 and chunk_size % 32 == 0)
+        if self.fused:
+            # the fused step's arrival counters must start at zero
+            self.step_ws = torch.zeros(
+                max(int(L.wall_decode_step_workspace(B, capacity, H, HQ, V, chunk_size)), 1),
+                dtype=torch.uint8, device=device)
 
     def append(self, k, v, g):
         """Appends Tn tokens: k [B,Tn,H,K], v [B,Tn,H,V], g [B,Tn,HQ,K];
@@ -208,10 +217,29 @@ class WallDecodeCache:
         return wall_attn_decode(q, self.v, p_curr, self.k_tilde, self.r_cache, self.sink,
                                 self.scale, self.C, T_kv=self.length)
 
-    def step(self, q, k, v, g):
-        """Appends one token and decodes its query; returns (o, lse)."""
-        P = self.append(k, v, g)
-        return self.decode(q, P[:, -1:])
+    def step(self, q, k, v, g, fused=None):
+        """Appends one token and decodes its query; returns (o, lse).
+        q [B,1,HQ,K], k [B,1,H,K], v [B,1,H,V], g [B,1,HQ,K].  ``fused=False``
+        takes the three-call path even where the fused step applies."""
+        if fused is None:
+            fused = self.fused
+        if not fused:
+            P = self.append(k, v, g)
+            return self.decode(q, P[:, -1:])
+        if not self.fused:
+            raise ValueError("the fused decode step does not cover this cache's shapes or dtype")
+        t = self.length
+        if t + 1 > self.cap:
+            raise ValueError("decode cache capacity exceeded")
+        B, HQ, V = self.B, self.HQ, self.V
+        o = torch.empty((B, 1, HQ, V), dtype=q.dtype, device=q.device)
+        lse = torch.empty((B, 1, HQ), dtype=torch.float32, device=q.device)
+        L.wall_decode_step(q.contiguous(), k.contiguous(), v.contiguous(), g.contiguous(),
+                           self.carry, self.k_tilde, self.v, self.r_cache, self.sink,
+                           self.scale or 0.0, self.C, t, B, self.cap, self.H, HQ, self.K, V,
+                           o, lse, self.step_ws)
+        self.length = t + 1
+        return o, lse
 
 
 def timing_enable(on=True):
@@ -225,7 +253,7 @@ def timing_read():
     """Per-stage {name: (launches, total_ms)} since the last read or enable;
     synchronizes on the recorded events and clears the totals."""
     import ctypes
-    n = 10
+    n = 11
     names = (ctypes.c_char_p * n)()
     launches = (ctypes.c_int * n)()
     ms = (ctypes.c_double * n)()

@@ -399,4 +399,46 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
   return rc;
 }
 
+size_t wall_decode_step_workspace(int B, int Tcap, int H, int HQ, int V, int C) {
+  if (B < 0 || Tcap < 1 || H < 1 || HQ < 1 || HQ % H != 0 || V < 1 || C < 1) return 0;
+  const int S = decode_splits(B, Tcap, H, C);
+  return align256(sizeof(float) * (size_t)B * HQ * S * (V + 2)) +
+         align256(sizeof(unsigned) * (size_t)B * HQ);
+}
+
+int wall_decode_step(const void* q, const void* k, const void* v, const void* g, int dtype,
+                     float* carry, void* k_tilde, void* v_cache, float* r_cache,
+                     const float* sink_bias, float scale, int C, int t, int B, int Tcap, int H,
+                     int HQ, int K, int V, void* o, float* lse, void* workspace,
+                     size_t workspace_bytes, wall_stream_t stream) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || t < 0 || Tcap < 1 || t >= Tcap || H < 1 || HQ < 1 || HQ % H != 0 || C < 1)
+    return WALL_ERR_INVALID_ARG;
+  if (dtype != WALL_BF16 || (K != 64 && K != 128) || (V != 64 && V != 128) || HQ / H > 8 ||
+      C % 32 != 0 || B > 65535 || H > 65535)
+    return WALL_ERR_UNSUPPORTED;
+  if (B == 0) return WALL_OK;
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(carry) ||
+      !ok_ptr(k_tilde) || !ok_ptr(v_cache) || !ok_ptr(r_cache) || !ok_ptr(o) ||
+      !ok_opt(sink_bias) || !ok_opt(lse))
+    return WALL_ERR_INVALID_ARG;
+  const size_t need = wall_decode_step_workspace(B, Tcap, H, HQ, V, C);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    return WALL_ERR_INVALID_ARG;
+  // partials sized for the largest split count the capacity allows, then the
+  // per-head arrival counters
+  const int S_cap = decode_splits(B, Tcap, H, C);
+  float* ws = static_cast<float*>(workspace);
+  unsigned* counters = reinterpret_cast<unsigned*>(
+      static_cast<char*>(workspace) + align256(sizeof(float) * (size_t)B * HQ * S_cap * (V + 2)));
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)K);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  timing_mark(T_STEP, st);
+  const int rc = decode_step(q, k, v, g, carry, k_tilde, v_cache, r_cache, sink_bias, sc, C, t,
+                             B, Tcap, H, HQ, K, V, o, lse, ws, counters,
+                             decode_splits(B, t, H, C), st);
+  timing_mark(T_STEP, st);
+  return rc;
+}
+
 }  // extern "C"

@@ -109,6 +109,21 @@ struct DecodeArgs {
   float* ws_ml;  // [B,HQ,splits,2]
 };
 
+// The one-token streaming step (append + decode in one launch): the new
+// token's inputs, the cache buffers it appends to and the per-head arrival
+// counters of the split partials.  Unused (all null) for a plain decode.
+struct StepArgs {
+  const void *k, *v, *g;  // [B,H,K], [B,H,V], [B,HQ,K] bf16: the new token
+  float* carry;           // [B,HQ,K] fp32: P at t-1 in, P at t out
+  void* kt;               // [B,Tcap,HQ,K] k_tilde, row t written
+  void* vc;               // [B,Tcap,H,V] value cache, row t written
+  float* rc;              // [B,ceil(Tcap/C),HQ,K] anchors, chunk t/C written if t%C == 0
+  unsigned* count;        // [B,HQ] split arrivals, zero between calls
+  void* o;                // [B,HQ,V] bf16
+  float* lse;             // [B,HQ] or nullptr
+  int t;                  // position of the new token (= cached tokens before it)
+};
+
 template <typename T, int KD, int VD>
 __global__ void decode_split_kernel(DecodeArgs a) {
   __shared__ float qh[32][KD];  // per warp (query head): scaled, anchored query
@@ -213,11 +228,134 @@ __global__ void decode_split_kernel(DecodeArgs a) {
 // workspace as the split kernel above and are merged the same way.
 constexpr int kDecTile = 32;
 
-template <int KD, int VD, int WPH>
-__global__ void __launch_bounds__(32 * 9, 1)
+// The merge and append of a streaming step for one (batch row, query head),
+// run by the finisher warp of the CTA whose split of that head arrived last
+// (all the head's split partials are in the workspace):
+//   P_t       = carry + g / ln 2 (per lane QPL channels), rounded as the scan
+//   own score = scale * q . k_new: the decay factor of a key at the query's
+//               own position is exp2(P_t - P_t) = 1, so no anchor enters
+//   appends   = r_cache[t/C] = P_t when t starts a chunk, k_tilde row t =
+//               k_new * exp2(R - P_t) rounded as the cache build rounds it,
+//               value row t, carry = P_t
+// Every split of this head read the carry and the chunk anchors before it
+// arrived, so the carry may be overwritten in place; row t and chunk t/C
+// (when t starts it) are outside the keys any split reads.
+template <int KD, int VD>
+__device__ __forceinline__ void step_merge_append(const DecodeArgs& a, const StepArgs& st, int b,
+                                                  int h, int kh, int g, int lane, float sl2) {
+  constexpr int VPL = VD / 32, QPL = KD / 32;
+  const long bh = (long)b * a.HQ + h;
+  if (lane == 0) st.count[bh] = 0u;  // every split of this call has arrived
+  float qv[QPL], pv[QPL];
+#pragma unroll
+  for (int i = 0; i < QPL; ++i) {
+    const long e = bh * KD + lane * QPL + i;
+    qv[i] = to_f32(static_cast<const T_bf16*>(a.q)[e]);
+    pv[i] = fmaf(kInvLn2, to_f32(static_cast<const T_bf16*>(st.g)[e]), st.carry[e]);
+  }
+  // the new token's chunk anchor, loaded early (written by an earlier call
+  // unless this token starts the chunk)
+  const int NC = (a.Tcap + a.C - 1) / a.C;
+  const long t = st.t, c = t / a.C;
+  const bool starts = t == c * a.C;
+  float* rrow = st.rc + (((long)b * NC + c) * a.HQ + h) * KD + lane * QPL;
+  float R[QPL];
+#pragma unroll
+  for (int i = 0; i < QPL; ++i) R[i] = starts ? pv[i] : rrow[i];
+
+  const T_bf16* kn = static_cast<const T_bf16*>(st.k) + ((long)b * a.H + kh) * KD + lane * QPL;
+  const T_bf16* vn = static_cast<const T_bf16*>(st.v) + ((long)b * a.H + kh) * VD + lane * VPL;
+  float kx[QPL], vx[VPL];
+  float d = 0.f;
+#pragma unroll
+  for (int i = 0; i < QPL; ++i) {
+    kx[i] = to_f32(kn[i]);
+    d = fmaf(qv[i], kx[i], d);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+  const float sd = d * sl2;  // log2 domain
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) vx[i] = to_f32(vn[i]);
+
+  // the partials: lanes stride the splits for (m, l); every lane then loads
+  // its value channels of eight splits at a time, all in flight together,
+  // so the merge costs a few L2 round trips whatever the split count
+  const long base = bh * a.splits;
+  const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + base;
+  const float sk = a.sink ? a.sink[h] * kLog2e : -INFINITY;
+  float m = fmaxf(sd, sk);
+  for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, __ldcg(ml + s).x);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const float fd = exp2f(sd - m);
+  float lp = 0.f;  // this lane's share of the splits' sums
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = fd * vx[i];
+  for (int s0 = 0; s0 < a.splits; s0 += 32) {
+    float f = 0.f;  // weight of split s0 + lane (0 for a split without keys)
+    if (s0 + lane < a.splits) {
+      const float2 x = __ldcg(ml + s0 + lane);
+      if (x.x != -INFINITY) {
+        f = exp2f(x.x - m);
+        lp = fmaf(x.y, f, lp);
+      }
+    }
+    const int n = min(32, a.splits - s0);
+    for (int j0 = 0; j0 < n; j0 += 8) {
+      float x[8][VPL];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float* po = a.ws_o + (base + s0 + min(j0 + j, n - 1)) * VD + lane * VPL;
+        if constexpr (VPL == 4) {
+          const float4 u = __ldcg(reinterpret_cast<const float4*>(po));
+          x[j][0] = u.x; x[j][1] = u.y; x[j][2] = u.z; x[j][3] = u.w;
+        } else {
+          const float2 u = __ldcg(reinterpret_cast<const float2*>(po));
+          x[j][0] = u.x; x[j][1] = u.y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float fj = __shfl_sync(0xffffffffu, f, (j0 + j) & 31);
+        if (j0 + j < n) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(x[j][i], fj, acc[i]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lp += __shfl_xor_sync(0xffffffffu, lp, off);
+  const float l = fd + (a.sink ? exp2f(sk - m) : 0.f) + lp;
+  const float inv = 1.f / l;
+  T_bf16* o = static_cast<T_bf16*>(st.o) + bh * VD + lane * VPL;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) o[i] = from_f32<T_bf16>(acc[i] * inv);
+  if (lane == 0 && st.lse) st.lse[bh] = (m + log2f(l)) * kLn2;
+
+  // append the token
+  T_bf16* krow = static_cast<T_bf16*>(st.kt) + (((long)b * a.Tcap + t) * a.HQ + h) * KD + lane * QPL;
+  float* crow = st.carry + bh * KD + lane * QPL;
+#pragma unroll
+  for (int i = 0; i < QPL; ++i) {
+    krow[i] = from_f32<T_bf16>(kx[i] * exp2f(R[i] - pv[i]));
+    if (starts) rrow[i] = pv[i];
+    crow[i] = pv[i];
+  }
+  if (g == 0) {
+    T_bf16* vrow = static_cast<T_bf16*>(st.vc) + (((long)b * a.Tcap + t) * a.H + kh) * VD + lane * VPL;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) vrow[i] = from_f32<T_bf16>(vx[i]);
+  }
+}
+
+template <int KD, int VD, int WPH, bool kStep>
+__global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, DecodeArgs a, int G,
-                         int n_items, int stages, int stage_bytes, int* status) {
+                         const __grid_constant__ CUtensorMap tm_v, DecodeArgs a, StepArgs st,
+                         int G, int n_items, int stages, int stage_bytes, int* status) {
   constexpr int VPL = VD / 32;  // value channels per lane
   constexpr int QPL = KD / 32;  // query channels per lane (for the scaled query)
   extern __shared__ uint8_t smem_raw[];
@@ -231,10 +369,15 @@ __global__ void __launch_bounds__(32 * 9, 1)
   float* qts = reinterpret_cast<float*>(smem + stages * stage_bytes);  // [nw][KD]
   float* xch = qts + nw * KD;                       // [G][32][VPL + 2]: second warp's state
   uint64_t* bars = reinterpret_cast<uint64_t*>(xch + G * 32 * (VPL + 2));
+  // a streaming step hands each head's split partial to the finisher warp
+  // through a shared-memory slot [G][VD + 2] (o, m, l) behind the barriers
+  float* pslot = reinterpret_cast<float*>(bars + 2 * stages + (kStep ? 4 : 2) * G);
   auto full = [&](int st) { return smem_u32(&bars[st]); };
   auto empty = [&](int st) { return smem_u32(&bars[stages + st]); };
   auto xfull = [&](int g) { return smem_u32(&bars[2 * stages + g]); };
   auto xempty = [&](int g) { return smem_u32(&bars[2 * stages + G + g]); };
+  auto pfull = [&](int g) { return smem_u32(&bars[2 * stages + 2 * G + g]); };
+  auto pempty = [&](int g) { return smem_u32(&bars[2 * stages + 3 * G + g]); };
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int NC = (a.Tcap + a.C - 1) / a.C;
   const int kps = a.keys_per_split;
@@ -246,6 +389,10 @@ __global__ void __launch_bounds__(32 * 9, 1)
     for (int g = 0; g < G; ++g) {
       mbar_init(xfull(g), 1);
       mbar_init(xempty(g), 1);
+      if (kStep) {
+        mbar_init(pfull(g), 1);
+        mbar_init(pempty(g), 1);
+      }
     }
     fence_barrier_init();
   }
@@ -311,7 +458,11 @@ __global__ void __launch_bounds__(32 * 9, 1)
 #pragma unroll
       for (int i = 0; i < QPL; ++i) {
         qv[i] = to_f32(q[qoff + lane * QPL + i]);
-        pv[i] = a.pc[qoff + lane * QPL + i];
+        if constexpr (kStep)  // P_t = P_{t-1} + g_t / ln 2, rounded as the prefix scan does
+          pv[i] = fmaf(kInvLn2, to_f32(static_cast<const T_bf16*>(st.g)[qoff + lane * QPL + i]),
+                       st.carry[qoff + lane * QPL + i]);
+        else
+          pv[i] = a.pc[qoff + lane * QPL + i];
       }
       float m = -INFINITY, l = 0.f, acc[VPL];
 #pragma unroll
@@ -435,15 +586,76 @@ __global__ void __launch_bounds__(32 * 9, 1)
           l = l * a0 + l1 * a1;
           m = mt;
         }
+        if (!__all_sync(0xffffffffu, got)) ok = false;  // the partial lacks the other warp's keys
         __syncwarp();
         if (lane == 0) mbar_arrive(xempty(g));
       }
-      const long part = ((long)b * a.HQ + h) * a.splits + s;
+      if constexpr (kStep) {
+        // to the finisher through shared memory: no global ordering on this
+        // warp's path.  A split that gave up never hands over, so its head
+        // is left unmerged and the status word reports the timeout.
+        const bool free_slot =
+            n_it == 0 || mbar_wait(pempty(g), (uint32_t)((n_it - 1) & 1), status);
+        if (!__all_sync(0xffffffffu, free_slot)) ok = false;
+        if (!ok) continue;
+        float* slot = pslot + g * (VD + 2);
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) a.ws_o[part * VD + lane * VPL + i] = acc[i];
-      if (lane == 0) {
-        a.ws_ml[part * 2] = m;
-        a.ws_ml[part * 2 + 1] = l;
+        for (int i = 0; i < VPL; ++i) slot[lane * VPL + i] = acc[i];
+        if (lane == 0) {
+          slot[VD] = m;
+          slot[VD + 1] = l;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pfull(g));
+      } else {
+        const long part = ((long)b * a.HQ + h) * a.splits + s;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) a.ws_o[part * VD + lane * VPL + i] = acc[i];
+        if (lane == 0) {
+          a.ws_ml[part * 2] = m;
+          a.ws_ml[part * 2 + 1] = l;
+        }
+      }
+    }
+  } else if constexpr (kStep) {
+    // ------------------------------------------------------------ finisher
+    // Per item: the G heads' partials from the slots to the workspace, one
+    // fence, one arrival per head; the CTA whose split arrives last for a
+    // head merges that head and appends the token (step_merge_append).
+    const float sl2 = a.scale * kLog2e;
+    int n_it = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_it) {
+      int b, kh, s;
+      item_of(it, b, kh, s);
+      bool ok = true;
+      for (int g = 0; g < G; ++g) {
+        const bool got = mbar_wait(pfull(g), (uint32_t)(n_it & 1), status);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        const float* slot = pslot + g * (VD + 2);
+        const long part = ((long)b * a.HQ + kh * G + g) * a.splits + s;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) a.ws_o[part * VD + lane * VPL + i] = slot[lane * VPL + i];
+        if (lane == 0) {
+          a.ws_ml[part * 2] = slot[VD];
+          a.ws_ml[part * 2 + 1] = slot[VD + 1];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pempty(g));
+      }
+      if (!ok) break;
+      __threadfence();  // this item's partials before its arrivals
+      __syncwarp();
+      unsigned prev = 0;
+      if (lane < G) prev = atomicAdd(st.count + (long)b * a.HQ + kh * G + lane, 1u);
+      const unsigned last =
+          __ballot_sync(0xffffffffu, lane < G && prev + 1 == (unsigned)a.splits);
+      if (last != 0u) {
+        __threadfence();  // the other splits' partials after their arrivals
+        for (int g = 0; g < G; ++g)
+          if ((last >> g) & 1u) step_merge_append<KD, VD>(a, st, b, kh * G + g, kh, g, lane, sl2);
       }
     }
   }
@@ -483,9 +695,12 @@ int launch_decode(const DecodeArgs& a, T* o, float* lse, cudaStream_t stream) {
 }
 
 // the streaming kernel's shared memory: stages of (G heads' key boxes, the
-// value box, anchors), the scaled queries and the barriers
-template <int KD, int VD, int WPH>
-int launch_decode_stream(const DecodeArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
+// value box, anchors), the scaled queries and the barriers.  A plain decode
+// merges the split partials in a second kernel; a streaming step merges them
+// inside the first (the last split of each head to finish) and launches once.
+template <int KD, int VD, int WPH, bool kStep>
+int launch_decode_stream(const DecodeArgs& a, const StepArgs& st, __nv_bfloat16* o, float* lse,
+                         cudaStream_t stream) {
   const int G = a.HQ / a.H;
   CUtensorMap tk, tv;
   if (!make_tile_map(&tk, a.kt, (long)a.B * a.Tcap, a.HQ, KD, kDecTile) ||
@@ -493,7 +708,8 @@ int launch_decode_stream(const DecodeArgs& a, __nv_bfloat16* o, float* lse, cuda
     return WALL_ERR_CUDA;
   const int oR = G * (KD / 64) * kDecTile * 128 + (VD / 64) * kDecTile * 128;
   const int stage_bytes = (oR + G * KD * 4 + 1023) & ~1023;
-  const int tail = G * WPH * KD * 4 + G * 32 * (VD / 32 + 2) * 4 + (2 * 4 + 2 * G) * 8;
+  const int tail = G * WPH * KD * 4 + G * 32 * (VD / 32 + 2) * 4 + (2 * 4 + 2 * G) * 8 +
+                   (kStep ? 2 * G * 8 + G * (VD + 2) * 4 : 0);
   const int budget = 227 * 1024 - 1024 - tail;
   int stages = budget / stage_bytes;
   if (stages > 4) stages = 4;
@@ -501,45 +717,56 @@ int launch_decode_stream(const DecodeArgs& a, __nv_bfloat16* o, float* lse, cuda
   const int smem = stages * stage_bytes + tail + 1024;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(decode_stream_kernel<KD, VD, WPH>,
+    if (cudaFuncSetAttribute(decode_stream_kernel<KD, VD, WPH, kStep>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
       return WALL_ERR_CUDA;
     attr = true;
   }
   const int n_items = a.B * a.H * a.splits;
   const int grid = n_items < 148 ? n_items : 148;
-  decode_stream_kernel<KD, VD, WPH><<<grid, 32 * (G * WPH + 1), smem, stream>>>(
-      tk, tv, a, G, n_items, stages, stage_bytes, device_status());
+  const int warps = G * WPH + 1 + (kStep ? 1 : 0);  // consumers, TMA, finisher
+  decode_stream_kernel<KD, VD, WPH, kStep><<<grid, 32 * warps, smem, stream>>>(
+      tk, tv, a, st, G, n_items, stages, stage_bytes, device_status());
   if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+  if (kStep) return WALL_OK;
   decode_merge_kernel<__nv_bfloat16><<<dim3(a.HQ, a.B), 128, 0, stream>>>(a, o, lse);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+template <int WPH, bool kStep>
+int launch_stream_dims(const DecodeArgs& a, const StepArgs& st, __nv_bfloat16* o, float* lse,
+                       cudaStream_t s) {
+  if (a.K == 128 && a.V == 128) return launch_decode_stream<128, 128, WPH, kStep>(a, st, o, lse, s);
+  if (a.K == 128) return launch_decode_stream<128, 64, WPH, kStep>(a, st, o, lse, s);
+  if (a.V == 128) return launch_decode_stream<64, 128, WPH, kStep>(a, st, o, lse, s);
+  return launch_decode_stream<64, 64, WPH, kStep>(a, st, o, lse, s);
+}
+
+// two warps per query head while they fit in the 9-warp CTA
+template <bool kStep>
+int launch_stream(const DecodeArgs& a, const StepArgs& st, __nv_bfloat16* o, float* lse,
+                  cudaStream_t s) {
+  return a.HQ / a.H <= 4 ? launch_stream_dims<2, kStep>(a, st, o, lse, s)
+                         : launch_stream_dims<1, kStep>(a, st, o, lse, s);
+}
+
+// the streaming kernel's domain: bf16, K and V in {64, 128}, up to 8 query
+// heads per kv head, tiles of 32 keys that never straddle a cache chunk, and
+// 16-byte aligned operands for the bulk copies
+bool stream_supported(const DecodeArgs& a) {
+  const int G = a.H > 0 ? a.HQ / a.H : 0;
+  const bool aligned = ((reinterpret_cast<uintptr_t>(a.kt) | reinterpret_cast<uintptr_t>(a.v) |
+                         reinterpret_cast<uintptr_t>(a.rc)) & 15) == 0;
+  return (a.K == 64 || a.K == 128) && (a.V == 64 || a.V == 128) && G >= 1 && G <= 8 &&
+         a.C % kDecTile == 0 && aligned;
 }
 
 template <typename T>
 int decode_dispatch(const DecodeArgs& a, void* o, float* lse, cudaStream_t s) {
   T* out = static_cast<T*>(o);
-  const int G = a.H > 0 ? a.HQ / a.H : 0;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-    // the streaming kernel: bf16, K and V in {64, 128}, up to 8 query heads
-    // per kv head, tiles of 32 keys that never straddle a cache chunk, and
-    // 16-byte aligned operands for the bulk copies
-    const bool aligned = ((reinterpret_cast<uintptr_t>(a.kt) | reinterpret_cast<uintptr_t>(a.v) |
-                           reinterpret_cast<uintptr_t>(a.rc)) & 15) == 0;
-    if ((a.K == 64 || a.K == 128) && (a.V == 64 || a.V == 128) && G >= 1 && G <= 8 &&
-        a.C % kDecTile == 0 && aligned) {
-      // two warps per query head while they fit in the 9-warp CTA
-      int rc;
-      if (G <= 4) {
-        if (a.K == 128 && a.V == 128) rc = launch_decode_stream<128, 128, 2>(a, out, lse, s);
-        else if (a.K == 128) rc = launch_decode_stream<128, 64, 2>(a, out, lse, s);
-        else if (a.V == 128) rc = launch_decode_stream<64, 128, 2>(a, out, lse, s);
-        else rc = launch_decode_stream<64, 64, 2>(a, out, lse, s);
-      } else {
-        if (a.K == 128 && a.V == 128) rc = launch_decode_stream<128, 128, 1>(a, out, lse, s);
-        else if (a.K == 128) rc = launch_decode_stream<128, 64, 1>(a, out, lse, s);
-        else if (a.V == 128) rc = launch_decode_stream<64, 128, 1>(a, out, lse, s);
-        else rc = launch_decode_stream<64, 64, 1>(a, out, lse, s);
-      }
+    if (stream_supported(a)) {
+      const int rc = launch_stream<false>(a, StepArgs{}, out, lse, s);
       if (rc != WALL_ERR_UNSUPPORTED) return rc;
     }
   }
@@ -548,6 +775,21 @@ int decode_dispatch(const DecodeArgs& a, void* o, float* lse, cudaStream_t s) {
   if (k64) return launch_decode<T, 64, 128>(a, out, lse, s);
   if (v64) return launch_decode<T, 128, 64>(a, out, lse, s);
   return launch_decode<T, 128, 128>(a, out, lse, s);
+}
+
+DecodeArgs decode_args(const void* q, const void* v, const float* p_curr, const void* k_tilde,
+                       const float* r_cache, const float* sink, float scale, int C, int B,
+                       int T_kv, int Tcap, int H, int HQ, int K, int V, float* ws, int splits) {
+  DecodeArgs a;
+  a.q = q; a.v = v; a.kt = k_tilde; a.pc = p_curr; a.rc = r_cache; a.sink = sink;
+  a.scale = scale; a.C = C; a.B = B; a.T_kv = T_kv; a.Tcap = Tcap; a.H = H; a.HQ = HQ;
+  a.K = K; a.V = V; a.splits = splits;
+  const long chunks = (T_kv + (long)C - 1) / C;
+  const long chunks_per_split = (chunks + splits - 1) / splits;
+  a.keys_per_split = (int)(chunks_per_split * C);
+  a.ws_o = ws;
+  a.ws_ml = ws + (long)B * HQ * splits * V;
+  return a;
 }
 
 }  // namespace
@@ -588,17 +830,25 @@ int attn_decode(const void* q, const void* v, const float* p_curr, const void* k
                 int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse, float* ws,
                 int splits, cudaStream_t stream) {
   if (B == 0) return WALL_OK;
-  DecodeArgs a;
-  a.q = q; a.v = v; a.kt = k_tilde; a.pc = p_curr; a.rc = r_cache; a.sink = sink;
-  a.scale = scale; a.C = C; a.B = B; a.T_kv = T_kv; a.Tcap = Tcap; a.H = H; a.HQ = HQ;
-  a.K = K; a.V = V; a.splits = splits;
-  const long chunks = (T_kv + (long)C - 1) / C;
-  const long chunks_per_split = (chunks + splits - 1) / splits;
-  a.keys_per_split = (int)(chunks_per_split * C);
-  a.ws_o = ws;
-  a.ws_ml = ws + (long)B * HQ * splits * V;
+  const DecodeArgs a = decode_args(q, v, p_curr, k_tilde, r_cache, sink, scale, C, B, T_kv, Tcap,
+                                   H, HQ, K, V, ws, splits);
   return dtype == WALL_BF16 ? decode_dispatch<__nv_bfloat16>(a, o, lse, stream)
                             : decode_dispatch<float>(a, o, lse, stream);
+}
+
+int decode_step(const void* q, const void* k, const void* v, const void* g, float* carry,
+                void* k_tilde, void* v_cache, float* r_cache, const float* sink, float scale,
+                int C, int t, int B, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
+                float* ws, unsigned* counters, int splits, cudaStream_t stream) {
+  if (B == 0) return WALL_OK;
+  // the cache holds positions [0, t); the new token is merged in by the kernel
+  const DecodeArgs a = decode_args(q, v_cache, nullptr, k_tilde, r_cache, sink, scale, C, B, t,
+                                   Tcap, H, HQ, K, V, ws, splits);
+  if (!stream_supported(a)) return WALL_ERR_UNSUPPORTED;
+  StepArgs st;
+  st.k = k; st.v = v; st.g = g; st.carry = carry; st.kt = k_tilde; st.vc = v_cache;
+  st.rc = r_cache; st.count = counters; st.o = o; st.lse = lse; st.t = t;
+  return launch_stream<true>(a, st, static_cast<__nv_bfloat16*>(o), lse, stream);
 }
 
 }  // namespace wall

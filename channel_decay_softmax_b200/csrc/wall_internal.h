@@ -16,7 +16,7 @@ namespace wall {
 void timing_mark(int slot, cudaStream_t stream);
 enum TimingSlot {
   T_PREFIX = 0, T_OPERANDS = 1, T_FWD = 2, T_BWD_PRE = 3, T_BWD_KEY = 4, T_BWD_DQ = 5,
-  T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9,
+  T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9, T_STEP = 10,
 };
 
 // ---- scans (wall_scan.cu) ----
@@ -106,5 +106,12 @@ int attn_decode(const void* q, const void* v, const float* p_curr, const void* k
                 const float* r_cache, const float* sink, float scale, int C, int dtype, int B,
                 int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
                 float* ws, int splits, cudaStream_t stream);
+// one streaming token: prefix update, cache append and decode in one launch;
+// WALL_ERR_UNSUPPORTED outside the streaming kernel's domain (bf16, K and V
+// in {64, 128}, HQ/H <= 8, C % 32 == 0, 16-byte aligned caches)
+int decode_step(const void* q, const void* k, const void* v, const void* g, float* carry,
+                void* k_tilde, void* v_cache, float* r_cache, const float* sink, float scale,
+                int C, int t, int B, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
+                float* ws, unsigned* counters, int splits, cudaStream_t stream);
 
 }  // namespace wall

@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(32 * kCarryParts)
   }
   if (carry_out != nullptr && valid && part == 0) {
     const float cin = carry_in != nullptr ? carry_in[(long)s * C + col] : 0.f;
-    carry_out[(long)s * C + col] = cin + mul * (float)all;
+    carry_out[(long)s * C + col] = fmaf(mul, (float)all, cin);
   }
 }
 
@@ -200,7 +200,8 @@ __global__ void __launch_bounds__(kThreadsScan)
       const float tk = acc[v] + yk;
       cmp[v] = (tk - acc[v]) - yk;
       acc[v] = tk;
-      o[v] = cin[v] + mul * acc[v];
+      // one fused rounding; the one-token decode step forms P the same way
+      o[v] = fmaf(mul, acc[v], cin[v]);
     }
     if (r < n) {
       if (VEC == 8) {

@@ -23,7 +23,8 @@ bool g_on = false;
 Slot g_slot[WALL_TIMING_SLOTS];
 const char* const kNames[WALL_TIMING_SLOTS] = {
     "prefix_scan", "operands", "fwd_tc", "bwd_pre", "bwd_keyblock",
-    "bwd_dq", "bwd_finalize", "reverse_scan", "decode", "cache_build"};
+    "bwd_dq", "bwd_finalize", "reverse_scan", "decode", "cache_build",
+    "decode_step"};
 
 }  // namespace
 

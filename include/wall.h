@@ -213,6 +213,57 @@ int wall_attn_decode_noalloc(const void* q, const void* v, const float* p_curr,
                              float scale, int C, int dtype, int B, int T_kv, int Tcap, int H,
                              int HQ, int K, int V, void* o, float* lse, wall_stream_t stream);
 
+/* wall_decode_step_workspace -- bytes of workspace wall_decode_step needs
+ * for a cache of capacity Tcap (enough for every t < Tcap). */
+size_t wall_decode_step_workspace(int B, int Tcap, int H, int HQ, int V, int C);
+
+/*
+ * wall_decode_step -- one token of the streaming decode loop in ONE launch:
+ * prefix update, cache append and decode (README "Decode": the prefix is the
+ * running sum of g / ln 2 and the cache holds k * exp2(R_c - P) with a
+ * per-chunk anchor R_c; appending a token and decoding it are the serving
+ * loop's two halves, fused here so a token costs one kernel launch).
+ *
+ * With t the number of tokens already cached (0 <= t < Tcap), for every batch
+ * row b and query head h (kv head h/G):
+ *   P_t = carry[b,h,:] + g[b,h,:] / ln 2            (fp32, one fused rounding,
+ *                                                    as wall_prefix_cumsum)
+ *   o, lse = decode of q[b,h,:] at P_t over positions 0 .. t: the cached
+ *            positions as wall_attn_decode scores them, plus the new token,
+ *            whose decay factor exp2(P_t - P_t) is 1, so its score is
+ *            scale * q . k[b,h/G,:] taken from the input directly
+ *   appends: r_cache[b,t/C,h,:] = P_t if t % C == 0 (a new chunk's anchor);
+ *            k_tilde[b,t,h,:] = k[b,h/G,:] * exp2(r_cache[b,t/C,h,:] - P_t)
+ *            rounded to bf16 as wall_build_kv_cache rounds it;
+ *            v_cache[b,t,h/G,:] = v[b,h/G,:];  carry[b,h,:] = P_t
+ * After the call the cache and carry are exactly what wall_prefix_cumsum
+ * (with carry_in / carry_out) and wall_build_kv_cache (t0 = t) would leave.
+ * In:  q [B,HQ,K], k [B,H,K], v [B,H,V], g [B,HQ,K] (bf16: `dtype` must be
+ *      WALL_BF16), sink_bias [HQ] fp32 or NULL, scale (<= 0: K^-0.5).
+ * In/out: carry [B,HQ,K] fp32 (P at t-1 in; zeros for t == 0 of a fresh
+ *      sequence), k_tilde [B,Tcap,HQ,K] bf16, v_cache [B,Tcap,H,V] bf16,
+ *      r_cache [B,ceil(Tcap/C),HQ,K] fp32: positions [0, t) are read, row t
+ *      (and chunk t/C when t starts it) written.
+ * Out: o [B,HQ,V] bf16, lse [B,HQ] fp32 natural log (may be NULL).
+ * Workspace: wall_decode_step_workspace(B, Tcap, H, HQ, V, C) bytes, 16-byte
+ * aligned, caller-owned.  Its tail holds per-head arrival counters of the
+ * split-KV partials: they must be ZERO before the first call (clear the whole
+ * workspace once) and every call that returns WALL_OK and whose status
+ * (wall_get_status) is WALL_OK leaves them zero again; after a device timeout
+ * clear the workspace before the next call.  Calls sharing a workspace must
+ * not overlap on the GPU.
+ * Supported: bf16, K and V in {64, 128}, HQ/H <= 8, C a multiple of 32;
+ * anything else returns WALL_ERR_UNSUPPORTED before any launch (append with
+ * wall_prefix_cumsum + wall_build_kv_cache and decode with wall_attn_decode
+ * instead).  Errors: WALL_ERR_INVALID_ARG for null or misaligned pointers,
+ * t outside [0, Tcap), a short workspace or bad shapes.
+ */
+int wall_decode_step(const void* q, const void* k, const void* v, const void* g, int dtype,
+                     float* carry, void* k_tilde, void* v_cache, float* r_cache,
+                     const float* sink_bias, float scale, int C, int t, int B, int Tcap, int H,
+                     int HQ, int K, int V, void* o, float* lse, void* workspace,
+                     size_t workspace_bytes, wall_stream_t stream);
+
 /*
  * wall_get_status -- synchronizes `stream`, returns the device status word
  * (WALL_OK or WALL_ERR_TIMEOUT) and clears it.  Returns WALL_ERR_CUDA if the
@@ -246,10 +297,11 @@ int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
  *   7 reverse_scan    the reverse scan(s) of wall_attn_bwd
  *   8 decode          wall_attn_decode (split and merge kernels)
  *   9 cache_build     wall_build_kv_cache
+ *  10 decode_step     wall_decode_step (one launch per token)
  * wall_timing_enable(1) starts recording (and clears the totals);
  * wall_timing_enable(0) stops.  Not thread-safe: one host thread at a time.
  */
-#define WALL_TIMING_SLOTS 10
+#define WALL_TIMING_SLOTS 11
 int wall_timing_enable(int on);
 
 /*

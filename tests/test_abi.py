@@ -104,6 +104,33 @@ def test_cache_and_decode_reject_bad_arguments(lib):
     assert dec(*args, 10, 10, 2, 4, 64, 64, FAKE, FAKE, FAKE, 8, None) == L.WALL_ERR_INVALID_ARG
 
 
+def test_decode_step_rejects_bad_arguments(lib):
+    st = lib.wall_decode_step
+    B, Tcap, H, HQ, K, V, C = 2, 256, 2, 8, 128, 128, 64
+    need = lib.wall_decode_step_workspace(B, Tcap, H, HQ, V, C)
+    # the counters follow the split partials sized for the capacity
+    al = lambda x: (x + 255) // 256 * 256
+    assert need > al(4 * B * HQ) and (need - al(4 * B * HQ)) % 256 == 0
+
+    def call(dtype=0, t=10, C=C, H=H, HQ=HQ, K=K, V=V, ws_bytes=need, q=FAKE, kt=FAKE,
+             carry=FAKE):
+        return st(q, FAKE, FAKE, FAKE, dtype, carry, kt, FAKE, FAKE, None, 0.0, C, t, B, Tcap,
+                  H, HQ, K, V, FAKE, None, FAKE, ws_bytes, None)
+
+    assert call(dtype=2) == L.WALL_ERR_INVALID_ARG           # unknown dtype
+    assert call(t=-1) == L.WALL_ERR_INVALID_ARG              # before the sequence
+    assert call(t=Tcap) == L.WALL_ERR_INVALID_ARG            # no room to append
+    assert call(dtype=1) == L.WALL_ERR_UNSUPPORTED           # fp32: three-call path instead
+    assert call(K=96) == L.WALL_ERR_UNSUPPORTED              # head size outside {64, 128}
+    assert call(C=48) == L.WALL_ERR_UNSUPPORTED              # chunk not a multiple of 32
+    assert call(H=1, HQ=16) == L.WALL_ERR_UNSUPPORTED        # 16 query heads per kv head
+    assert call(q=None) == L.WALL_ERR_INVALID_ARG
+    assert call(kt=FAKE + 8) == L.WALL_ERR_INVALID_ARG       # misaligned cache
+    assert call(carry=None) == L.WALL_ERR_INVALID_ARG
+    assert call(ws_bytes=need - 1) == L.WALL_ERR_INVALID_ARG  # workspace too small
+    assert lib.wall_decode_step_workspace(1, 0, 1, 1, 64, 64) == 0
+
+
 def test_prefix_rejects_bad_arguments(lib):
     pc = lib.wall_prefix_cumsum
     assert pc(FAKE, 3, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG

@@ -123,10 +123,11 @@ def test_decode_single_step_full_size_sampled():
         assert_fwd(s.dtype, o[b, 0], o_ref[0, -1], lse[b, 0], l_ref[0, -1], what=f"b={b}")
 
 
-def _streaming(s, n_stream, check_prefill):
+def _streaming(s, n_stream, check_prefill, fused=None):
     """Build the cache from [0, T - n) then append n tokens one by one; each
     decoded row must equal the oracle's forward row (and the GPU prefill
-    forward row)."""
+    forward row).  ``fused`` picks the one-launch step or the three-call
+    append + decode (default: the fused step where it applies)."""
     x = _stack(s, n_rows=n_stream)
     k, v, g = x["k"].to(DEV), x["v"].to(DEV), x["g"].to(DEV)
     q_tail = x["q"].to(DEV)
@@ -137,7 +138,7 @@ def _streaming(s, n_stream, check_prefill):
     outs, lses = [], []
     for t in range(T0, s.T):
         o, lse = cache.step(q_tail[:, t - T0:t - T0 + 1], k[:, t:t + 1], v[:, t:t + 1],
-                            g[:, t:t + 1])
+                            g[:, t:t + 1], fused=fused)
         outs.append(o)
         lses.append(lse)
     torch.cuda.synchronize()
@@ -156,8 +157,74 @@ def _streaming(s, n_stream, check_prefill):
         assert_fwd(s.dtype, o_stream, o_pf[:, T0:], what="stream vs prefill")
 
 
-def test_streaming_loop_small():
-    _streaming(_small_decode_spec(T=700), 64, check_prefill=True)
+@pytest.mark.parametrize("fused", [True, False], ids=["fused_step", "three_call"])
+def test_streaming_loop_small(fused):
+    _streaming(_small_decode_spec(T=700), 64, check_prefill=True, fused=fused)
+
+
+def _step_cache(s, x, T0, fused, sink=None):
+    """Cache of capacity T with positions [0, T0) appended at once, then
+    T - T0 single-token steps; returns the cache and the decoded rows."""
+    k, v, g, q = (x[n].to(DEV) for n in ("k", "v", "g", "q"))
+    cache = api.WallDecodeCache(s.B, s.H, s.HQ, s.K, s.V, capacity=s.T, chunk_size=s.chunk,
+                                dtype=s.dtype, device=DEV, scale=s.scale, sink_bias=sink)
+    if T0 > 0:
+        cache.append(k[:, :T0], v[:, :T0], g[:, :T0])
+    outs, lses = [], []
+    for t in range(T0, s.T):
+        o, lse = cache.step(q[:, t - T0:t - T0 + 1], k[:, t:t + 1], v[:, t:t + 1],
+                            g[:, t:t + 1], fused=fused)
+        outs.append(o)
+        lses.append(lse)
+    torch.cuda.synchronize()
+    return cache, torch.cat(outs, 1), torch.cat(lses, 1)
+
+
+def test_decode_step_matches_three_call_path():
+    """The fused step leaves the carry, k_tilde, v and r_cache bit for bit as
+    the prefix scan + cache build + value copy do (the same fp32 operations:
+    P_t = carry + g / ln 2 in one fused rounding, k * exp2(R - P_t) rounded
+    to bf16), across chunk starts at 128 and 192.  Its decoded rows agree to
+    bf16 rounding: the new token's own score comes from k itself (factor
+    exp2(0) = 1), not from its rounded k_tilde row.  Every call leaves the
+    per-head arrival counters at zero."""
+    s = _small_decode_spec(B=2, T=300, HQ=8, H=2)
+    T0 = 100
+    x = _stack(s, n_rows=s.T - T0)
+    cf, of, lf = _step_cache(s, x, T0, fused=True)
+    c3, o3, l3 = _step_cache(s, x, T0, fused=False)
+    assert torch.equal(cf.carry, c3.carry)
+    assert torch.equal(cf.k_tilde, c3.k_tilde)
+    assert torch.equal(cf.v, c3.v)
+    assert torch.equal(cf.r_cache, c3.r_cache)
+    assert_fwd(s.dtype, of, o3, lf, l3, what="fused vs three-call")
+    al = lambda n: (n + 255) // 256 * 256
+    counters = cf.step_ws[-al(4 * s.B * s.HQ):]
+    assert int(counters.count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("HQ,H,K,V,C,sink", [
+    (8, 1, 64, 64, 32, True),     # 8 heads per kv head (one warp per head), sink
+    (4, 2, 128, 64, 64, False),   # K != V
+    (2, 2, 64, 128, 96, True),    # no grouping, a chunk that is not a power of two
+])
+def test_decode_step_from_empty_cache(HQ, H, K, V, C, sink):
+    """Streaming from an empty cache (t = 0 decodes the token against itself
+    only): every row equals the oracle's forward row, with the sink logit."""
+    s = _small_decode_spec(B=2, T=200, HQ=HQ, H=H, K=K, V=V, chunk=C)
+    x = _stack(s, n_rows=s.T)
+    sk = None
+    if sink:
+        gen = torch.Generator().manual_seed(77)
+        sk = torch.randn((HQ,), generator=gen, dtype=torch.float32)
+    cache, o, lse = _step_cache(s, x, 0, fused=True,
+                                sink=sk.to(DEV) if sk is not None else None)
+    assert cache.fused
+    for b in range(s.B):
+        o_ref, l_ref = wo.forward(x["q"][b:b + 1], x["k"][b:b + 1], x["v"][b:b + 1],
+                                  x["g"][b:b + 1], scale=s.scale, sink_bias=sk,
+                                  rows=(0, s.T), q_rows_only=True)
+        assert_fwd(s.dtype, o[b], o_ref[0], lse[b], l_ref[0], what=f"step b={b}")
 
 
 @pytest.mark.slow
