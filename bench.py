@@ -9,8 +9,9 @@ step = prefix scan + forward + backward (dq, dk, dv, dg with the reverse
 scan), counting causal FLOPs: forward 2 * pairs * (K + V) per head,
 backward 2.5x that.  The same line carries the decode numbers (B=32,
 T_kv=32768, HQ=32, H=8, K=V=128, C=64): GB/s and tokens/s of one decode
-step, the cache build and prefix scan GB/s, and the 64-token streaming
-append loop.
+step, the cache build and prefix scan GB/s, the 64-token streaming
+append loop, and the same 64 positions' queries as one chunk against the
+cache (multi-token decode / chunked prefill).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
 the same workload on its own data (weak scaling, no collective on the data
@@ -324,6 +325,7 @@ def bench_train_e2e(args, x, s, step_flops, world):
 
 
 def bench_decode(args, rank, peaks):
+    from channel_decay_softmax_b200 import _lib as L
     from channel_decay_softmax_b200 import api
 
     over = {"B": args.decode_batch} if args.decode_batch else {}
@@ -335,23 +337,34 @@ def bench_decode(args, rank, peaks):
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     out = {}
+
+    def timed(fn, reps=3):
+        """ms per call of fn after one warm-up call (outputs preallocated)"""
+        fn()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
     # prefix scan over the whole cache's gates (B*T*HQ*K elements)
-    a, b = ev(), ev()
-    a.record(stream)
-    P = api.prefix_cumsum(d["g"])
-    b.record(stream)
-    torch.cuda.synchronize()
+    Bq, Tg, HQ, K = d["g"].shape
+    P = torch.empty((Bq, Tg, HQ, K), dtype=torch.float32, device="cuda")
+    ms_p = timed(lambda: L.wall_prefix_cumsum(d["g"], P, Bq, Tg, HQ, K))
     n_el = d["g"].numel()
-    out["prefix_gbs"] = n_el * (2 + 4) / (a.elapsed_time(b) * 1e-3) / 1e9
+    out["prefix_gbs"] = n_el * (2 + 4) / (ms_p * 1e-3) / 1e9
     # cache build over positions [0, T)
-    a, b = ev(), ev()
-    a.record(stream)
-    kt, rc = api.build_wall_kv_cache(d["k"], P, chunk_size=s.chunk)
-    b.record(stream)
-    torch.cuda.synchronize()
+    kt = torch.empty((s.B, T, s.HQ, s.K), dtype=s.dtype, device="cuda")
+    rc = torch.empty((s.B, I.ceil_div(T, s.chunk), s.HQ, s.K), dtype=torch.float32, device="cuda")
+    ms_cb = timed(lambda: L.wall_build_kv_cache(d["k"], P, s.B, T, s.H, s.HQ, s.K, s.chunk, 0,
+                                                kt, rc, T))
     cb_bytes = d["k"].numel() * 2 + P.numel() * 4 + kt.numel() * 2 + rc.numel() * 4
-    out["cache_build_gbs"] = cb_bytes / (a.elapsed_time(b) * 1e-3) / 1e9
+    out["cache_build_gbs"] = cb_bytes / (ms_cb * 1e-3) / 1e9
     p_last = P[:, -1:].contiguous()
+    p_tail = P[:, T - n_stream:].contiguous()
     del P
     q_last = d["q_tail"][:, -1:].contiguous()
 
@@ -375,6 +388,32 @@ def bench_decode(args, rank, peaks):
     out.update(decode_ms=ms, decode_gbs=gbs, decode_frac_hbm=gbs / peaks["hbm_gbs"],
                tokens_per_s=s.B / (ms * 1e-3), decode_bytes=nbytes,
                decode_launches_per_step=2)
+    # the last 64 positions' queries as one chunk against the full cache
+    # (multi-token decode / chunked prefill: row i at position T - 64 + i)
+
+    def chunk():
+        return api.wall_attn_decode_chunk(d["q_tail"], d["v"], p_tail, kt, rc, scale=s.scale,
+                                          cache_chunk_size=s.chunk)
+
+    for _ in range(max(3, args.warmup)):
+        chunk()
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(reps):
+        chunk()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_c = a.elapsed_time(b) / reps
+    esz = 2
+    c_bytes = (kt.numel() * esz + d["v"].numel() * esz + rc.numel() * 4 +
+               s.B * n_stream * s.HQ * (s.K * esz + s.K * 4 + s.V * esz + 4))
+    c_flops = 2.0 * s.B * s.HQ * (s.K + s.V) * sum(t + 1 for t in range(T - n_stream, T))
+    out.update(chunk_rows=n_stream, chunk_ms=ms_c,
+               chunk_gbs=c_bytes / (ms_c * 1e-3) / 1e9,
+               chunk_frac_hbm=c_bytes / (ms_c * 1e-3) / 1e9 / peaks["hbm_gbs"],
+               chunk_tokens_per_s=s.B * n_stream / (ms_c * 1e-3),
+               chunk_tflops=c_flops / (ms_c * 1e-3) / 1e12, chunk_launches=2)
     del kt, rc
     torch.cuda.empty_cache()
     # streaming append loop: cache of [0, T0) then 64 appended tokens, once
@@ -544,12 +583,14 @@ def main(argv=None):
         if dec is not None:
             line["decode"] = dec
         if world == 1 and not args.no_cpu:
-            v, sec, threads = oracle_sample_tflops(int(os.environ.get("WALL_CPU_T", "1536")))
+            # about 10-15 s of host work (the cost grows with the square of
+            # the sampled rows)
+            v, sec, threads = oracle_sample_tflops(int(os.environ.get("WALL_CPU_T", "4608")))
             line["cpu_baseline"] = {
                 "value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                 "seconds": sec,
                 "sample": "fp64 oracle fwd+bwd on rows [0,%s) of the T=8192 workload, all 16 "
-                          "heads" % os.environ.get("WALL_CPU_T", "1536")}
+                          "heads" % os.environ.get("WALL_CPU_T", "4608")}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

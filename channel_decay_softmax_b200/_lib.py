@@ -20,7 +20,8 @@ EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn
            "wall_attn_fwd", "wall_attn_bwd_workspace", "wall_attn_bwd", "wall_build_kv_cache",
            "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
            "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
-           "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step"]
+           "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step",
+           "wall_attn_decode_chunk_workspace", "wall_attn_decode_chunk"]
 
 _lib = None
 
@@ -81,6 +82,11 @@ def lib():
         L.wall_decode_step.restype = i
         L.wall_decode_step.argtypes = [vp, vp, vp, vp, i, fp, vp, vp, fp, fp, f, i, i, i, i, i,
                                        i, i, i, vp, fp, vp, sz, vp]
+        L.wall_attn_decode_chunk_workspace.restype = sz
+        L.wall_attn_decode_chunk_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.wall_attn_decode_chunk.restype = i
+        L.wall_attn_decode_chunk.argtypes = [vp, vp, fp, vp, fp, fp, f, i, i, i, i, i, i, i, i,
+                                             i, i, vp, fp, vp, sz, vp]
         _lib = L
     return _lib
 
@@ -206,3 +212,17 @@ def wall_decode_step(q, k, v, g, carry, k_tilde, v_cache, r_cache, sink_bias, sc
         _p(q), _p(k), _p(v), _p(g), dtype_code(q.dtype), _p(carry), _p(k_tilde), _p(v_cache),
         _p(r_cache), _p(sink_bias), float(scale), C, t, B, Tcap, H, HQ, K, V, _p(o), _p(lse),
         _p(workspace), ws_bytes, _stream(stream)))
+
+
+def wall_attn_decode_chunk_workspace(dtype, B, Tq, T_kv, H, HQ, K, V, C) -> int:
+    return lib().wall_attn_decode_chunk_workspace(dtype, B, Tq, T_kv, H, HQ, K, V, C)
+
+
+def wall_attn_decode_chunk(q, v, p, k_tilde, r_cache, sink_bias, scale, C, B, Tq, T_kv, Tcap, H,
+                           HQ, K, V, o, lse, workspace, stream=None):
+    """Tq queries per batch row at the last Tq cached positions, one call."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_attn_decode_chunk", lib().wall_attn_decode_chunk(
+        _p(q), _p(v), _p(p), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
+        dtype_code(q.dtype), B, Tq, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _p(workspace),
+        ws_bytes, _stream(stream)))

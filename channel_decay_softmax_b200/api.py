@@ -163,6 +163,30 @@ def wall_attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias=None, scale=None,
     return o, lse
 
 
+def wall_attn_decode_chunk(q, v, p, k_tilde, r_cache, sink_bias=None, scale=None,
+                           cache_chunk_size=64, T_kv=None):
+    """Multi-token decode / chunked prefill against the pre-rescaled cache:
+    q [B,Tq,HQ,K] and p [B,Tq,HQ,K] (P at their positions) are the queries of
+    the last Tq of the first T_kv cached positions (default: all), each
+    attending causally to the cache up to its own position.  Returns
+    (o [B,Tq,HQ,V], lse [B,Tq,HQ])."""
+    B, Tcap, HQ, K = k_tilde.shape
+    H, V = v.shape[2], v.shape[3]
+    Tq = q.shape[1]
+    T_kv = Tcap if T_kv is None else int(T_kv)
+    if v.shape[1] != Tcap:
+        raise ValueError("v and k_tilde must have the same capacity")
+    o = torch.empty((B, Tq, HQ, V), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, Tq, HQ), dtype=torch.float32, device=q.device)
+    C = int(cache_chunk_size)
+    ws = _ws(L.wall_attn_decode_chunk_workspace(L.dtype_code(q.dtype), B, Tq, T_kv, H, HQ, K, V,
+                                                C), q.device)
+    sk = sink_bias.contiguous().float() if sink_bias is not None else None
+    L.wall_attn_decode_chunk(q.contiguous(), v, p.contiguous(), k_tilde, r_cache, sk,
+                             scale or 0.0, C, B, Tq, T_kv, Tcap, H, HQ, K, V, o, lse, ws)
+    return o, lse
+
+
 class WallDecodeCache:
     """Append-as-you-go decode state (README "Decode": the streaming serving
     loop): cache buffers of a fixed capacity plus the running prefix.
@@ -217,6 +241,14 @@ class WallDecodeCache:
         return wall_attn_decode(q, self.v, p_curr, self.k_tilde, self.r_cache, self.sink,
                                 self.scale, self.C, T_kv=self.length)
 
+    def extend(self, q, k, v, g):
+        """Appends Tn tokens and attends all their queries at once (chunked
+        prefill / multi-token decode): q [B,Tn,HQ,K], k [B,Tn,H,K],
+        v [B,Tn,H,V], g [B,Tn,HQ,K]; returns (o [B,Tn,HQ,V], lse [B,Tn,HQ])."""
+        P = self.append(k, v, g)
+        return wall_attn_decode_chunk(q, self.v, P, self.k_tilde, self.r_cache, self.sink,
+                                      self.scale, self.C, T_kv=self.length)
+
     def step(self, q, k, v, g, fused=None):
         """Appends one token and decodes its query; returns (o, lse).
         q [B,1,HQ,K], k [B,1,H,K], v [B,1,H,V], g [B,1,HQ,K].  ``fused=False``
@@ -253,7 +285,7 @@ def timing_read():
     """Per-stage {name: (launches, total_ms)} since the last read or enable;
     synchronizes on the recorded events and clears the totals."""
     import ctypes
-    n = 11
+    n = 12
     names = (ctypes.c_char_p * n)()
     launches = (ctypes.c_int * n)()
     ms = (ctypes.c_double * n)()

@@ -147,6 +147,29 @@ BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
 
 inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
+// wall_attn_decode_chunk's workspace: the anchored queries and their block
+// anchors (tensor-core path) or the split partials (split path)
+struct ChunkWs {
+  bool tc;
+  int splits;
+  size_t qh, anchors, total;
+};
+ChunkWs chunk_ws_layout(int dtype, int B, int Tq, int T_kv, int H, int HQ, int K, int V, int C) {
+  ChunkWs w;
+  w.tc = decode_chunk_tc_supported(dtype, K, V, C);
+  w.splits = 0;
+  w.qh = w.anchors = 0;
+  if (w.tc) {
+    const size_t nqb = (size_t)B * ((Tq + 127) / 128);
+    w.anchors = align256((size_t)2 * B * Tq * HQ * K);
+    w.total = w.anchors + align256(sizeof(float) * nqb * HQ * K);
+  } else {
+    w.splits = decode_chunk_splits(B, Tq, T_kv, H, C);
+    w.total = align256(sizeof(float) * (size_t)B * Tq * HQ * w.splits * (V + 2));
+  }
+  return w;
+}
+
 }  // namespace
 
 int* device_status() { return status_ptr(); }
@@ -396,6 +419,51 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
                              Tcap, H, HQ, K, V, o, lse, static_cast<float*>(workspace), S,
                              reinterpret_cast<cudaStream_t>(stream));
   timing_mark(T_DECODE, reinterpret_cast<cudaStream_t>(stream));
+  return rc;
+}
+
+size_t wall_attn_decode_chunk_workspace(int dtype, int B, int Tq, int T_kv, int H, int HQ, int K,
+                                        int V, int C) {
+  if (B < 0 || Tq < 0 || T_kv < 1 || Tq > T_kv || H < 1 || HQ < 1 || HQ % H != 0 || K < 1 ||
+      V < 1 || C < 1)
+    return 0;
+  return chunk_ws_layout(dtype, B, Tq, T_kv, H, HQ, K, V, C).total;
+}
+
+int wall_attn_decode_chunk(const void* q, const void* v, const float* p, const void* k_tilde,
+                           const float* r_cache, const float* sink_bias, float scale, int C,
+                           int dtype, int B, int Tq, int T_kv, int Tcap, int H, int HQ, int K,
+                           int V, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                           wall_stream_t stream) {
+  if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
+  if (B < 0 || Tq < 0 || T_kv < 1 || Tq > T_kv || Tcap < T_kv || H < 1 || HQ < 1 ||
+      HQ % H != 0 || C < 1)
+    return WALL_ERR_INVALID_ARG;
+  if (!ok_head_dim(K) || !ok_head_dim(V) || HQ / H > 32) return WALL_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || HQ > 65535) return WALL_ERR_UNSUPPORTED;
+  if ((long)B * Tq == 0) return WALL_OK;
+  const ChunkWs w = chunk_ws_layout(dtype, B, Tq, T_kv, H, HQ, K, V, C);
+  // grid rows: query rows (split path) or 128-row query blocks (tensor cores)
+  if ((long)B * (w.tc ? (Tq + 127) / 128 : Tq) > 65535) return WALL_ERR_UNSUPPORTED;
+  if (!ok_ptr(q) || !ok_ptr(v) || !ok_ptr(p) || !ok_ptr(k_tilde) || !ok_ptr(r_cache) ||
+      !ok_ptr(o) || !ok_opt(sink_bias) || !ok_opt(lse))
+    return WALL_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace))
+    return WALL_ERR_INVALID_ARG;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)K);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  timing_mark(T_CHUNK, st);
+  int rc;
+  if (w.tc)
+    rc = attn_decode_chunk_tc(q, v, p, k_tilde, r_cache, sink_bias, sc, C, B, Tq, T_kv, Tcap, H,
+                              HQ, K, reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh)),
+                              reinterpret_cast<float*>(at(workspace, w.anchors)), o, lse,
+                              status_ptr(), st);
+  else
+    rc = attn_decode_chunk_split(q, v, p, k_tilde, r_cache, sink_bias, sc, C, dtype, B, Tq, T_kv,
+                                 Tcap, H, HQ, K, V, o, lse, static_cast<float*>(workspace),
+                                 w.splits, st);
+  timing_mark(T_CHUNK, st);
   return rc;
 }
 

@@ -69,16 +69,25 @@ struct FwdTcParams {
   int window;
   int n_blocks;          // grid bound on 128-row blocks
   int* status;
+  // a chunk of queries against the decode cache (kCache kernels only): keys
+  // are k_tilde rows, whose factor against the query block is
+  // 2^(R_I - R_c) with R_c the anchor of the key's cache chunk
+  const float* rc;       // r_cache [B, NC, HQ, K]
+  int C, NC;             // cache chunk size, r_cache chunks per batch row
+  int t_off;             // cache position of query row 0 (T_kv - Tq)
+  int T_kv;              // cached positions per batch row
 };
 
-template <int KD>
+template <int KD, bool kCache>
 struct Smem {
+  // anchor rows per key stage: a cache tile spans up to 128 / 32 chunks
+  static constexpr int kRJRows = kCache ? 4 : 1;
   static constexpr int kT = BN * KD * 2;          // one 128-row bf16 tile
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kT;              // kKS stages
   static constexpr int oV = oK + kKS * kT;        // kVS stages
-  static constexpr int oRJ = oV + kVS * kT;        // float[kKS][KD] key-block anchors
-  static constexpr int oGS = oRJ + kKS * KD * 4;  // float[8 warps][BN] key prefix
+  static constexpr int oRJ = oV + kVS * kT;        // float[kKS][kRJRows][KD] key anchors
+  static constexpr int oGS = oRJ + kKS * kRJRows * KD * 4;  // float[8 warps][BN] key prefix
   static constexpr int oX = oGS + 8 * BN * 4;     // float[2 groups][2][BM]: m, l
   static constexpr int oBar = oX + 2 * 2 * BM * 4;
   static constexpr int kBars = 22;
@@ -131,11 +140,19 @@ __device__ __forceinline__ uint32_t pow2_bf16(float k) {
   return e < -126 ? 0u : e > 127 ? 0x7F80u : uint32_t(e + 127) << 7;
 }
 
-template <int KD>
+// Cache position of the first key tile's chunk and the number of the tile's
+// chunks that hold cached positions (kCache kernels).
+__device__ __forceinline__ int cache_tile_chunks(const FwdTcParams& p, int j0, int& c0) {
+  c0 = j0 / p.C;
+  const int nc = p.C >= BN ? 1 : BN / p.C;
+  return min(nc, (p.T_kv + p.C - 1) / p.C - c0);
+}
+
+template <int KD, bool kCache>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, FwdTcParams p) {
-  using Lay = Smem<KD>;
+  using Lay = Smem<KD, kCache>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -157,10 +174,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!seq_block(p.seqs, BM, flat, seq, blk)) return;
   const int blk_off = flat - blk;
   const long s0 = p.seqs.start(seq);
-  const int L = p.seqs.len(seq);
+  const int Lq = p.seqs.len(seq);            // query rows of this sequence
+  // keys: the same rows, or the cache's positions; query row i sits at
+  // position i, or t_off + i in the cache
+  const int L = kCache ? p.T_kv : Lq;
+  const int pos0 = kCache ? p.t_off : 0;
   const int i0 = blk * BM;
-  const int ni = min(BM, L - i0);
-  const int jb_hi = (i0 + ni - 1) / BN;
+  const int ni = min(BM, Lq - i0);
+  const int jb_hi = (pos0 + i0 + ni - 1) / BN;
   const int jb_lo = p.window > 0 ? max(0, i0 - p.window + 1) / BN : 0;
   const int nT = jb_hi - jb_lo + 1;
 
@@ -210,14 +231,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = t % kKS;
         if (t >= kKS && !wait_bar(bar(B_KEMPTY + st), (t / kKS - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(B_KFULL + st), Lay::kT + K * 4);
-        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
-        for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k, bar(B_KFULL + st),
-                      b * 64, h, row);
-        bulk_load(sbase + Lay::oRJ + st * K * 4,
-                  p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
-                  bar(B_KFULL + st));
+        const uint32_t rj_dst = sbase + Lay::oRJ + st * Lay::kRJRows * K * 4;
+        if constexpr (kCache) {
+          // k_tilde rows of batch row `seq` (zeros past T_kv) and the
+          // anchors of the tile's cached chunks
+          const int j0 = (jb_lo + t) * BN;
+          int c0;
+          const int nc = cache_tile_chunks(p, j0, c0);
+          mbar_expect_tx(bar(B_KFULL + st), Lay::kT + nc * K * 4);
+          for (int b = 0; b < K / 64; ++b)
+            tma_load_4d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k,
+                        bar(B_KFULL + st), b * 64, h, j0, seq);
+          for (int x = 0; x < nc; ++x)
+            bulk_load(rj_dst + x * K * 4, p.rc + (((long)seq * p.NC + c0 + x) * HQ + h) * K,
+                      K * 4, bar(B_KFULL + st));
+        } else {
+          mbar_expect_tx(bar(B_KFULL + st), Lay::kT + K * 4);
+          const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+          for (int b = 0; b < K / 64; ++b)
+            tma_load_3d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k,
+                        bar(B_KFULL + st), b * 64, h, row);
+          bulk_load(rj_dst, p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
+                    bar(B_KFULL + st));
+        }
         issued = t + 1;
       }
       // no bulk copy may still be landing in this CTA's shared memory at exit
@@ -232,10 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t >= kVS && !wait_bar(bar(B_VEMPTY + st), (t / kVS - 1) & 1, p.status, abort_flag))
           break;
         mbar_expect_tx(bar(B_VFULL + st), Lay::kT);
-        const int row = (int)(s0 + (long)(jb_lo + t) * BN);
-        for (int b = 0; b < V / 64; ++b)
-          tma_load_3d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v, bar(B_VFULL + st),
-                      b * 64, kh, row);
+        if constexpr (kCache) {
+          for (int b = 0; b < V / 64; ++b)
+            tma_load_4d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v,
+                        bar(B_VFULL + st), b * 64, kh, (jb_lo + t) * BN, seq);
+        } else {
+          const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+          for (int b = 0; b < V / 64; ++b)
+            tma_load_3d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v,
+                        bar(B_VFULL + st), b * 64, kh, row);
+        }
         issued = t + 1;
       }
       for (int t = max(0, issued - kVS); t < issued; ++t)
@@ -310,31 +352,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool got = wait_bar(bar(B_KFULL + st), (t / kKS) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) break;
       }
-      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
-      __nv_bfloat162 d[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
-                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
-        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
-      }
+      const float* rj =
+          reinterpret_cast<const float*>(smem + Lay::oRJ + st * Lay::kRJRows * K * 4) + ch * 8;
       uint8_t* kt = smem + Lay::oK + st * Lay::kT + (ch / 8) * (BN * 128);
-      constexpr int kBatch = 8;
+      if constexpr (kCache) {
+        // factor 2^(R_I - R_c) per cache chunk of the tile: not a power of
+        // two, so it is rounded to bf16 and applied with packed bf16
+        // multiplies (two roundings of 2^-9 on the key, as fine as the
+        // k_tilde rounding itself); rows of a chunk that holds no cached
+        // position are zeros and get factor 0
+        int c0;
+        const int nvalid = cache_tile_chunks(p, (jb_lo + t) * BN, c0);
+        const int crows = p.C >= BN ? BN : p.C;  // tile rows per chunk
+        for (int x = 0; x * crows < BN; ++x) {
+          __nv_bfloat162 f[4];
 #pragma unroll
-      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
-        uint4 v[kBatch];
+          for (int e = 0; e < 4; ++e)
+            f[e] = x < nvalid ? __floats2bfloat162_rn(exp2f(ri[2 * e] - rj[x * K + 2 * e]),
+                                                      exp2f(ri[2 * e + 1] - rj[x * K + 2 * e + 1]))
+                              : __floats2bfloat162_rn(0.f, 0.f);
+          constexpr int kBatch = 4;
+          for (int m0 = x * crows / kRowStep; m0 < (x + 1) * crows / kRowStep; m0 += kBatch) {
+            uint4 v[kBatch];
 #pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          const int r = rs + (m0 + x) * kRowStep;
-          v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+            for (int y = 0; y < kBatch; ++y) {
+              const int r = rs + (m0 + y) * kRowStep;
+              v[y] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+            }
+#pragma unroll
+            for (int y = 0; y < kBatch; ++y) {
+              const int r = rs + (m0 + y) * kRowStep;
+              __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[y]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], f[e]);
+              *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[y];
+            }
+          }
         }
+      } else {
+        __nv_bfloat162 d[4];
 #pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          const int r = rs + (m0 + x) * kRowStep;
-          __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                             (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+          d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+        }
+        constexpr int kBatch = 8;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
-          *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
+        for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+          uint4 v[kBatch];
+#pragma unroll
+          for (int x = 0; x < kBatch; ++x) {
+            const int r = rs + (m0 + x) * kRowStep;
+            v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+          }
+#pragma unroll
+          for (int x = 0; x < kBatch; ++x) {
+            const int r = rs + (m0 + x) * kRowStep;
+            __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
+            *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
+          }
         }
       }
       fence_proxy_async_smem();
@@ -346,19 +425,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - 4) >> 2;          // 0: even key tiles, 1: odd ones
     const int quarter = warp & 3;             // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;        // query row within the block
-    const int i = i0 + r;                     // row within the sequence
+    const int qi = i0 + r;                    // query row within the sequence
+    const int i = pos0 + qi;                  // its position among the keys
     const bool row_ok = r < ni;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const bool has_gs = p.GS != nullptr;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
-    const float gs_i = (has_gs && row_ok) ? p.GS[(s0 + i) * HQ + h] * kLog2e : 0.f;
+    const float gs_i = (has_gs && row_ok) ? p.GS[(s0 + qi) * HQ + h] * kLog2e : 0.f;
     const uint32_t s_addr = tmem + lane_base + grp * 128;
     const uint32_t o_addr = tmem + lane_base + 256 + grp * V;
     float* gsk = sGS + (warp - 4) * BN;  // this warp's copy of the key prefix (or zeros)
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
+    // a chunk of fewer than 128 queries leaves whole warps without a row:
+    // they only keep step with their group (S ready, P "written")
+    const bool idle = kCache && !__any_sync(0xffffffffu, row_ok);
     for (int t = grp; t < nT; t += 2) {
       const int j0 = (jb_lo + t) * BN;
+      if (idle) {
+        const bool got = wait_bar(bar(B_SFULL + grp), (t >> 1) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PFULL + grp));
+        continue;
+      }
       if (has_gs || t == grp) {
         __syncwarp();
         for (int c = lane; c < BN; c += 32) {
@@ -376,8 +466,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // common case -- a fully visible tile without a scalar gate -- is a
       // plain multiply; the decision is warp-uniform and hoisted out of the
       // element loops.
-      const bool fast = __all_sync(0xffffffffu, row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
-                                                    (i - j0 < win) && !has_gs);
+      // (rows past a cache chunk's queries compute on finite stand-in
+      // queries and are never stored, so they do not hold the warp back)
+      const bool fast =
+          __all_sync(0xffffffffu, (kCache && !row_ok) ||
+                                      (row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
+                                       (i - j0 < win) && !has_gs));
       const float sl2 = p.scale_log2;
       const float bias_i = has_gs ? gs_i : 0.f;
       bool done = false;
@@ -534,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.sink) lt += exp2f(p.sink[h] * kLog2e - m_f);
       const float inv = 1.f / lt;
       const float f0 = a0 * inv, f1 = a1 * inv;
-      __nv_bfloat16* orow = p.o + ((s0 + i) * HQ + h) * (long)V;
+      __nv_bfloat16* orow = p.o + ((s0 + qi) * HQ + h) * (long)V;
       // each group writes half of the channels; O_odd exists only if the odd
       // group had tiles (warp-uniform)
 #pragma unroll 1
@@ -561,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (grp == 0 && row_ok && p.lse) p.lse[(s0 + i) * HQ + h] = (m_f + log2f(lt)) * kLn2;
+      if (grp == 0 && row_ok && p.lse) p.lse[(s0 + qi) * HQ + h] = (m_f + log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
@@ -615,10 +709,12 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
 #pragma unroll
     for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(pv[c] - rv[c]);
     store8(qh + (row * HQ + hh) * K + g8 * 8, y);
-    load8(k + (row * H + hh / G) * K + g8 * 8, x);
+    if (k != nullptr) {  // without keys: the query operand and anchors only
+      load8(k + (row * H + hh / G) * K + g8 * 8, x);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(rv[c] - pv[c]);
-    store8(khat + (row * HQ + hh) * K + g8 * 8, y);
+      for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(rv[c] - pv[c]);
+      store8(khat + (row * HQ + hh) * K + g8 * 8, y);
+    }
     if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, rv);
   }
 }
@@ -636,8 +732,8 @@ int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, in
     return WALL_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(fwd_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<KD>::kAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(fwd_tc_kernel<KD, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<KD, false>::kAlloc) != cudaSuccess)
       return WALL_ERR_CUDA;
     attr = true;
   }
@@ -653,8 +749,34 @@ int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, in
   p.window = pb.window;
   p.n_blocks = ws.n_blocks128;
   p.status = status;
+  p.rc = nullptr;
+  p.C = p.NC = p.t_off = p.T_kv = 0;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  fwd_tc_kernel<KD><<<grid, kThreads, Smem<KD>::kAlloc, stream>>>(tq, tk, tv, p);
+  fwd_tc_kernel<KD, false><<<grid, kThreads, Smem<KD, false>::kAlloc, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+// A chunk of queries against the decode cache: Qh, the query-block anchors,
+// then the forward kernel in its cache form (keys = k_tilde rows, values =
+// the value cache, both read through maps that end at T_kv).
+template <int KD>
+int launch_decode_chunk_tc(const FwdTcParams& p0, const void* k_tilde, const void* v, int B,
+                           int Tq, int T_kv, int Tcap, int H, int HQ, const __nv_bfloat16* qh,
+                           cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, qh, (long)B * Tq, HQ, KD, BM) ||
+      !make_cache_map(&tk, k_tilde, B, T_kv, Tcap, HQ, KD, BN) ||
+      !make_cache_map(&tv, v, B, T_kv, Tcap, H, KD, BN))
+    return WALL_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(fwd_tc_kernel<KD, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<KD, true>::kAlloc) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    attr = true;
+  }
+  dim3 grid(HQ, p0.n_blocks);
+  fwd_tc_kernel<KD, true><<<grid, kThreads, Smem<KD, true>::kAlloc, stream>>>(tq, tk, tv, p0);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
@@ -674,6 +796,48 @@ int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, c
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), P, pb.seqs,
       pb.HQ, pb.H, pb.K, ws.qh, ws.kh, ws.anchors);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+bool decode_chunk_tc_supported(int dtype, int K, int V, int C) {
+  return dtype == WALL_BF16 && K == V && (K == 64 || K == 128) && C >= 32 && C % 32 == 0 &&
+         (BN % C == 0 || C % BN == 0);
+}
+
+int attn_decode_chunk_tc(const void* q, const void* v, const float* p, const void* k_tilde,
+                         const float* r_cache, const float* sink, float scale, int C, int B,
+                         int Tq, int T_kv, int Tcap, int H, int HQ, int K, __nv_bfloat16* qh,
+                         float* anchors, void* o, float* lse, int* status, cudaStream_t stream) {
+  if ((long)B * Tq == 0) return WALL_OK;
+  Seqs seqs;
+  seqs.cu = nullptr;
+  seqs.n = B;
+  seqs.T = Tq;
+  seqs.rows = (long)B * Tq;
+  // Qh = q * 2^(p - R_I) and the query-block anchors R_I = floor(p at the
+  // block's first row), as the training forward prepares its queries
+  const int per_seq = (148 * 8 + B - 1) / B;
+  anchor_operands_kernel<<<dim3(per_seq < 1 ? 1 : per_seq, B), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), nullptr, p, seqs, HQ, H, K, qh, nullptr, anchors);
+  if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+  FwdTcParams pr;
+  pr.anchors = anchors;
+  pr.GS = nullptr;
+  pr.sink = sink;
+  pr.o = static_cast<__nv_bfloat16*>(o);
+  pr.lse = lse;
+  pr.seqs = seqs;
+  pr.HQ = HQ; pr.H = H; pr.K = K; pr.V = K;
+  pr.scale_log2 = scale * kLog2e;
+  pr.window = 0;
+  pr.n_blocks = B * ((Tq + BM - 1) / BM);
+  pr.status = status;
+  pr.rc = r_cache;
+  pr.C = C;
+  pr.NC = (Tcap + C - 1) / C;
+  pr.t_off = T_kv - Tq;
+  pr.T_kv = T_kv;
+  return K == 128 ? launch_decode_chunk_tc<128>(pr, k_tilde, v, B, Tq, T_kv, Tcap, H, HQ, qh, stream)
+                  : launch_decode_chunk_tc<64>(pr, k_tilde, v, B, Tq, T_kv, Tcap, H, HQ, qh, stream);
 }
 
 int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,

@@ -105,8 +105,12 @@ struct DecodeArgs {
   const float *pc, *rc, *sink;
   float scale;
   int C, B, T_kv, Tcap, H, HQ, K, V, splits, keys_per_split;
-  float* ws_o;   // [B,HQ,splits,V]
-  float* ws_ml;  // [B,HQ,splits,2]
+  float* ws_o;   // [B,Tq,HQ,splits,V]
+  float* ws_ml;  // [B,Tq,HQ,splits,2]
+  // query rows per batch row (1 for a decode step): q, p_curr, the partials
+  // and the outputs hold B*Tq rows, row i of batch row b at cache position
+  // T_kv - Tq + i, which sees the keys up to and including that position
+  int Tq;
 };
 
 // The one-token streaming step (append + decode in one launch): the new
@@ -127,7 +131,9 @@ struct StepArgs {
 template <typename T, int KD, int VD>
 __global__ void decode_split_kernel(DecodeArgs a) {
   __shared__ float qh[32][KD];  // per warp (query head): scaled, anchored query
-  const int s = blockIdx.x, kh = blockIdx.y, b = blockIdx.z;
+  const int s = blockIdx.x, kh = blockIdx.y;
+  const int z = blockIdx.z;     // query row: batch row b, row z - b * Tq of its chunk
+  const int b = z / a.Tq;
   const int G = a.HQ / a.H;
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = kh * G + w;
@@ -137,14 +143,14 @@ __global__ void decode_split_kernel(DecodeArgs a) {
   const T* kt = static_cast<const T*>(a.kt);
   const int NC = (a.Tcap + a.C - 1) / a.C;
   const long k0 = (long)s * a.keys_per_split;
-  const long k1 = min((long)a.T_kv, k0 + a.keys_per_split);
+  const long k1 = min((long)a.T_kv - a.Tq + 1 + (z - (long)b * a.Tq), k0 + a.keys_per_split);
   constexpr int VPL = VD / 32;  // value channels per lane
   float m = -INFINITY, l = 0.f;
   float acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   const float sl2 = a.scale * kLog2e;
-  const long qoff = ((long)b * a.HQ + h) * K;
+  const long qoff = ((long)z * a.HQ + h) * K;
   for (long cs = k0; cs < k1; cs += a.C) {
     const long c = cs / a.C;
     // query scaled for this chunk: scale*log2e * q * exp2(p_curr - R_c)
@@ -203,7 +209,7 @@ __global__ void decode_split_kernel(DecodeArgs a) {
     }
     __syncwarp();
   }
-  const long part = ((long)b * a.HQ + h) * a.splits + s;
+  const long part = ((long)z * a.HQ + h) * a.splits + s;
   if (lane * VPL < V) {
 #pragma unroll
     for (int i = 0; i < VPL; ++i) a.ws_o[part * V + lane * VPL + i] = acc[i];
@@ -687,10 +693,11 @@ __global__ void decode_merge_kernel(DecodeArgs a, T* __restrict__ o, float* __re
 template <typename T, int KD, int VD>
 int launch_decode(const DecodeArgs& a, T* o, float* lse, cudaStream_t stream) {
   const int G = a.HQ / a.H;
-  dim3 grid(a.splits, a.H, a.B);
+  dim3 grid(a.splits, a.H, a.B * a.Tq);
   decode_split_kernel<T, KD, VD><<<grid, 32 * G, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
-  decode_merge_kernel<T><<<dim3(a.HQ, a.B), 128, 0, stream>>>(a, o, lse);
+  // the merge indexes query rows as batch rows: B*Tq of them
+  decode_merge_kernel<T><<<dim3(a.HQ, a.B * a.Tq), 128, 0, stream>>>(a, o, lse);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
@@ -783,7 +790,7 @@ DecodeArgs decode_args(const void* q, const void* v, const float* p_curr, const 
   DecodeArgs a;
   a.q = q; a.v = v; a.kt = k_tilde; a.pc = p_curr; a.rc = r_cache; a.sink = sink;
   a.scale = scale; a.C = C; a.B = B; a.T_kv = T_kv; a.Tcap = Tcap; a.H = H; a.HQ = HQ;
-  a.K = K; a.V = V; a.splits = splits;
+  a.K = K; a.V = V; a.splits = splits; a.Tq = 1;
   const long chunks = (T_kv + (long)C - 1) / C;
   const long chunks_per_split = (chunks + splits - 1) / splits;
   a.keys_per_split = (int)(chunks_per_split * C);
@@ -823,6 +830,36 @@ int decode_splits(int B, int T_kv, int H, int C) {
   if (s > chunks) s = chunks;
   if (s < 1) s = 1;
   return (int)s;
+}
+
+// Splits for a chunk of Tq query rows per batch row: the same waves, with
+// every query row a unit of its own.
+int decode_chunk_splits(int B, int Tq, int T_kv, int H, int C) {
+  return decode_splits(B * Tq, T_kv, H, C);
+}
+
+int attn_decode_chunk_split(const void* q, const void* v, const float* p, const void* k_tilde,
+                            const float* r_cache, const float* sink, float scale, int C,
+                            int dtype, int B, int Tq, int T_kv, int Tcap, int H, int HQ, int K,
+                            int V, void* o, float* lse, float* ws, int splits,
+                            cudaStream_t stream) {
+  if ((long)B * Tq == 0) return WALL_OK;
+  DecodeArgs a = decode_args(q, v, p, k_tilde, r_cache, sink, scale, C, B, T_kv, Tcap, H, HQ, K,
+                             V, ws, splits);
+  a.Tq = Tq;
+  a.ws_ml = ws + (long)B * Tq * HQ * splits * V;
+  if (dtype == WALL_BF16) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(o);
+    if (K <= 64 && V <= 64) return launch_decode<__nv_bfloat16, 64, 64>(a, out, lse, stream);
+    if (K <= 64) return launch_decode<__nv_bfloat16, 64, 128>(a, out, lse, stream);
+    if (V <= 64) return launch_decode<__nv_bfloat16, 128, 64>(a, out, lse, stream);
+    return launch_decode<__nv_bfloat16, 128, 128>(a, out, lse, stream);
+  }
+  float* out = static_cast<float*>(o);
+  if (K <= 64 && V <= 64) return launch_decode<float, 64, 64>(a, out, lse, stream);
+  if (K <= 64) return launch_decode<float, 64, 128>(a, out, lse, stream);
+  if (V <= 64) return launch_decode<float, 128, 64>(a, out, lse, stream);
+  return launch_decode<float, 128, 128>(a, out, lse, stream);
 }
 
 int attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,

@@ -16,7 +16,7 @@ namespace wall {
 void timing_mark(int slot, cudaStream_t stream);
 enum TimingSlot {
   T_PREFIX = 0, T_OPERANDS = 1, T_FWD = 2, T_BWD_PRE = 3, T_BWD_KEY = 4, T_BWD_DQ = 5,
-  T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9, T_STEP = 10,
+  T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9, T_STEP = 10, T_CHUNK = 11,
 };
 
 // ---- scans (wall_scan.cu) ----
@@ -87,6 +87,27 @@ int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, i
 // ---- TMA tensor maps (wall_tma.cu) ----
 bool make_tile_map(CUtensorMap* m, const void* base, long rows, int heads, int dim,
                    int box_rows);
+
+bool make_cache_map(CUtensorMap* m, const void* base, int B, int T, int Tcap, int heads, int dim,
+                    int box_rows);
+
+// ---- a chunk of Tq queries against the decode cache (multi-token decode,
+// chunked prefill); query row i of batch row b sits at cache position
+// T_kv - Tq + i ----
+// tensor-core path (wall_attn_fwd_sm100.cu): bf16, K == V in {64, 128},
+// C a multiple of 32 that divides 128 or is a multiple of 128
+bool decode_chunk_tc_supported(int dtype, int K, int V, int C);
+int attn_decode_chunk_tc(const void* q, const void* v, const float* p, const void* k_tilde,
+                         const float* r_cache, const float* sink, float scale, int C, int B,
+                         int Tq, int T_kv, int Tcap, int H, int HQ, int K, __nv_bfloat16* qh,
+                         float* anchors, void* o, float* lse, int* status, cudaStream_t stream);
+// general path (wall_decode.cu): the split decode with one grid row per query
+int decode_chunk_splits(int B, int Tq, int T_kv, int H, int C);
+int attn_decode_chunk_split(const void* q, const void* v, const float* p, const void* k_tilde,
+                            const float* r_cache, const float* sink, float scale, int C,
+                            int dtype, int B, int Tq, int T_kv, int Tcap, int H, int HQ, int K,
+                            int V, void* o, float* lse, float* ws, int splits,
+                            cudaStream_t stream);
 
 // ---- SIMT fp32 attention (wall_attn_simt.cu) ----
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);

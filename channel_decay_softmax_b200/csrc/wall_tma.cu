@@ -42,4 +42,22 @@ bool make_tile_map(CUtensorMap* m, const void* base, long rows, int heads, int d
   return r == CUDA_SUCCESS;
 }
 
+// A [B, Tcap, heads, dim] bf16 cache of which the first T rows of every batch
+// row are read, viewed as the 4-D tensor (dim, heads, T, B) with batch rows
+// Tcap rows apart; rows at or past T read as zeros.  Box as above.
+bool make_cache_map(CUtensorMap* m, const void* base, int B, int T, int Tcap, int heads, int dim,
+                    int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || B <= 0 || T <= 0 || Tcap < T || dim % 64 != 0) return false;
+  cuuint64_t gdim[4] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t gstride[3] = {(cuuint64_t)dim * 2, (cuuint64_t)dim * heads * 2,
+                           (cuuint64_t)Tcap * heads * dim * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim, gstride,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace wall

@@ -264,6 +264,49 @@ int wall_decode_step(const void* q, const void* k, const void* v, const void* g,
                      int HQ, int K, int V, void* o, float* lse, void* workspace,
                      size_t workspace_bytes, wall_stream_t stream);
 
+/* wall_attn_decode_chunk_workspace -- bytes of workspace wall_attn_decode_chunk
+ * needs for these arguments (its path depends on dtype, K, V and C). */
+size_t wall_attn_decode_chunk_workspace(int dtype, int B, int Tq, int T_kv, int H, int HQ, int K,
+                                        int V, int C);
+
+/*
+ * wall_attn_decode_chunk -- Tq queries per batch row against the pre-rescaled
+ * cache at once: multi-token decode and chunked prefill.  The queries are the
+ * LAST Tq cached positions (bottom-right aligned causal mask, as the course
+ * slides on attention masks align a short query block with a longer key
+ * sequence): query row i of batch row b sits at position t_i = T_kv - Tq + i
+ * and sees the cached keys 0 .. t_i.  Append the chunk's keys and values
+ * first (wall_prefix_cumsum with the carry, wall_build_kv_cache with
+ * t0 = T_kv - Tq); then for each (b, i, h), with c(j) = j / C,
+ *   s_j = scale * sum_n q[b,i,h,n] exp2(p[b,i,h,n] - r_cache[b,c(j),h,n])
+ *                  * k_tilde[b,j,h,n],       j = 0 .. t_i
+ *   o[b,i,h,:] = sum_j softmax(s, sink)_j v[b,j,h/G,:],  lse = log-sum-exp
+ * which is wall_attn_decode of that row with T_kv = t_i + 1 (README "Decode":
+ * the pre-rescaled cache with per-chunk anchors), and equals the training
+ * forward's row t_i.
+ * In:  q [B,Tq,HQ,K] (`dtype`), p [B,Tq,HQ,K] fp32 (P at the queries'
+ *      positions), k_tilde [B,Tcap,HQ,K] and v [B,Tcap,H,V] (`dtype`, the
+ *      first T_kv positions are read), r_cache [B,ceil(Tcap/C),HQ,K] fp32,
+ *      sink_bias [HQ] fp32 or NULL.  1 <= T_kv <= Tcap, 0 <= Tq <= T_kv.
+ * Out: o [B,Tq,HQ,V] (`dtype`), lse [B,Tq,HQ] fp32 natural log (may be NULL).
+ * Workspace: wall_attn_decode_chunk_workspace(...) bytes, 16-byte aligned,
+ * caller-owned; no state is kept in it between calls.
+ * Paths: bf16 with K == V in {64, 128} and C a multiple of 32 that divides
+ * 128 or is a multiple of 128 runs on the tensor cores (tcgen05, one CTA per
+ * 128 query rows of a (batch row, head), key tiles of 128 cached positions
+ * scaled per chunk by 2^(R_I - R_c) with R_I the query block's integer
+ * anchor); every other supported shape (bf16 or fp32, K and V multiples of 8
+ * up to 128, HQ/H <= 32, B*Tq <= 65535) runs the split-KV decode with one
+ * grid row per query.  Errors: WALL_ERR_INVALID_ARG for null or misaligned
+ * pointers, bad shapes or a short workspace; WALL_ERR_UNSUPPORTED outside
+ * both paths.
+ */
+int wall_attn_decode_chunk(const void* q, const void* v, const float* p, const void* k_tilde,
+                           const float* r_cache, const float* sink_bias, float scale, int C,
+                           int dtype, int B, int Tq, int T_kv, int Tcap, int H, int HQ, int K,
+                           int V, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                           wall_stream_t stream);
+
 /*
  * wall_get_status -- synchronizes `stream`, returns the device status word
  * (WALL_OK or WALL_ERR_TIMEOUT) and clears it.  Returns WALL_ERR_CUDA if the
@@ -298,10 +341,11 @@ int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
  *   8 decode          wall_attn_decode (split and merge kernels)
  *   9 cache_build     wall_build_kv_cache
  *  10 decode_step     wall_decode_step (one launch per token)
+ *  11 decode_chunk    wall_attn_decode_chunk (operands and attention)
  * wall_timing_enable(1) starts recording (and clears the totals);
  * wall_timing_enable(0) stops.  Not thread-safe: one host thread at a time.
  */
-#define WALL_TIMING_SLOTS 11
+#define WALL_TIMING_SLOTS 12
 int wall_timing_enable(int on);
 
 /*

@@ -131,6 +131,39 @@ def test_decode_step_rejects_bad_arguments(lib):
     assert lib.wall_decode_step_workspace(1, 0, 1, 1, 64, 64) == 0
 
 
+def test_decode_chunk_rejects_bad_arguments(lib):
+    ch = lib.wall_attn_decode_chunk
+    wsf = lib.wall_attn_decode_chunk_workspace
+    B, Tq, T_kv, Tcap, H, HQ, K, V, C = 2, 64, 1000, 1024, 2, 8, 128, 128, 64
+    al = lambda x: (x + 255) // 256 * 256
+    # tensor-core path: anchored queries (bf16) and 128-row block anchors (fp32)
+    tc = al(2 * B * Tq * HQ * K) + al(4 * B * 1 * HQ * K)
+    assert wsf(0, B, Tq, T_kv, H, HQ, K, V, C) == tc
+    # split path (fp32): per query row and split, the partial (o, m, l)
+    split = wsf(1, B, Tq, T_kv, H, HQ, K, V, C)
+    assert split > 0 and split % (4 * B * Tq * HQ * (V + 2)) < 256
+    assert wsf(0, B, Tq + 1, Tq, H, HQ, K, V, C) == 0          # more queries than positions
+
+    def call(dtype=0, Tq=Tq, T_kv=T_kv, Tcap=Tcap, C=C, H=H, HQ=HQ, K=K, V=V, ws_bytes=tc,
+             q=FAKE, kt=FAKE, B=B):
+        return ch(q, FAKE, FAKE, kt, FAKE, None, 0.0, C, dtype, B, Tq, T_kv, Tcap, H, HQ, K, V,
+                  FAKE, None, FAKE, ws_bytes, None)
+
+    assert call(dtype=3) == L.WALL_ERR_INVALID_ARG
+    assert call(Tq=T_kv + 1) == L.WALL_ERR_INVALID_ARG        # queries past the cache
+    assert call(Tcap=T_kv - 1) == L.WALL_ERR_INVALID_ARG      # cache shorter than T_kv
+    assert call(T_kv=0, Tq=0) == L.WALL_ERR_INVALID_ARG
+    assert call(HQ=7) == L.WALL_ERR_INVALID_ARG               # HQ % H != 0
+    assert call(K=136) == L.WALL_ERR_UNSUPPORTED              # head size beyond 128
+    assert call(H=1, HQ=64) == L.WALL_ERR_UNSUPPORTED         # 64 query heads per kv head
+    assert call(q=None) == L.WALL_ERR_INVALID_ARG
+    assert call(kt=FAKE + 4) == L.WALL_ERR_INVALID_ARG        # misaligned cache
+    assert call(ws_bytes=tc - 1) == L.WALL_ERR_INVALID_ARG    # workspace too small
+    assert call(dtype=1, ws_bytes=tc) == L.WALL_ERR_INVALID_ARG  # fp32 needs the split partials
+    assert call(dtype=1, Tq=700, T_kv=700, B=100) == L.WALL_ERR_UNSUPPORTED  # 70000 grid rows
+    assert call(Tq=0) == L.WALL_OK                            # empty: nothing launched
+
+
 def test_prefix_rejects_bad_arguments(lib):
     pc = lib.wall_prefix_cumsum
     assert pc(FAKE, 3, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG
