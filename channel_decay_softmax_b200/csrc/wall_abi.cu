@@ -117,8 +117,13 @@ FwdWs fwd_ws_layout(const AttnProblem& pb, int has_gs) {
   return w;
 }
 
+// The stored dS tiles of the tensor-core backward (dense sequences): at most
+// this much workspace, beyond it the dq kernel recomputes S, P and dP.
+constexpr size_t kMaxDsBytes = size_t(8) << 30;
+
 struct BwdWs {
-  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, qh, kh, anchors, total;
+  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, qh, kh, anchors, dS, total;
+  bool has_ds;
   int n_blocks128;
 };
 BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
@@ -140,6 +145,17 @@ BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
     w.qh = off;      off += align256((size_t)2 * rows * HQ * K);
     w.kh = off;      off += align256((size_t)2 * rows * HQ * K);
     w.anchors = off; off += align256(sizeof(float) * (size_t)w.n_blocks128 * HQ * K);
+  }
+  w.dS = off;
+  w.has_ds = false;
+  if (fwd_tc_supported(pb) && pb.extra_blocks == 0) {
+    // dS^T tiles (bf16, 128 x 128) of every (batch row, head, I, J <= I)
+    const size_t nb = (size_t)(pb.T + 127) / 128;
+    const size_t bytes = (size_t)pb.B * HQ * (nb * (nb + 1) / 2) * 128 * 128 * 2;
+    if (bytes > 0 && bytes <= kMaxDsBytes) {
+      w.has_ds = true;
+      off += align256(bytes);
+    }
   }
   w.total = off;
   return w;
@@ -334,6 +350,9 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   a.dvh32 = reinterpret_cast<float*>(at(workspace, w.dvh32));
   a.dgs_row = reinterpret_cast<float*>(at(workspace, w.dgs_row));
   a.dgs_col = reinterpret_cast<float*>(at(workspace, w.dgs_col));
+  // dq from stored dS tiles: dense causal without a window, tensor-core path
+  a.dS = (w.has_ds && pb.window == 0)
+             ? reinterpret_cast<__nv_bfloat16*>(at(workspace, w.dS)) : nullptr;
   a.GS = nullptr;
   if (g_scalar) {
     float* gs = reinterpret_cast<float*>(at(workspace, w.gs));

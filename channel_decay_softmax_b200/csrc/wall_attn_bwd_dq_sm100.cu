@@ -447,6 +447,256 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// dq from the dS tiles the key-block kernel stored (dense causal problems
+// without a window): for the CTA's query block I and every key tile J <= I,
+//   dQa += dS_IJ Kt_J,   Kt_J = Kh_J (.) 2^(R_I - R_J)  (exact, in place)
+// one contraction per tile instead of four (S, dP and this one recomputed,
+// and the exponentials); HBM carries the dS tiles, L2 keeps Kh.
+//
+// CTA = 8 warps (256 threads):
+//   warp 0      TMA, lane 0: per tile the dS tile (two 64-query boxes of 128
+//               key rows), Kh_J and its block anchors (kDS stages)
+//   warp 1      TMEM owner (128 columns) and MMA issuer: A = dS (queries x
+//               keys, MN-major: queries contiguous in the stored rows),
+//               B = Kt (keys x channels, MN-major)
+//   warps 2-3   Kt_J = Kh_J (.) d in place, as in the kernel above
+//   warps 4-7   epilogue: dQa rows -> fp32 workspace
+constexpr int kDS = 3;  // stages
+constexpr int kDsThreads = 256;
+
+template <int KD>
+struct QSmem {
+  static constexpr int kDsT = 128 * 128 * 2;  // one stored dS tile
+  static constexpr int kKT = BN * KD * 2;     // one Kh tile
+  static constexpr int oDS = 0;               // kDS stages
+  static constexpr int oK = oDS + kDS * kDsT;  // kDS stages
+  static constexpr int oRJ = oK + kDS * kKT;   // float[kDS][KD]
+  static constexpr int oBar = oRJ + kDS * KD * 4;
+  static constexpr int kBars = 3 * kDS + 2;
+  static constexpr int oMisc = oBar + kBars * 8;
+  static constexpr int kBytes = oMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KB alignment
+};
+static_assert(QSmem<128>::kAlloc <= 227 * 1024, "shared memory");
+
+enum QBar { QS_FULL = 0, QS_READY = kDS, QS_EMPTY = 2 * kDS, QS_DONE = 3 * kDS, QS_MMA = 3 * kDS + 1 };
+
+template <int KD>
+__global__ void __launch_bounds__(kDsThreads, 1)
+    bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_ds,
+                     const __grid_constant__ CUtensorMap tm_k, DqParams p, int ds_nb) {
+  using Lay = QSmem<KD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oMisc + 4);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.x;
+  const int HQ = p.HQ, K = KD;
+  // longest query blocks first
+  const int flat = p.n_blocks - 1 - (int)blockIdx.y;
+  int seq, blk;
+  if (!seq_block(p.seqs, BM, flat, seq, blk)) return;
+  const int blk_off = flat - blk;
+  const long s0 = p.seqs.start(seq);
+  const int L = p.seqs.len(seq);
+  const int i0 = blk * BM;
+  const int ni = min(BM, L - i0);
+  const int nT = blk + 1;  // key tiles 0 .. I
+  const long tile0 =
+      ((long)seq * HQ + h) * ((long)ds_nb * (ds_nb + 1) / 2) + (long)blk * (blk + 1) / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDS; ++s) {
+      mbar_init(bar(QS_FULL + s), 1);
+      mbar_init(bar(QS_READY + s), 2);
+      mbar_init(bar(QS_EMPTY + s), 1);
+    }
+    mbar_init(bar(QS_DONE), 1);
+    mbar_init(bar(QS_MMA), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_ds);
+      tma_prefetch_desc(&tm_k);
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kDS;
+        if (t >= kDS && !wait_bar(bar(QS_EMPTY + st), (t / kDS - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(QS_FULL + st), Lay::kDsT + Lay::kKT + K * 4);
+        const int drow = (int)((tile0 + t) * 128);
+        for (int b = 0; b < 2; ++b)
+          tma_load_2d(sbase + Lay::oDS + st * Lay::kDsT + b * (128 * 128), &tm_ds,
+                      bar(QS_FULL + st), b * 64, drow);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k, bar(QS_FULL + st),
+                      b * 64, h, (int)(s0 + (long)t * BN));
+        bulk_load(sbase + Lay::oRJ + st * K * 4, p.anchors + ((long)(blk_off + t) * HQ + h) * K,
+                  K * 4, bar(QS_FULL + st));
+        issued = t + 1;
+      }
+      // no copy may still be in flight when the CTA exits
+      for (int t = max(0, issued - kDS); t < issued; ++t)
+        mbar_wait(bar(QS_FULL + t % kDS), (t / kDS) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(BM, KD, true, true);
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kDS;
+        if (!wait_bar(bar(QS_READY + st), (t / kDS) & 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        // K = 16 keys per MMA: rows 16kk .. 16kk+15 of both operands; the two
+        // 64-wide M (N) boxes of dS (Kt) are 128 rows x 128 B apart
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ss(tmem,
+                       sdesc_sw128(sbase + Lay::oDS + st * Lay::kDsT + kk * 16 * 128, 128 * 128,
+                                   1024),
+                       sdesc_sw128(sbase + Lay::oK + st * Lay::kKT + kk * 16 * 128, BN * 128,
+                                   1024),
+                       id, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(QS_EMPTY + st));
+      }
+      umma_commit(bar(QS_DONE));
+      umma_commit(bar(QS_MMA));
+      mbar_wait(bar(QS_MMA), 0, p.status);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ key rescale
+    constexpr int kChunks = KD / 8;
+    constexpr int kRowStep = 64 / kChunks;
+    constexpr int kRows = BN / kRowStep;
+    const int tid = threadIdx.x - 64;
+    const int ch = tid % kChunks;
+    const int rs = tid / kChunks;
+    float ri[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
+    for (int t = 0; t < nT; ++t) {
+      const int st = t % kDS;
+      {
+        const bool got = wait_bar(bar(QS_FULL + st), (t / kDS) & 1, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) break;
+      }
+      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
+      __nv_bfloat162 d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+      }
+      uint8_t* kt = smem + Lay::oK + st * Lay::kKT + (ch / 8) * (BN * 128);
+      constexpr int kBatch = 8;
+#pragma unroll
+      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int r = rs + (m0 + x) * kRowStep;
+          v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+        }
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          const int r = rs + (m0 + x) * kRowStep;
+          __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
+          *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(QS_READY + st));
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const bool ok = __all_sync(0xffffffffu, wait_bar(bar(QS_DONE), 0, p.status, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      float* out = p.dq32 + ((s0 + i0 + r) * HQ + h) * (long)K;
+#pragma unroll 1
+      for (int c = 0; c < KD; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + c, v);
+        tmem_wait_ld();
+        if (r < ni) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(out + c + e) =
+                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+template <int KD>
+int launch_dq_ds(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
+                 cudaStream_t stream) {
+  const int nb = (pb.T + BM - 1) / BM;
+  const long tiles = (long)pb.B * pb.HQ * ((long)nb * (nb + 1) / 2);
+  CUtensorMap tds, tk;
+  if (!make_rows128_map(&tds, a.dS, tiles * 128, 128, 64) ||
+      !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN))
+    return WALL_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(bwd_dq_ds_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QSmem<KD>::kAlloc) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    attr = true;
+  }
+  DqParams p;
+  p.anchors = ws.anchors;
+  p.lse = a.lse;
+  p.D = a.D;
+  p.GS = a.GS;
+  p.dq32 = a.dq32;
+  p.seqs = pb.seqs;
+  p.HQ = pb.HQ;
+  p.H = pb.H;
+  p.scale_log2 = pb.scale * kLog2e;
+  p.window = pb.window;
+  p.n_blocks = ws.n_blocks128;
+  p.status = status;
+  dim3 grid(pb.HQ, ws.n_blocks128);
+  bwd_dq_ds_kernel<KD><<<grid, kDsThreads, QSmem<KD>::kAlloc, stream>>>(tds, tk, p, nb);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
 template <int KD>
 int launch_dq(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
               cudaStream_t stream) {
@@ -486,6 +736,10 @@ int launch_dq(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* s
 int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                    cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
+  if (a.dS) {  // the key-block kernel stored dS (dense causal, no window)
+    return pb.K == 128 ? launch_dq_ds<128>(pb, a, ws, status, stream)
+                       : launch_dq_ds<64>(pb, a, ws, status, stream);
+  }
   return pb.K == 128 ? launch_dq<128>(pb, a, ws, status, stream)
                      : launch_dq<64>(pb, a, ws, status, stream);
 }

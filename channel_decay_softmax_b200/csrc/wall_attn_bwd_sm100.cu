@@ -11,7 +11,10 @@
 //   dV_J  += P^T dO_I               (P^T from TMEM)
 //   dKa_J += dS^T Qt_I              (dS^T from TMEM); dk_j = scale 2^(R_J - P_j) dKa_j
 // dq comes from a separate query-block kernel (wall_attn_bwd_dq_sm100.cu), so
-// no fp32 atomics are needed.
+// no fp32 atomics are needed.  For dense causal problems without a window
+// this kernel also stores every dS tile it forms (bf16, as the dK MMA reads
+// it), and the dq kernel is then one contraction dQa = dS Kt per tile instead
+// of recomputing S, P, dP and dS.
 // The gate gradient needs dk per query head before the GQA sum; it is fused
 // into the finalize kernel as dL = q (.) dq - k (.) dk^(h) (blog, fast
 // training section 2: the key-side term is -K_j (.) dK_j), followed by the
@@ -39,6 +42,8 @@
 //               epilogue at the end
 #include <cuda.h>
 
+#include <string.h>
+
 #include <type_traits>
 
 #include "sm100_ptx.cuh"
@@ -64,6 +69,11 @@ struct BwdTcParams {
   float* dkh32;             // [rows, HQ, K]
   float* dvh32;             // [rows, HQ, V]
   float* dgs_col;           // [rows, HQ] or nullptr
+  // dS^T tiles for the dq kernel, or nullptr: tile (b, h, I, J), J <= I, at
+  // ((b * HQ + h) * nb(nb+1)/2 + I(I+1)/2 + J) * 128 * 128, rows = keys,
+  // 128 queries per row (dense sequences of nb 128-row blocks, no window)
+  __nv_bfloat16* dS;
+  int ds_nb;
   Seqs seqs;
   int HQ, H;
   float scale, scale_log2;
@@ -87,9 +97,14 @@ struct BSmem {
   static constexpr int oBar = oRI + kStages * KD * 4;
   static constexpr int kBars = 20;
   static constexpr int oMisc = oBar + kBars * 8;
-  static constexpr int kBytes = oMisc + 16;
+  // per softmax warp: its 32 keys x 32 queries of dS^T (bf16) on their way
+  // to the stored tile by TMA
+  static constexpr int oStg = (oMisc + 16 + 1023) & ~1023;
+  static constexpr int kStg = 32 * 32 * 2;
+  static constexpr int kBytes = oStg + 8 * kStg;
   static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(BSmem<128>::kAlloc <= 227 * 1024, "shared memory");
 
 enum BBar {
   KV_FULL = 0,
@@ -154,7 +169,7 @@ template <int KD, bool kGS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  BwdTcParams p) {
+                  const __grid_constant__ CUtensorMap tm_ds, BwdTcParams p) {
   using Lay = BSmem<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -421,6 +436,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gs_j = (kGS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     const uint32_t scol = kColS + half * 64, dcol = kColDP + half * 64;
+    // the stored dS tile (I0, J), I0 = J: tile
+    // (b * HQ + h) * nb(nb+1)/2 + I(I+1)/2 + J, rows = keys, 128 queries each;
+    // this warp's 32 keys x 32 queries go through its staging block
+    const bool store_ds = p.dS != nullptr;
+    long ds_tile = store_ds ? ((long)seq * HQ + h) * ((long)p.ds_nb * (p.ds_nb + 1) / 2) +
+                                  (long)I0 * (I0 + 1) / 2 + blk
+                            : 0;
+    uint8_t* stg = smem + Lay::oStg + (warp - 4) * Lay::kStg;
     float colsum = 0.f;
     bool ok = true;
     for (int t = 0; t < nT && ok; ++t) {
@@ -526,7 +549,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(DS_READY));
+      if (store_ds) {
+        // off the MMA's path: the same bf16 values, 32 queries at a time,
+        // this key's 64 bytes into the staging block (64-byte swizzle: the
+        // 16-byte chunk index XOR bits 1-2 of the row, conflict-free) once
+        // the previous store has read it, then one TMA store of the warp's
+        // 32 keys x 32 queries
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint4 v = make_uint4(pack_bf16x2(pv[c + 8 * e], pv[c + 8 * e + 1]),
+                                       pack_bf16x2(pv[c + 8 * e + 2], pv[c + 8 * e + 3]),
+                                       pack_bf16x2(pv[c + 8 * e + 4], pv[c + 8 * e + 5]),
+                                       pack_bf16x2(pv[c + 8 * e + 6], pv[c + 8 * e + 7]));
+            *reinterpret_cast<uint4*>(stg + lane * 64 + ((e ^ ((lane >> 1) & 3)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_ds, smem_u32(stg), half * 64 + c, (int)(ds_tile * BK + quarter * 32));
+            bulk_commit();
+          }
+        }
+        // tile (I + 1, J) follows tile (I, J) after the I + 1 tiles of row I
+        ds_tile += I0 + t + 1;
+      }
     }
+    // the stored tiles are complete before the CTA can exit
+    if (store_ds && lane == 0) bulk_wait_all();
     // ---- dK, dV epilogue.  Thread = key row in TMEM, but a row per thread
     // makes every global access of a warp touch 32 rows: the accumulators go
     // through shared memory (free once every MMA has completed), then each
@@ -746,11 +799,16 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict
 template <int KD, bool kGS>
 int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                   cudaStream_t stream) {
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tds;
   if (!make_tile_map(&tq, ws.qh, pb.rows, pb.HQ, KD, BQ) ||
       !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BK) ||
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BK) ||
       !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BQ))
+    return WALL_ERR_CUDA;
+  memset(&tds, 0, sizeof(tds));  // unused without stored dS tiles
+  const int nb = (pb.T + BQ - 1) / BQ;
+  if (a.dS && !make_rows128_map(&tds, a.dS, (long)pb.B * pb.HQ * ((long)nb * (nb + 1) / 2) * BK,
+                                32, 32))
     return WALL_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
@@ -769,6 +827,8 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.dkh32 = a.dkh32;
   p.dvh32 = a.dvh32;
   p.dgs_col = a.GS ? a.dgs_col : nullptr;
+  p.dS = a.dS;
+  p.ds_nb = (pb.T + BQ - 1) / BQ;
   p.seqs = pb.seqs;
   p.HQ = pb.HQ;
   p.H = pb.H;
@@ -778,7 +838,7 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.n_blocks = ws.n_blocks128;
   p.status = status;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  bwd_tc_kernel<KD, kGS><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tq, tk, tv, to, p);
+  bwd_tc_kernel<KD, kGS><<<grid, kThreads, BSmem<KD>::kAlloc, stream>>>(tq, tk, tv, to, tds, p);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

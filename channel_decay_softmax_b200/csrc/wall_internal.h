@@ -61,6 +61,10 @@ struct BwdArgs {
   float* dgs_row; // [rows,HQ]
   float* dgs_col; // [rows,HQ]
   float* dsink;   // [HQ] or nullptr (accumulated atomically, zeroed by the caller)
+  // tensor-core path, dense causal without a window: the key-block kernel
+  // stores its dS tiles here and dq is one contraction per tile; nullptr:
+  // the dq kernel recomputes S, P, dP and dS
+  __nv_bfloat16* dS;  // [B * HQ * nb(nb+1)/2, 128, 128], nb = ceil(T / 128)
 };
 
 // ---- tensor-core forward (wall_attn_fwd_sm100.cu) ----
@@ -88,6 +92,7 @@ int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, i
 bool make_tile_map(CUtensorMap* m, const void* base, long rows, int heads, int dim,
                    int box_rows);
 
+bool make_rows128_map(CUtensorMap* m, const void* base, long rows, int box_rows, int box_cols);
 bool make_cache_map(CUtensorMap* m, const void* base, int B, int T, int Tcap, int heads, int dim,
                     int box_rows);
 

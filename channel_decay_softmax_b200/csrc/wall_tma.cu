@@ -60,4 +60,21 @@ bool make_cache_map(CUtensorMap* m, const void* base, int B, int T, int Tcap, in
   return r == CUDA_SUCCESS;
 }
 
+// A [rows, 128] bf16 array of stored 128 x 128 tiles viewed as the 2-D tensor
+// (128, rows).  Loads: one box is 64 columns (128 B, 128-byte swizzle) x
+// box_rows rows.  Stores: 32 columns (64 B, 64-byte swizzle) x box_rows.
+bool make_rows128_map(CUtensorMap* m, const void* base, long rows, int box_rows, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || (box_cols != 32 && box_cols != 64)) return false;
+  cuuint64_t gdim[2] = {128, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {256};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace wall

@@ -185,7 +185,14 @@ def test_workspace_sizes(lib):
     tc = 2 * al(2 * rows * HQ * K) + al(4 * nblk * HQ * K)
     assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 0, 0) == simt        # fp32
     assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 1, 0) == simt + al(4 * rows * HQ)
-    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc   # bf16
+    # bf16 dense: the stored dS tiles (bf16 128 x 128) of every (b, h, I, J <= I)
+    nb = (T + 127) // 128
+    ds = al(B * HQ * nb * (nb + 1) // 2 * 128 * 128 * 2)
+    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc + ds
+    # varlen packing (B == 1, n_seq > 0): no stored tiles, dq recomputes them
+    simt1 = al(4 * T * HQ) + 2 * al(4 * T * HQ * K) + al(4 * T * HQ * V) + 2 * al(4 * T * HQ)
+    tc1 = 2 * al(2 * T * HQ * K) + al(4 * ((T + 127) // 128 + 3) * HQ * K)
+    assert lib.wall_attn_bwd_workspace(0, 1, T, 4, HQ, K, V, 0, 3) == simt1 + tc1
     assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, 32, 32, 0, 0) == \
         al(4 * rows * HQ) + 2 * al(4 * rows * HQ * 32) + al(4 * rows * HQ * 32) + \
         2 * al(4 * rows * HQ)                                                     # SIMT bf16

@@ -204,3 +204,24 @@ def test_backward_reuses_forward_operands_bit_exactly():
     torch.cuda.synchronize()
     for name, ta, tb in zip(("dq", "dk", "dv", "dg"), a[:4], b[:4]):
         assert torch.equal(ta, tb), name
+
+
+@pytest.mark.parametrize("K", [64, 128])
+def test_dq_from_stored_ds_matches_recompute(K):
+    """Dense causal bf16 problems store the key-block kernel's dS tiles and
+    take dq as one contraction per tile; a window longer than the sequence
+    (the same attention) sends dq through the recomputing query-block kernel
+    instead.  Both match the oracle, with the scalar gate and sink, and agree
+    with each other to bf16 rounding."""
+    T = 700
+    s = I.spec(2, T=T, K=K, V=K, g_scalar=True, sink=True)
+    x_cpu = I.training_inputs(s)
+    _check_all(s, x_cpu, what=f"stored dS K={K}")
+    s_w = I.spec(2, T=T, K=K, V=K, g_scalar=True, sink=True, window=T + 1)
+    x_w = dict(x_cpu, window_size=T + 1)
+    _check_all(s_w, x_w, what=f"recompute K={K}")
+    _, _, _, ga = _run_gpu(_to(x_cpu))
+    _, _, _, gb = _run_gpu(_to(x_w))
+    for name, ta, tb in zip(("dq", "dk", "dv", "dg"), ga[:4], gb[:4]):
+        e = float((ta.float() - tb.float()).norm() / tb.float().norm())
+        assert e < 1e-2, (name, e)
