@@ -494,8 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float cx = cr[c + e + x];
               const float arg = fmaf(__uint_as_float(sv[c + e + x]), p.scale_log2,
                                      kGS ? cx - gs_j : cx);
-              // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
-              const float ev = ((e + x) & 7) >= 5 ? exp2_fma(arg) : exp2f(arg);
+              // all on MUFU: moving part of them to an FMA-pipe polynomial
+              // costs more issue slots than it frees on MUFU (measured)
+              const float ev = exp2f(arg);
               if constexpr (decltype(masked)::value) {
                 const int i = i0 + c + e + x;
                 const bool vis = key_ok & (i < L) & (jj <= i) & (i - jj < win);

@@ -56,6 +56,7 @@ constexpr int kThreads = 384;
 constexpr int kKS = 3;                    // key stages
 constexpr int kVS = 2;                    // value stages
 constexpr float kRescaleThreshold = 8.f;  // log2 units: lazy O rescale
+constexpr float kRescaleBound = 256.f;    // 2^kRescaleThreshold
 
 struct FwdTcParams {
   const float* anchors;  // [nblk, HQ, K]
@@ -476,12 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float bias_i = has_gs ? gs_i : 0.f;
       bool done = false;
       // One pass when every row's running max is set: exponentials against
-      // it, P held packed in registers and stored only if no row's max grew
-      // past the lazy threshold; otherwise S, still intact in TMEM, goes
-      // through the two passes below (max, O rescale, exponentials).
+      // it, P held packed in registers and stored only if no row's sum
+      // exceeds 2^threshold (then no term does, so no row's max grew past
+      // the lazy threshold; an overflow or NaN fails the test too);
+      // otherwise S, still intact in TMEM, goes through the two passes below
+      // (max, O rescale, exponentials).  The row max itself is not formed
+      // here: issue slots, not the exponential unit, bound this loop.
       if (fast && __all_sync(0xffffffffu, m_use != -INFINITY)) {
         uint32_t pk1[64];
-        float r0 = 0.f, r1 = 0.f, mxx = -INFINITY;
+        float r0 = 0.f, r1 = 0.f;
 #pragma unroll
         for (int c = 0; c < BN; c += 64) {
           uint32_t sv[64];
@@ -490,18 +494,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
-            const float x0 = fmaf(__uint_as_float(sv[e]), sl2, -m_use);
-            const float x1 = fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use);
-            mxx = fmaxf(mxx, fmaxf(x0, x1));
-            // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
-            const float p0 = (e & 7) >= 5 ? exp2_fma(x0) : exp2f(x0);
-            const float p1 = ((e + 1) & 7) >= 5 ? exp2_fma(x1) : exp2f(x1);
+            const float p0 = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
+            const float p1 = exp2f(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
             r0 += p0;
             r1 += p1;
             pk1[(c + e) / 2] = pack_bf16x2(p0, p1);
           }
         }
-        if (!__any_sync(0xffffffffu, mxx > kRescaleThreshold)) {
+        if (!__any_sync(0xffffffffu, !(r0 + r1 <= kRescaleBound))) {
           // keys [32c, 32c+32) -> columns [16c, 16c+16): all of S was read
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_st16(s_addr + c * 16, pk1 + c * 16);
@@ -574,9 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (fast) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float x = fmaf(__uint_as_float(sv[e]), sl2, -m_eff);
-              // 3 of every 8 exponentials on the FMA pipe, the rest on MUFU
-              e32[e] = (e & 7) >= 5 ? exp2_fma(x) : exp2f(x);
+              e32[e] = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_eff));
             }
           } else {
 #pragma unroll
