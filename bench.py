@@ -198,11 +198,11 @@ def bench_train(args, world, rank, peaks):
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
-        P = api.prefix_cumsum(g)
         if ev is not None:
             ev[0].record(stream)
-        # the forward's anchored operands are reused by the backward
-        o, lse, fws = api.wall_attn_fwd(q, k, v, P, s.scale, return_workspace=True)
+        # the prefix scan fused into the forward's operand pass; the
+        # forward's anchored operands are reused by the backward
+        o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, s.scale, return_workspace=True)
         if ev is not None:
             ev[1].record(stream)
         out = api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, fwd_workspace=fws)
@@ -238,12 +238,13 @@ def bench_train(args, world, rank, peaks):
     ms_max = max_over_ranks(ms, world)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    # launches of this library inside one step: prefix scan 3 (chunk sums,
-    # carries, chunk scans); forward: operand preparation 1 + tcgen05 forward
-    # 1; backward (reusing the forward's operands): D/sink pre-pass 1, tcgen05
-    # key-block (dK, dV) 1, tcgen05 query-block (dq) 1, finalize 1, reverse
-    # scan 3
-    launches_per_step = 12
+    # launches of this library inside one step: forward: prefix chunk sums
+    # and carries 2, chunk scans fused with the operand preparation 1,
+    # tcgen05 forward 1; backward (reusing the forward's operands): D/sink
+    # pre-pass 1, tcgen05 key-block (dK, dV, dS tiles) 1, dk/dv group sums 1,
+    # tcgen05 query-block dq 1, dq/dL finalize with dL's chunk sums 1,
+    # reverse-scan carries and chunk scans 2
+    launches_per_step = 11
     res = dict(ms=ms_max, value=world * step_flops / (ms_max * 1e-3) / 1e12,
                fwd_ms=fwd_ms, bwd_ms=bwd_ms,
                fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,
@@ -286,8 +287,8 @@ def bench_train_e2e(args, x, s, step_flops, world):
                 d[n].copy_(host_in[n], non_blocking=True)
             inputs_ready[b].record(s_h2d)
         s_comp.wait_event(inputs_ready[b])
-        P = api.prefix_cumsum(d["g"])
-        o, lse, fws = api.wall_attn_fwd(d["q"], d["k"], d["v"], P, s.scale, return_workspace=True)
+        o, lse, P, fws = api.wall_attn_fwd_gate(d["q"], d["k"], d["v"], d["g"], s.scale,
+                                                return_workspace=True)
         dq, dk, dv, dg, _, _ = api.wall_attn_bwd(d["dO"], d["q"], d["k"], d["v"], P, o, lse,
                                                  s.scale, fwd_workspace=fws)
         inputs_free[b].record(s_comp)

@@ -21,7 +21,8 @@ EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn
            "wall_attn_decode_workspace", "wall_attn_decode", "wall_get_status",
            "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
            "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step",
-           "wall_attn_decode_chunk_workspace", "wall_attn_decode_chunk"]
+           "wall_attn_decode_chunk_workspace", "wall_attn_decode_chunk",
+           "wall_attn_fwd_gate_workspace", "wall_attn_fwd_gate"]
 
 _lib = None
 
@@ -82,6 +83,11 @@ def lib():
         L.wall_decode_step.restype = i
         L.wall_decode_step.argtypes = [vp, vp, vp, vp, i, fp, vp, vp, fp, fp, f, i, i, i, i, i,
                                        i, i, i, vp, fp, vp, sz, vp]
+        L.wall_attn_fwd_gate_workspace.restype = sz
+        L.wall_attn_fwd_gate_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.wall_attn_fwd_gate.restype = i
+        L.wall_attn_fwd_gate.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, f, fp, fp, i, ip,
+                                         i, fp, vp, fp, vp, sz, vp]
         L.wall_attn_decode_chunk_workspace.restype = sz
         L.wall_attn_decode_chunk_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
         L.wall_attn_decode_chunk.restype = i
@@ -226,3 +232,18 @@ def wall_attn_decode_chunk(q, v, p, k_tilde, r_cache, sink_bias, scale, C, B, Tq
         _p(q), _p(v), _p(p), _p(k_tilde), _p(r_cache), _p(sink_bias), float(scale), C,
         dtype_code(q.dtype), B, Tq, T_kv, Tcap, H, HQ, K, V, _p(o), _p(lse), _p(workspace),
         ws_bytes, _stream(stream)))
+
+
+def wall_attn_fwd_gate_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> int:
+    return lib().wall_attn_fwd_gate_workspace(dtype_code(dtype), B, T, H, HQ, K, V,
+                                              int(bool(has_g_scalar)), n_seq)
+
+
+def wall_attn_fwd_gate(q, k, v, g, B, T, H, HQ, K, V, scale, g_scalar, sink_bias, window_size,
+                       cu_seqlens, n_seq, P, o, lse, workspace, stream=None):
+    """Prefix scan and forward in one call; P is written for the backward."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("wall_attn_fwd_gate", lib().wall_attn_fwd_gate(
+        _p(q), _p(k), _p(v), _p(g), dtype_code(q.dtype), B, T, H, HQ, K, V, float(scale),
+        _p(g_scalar), _p(sink_bias), int(window_size), _p(cu_seqlens), n_seq, _p(P), _p(o),
+        _p(lse), _p(workspace), ws_bytes, _stream(stream)))

@@ -69,6 +69,26 @@ def wall_attn_fwd(q, k, v, P, scale=None, g_scalar=None, sink_bias=None, window_
     return (o, lse, ws) if return_workspace else (o, lse)
 
 
+def wall_attn_fwd_gate(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size=None,
+                       cu_seqlens=None, return_workspace=False):
+    """Prefix scan and forward in one call, the prefix fused into the
+    forward's operand pass; returns (o, lse, P), or (o, lse, P, workspace)
+    with return_workspace (the workspace serves wall_attn_bwd as its
+    fwd_workspace).  P and o are bit for bit those of prefix_cumsum followed
+    by wall_attn_fwd."""
+    g = g.contiguous()
+    B, T, H, HQ, K, V = _shape_checks(q, k, v, g)
+    nseq = _n_seq(cu_seqlens, B)
+    o = torch.empty((B, T, HQ, V), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, T, HQ), dtype=torch.float32, device=q.device)
+    P = torch.empty((B, T, HQ, K), dtype=torch.float32, device=q.device)
+    ws = _ws(L.wall_attn_fwd_gate_workspace(q.dtype, B, T, H, HQ, K, V, g_scalar is not None,
+                                            nseq), q.device)
+    L.wall_attn_fwd_gate(q, k, v, g, B, T, H, HQ, K, V, scale or 0.0, g_scalar, sink_bias,
+                         window_size or 0, cu_seqlens, nseq, P, o, lse, ws)
+    return (o, lse, P, ws) if return_workspace else (o, lse, P)
+
+
 def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=None,
                   window_size=None, cu_seqlens=None, want_dsink=False, fwd_workspace=None):
     """Backward; returns dq, dk, dv, dg, dg_scalar (or None), dsink (or None).
@@ -99,9 +119,8 @@ class WallAttnFunction(torch.autograd.Function):
             raise TypeError("q, k, v and g must share one dtype")
         gs = g_scalar.contiguous().float() if g_scalar is not None else None
         sk = sink_bias.contiguous().float() if sink_bias is not None else None
-        P = prefix_cumsum(g, cu_seqlens)
-        o, lse, fws = wall_attn_fwd(q, k, v, P, scale, gs, sk, window_size, cu_seqlens,
-                                    return_workspace=True)
+        o, lse, P, fws = wall_attn_fwd_gate(q, k, v, g, scale, gs, sk, window_size, cu_seqlens,
+                                            return_workspace=True)
         ctx.save_for_backward(q, k, v, P, o, lse, gs, sk, cu_seqlens, fws)
         ctx.scale, ctx.window_size = scale, window_size
         ctx.gs_dtype = g_scalar.dtype if g_scalar is not None else None

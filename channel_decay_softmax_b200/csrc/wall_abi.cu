@@ -303,6 +303,69 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
   return attn_fwd_simt(pb, a, s);
 }
 
+size_t wall_attn_fwd_gate_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                                    int has_g_scalar, int n_seq) {
+  AttnProblem pb;
+  if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
+  if (n_seq > 0 && B == 1) pb.extra_blocks = n_seq;
+  const FwdWs w = fwd_ws_layout(pb, has_g_scalar);
+  // the forward's own layout first (wall_attn_bwd may reuse it), then the
+  // chunk carries of the fused prefix pass
+  return w.total + (fwd_tc_supported(pb) ? align256(sizeof(float) * pb.rows * HQ * K) : 0);
+}
+
+int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* g, int dtype,
+                       int B, int T, int H, int HQ, int K, int V, float scale,
+                       const float* g_scalar, const float* sink_bias, int window_size,
+                       const int32_t* cu_seqlens, int n_seq, float* P, void* o, float* lse,
+                       void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  AttnProblem pb;
+  int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
+  if (rc) return rc;
+  if (pb.rows == 0) return WALL_OK;
+  if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(P) || !ok_ptr(o))
+    return WALL_ERR_INVALID_ARG;
+  if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(lse)) return WALL_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws_layout(pb, g_scalar != nullptr);
+  const bool tc = fwd_tc_supported(pb);
+  const size_t need = w.total + (tc ? align256(sizeof(float) * pb.rows * HQ * K) : 0);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return WALL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cu_seqlens) {
+    rc = check_cu(cu_seqlens, n_seq, pb.rows, s);
+    if (rc) return rc;
+  }
+  FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.P = P; a.sink = sink_bias; a.o = o; a.lse = lse;
+  a.GS = nullptr;
+  if (g_scalar) {
+    float* gs = reinterpret_cast<float*>(at(workspace, w.gs));
+    rc = scan_prefix_plain(g_scalar, gs, HQ, pb.seqs, s);
+    if (rc) return rc;
+    a.GS = gs;
+  }
+  if (!tc) {
+    timing_mark(T_PREFIX, s);
+    rc = scan_prefix_log2(g, dtype, P, (long)HQ * K, pb.seqs, nullptr, nullptr, s);
+    timing_mark(T_PREFIX, s);
+    if (rc) return rc;
+    return attn_fwd_simt(pb, a, s);
+  }
+  TcFwdWs tw;
+  tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
+  tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
+  tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+  tw.n_blocks128 = w.n_blocks128;
+  rc = scan_prefix_operands(static_cast<const __nv_bfloat16*>(g),
+                            static_cast<const __nv_bfloat16*>(q),
+                            static_cast<const __nv_bfloat16*>(k), P,
+                            reinterpret_cast<float*>(at(workspace, w.total)), HQ, H, K, pb.seqs,
+                            tw.qh, tw.kh, tw.anchors, s);
+  if (rc) return rc;
+  return attn_fwd_tc(pb, a, tw, status_ptr(), s, /*prepared=*/true);
+}
+
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                int has_g_scalar, int n_seq) {
   AttnProblem pb;
@@ -375,20 +438,26 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
       tw.kh = reinterpret_cast<__nv_bfloat16*>(at(fws, fw.kh));
       tw.anchors = reinterpret_cast<float*>(at(fws, fw.anchors));
     }
-    rc = attn_bwd_tc(pb, a, tw, !reuse, dq, dk, dv, status_ptr(), s);
+    // dg as well: dL's reverse scan starts inside the finalize pass
+    rc = attn_bwd_tc(pb, a, tw, !reuse, dq, dk, dv, dg, status_ptr(), s);
     if (rc) return rc;
   } else {
     rc = attn_bwd_simt(pb, a, s);
     if (rc) return rc;
     rc = attn_bwd_reduce(pb, a, dq, dk, dv, s);
     if (rc) return rc;
+    // dg = reverse cumulative sum of dL (held in dq32 after the reduce);
+    // the per-head dk buffer is dead after the reduce: chunk scratch
+    timing_mark(T_REV_SCAN, s);
+    rc = scan_reverse(a.dq32, dg, dtype, a.dkh32, (long)HQ * K, pb.seqs, s);
+    timing_mark(T_REV_SCAN, s);
+    if (rc) return rc;
   }
-  // dg = reverse cumulative sum of dL (held in dq32 after the reduce)
-  // the per-head dk buffer is dead after the finalize: chunk scratch
-  timing_mark(T_REV_SCAN, s);
-  rc = scan_reverse(a.dq32, dg, dtype, a.dkh32, (long)HQ * K, pb.seqs, s);
-  if (!rc && g_scalar) rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, a.dgs_col, HQ, pb.seqs, s);
-  timing_mark(T_REV_SCAN, s);
+  if (g_scalar) {
+    timing_mark(T_REV_SCAN, s);
+    rc = scan_reverse(a.dgs_row, dg_scalar, WALL_FP32, a.dgs_col, HQ, pb.seqs, s);
+    timing_mark(T_REV_SCAN, s);
+  }
   return rc;
 }
 

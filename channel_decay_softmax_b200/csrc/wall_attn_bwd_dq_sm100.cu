@@ -460,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warp 1      TMEM owner (128 columns) and MMA issuer: A = dS (queries x
 //               keys, MN-major: queries contiguous in the stored rows),
 //               B = Kt (keys x channels, MN-major)
-//   warps 2-3   Kt_J = Kh_J (.) d in place, as in the kernel above
+//   warps 2-5   Kt_J = Kh_J (.) d in place, as in the kernel above (four
+//               warps: with two, the in-place scaling set the tile rate)
 //   warps 4-7   epilogue: dQa rows -> fp32 workspace
 constexpr int kDS = 3;  // stages
 constexpr int kDsThreads = 256;
@@ -515,7 +516,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDS; ++s) {
       mbar_init(bar(QS_FULL + s), 1);
-      mbar_init(bar(QS_READY + s), 2);
+      mbar_init(bar(QS_READY + s), 4);
       mbar_init(bar(QS_EMPTY + s), 1);
     }
     mbar_init(bar(QS_DONE), 1);
@@ -582,75 +583,78 @@ __global__ void __launch_bounds__(kDsThreads, 1)
       umma_commit(bar(QS_MMA));
       mbar_wait(bar(QS_MMA), 0, p.status);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ key rescale
-    constexpr int kChunks = KD / 8;
-    constexpr int kRowStep = 64 / kChunks;
-    constexpr int kRows = BN / kRowStep;
-    const int tid = threadIdx.x - 64;
-    const int ch = tid % kChunks;
-    const int rs = tid / kChunks;
-    float ri[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
-    for (int t = 0; t < nT; ++t) {
-      const int st = t % kDS;
-      {
-        const bool got = wait_bar(bar(QS_FULL + st), (t / kDS) & 1, p.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) break;
-      }
-      const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
-      __nv_bfloat162 d[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
-                           (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
-        d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
-      }
-      uint8_t* kt = smem + Lay::oK + st * Lay::kKT + (ch / 8) * (BN * 128);
-      constexpr int kBatch = 8;
-#pragma unroll
-      for (int m0 = 0; m0 < kRows; m0 += kBatch) {
-        uint4 v[kBatch];
-#pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          const int r = rs + (m0 + x) * kRowStep;
-          v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
-        }
-#pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          const int r = rs + (m0 + x) * kRowStep;
-          __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
-          *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(QS_READY + st));
-    }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const bool ok = __all_sync(0xffffffffu, wait_bar(bar(QS_DONE), 0, p.status, abort_flag));
-    if (ok) {
-      tc_fence_after();
-      float* out = p.dq32 + ((s0 + i0 + r) * HQ + h) * (long)K;
-#pragma unroll 1
-      for (int c = 0; c < KD; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + c, v);
-        tmem_wait_ld();
-        if (r < ni) {
+    if (warp < 6) {
+      // ------------------------------------------------------------ key rescale
+      constexpr int kChunks = KD / 8;
+      constexpr int kRowStep = 128 / kChunks;
+      constexpr int kRows = BN / kRowStep;
+      const int tid = threadIdx.x - 64;
+      const int ch = tid % kChunks;
+      const int rs = tid / kChunks;
+      float ri[8];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(out + c + e) =
-                make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+      for (int e = 0; e < 8; ++e)
+        ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kDS;
+        {
+          const bool got = wait_bar(bar(QS_FULL + st), (t / kDS) & 1, p.status, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) break;
+        }
+        const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
+        __nv_bfloat162 d[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t b = pow2_bf16(ri[2 * e] - rj[2 * e]) |
+                             (pow2_bf16(ri[2 * e + 1] - rj[2 * e + 1]) << 16);
+          d[e] = *reinterpret_cast<const __nv_bfloat162*>(&b);
+        }
+        uint8_t* kt = smem + Lay::oK + st * Lay::kKT + (ch / 8) * (BN * 128);
+        constexpr int kBatch = 8;
+#pragma unroll
+        for (int m0 = 0; m0 < kRows; m0 += kBatch) {
+          uint4 v[kBatch];
+#pragma unroll
+          for (int x = 0; x < kBatch; ++x) {
+            const int r = rs + (m0 + x) * kRowStep;
+            v[x] = *reinterpret_cast<const uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+          }
+#pragma unroll
+          for (int x = 0; x < kBatch; ++x) {
+            const int r = rs + (m0 + x) * kRowStep;
+            __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(&v[x]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[e] = __hmul2(w[e], d[e]);
+            *reinterpret_cast<uint4*>(kt + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v[x];
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(QS_READY + st));
+      }
+    }
+    if (warp >= 4) {
+      // ------------------------------------------------------------ epilogue
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;
+      const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+      const bool ok = __all_sync(0xffffffffu, wait_bar(bar(QS_DONE), 0, p.status, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        float* out = p.dq32 + ((s0 + i0 + r) * HQ + h) * (long)K;
+#pragma unroll 1
+        for (int c = 0; c < KD; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + c, v);
+          tmem_wait_ld();
+          if (r < ni) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(out + c + e) =
+                  make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                              __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
         }
       }
     }

@@ -720,17 +720,15 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-// dq = scale * 2^(P - R_I) (.) dq32 for the tensor-core path (R_I = floor of P
-// at the row's 128-row block start), then dL = q (.) dq - k (.) dk^(h) over dq32;
-// dk, dv = group sums; dGS = row + column parts.
+// dk, dv = sums of the per-query-head dk^(h), dv^(h) over each GQA group;
+// dGS = row + column parts.  (dq and the gate-gradient summand dL come from
+// finalize_dq_dl_sums, fused with the reverse scan's first pass.)
 template <typename T>
-__global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                    const float* __restrict__ P, Seqs seqs, int HQ, int H, int K,
-                                    int V, float scale, float* __restrict__ dq32,
+__global__ void bwd_finalize_kernel(Seqs seqs, int HQ, int H, int K, int V,
                                     const float* __restrict__ dkh32,
                                     const float* __restrict__ dvh32, float* __restrict__ dgs_row,
-                                    const float* __restrict__ dgs_col, T* __restrict__ dq,
-                                    T* __restrict__ dk, T* __restrict__ dv) {
+                                    const float* __restrict__ dgs_col, T* __restrict__ dk,
+                                    T* __restrict__ dv) {
   const int s = blockIdx.y;
   const long s0 = seqs.start(s);
   const int L = seqs.len(s);
@@ -738,31 +736,6 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ q, const T* __restrict
   const long stride = (long)gridDim.x * blockDim.x;
   const long tid0 = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const int kg = K / 8;
-  const long nq = (long)L * HQ * kg;
-  for (long e = tid0; e < nq; e += stride) {
-    const int g8 = (int)(e % kg);
-    const int hh = (int)((e / kg) % HQ);
-    const int t = (int)(e / ((long)kg * HQ));
-    const long row = s0 + t;
-    const long arow = s0 + (long)(t / 128) * 128;
-    const long off = (row * HQ + hh) * K + g8 * 8;
-    float pv[8], rv[8], a[8], qq[8], kk[8], dkv[8], out[8];
-    load8(P + off, pv);
-    load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
-#pragma unroll
-    for (int x = 0; x < 8; ++x) rv[x] = floorf(rv[x]);
-    load8(dq32 + off, a);
-    load8(q + off, qq);
-    load8(k + (row * H + hh / G) * K + g8 * 8, kk);
-    load8(dkh32 + off, dkv);
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      a[x] *= scale * exp2f(pv[x] - rv[x]);
-      out[x] = qq[x] * a[x] - kk[x] * dkv[x];
-    }
-    store8(dq + off, a);
-    store8(dq32 + off, out);
-  }
   const long nk = (long)L * H * kg;
   for (long e = tid0; e < nk; e += stride) {
     const int g8 = (int)(e % kg);
@@ -853,7 +826,7 @@ int launch_bwd_tc_gs(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws,
 }  // namespace
 
 int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool prepare, void* dq,
-                void* dk, void* dv, int* status, cudaStream_t stream) {
+                void* dk, void* dv, void* dg, int* status, cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
   int rc = WALL_OK;
   if (prepare) {  // else the forward's operands are reused
@@ -877,19 +850,36 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
                    : launch_bwd_tc_gs<64>(pb, a, ws, status, stream);
   timing_mark(T_BWD_KEY, stream);
   if (rc) return rc;
+  // dk, dv group sums and the scalar-gate parts need only the key-block
+  // kernel; they run before dL overwrites dk^(h)'s chunk rows with its sums
+  timing_mark(T_BWD_FIN, stream);
+  {
+    dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
+    bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        pb.seqs, pb.HQ, pb.H, pb.K, pb.V, a.dkh32, a.dvh32, a.GS ? a.dgs_row : nullptr,
+        a.GS ? a.dgs_col : nullptr, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv));
+    if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+  }
+  timing_mark(T_BWD_FIN, stream);
   timing_mark(T_BWD_DQ, stream);
   rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
   timing_mark(T_BWD_DQ, stream);
   if (rc) return rc;
+  // dq, dL and dL's chunk sums in one pass, then the reverse scan's
+  // carries and chunk scans give dg
   timing_mark(T_BWD_FIN, stream);
-  dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
-  bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.P,
-      pb.seqs, pb.HQ, pb.H, pb.K, pb.V, pb.scale, a.dq32, a.dkh32, a.dvh32,
-      a.GS ? a.dgs_row : nullptr, a.GS ? a.dgs_col : nullptr, static_cast<__nv_bfloat16*>(dq),
-      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+  rc = finalize_dq_dl_sums(static_cast<const __nv_bfloat16*>(a.q),
+                           static_cast<const __nv_bfloat16*>(a.k), a.P, a.dq32, a.dkh32,
+                           static_cast<__nv_bfloat16*>(dq), pb.HQ, pb.H, pb.K, pb.scale,
+                           pb.seqs, stream);
   timing_mark(T_BWD_FIN, stream);
-  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+  if (rc) return rc;
+  timing_mark(T_REV_SCAN, stream);
+  rc = scan_reverse_from_sums(a.dq32, dg, WALL_BF16, a.dkh32, (long)pb.HQ * pb.K, pb.seqs,
+                              stream);
+  timing_mark(T_REV_SCAN, stream);
+  return rc;
 }
 
 }  // namespace wall

@@ -839,12 +839,15 @@ int attn_decode_chunk_tc(const void* q, const void* v, const float* p, const voi
 }
 
 int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
-                cudaStream_t stream) {
+                cudaStream_t stream, bool prepared) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
-  timing_mark(T_OPERANDS, stream);
-  int rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
-  timing_mark(T_OPERANDS, stream);
-  if (rc) return rc;
+  int rc = WALL_OK;
+  if (!prepared) {
+    timing_mark(T_OPERANDS, stream);
+    rc = attn_prepare_operands(pb, a.q, a.k, a.P, ws, stream);
+    timing_mark(T_OPERANDS, stream);
+    if (rc) return rc;
+  }
   timing_mark(T_FWD, stream);
   rc = pb.K == 128 ? launch_fwd_tc<128>(pb, a, ws, status, stream)
                    : launch_fwd_tc<64>(pb, a, ws, status, stream);

@@ -23,6 +23,22 @@ enum TimingSlot {
 int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seqs,
                      const float* carry_in, float* carry_out, cudaStream_t stream);
 int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream);
+// the forward prefix fused with the tensor-core operand preparation: P (as
+// scan_prefix_log2 forms it, bit for bit), Qh, Kh and the 128-row block
+// anchors (as attn_prepare_operands forms them); scratch: fp32 [rows, HQ*K]
+// for the chunk carries, not P
+int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                         float* P, float* scratch, int HQ, int H, int K, const Seqs& seqs,
+                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors,
+                         cudaStream_t stream);
+// the tensor-core backward's dq finalize fused with pass 1 of dL's reverse
+// scan: dq (bf16), dL over dq32, chunk sums of dL into dkh32's chunk rows
+int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* P,
+                        float* dq32, float* dkh32, __nv_bfloat16* dq, int HQ, int H, int K,
+                        float scale, const Seqs& seqs, cudaStream_t stream);
+// passes 2 and 3 of the reverse scan, the chunk sums already in scratch
+int scan_reverse_from_sums(const float* x, void* y, int out_dtype, float* scratch, long C,
+                           const Seqs& seqs, cudaStream_t stream);
 int scan_reverse(const float* x, void* y, int out_dtype, float* scratch, long C,
                  const Seqs& seqs, cudaStream_t stream);
 
@@ -77,13 +93,15 @@ struct TcFwdWs {
 bool fwd_tc_supported(const AttnProblem& pb);
 int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
                           const TcFwdWs& ws, cudaStream_t stream);
+// prepared: ws already holds Qh, Kh and the anchors (the fused prefix pass)
 int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int* status,
-                cudaStream_t stream);
+                cudaStream_t stream, bool prepared = false);
 
 // ---- tensor-core backward (wall_attn_bwd_sm100.cu) ----
 // prepare: false when ws already holds the forward's anchored operands
+// also writes dg (the reverse scan of dL) on this path
 int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool prepare,
-                void* dq, void* dk, void* dv, int* status, cudaStream_t stream);
+                void* dq, void* dk, void* dv, void* dg, int* status, cudaStream_t stream);
 // raw dq (without the per-row anchor factor) into a.dq32 (wall_attn_bwd_dq_sm100.cu)
 int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                    cudaStream_t stream);

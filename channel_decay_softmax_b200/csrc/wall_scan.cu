@@ -214,6 +214,201 @@ __global__ void __launch_bounds__(kThreadsScan)
   }
 }
 
+// pass 3 of the forward scan fused with the tensor-core forward's operand
+// preparation (the prefix enters the forward without an HBM round trip of
+// its own): per (sequence, chunk, 8 columns of one query head) the same
+// compensated scan from the chunk's carry as chunk_scan_kernel, bit for bit,
+// writing P, and for each row
+//   Qh = q * 2^(P - R),  Kh = k * 2^(R - P),  R = floor(P at the row's
+//   128-row block start)   (the anchors, written at the block start row)
+// as the forward's preparation kernel forms them.  R of a block whose start
+// lies in an earlier chunk is that row's prefix, rebuilt from its chunk's
+// carry: the scan's first step is carry + g, then one fused rounding.
+// The carries come from a scratch that is not P, so no thread reads a carry
+// another one has overwritten.
+constexpr int kInFlightOps = 8;
+// at most 128 registers: four CTAs per SM, so the 512 CTAs of the T = 8192
+// problem run in one wave (with 150 registers they needed 1.15 waves and
+// took 50 % longer)
+__global__ void __launch_bounds__(kThreadsScan, 4)
+    chunk_scan_operands_kernel(const __nv_bfloat16* __restrict__ g,
+                               const __nv_bfloat16* __restrict__ q,
+                               const __nv_bfloat16* __restrict__ k,
+                               const float* __restrict__ scratch, float* __restrict__ P, long C,
+                               Seqs seqs, int HQ, int H, int K, __nv_bfloat16* __restrict__ qh,
+                               __nv_bfloat16* __restrict__ kh, float* __restrict__ anchors) {
+  constexpr int BA = 128;  // anchor block rows of the tensor-core kernels
+  __shared__ int s_blk_off;
+  int s, kc;
+  if (!seq_block(seqs, kChunk, (int)blockIdx.x, s, kc)) return;  // uniform in the CTA
+  const long start = seqs.start(s);
+  const long len = seqs.len(s);
+  const long lr0 = (long)kc * kChunk;
+  if (lr0 >= len) return;  // uniform in the CTA
+  if (threadIdx.x == 0) {
+    int off = 0;
+    if (seqs.cu) {
+      for (int x = 0; x < s; ++x) off += (seqs.len(x) + BA - 1) / BA;
+    } else {
+      off = s * ((seqs.T + BA - 1) / BA);
+    }
+    s_blk_off = off;
+  }
+  __syncthreads();
+  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * 8;
+  if (col >= C) return;
+  const int n = (int)min((long)kChunk, len - lr0);
+  const int hh = (int)(col / K), n0 = (int)(col % K);
+  const int G = HQ / H;
+  // R: the anchor of the 128-row block this chunk lies in
+  const long lb = (lr0 / BA) * BA;
+  float R[8];
+  {
+    const float* cb = scratch + chunk_row(start, len, (int)(lb / kChunk), false) * C + col;
+    float gb[8];
+    load8(g + (start + lb) * C + col, gb);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) R[v] = floorf(fmaf(kInvLn2, cb[v] + gb[v], 0.f));
+  }
+  float acc[8], cmp[8];
+  {
+    const float* c = scratch + chunk_row(start, len, kc, false) * C + col;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      acc[v] = c[v];
+      cmp[v] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int r0 = 0; r0 < kChunk; r0 += kInFlightOps) {
+    float a[kInFlightOps][8];
+    uint4 qa[kInFlightOps], ka[kInFlightOps];
+#pragma unroll
+    for (int r = 0; r < kInFlightOps; ++r) {
+      const long pr = start + lr0 + (r0 + r < n ? r0 + r : 0);
+      load8(g + pr * C + col, a[r]);
+      qa[r] = *reinterpret_cast<const uint4*>(q + pr * C + col);
+      ka[r] = *reinterpret_cast<const uint4*>(k + (pr * H + hh / G) * K + n0);
+    }
+#pragma unroll
+    for (int rr = 0; rr < kInFlightOps; ++rr) {
+      const int r = r0 + rr;
+      const long lr = lr0 + r;
+      const long pr = start + lr;
+      float o[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float yk = a[rr][v] - cmp[v];
+        const float tk = acc[v] + yk;
+        cmp[v] = (tk - acc[v]) - yk;
+        acc[v] = tk;
+        o[v] = fmaf(kInvLn2, acc[v], 0.f);
+      }
+      if (r < n) {
+        store8(P + pr * C + col, o);
+        float x[8], y[8];
+        const __nv_bfloat162* qv = reinterpret_cast<const __nv_bfloat162*>(&qa[rr]);
+        const __nv_bfloat162* kv = reinterpret_cast<const __nv_bfloat162*>(&ka[rr]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float2 f = __bfloat1622float2(qv[v]);
+          x[2 * v] = f.x;
+          x[2 * v + 1] = f.y;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) y[v] = x[v] * exp2f(o[v] - R[v]);
+        store8(qh + pr * C + col, y);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float2 f = __bfloat1622float2(kv[v]);
+          x[2 * v] = f.x;
+          x[2 * v + 1] = f.y;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) y[v] = x[v] * exp2f(R[v] - o[v]);
+        store8(kh + pr * C + col, y);
+        if (lr == lb)
+          store8(anchors + ((long)(s_blk_off + lr / BA) * HQ + hh) * K + n0, R);
+      }
+    }
+  }
+}
+
+// The backward's dq finalize fused with pass 1 of the reverse scan of dL
+// (tensor-core path): per (sequence, chunk in reverse order, 8 columns of one
+// query head), for each row
+//   dq = scale * 2^(P - R_I) (.) dq32          R_I = floor(P at the row's
+//                                              128-row block start)
+//   dL = q (.) dq - k (.) dk^(h)               (fp32, written over dq32)
+// and the chunk's compensated sum of dL in the order chunk_sum_kernel adds
+// it, into the chunk row of `scratch` (dk^(h) itself: this thread has read
+// that row's dk^(h) by then, and no other thread reads this chunk's rows).
+__global__ void __launch_bounds__(kThreadsScan, 4)
+    finalize_dl_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                       const float* __restrict__ P, float* __restrict__ dq32,
+                       const float* __restrict__ dkh32, float* __restrict__ scratch,
+                       __nv_bfloat16* __restrict__ dq, long C, Seqs seqs, int HQ, int H, int K,
+                       float scale) {
+  constexpr int BA = 128;
+  int s, kc;
+  if (!seq_block(seqs, kChunk, (int)blockIdx.x, s, kc)) return;
+  const long start = seqs.start(s);
+  const long len = seqs.len(s);
+  const long lr0 = (long)kc * kChunk;
+  if (lr0 >= len) return;
+  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * 8;
+  if (col >= C) return;
+  const int n = (int)min((long)kChunk, len - lr0);
+  const int hh = (int)(col / K), n0 = (int)(col % K);
+  const int G = HQ / H;
+  float sum[8], cmp[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) sum[v] = cmp[v] = 0.f;
+#pragma unroll 1
+  for (int r0 = 0; r0 < kChunk; r0 += kInFlightOps) {
+    float dl[kInFlightOps][8];
+#pragma unroll
+    for (int r = 0; r < kInFlightOps; ++r) {
+      const bool in = r0 + r < n;
+      const long lr = lr0 + (in ? r0 + r : 0);
+      const long pr = start + len - 1 - lr;  // reverse scan order
+      const long off = pr * C + col;
+      const long arow = start + ((pr - start) / BA) * BA;
+      float pv[8], rv[8], a[8], qq[8], kk[8], dkv[8];
+      load8(P + off, pv);
+      load8(P + arow * C + col, rv);
+      load8(dq32 + off, a);
+      load8(q + off, qq);
+      load8(k + (pr * H + hh / G) * K + n0, kk);
+      load8(dkh32 + off, dkv);
+      float o[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        a[v] *= scale * exp2f(pv[v] - floorf(rv[v]));
+        o[v] = qq[v] * a[v] - kk[v] * dkv[v];
+        dl[r][v] = in ? o[v] : 0.f;
+      }
+      if (in) {
+        store8(dq + off, a);
+        store8(dq32 + off, o);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kInFlightOps; ++r) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float yk = dl[r][v] - cmp[v];
+        const float tk = sum[v] + yk;
+        cmp[v] = (tk - sum[v]) - yk;
+        sum[v] = tk;
+      }
+    }
+  }
+  float* dst = scratch + chunk_row(start, len, kc, true) * C + col;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) dst[v] = sum[v];
+}
+
 template <typename Tin, typename Tout, bool kReverse, int VEC>
 int launch_scan_vec(const Tin* x, Tout* y, float* scratch, long C, const Seqs& seqs, float mul,
                     const float* carry_in, float* carry_out, cudaStream_t stream) {
@@ -257,6 +452,72 @@ int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seq
                                                     seqs, kInvLn2, carry_in, carry_out, stream);
   return launch_scan<float, float, false>(static_cast<const float*>(g), P, P, C, seqs, kInvLn2,
                                           carry_in, carry_out, stream);
+}
+
+int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                         float* P, float* scratch, int HQ, int H, int K, const Seqs& seqs,
+                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors,
+                         cudaStream_t stream) {
+  const long C = (long)HQ * K;
+  if (seqs.n == 0 || C == 0) return WALL_OK;
+  if (C % 8 != 0) return WALL_ERR_UNSUPPORTED;
+  const long groups = (C / 8 + kThreadsScan - 1) / kThreadsScan;
+  const long chunks = seqs.cu ? (seqs.rows + kChunk - 1) / kChunk + seqs.n
+                              : (long)seqs.n * ((seqs.T + kChunk - 1) / kChunk);
+  if (groups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  if (chunks == 0) return WALL_OK;
+  const dim3 grid((unsigned)chunks, (unsigned)groups);
+  timing_mark(T_PREFIX, stream);
+  chunk_sum_kernel<__nv_bfloat16, 8, false><<<grid, kThreadsScan, 0, stream>>>(g, scratch, C, seqs);
+  const dim3 cgrid((unsigned)((C + 31) / 32), (unsigned)seqs.n);
+  carry_kernel<false><<<cgrid, 32 * kCarryParts, 0, stream>>>(scratch, C, seqs, kInvLn2, nullptr,
+                                                              nullptr);
+  timing_mark(T_PREFIX, stream);
+  timing_mark(T_OPERANDS, stream);
+  chunk_scan_operands_kernel<<<grid, kThreadsScan, 0, stream>>>(g, q, k, scratch, P, C, seqs, HQ,
+                                                                H, K, qh, kh, anchors);
+  timing_mark(T_OPERANDS, stream);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* P,
+                        float* dq32, float* dkh32, __nv_bfloat16* dq, int HQ, int H, int K,
+                        float scale, const Seqs& seqs, cudaStream_t stream) {
+  const long C = (long)HQ * K;
+  if (seqs.n == 0 || C == 0) return WALL_OK;
+  if (C % 8 != 0) return WALL_ERR_UNSUPPORTED;
+  const long groups = (C / 8 + kThreadsScan - 1) / kThreadsScan;
+  const long chunks = seqs.cu ? (seqs.rows + kChunk - 1) / kChunk + seqs.n
+                              : (long)seqs.n * ((seqs.T + kChunk - 1) / kChunk);
+  if (groups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  if (chunks == 0) return WALL_OK;
+  finalize_dl_kernel<<<dim3((unsigned)chunks, (unsigned)groups), kThreadsScan, 0, stream>>>(
+      q, k, P, dq32, dkh32, dkh32, dq, C, seqs, HQ, H, K, scale);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+int scan_reverse_from_sums(const float* x, void* y, int out_dtype, float* scratch, long C,
+                           const Seqs& seqs, cudaStream_t stream) {
+  if (seqs.n == 0 || C == 0) return WALL_OK;
+  if (C % 8 != 0 || ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y) |
+                      reinterpret_cast<uintptr_t>(scratch)) % 16) != 0)
+    return WALL_ERR_UNSUPPORTED;
+  const long groups = (C / 8 + kThreadsScan - 1) / kThreadsScan;
+  const long chunks = seqs.cu ? (seqs.rows + kChunk - 1) / kChunk + seqs.n
+                              : (long)seqs.n * ((seqs.T + kChunk - 1) / kChunk);
+  if (groups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  if (chunks == 0) return WALL_OK;
+  const dim3 grid((unsigned)chunks, (unsigned)groups);
+  const dim3 cgrid((unsigned)((C + 31) / 32), (unsigned)seqs.n);
+  carry_kernel<true><<<cgrid, 32 * kCarryParts, 0, stream>>>(scratch, C, seqs, 1.f, nullptr,
+                                                             nullptr);
+  if (out_dtype == WALL_BF16)
+    chunk_scan_kernel<float, __nv_bfloat16, 8, true><<<grid, kThreadsScan, 0, stream>>>(
+        x, static_cast<__nv_bfloat16*>(y), scratch, C, seqs, 1.f, nullptr);
+  else
+    chunk_scan_kernel<float, float, 8, true><<<grid, kThreadsScan, 0, stream>>>(
+        x, static_cast<float*>(y), scratch, C, seqs, 1.f, nullptr);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
 int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream) {

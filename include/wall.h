@@ -118,6 +118,33 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
                   void* o, float* lse, void* workspace, size_t workspace_bytes,
                   wall_stream_t stream);
 
+/* wall_attn_fwd_gate_workspace -- bytes of workspace wall_attn_fwd_gate needs:
+ * wall_attn_fwd_workspace's layout first, then the prefix scan's chunk
+ * carries (fp32 [B*T, HQ*K]) on the tensor-core path. */
+size_t wall_attn_fwd_gate_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
+                                    int has_g_scalar, int n_seq);
+
+/*
+ * wall_attn_fwd_gate -- wall_prefix_cumsum and wall_attn_fwd in one call,
+ * with the prefix fused into the forward (blog "Wall Attention", fast
+ * training section 1: the anchored factors come from the prefix P of the
+ * gates; README "Decode": P = cumsum(g) / ln 2).  From the gates g
+ * [B,T,HQ,K] (`dtype`) it writes P [B,T,HQ,K] fp32 -- bit for bit what
+ * wall_prefix_cumsum writes, for wall_attn_bwd -- and o, lse exactly as
+ * wall_attn_fwd computes them from that P.  On the tensor-core path the
+ * scan's last pass also forms the anchored operands, so P is not read back
+ * (one pass over q, k, g instead of a scan and a preparation pass).  The
+ * workspace (wall_attn_fwd_gate_workspace bytes, 16-byte aligned) begins with
+ * wall_attn_fwd's layout, so it can be handed to wall_attn_bwd as its
+ * fwd_workspace.  Arguments, options, errors and the supported cases are
+ * those of wall_attn_fwd, plus g (non-null, 16-byte aligned).
+ */
+int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* g, int dtype,
+                       int B, int T, int H, int HQ, int K, int V, float scale,
+                       const float* g_scalar, const float* sink_bias, int window_size,
+                       const int32_t* cu_seqlens, int n_seq, float* P, void* o, float* lse,
+                       void* workspace, size_t workspace_bytes, wall_stream_t stream);
+
 /* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs. */
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                int has_g_scalar, int n_seq);

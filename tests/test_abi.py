@@ -164,6 +164,29 @@ def test_decode_chunk_rejects_bad_arguments(lib):
     assert call(Tq=0) == L.WALL_OK                            # empty: nothing launched
 
 
+def test_fwd_gate_workspace_and_checks(lib):
+    al = lambda x: (x + 255) // 256 * 256
+    B, T, H, HQ, K, V = 2, 100, 4, 8, 64, 64
+    fwd = lib.wall_attn_fwd_workspace(0, B, T, H, HQ, K, V, 0, 0)
+    # the forward's layout, then the prefix scan's chunk carries [B*T, HQ*K] fp32
+    assert lib.wall_attn_fwd_gate_workspace(0, B, T, H, HQ, K, V, 0, 0) == \
+        fwd + al(4 * B * T * HQ * K)
+    # fp32 (SIMT path): no anchored operands, no carries
+    assert lib.wall_attn_fwd_gate_workspace(1, B, T, H, HQ, K, V, 0, 0) == \
+        lib.wall_attn_fwd_workspace(1, B, T, H, HQ, K, V, 0, 0)
+    need = lib.wall_attn_fwd_gate_workspace(0, B, T, H, HQ, K, V, 0, 0)
+
+    def call(g=FAKE, P=FAKE, HQ=HQ, ws_bytes=need, dtype=0):
+        return lib.wall_attn_fwd_gate(FAKE, FAKE, FAKE, g, dtype, B, T, H, HQ, K, V, 0.0, None,
+                                      None, 0, None, 0, P, FAKE, FAKE, FAKE, ws_bytes, None)
+
+    assert call(g=None) == L.WALL_ERR_INVALID_ARG
+    assert call(P=None) == L.WALL_ERR_INVALID_ARG
+    assert call(HQ=6) == L.WALL_ERR_INVALID_ARG
+    assert call(ws_bytes=need - 1) == L.WALL_ERR_INVALID_ARG
+    assert call(dtype=7) == L.WALL_ERR_INVALID_ARG
+
+
 def test_prefix_rejects_bad_arguments(lib):
     pc = lib.wall_prefix_cumsum
     assert pc(FAKE, 3, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG

@@ -225,3 +225,35 @@ def test_dq_from_stored_ds_matches_recompute(K):
     for name, ta, tb in zip(("dq", "dk", "dv", "dg"), ga[:4], gb[:4]):
         e = float((ta.float() - tb.float()).norm() / tb.float().norm())
         assert e < 1e-2, (name, e)
+
+
+@pytest.mark.parametrize("case", ["cfg2", "cfg4_reduced", "fp32_options"])
+def test_fwd_gate_equals_prefix_then_forward(case):
+    """wall_attn_fwd_gate fuses the prefix scan into the forward's operand
+    pass: P must be bit for bit wall_prefix_cumsum's, o and lse bit for bit
+    wall_attn_fwd's from that P, and its workspace must serve the backward as
+    the forward's does (dense, varlen with every option, fp32)."""
+    if case == "cfg2":
+        s = I.spec(2)
+    elif case == "cfg4_reduced":
+        s = I.spec(4, len_lo=64, len_hi=600, window=128)
+    else:
+        s = I.spec(4, dtype=torch.float32, K=64, V=64, HQ=4, H=2, window=100, len_lo=1,
+                   len_hi=300)
+    x = _to(I.training_inputs(s))
+    q, k, v, g, cu = x["q"], x["k"], x["v"], x["g"], x["cu_seqlens"]
+    kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=x["window_size"],
+              cu_seqlens=cu)
+    P = api.prefix_cumsum(g, cu)
+    o, lse, fws = api.wall_attn_fwd(q, k, v, P, x["scale"], return_workspace=True, **kw)
+    o2, lse2, P2, gws = api.wall_attn_fwd_gate(q, k, v, g, x["scale"], return_workspace=True,
+                                               **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(P2, P)
+    assert torch.equal(o2, o)
+    assert torch.equal(lse2, lse)
+    a = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], fwd_workspace=fws, **kw)
+    b = api.wall_attn_bwd(x["dO"], q, k, v, P2, o2, lse2, x["scale"], fwd_workspace=gws, **kw)
+    torch.cuda.synchronize()
+    for name, ta, tb in zip(("dq", "dk", "dv", "dg"), a[:4], b[:4]):
+        assert torch.equal(ta, tb), name
