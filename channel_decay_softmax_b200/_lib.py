@@ -22,7 +22,7 @@ EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn
            "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
            "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step",
            "wall_attn_decode_chunk_workspace", "wall_attn_decode_chunk",
-           "wall_attn_fwd_gate_workspace", "wall_attn_fwd_gate"]
+           "wall_attn_fwd_gate_workspace", "wall_attn_fwd_gate", "wall_timing_enable_slots"]
 
 _lib = None
 
@@ -75,6 +75,8 @@ def lib():
                                                i, vp, fp, vp]
         L.wall_timing_enable.restype = i
         L.wall_timing_enable.argtypes = [i]
+        L.wall_timing_enable_slots.restype = i
+        L.wall_timing_enable_slots.argtypes = [ctypes.c_uint]
         L.wall_timing_read.restype = i
         L.wall_timing_read.argtypes = [i, ctypes.POINTER(ctypes.c_char_p),
                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]

@@ -300,6 +300,19 @@ def timing_enable(on=True):
     L._check("wall_timing_enable", L.lib().wall_timing_enable(1 if on else 0))
 
 
+TIMING_SLOTS = ("prefix_scan", "operands", "fwd_tc", "bwd_pre", "bwd_keyblock", "bwd_dq",
+                "bwd_finalize", "reverse_scan", "decode", "cache_build", "decode_step",
+                "decode_chunk")
+
+
+def timing_enable_slots(names):
+    """Times only the named stages (see TIMING_SLOTS); an empty list stops."""
+    mask = 0
+    for n in names:
+        mask |= 1 << TIMING_SLOTS.index(n)
+    L._check("wall_timing_enable_slots", L.lib().wall_timing_enable_slots(mask))
+
+
 def timing_read():
     """Per-stage {name: (launches, total_ms)} since the last read or enable;
     synchronizes on the recorded events and clears the totals."""

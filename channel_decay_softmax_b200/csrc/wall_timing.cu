@@ -19,7 +19,7 @@ struct Slot {
   int used = 0;                 // events recorded since the last read
 };
 
-bool g_on = false;
+unsigned g_mask = 0;  // timed slots
 Slot g_slot[WALL_TIMING_SLOTS];
 const char* const kNames[WALL_TIMING_SLOTS] = {
     "prefix_scan", "operands", "fwd_tc", "bwd_pre", "bwd_keyblock",
@@ -29,7 +29,7 @@ const char* const kNames[WALL_TIMING_SLOTS] = {
 }  // namespace
 
 void timing_mark(int slot, cudaStream_t stream) {
-  if (!g_on || slot < 0 || slot >= WALL_TIMING_SLOTS) return;
+  if (slot < 0 || slot >= WALL_TIMING_SLOTS || !((g_mask >> slot) & 1u)) return;
   Slot& s = g_slot[slot];
   if (s.used == (int)s.ev.size()) {
     cudaEvent_t e;
@@ -43,7 +43,15 @@ void timing_mark(int slot, cudaStream_t stream) {
 
 extern "C" int wall_timing_enable(int on) {
   using namespace wall;
-  g_on = on != 0;
+  g_mask = on != 0 ? (1u << WALL_TIMING_SLOTS) - 1u : 0u;
+  for (auto& s : g_slot) s.used = 0;
+  return WALL_OK;
+}
+
+extern "C" int wall_timing_enable_slots(unsigned mask) {
+  using namespace wall;
+  if (mask >> WALL_TIMING_SLOTS) return WALL_ERR_INVALID_ARG;
+  g_mask = mask;
   for (auto& s : g_slot) s.used = 0;
   return WALL_OK;
 }

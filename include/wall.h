@@ -376,6 +376,14 @@ int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
 int wall_timing_enable(int on);
 
 /*
+ * wall_timing_enable_slots -- as wall_timing_enable, for the slots whose bit
+ * is set in `mask` only (bit i = slot i; 0 stops timing), so a measurement
+ * can time one stage without recording events around all the others.
+ * Returns WALL_ERR_INVALID_ARG for bits past WALL_TIMING_SLOTS.
+ */
+int wall_timing_enable_slots(unsigned mask);
+
+/*
  * wall_timing_read -- for slots [0, n) (n <= WALL_TIMING_SLOTS) writes the
  * number of timed launches since the last read (or enable) and their total
  * device time in milliseconds, then clears them.  Synchronizes on the

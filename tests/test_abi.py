@@ -187,6 +187,14 @@ def test_fwd_gate_workspace_and_checks(lib):
     assert call(dtype=7) == L.WALL_ERR_INVALID_ARG
 
 
+def test_timing_slot_mask(lib):
+    # host-only: the mask selects slots; bits past the slot count are refused
+    assert lib.wall_timing_enable_slots(1 << 4) == L.WALL_OK
+    assert lib.wall_timing_enable_slots(1 << 12) == L.WALL_ERR_INVALID_ARG
+    assert lib.wall_timing_enable_slots(0) == L.WALL_OK
+    assert lib.wall_timing_enable(0) == L.WALL_OK
+
+
 def test_prefix_rejects_bad_arguments(lib):
     pc = lib.wall_prefix_cumsum
     assert pc(FAKE, 3, FAKE, 1, 8, 4, 64, None, 0, None, None, None) == L.WALL_ERR_INVALID_ARG
