@@ -455,33 +455,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and the exponentials); HBM carries the dS tiles, L2 keeps Kh.
 //
 // CTA = 8 warps (256 threads):
-//   warp 0      TMA, lane 0: per tile the dS tile (two 64-query boxes of 128
-//               key rows), Kh_J and its block anchors (kDS stages)
+//   warp 0      TMA, lane 0: the dS ring (two 64-query boxes of 128 key rows
+//               per tile, 4 stages, from HBM); lane 1: the key ring (Kh_J and
+//               its block anchors, 3 stages, mostly from L2).  The rings have
+//               barriers of their own, so the keys are scaled while the slower
+//               dS tiles are still in flight.
 //   warp 1      TMEM owner (128 columns) and MMA issuer: A = dS (queries x
 //               keys, MN-major: queries contiguous in the stored rows),
 //               B = Kt (keys x channels, MN-major)
 //   warps 2-5   Kt_J = Kh_J (.) d in place, as in the kernel above (four
 //               warps: with two, the in-place scaling set the tile rate)
 //   warps 4-7   epilogue: dQa rows -> fp32 workspace
-constexpr int kDS = 3;  // stages
+constexpr int kDSS = 4;  // dS stages
+constexpr int kKS3 = 3;  // key stages
 constexpr int kDsThreads = 256;
 
 template <int KD>
 struct QSmem {
-  static constexpr int kDsT = 128 * 128 * 2;  // one stored dS tile
-  static constexpr int kKT = BN * KD * 2;     // one Kh tile
-  static constexpr int oDS = 0;               // kDS stages
-  static constexpr int oK = oDS + kDS * kDsT;  // kDS stages
-  static constexpr int oRJ = oK + kDS * kKT;   // float[kDS][KD]
-  static constexpr int oBar = oRJ + kDS * KD * 4;
-  static constexpr int kBars = 3 * kDS + 2;
+  static constexpr int kDsT = 128 * 128 * 2;    // one stored dS tile
+  static constexpr int kKT = BN * KD * 2;       // one Kh tile
+  static constexpr int oDS = 0;                 // kDSS stages
+  static constexpr int oK = oDS + kDSS * kDsT;  // kKS3 stages
+  static constexpr int oRJ = oK + kKS3 * kKT;   // float[kKS3][KD]
+  static constexpr int oBar = oRJ + kKS3 * KD * 4;
+  static constexpr int kBars = 2 * kDSS + 3 * kKS3 + 2;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int kBytes = oMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KB alignment
 };
 static_assert(QSmem<128>::kAlloc <= 227 * 1024, "shared memory");
 
-enum QBar { QS_FULL = 0, QS_READY = kDS, QS_EMPTY = 2 * kDS, QS_DONE = 3 * kDS, QS_MMA = 3 * kDS + 1 };
+enum QBar {
+  D_FULL = 0,                     // + dS stage
+  D_EMPTY = kDSS,                 // + dS stage
+  K_FULL3 = 2 * kDSS,             // + key stage
+  K_READY3 = 2 * kDSS + kKS3,     // + key stage, 4 scaling warps
+  K_EMPTY3 = 2 * kDSS + 2 * kKS3,  // + key stage
+  QS_DONE = 2 * kDSS + 3 * kKS3,
+  QS_MMA = QS_DONE + 1,
+};
 
 template <int KD>
 __global__ void __launch_bounds__(kDsThreads, 1)
@@ -514,10 +526,14 @@ __global__ void __launch_bounds__(kDsThreads, 1)
       ((long)seq * HQ + h) * ((long)ds_nb * (ds_nb + 1) / 2) + (long)blk * (blk + 1) / 2;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDS; ++s) {
-      mbar_init(bar(QS_FULL + s), 1);
-      mbar_init(bar(QS_READY + s), 4);
-      mbar_init(bar(QS_EMPTY + s), 1);
+    for (int s = 0; s < kDSS; ++s) {
+      mbar_init(bar(D_FULL + s), 1);
+      mbar_init(bar(D_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kKS3; ++s) {
+      mbar_init(bar(K_FULL3 + s), 1);
+      mbar_init(bar(K_READY3 + s), 4);
+      mbar_init(bar(K_EMPTY3 + s), 1);
     }
     mbar_init(bar(QS_DONE), 1);
     mbar_init(bar(QS_MMA), 1);
@@ -536,36 +552,50 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
+      // the dS ring
       tma_prefetch_desc(&tm_ds);
-      tma_prefetch_desc(&tm_k);
       int issued = 0;
       for (int t = 0; t < nT; ++t) {
-        const int st = t % kDS;
-        if (t >= kDS && !wait_bar(bar(QS_EMPTY + st), (t / kDS - 1) & 1, p.status, abort_flag))
+        const int st = t % kDSS;
+        if (t >= kDSS && !wait_bar(bar(D_EMPTY + st), (t / kDSS - 1) & 1, p.status, abort_flag))
           break;
-        mbar_expect_tx(bar(QS_FULL + st), Lay::kDsT + Lay::kKT + K * 4);
+        mbar_expect_tx(bar(D_FULL + st), Lay::kDsT);
         const int drow = (int)((tile0 + t) * 128);
         for (int b = 0; b < 2; ++b)
           tma_load_2d(sbase + Lay::oDS + st * Lay::kDsT + b * (128 * 128), &tm_ds,
-                      bar(QS_FULL + st), b * 64, drow);
-        for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k, bar(QS_FULL + st),
-                      b * 64, h, (int)(s0 + (long)t * BN));
-        bulk_load(sbase + Lay::oRJ + st * K * 4, p.anchors + ((long)(blk_off + t) * HQ + h) * K,
-                  K * 4, bar(QS_FULL + st));
+                      bar(D_FULL + st), b * 64, drow);
         issued = t + 1;
       }
       // no copy may still be in flight when the CTA exits
-      for (int t = max(0, issued - kDS); t < issued; ++t)
-        mbar_wait(bar(QS_FULL + t % kDS), (t / kDS) & 1, p.status);
+      for (int t = max(0, issued - kDSS); t < issued; ++t)
+        mbar_wait(bar(D_FULL + t % kDSS), (t / kDSS) & 1, p.status);
+    } else if (lane == 1) {
+      // the key ring
+      tma_prefetch_desc(&tm_k);
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % kKS3;
+        if (t >= kKS3 && !wait_bar(bar(K_EMPTY3 + st), (t / kKS3 - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_expect_tx(bar(K_FULL3 + st), Lay::kKT + K * 4);
+        for (int b = 0; b < K / 64; ++b)
+          tma_load_3d(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k, bar(K_FULL3 + st),
+                      b * 64, h, (int)(s0 + (long)t * BN));
+        bulk_load(sbase + Lay::oRJ + st * K * 4, p.anchors + ((long)(blk_off + t) * HQ + h) * K,
+                  K * 4, bar(K_FULL3 + st));
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - kKS3); t < issued; ++t)
+        mbar_wait(bar(K_FULL3 + t % kKS3), (t / kKS3) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       const uint32_t id = idesc_bf16(BM, KD, true, true);
       for (int t = 0; t < nT; ++t) {
-        const int st = t % kDS;
-        if (!wait_bar(bar(QS_READY + st), (t / kDS) & 1, p.status, abort_flag)) break;
+        const int st = t % kDSS, kt = t % kKS3;
+        if (!wait_bar(bar(D_FULL + st), (t / kDSS) & 1, p.status, abort_flag)) break;
+        if (!wait_bar(bar(K_READY3 + kt), (t / kKS3) & 1, p.status, abort_flag)) break;
         tc_fence_after();
         // K = 16 keys per MMA: rows 16kk .. 16kk+15 of both operands; the two
         // 64-wide M (N) boxes of dS (Kt) are 128 rows x 128 B apart
@@ -574,10 +604,11 @@ __global__ void __launch_bounds__(kDsThreads, 1)
           umma_bf16_ss(tmem,
                        sdesc_sw128(sbase + Lay::oDS + st * Lay::kDsT + kk * 16 * 128, 128 * 128,
                                    1024),
-                       sdesc_sw128(sbase + Lay::oK + st * Lay::kKT + kk * 16 * 128, BN * 128,
+                       sdesc_sw128(sbase + Lay::oK + kt * Lay::kKT + kk * 16 * 128, BN * 128,
                                    1024),
                        id, (t > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(QS_EMPTY + st));
+        umma_commit(bar(D_EMPTY + st));
+        umma_commit(bar(K_EMPTY3 + kt));
       }
       umma_commit(bar(QS_DONE));
       umma_commit(bar(QS_MMA));
@@ -597,9 +628,9 @@ __global__ void __launch_bounds__(kDsThreads, 1)
       for (int e = 0; e < 8; ++e)
         ri[e] = __ldg(p.anchors + ((long)(blk_off + blk) * HQ + h) * K + ch * 8 + e);
       for (int t = 0; t < nT; ++t) {
-        const int st = t % kDS;
+        const int st = t % kKS3;
         {
-          const bool got = wait_bar(bar(QS_FULL + st), (t / kDS) & 1, p.status, abort_flag);
+          const bool got = wait_bar(bar(K_FULL3 + st), (t / kKS3) & 1, p.status, abort_flag);
           if (!__all_sync(0xffffffffu, got)) break;
         }
         const float* rj = reinterpret_cast<const float*>(smem + Lay::oRJ + st * K * 4) + ch * 8;
@@ -631,7 +662,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(QS_READY + st));
+        if (lane == 0) mbar_arrive(bar(K_READY3 + st));
       }
     }
     if (warp >= 4) {
