@@ -214,9 +214,48 @@ __global__ void __launch_bounds__(kThreadsScan)
   }
 }
 
+// VW consecutive elements as floats (VW = 4: 8 B of bf16 / 16 B of fp32).
+template <int VW>
+__device__ __forceinline__ void loadw(const __nv_bfloat16* p, float* out) {
+  if constexpr (VW == 8) {
+    load8(p, out);
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+  }
+}
+template <int VW>
+__device__ __forceinline__ void loadw(const float* p, float* out) {
+  if constexpr (VW == 8) {
+    load8(p, out);
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+  }
+}
+template <int VW>
+__device__ __forceinline__ void storew(__nv_bfloat16* p, const float* in) {
+  if constexpr (VW == 8) {
+    store8(p, in);
+  } else {
+    __nv_bfloat162 h[2] = {__floats2bfloat162_rn(in[0], in[1]), __floats2bfloat162_rn(in[2], in[3])};
+    *reinterpret_cast<uint2*>(p) = *reinterpret_cast<const uint2*>(h);
+  }
+}
+template <int VW>
+__device__ __forceinline__ void storew(float* p, const float* in) {
+  if constexpr (VW == 8) {
+    store8(p, in);
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(in[0], in[1], in[2], in[3]);
+  }
+}
+
 // pass 3 of the forward scan fused with the tensor-core forward's operand
 // preparation (the prefix enters the forward without an HBM round trip of
-// its own): per (sequence, chunk, 8 columns of one query head) the same
+// its own): per (sequence, chunk, VW columns of one query head) the same
 // compensated scan from the chunk's carry as chunk_scan_kernel, bit for bit,
 // writing P, and for each row
 //   Qh = q * 2^(P - R),  Kh = k * 2^(R - P),  R = floor(P at the row's
@@ -225,11 +264,14 @@ __global__ void __launch_bounds__(kThreadsScan)
 // lies in an earlier chunk is that row's prefix, rebuilt from its chunk's
 // carry: the scan's first step is carry + g, then one fused rounding.
 // The carries come from a scratch that is not P, so no thread reads a carry
-// another one has overwritten.
+// another one has overwritten.  A thread walks its chunk's rows in order, so
+// the walkers are latency-bound: 4 columns per thread instead of 8 doubles
+// the threads in flight here (0.048 -> 0.039 ms at T = 8192); the dL walker
+// below is faster with 8 (0.046 against 0.053 ms).
 constexpr int kInFlightOps = 8;
-// at most 128 registers: four CTAs per SM, so the 512 CTAs of the T = 8192
-// problem run in one wave (with 150 registers they needed 1.15 waves and
-// took 50 % longer)
+constexpr int kWalkOps = 4;
+constexpr int kWalkDl = 8;
+template <int VW>
 __global__ void __launch_bounds__(kThreadsScan, 4)
     chunk_scan_operands_kernel(const __nv_bfloat16* __restrict__ g,
                                const __nv_bfloat16* __restrict__ q,
@@ -255,49 +297,48 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
     s_blk_off = off;
   }
   __syncthreads();
-  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * 8;
+  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * VW;
   if (col >= C) return;
   const int n = (int)min((long)kChunk, len - lr0);
   const int hh = (int)(col / K), n0 = (int)(col % K);
   const int G = HQ / H;
   // R: the anchor of the 128-row block this chunk lies in
   const long lb = (lr0 / BA) * BA;
-  float R[8];
+  float R[VW];
   {
     const float* cb = scratch + chunk_row(start, len, (int)(lb / kChunk), false) * C + col;
-    float gb[8];
-    load8(g + (start + lb) * C + col, gb);
+    float gb[VW];
+    loadw<VW>(g + (start + lb) * C + col, gb);
 #pragma unroll
-    for (int v = 0; v < 8; ++v) R[v] = floorf(fmaf(kInvLn2, cb[v] + gb[v], 0.f));
+    for (int v = 0; v < VW; ++v) R[v] = floorf(fmaf(kInvLn2, cb[v] + gb[v], 0.f));
   }
-  float acc[8], cmp[8];
+  float acc[VW], cmp[VW];
   {
     const float* c = scratch + chunk_row(start, len, kc, false) * C + col;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
+    for (int v = 0; v < VW; ++v) {
       acc[v] = c[v];
       cmp[v] = 0.f;
     }
   }
 #pragma unroll
   for (int r0 = 0; r0 < kChunk; r0 += kInFlightOps) {
-    float a[kInFlightOps][8];
-    uint4 qa[kInFlightOps], ka[kInFlightOps];
+    float a[kInFlightOps][VW], qa[kInFlightOps][VW], ka[kInFlightOps][VW];
 #pragma unroll
     for (int r = 0; r < kInFlightOps; ++r) {
       const long pr = start + lr0 + (r0 + r < n ? r0 + r : 0);
-      load8(g + pr * C + col, a[r]);
-      qa[r] = *reinterpret_cast<const uint4*>(q + pr * C + col);
-      ka[r] = *reinterpret_cast<const uint4*>(k + (pr * H + hh / G) * K + n0);
+      loadw<VW>(g + pr * C + col, a[r]);
+      loadw<VW>(q + pr * C + col, qa[r]);
+      loadw<VW>(k + (pr * H + hh / G) * K + n0, ka[r]);
     }
 #pragma unroll
     for (int rr = 0; rr < kInFlightOps; ++rr) {
       const int r = r0 + rr;
       const long lr = lr0 + r;
       const long pr = start + lr;
-      float o[8];
+      float o[VW];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
+      for (int v = 0; v < VW; ++v) {
         const float yk = a[rr][v] - cmp[v];
         const float tk = acc[v] + yk;
         cmp[v] = (tk - acc[v]) - yk;
@@ -305,44 +346,31 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
         o[v] = fmaf(kInvLn2, acc[v], 0.f);
       }
       if (r < n) {
-        store8(P + pr * C + col, o);
-        float x[8], y[8];
-        const __nv_bfloat162* qv = reinterpret_cast<const __nv_bfloat162*>(&qa[rr]);
-        const __nv_bfloat162* kv = reinterpret_cast<const __nv_bfloat162*>(&ka[rr]);
+        storew<VW>(P + pr * C + col, o);
+        float y[VW];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float2 f = __bfloat1622float2(qv[v]);
-          x[2 * v] = f.x;
-          x[2 * v + 1] = f.y;
-        }
+        for (int v = 0; v < VW; ++v) y[v] = qa[rr][v] * exp2f(o[v] - R[v]);
+        storew<VW>(qh + pr * C + col, y);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) y[v] = x[v] * exp2f(o[v] - R[v]);
-        store8(qh + pr * C + col, y);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float2 f = __bfloat1622float2(kv[v]);
-          x[2 * v] = f.x;
-          x[2 * v + 1] = f.y;
-        }
-#pragma unroll
-        for (int v = 0; v < 8; ++v) y[v] = x[v] * exp2f(R[v] - o[v]);
-        store8(kh + pr * C + col, y);
+        for (int v = 0; v < VW; ++v) y[v] = ka[rr][v] * exp2f(R[v] - o[v]);
+        storew<VW>(kh + pr * C + col, y);
         if (lr == lb)
-          store8(anchors + ((long)(s_blk_off + lr / BA) * HQ + hh) * K + n0, R);
+          storew<VW>(anchors + ((long)(s_blk_off + lr / BA) * HQ + hh) * K + n0, R);
       }
     }
   }
 }
 
 // The backward's dq finalize fused with pass 1 of the reverse scan of dL
-// (tensor-core path): per (sequence, chunk in reverse order, 8 columns of one
-// query head), for each row
+// (tensor-core path): per (sequence, chunk in reverse order, VW columns of
+// one query head), for each row
 //   dq = scale * 2^(P - R_I) (.) dq32          R_I = floor(P at the row's
 //                                              128-row block start)
 //   dL = q (.) dq - k (.) dk^(h)               (fp32, written over dq32)
 // and the chunk's compensated sum of dL in the order chunk_sum_kernel adds
 // it, into the chunk row of `scratch` (dk^(h) itself: this thread has read
 // that row's dk^(h) by then, and no other thread reads this chunk's rows).
+template <int VW>
 __global__ void __launch_bounds__(kThreadsScan, 4)
     finalize_dl_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const float* __restrict__ P, float* __restrict__ dq32,
@@ -356,17 +384,17 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
   const long len = seqs.len(s);
   const long lr0 = (long)kc * kChunk;
   if (lr0 >= len) return;
-  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * 8;
+  const long col = ((long)blockIdx.y * kThreadsScan + threadIdx.x) * VW;
   if (col >= C) return;
   const int n = (int)min((long)kChunk, len - lr0);
   const int hh = (int)(col / K), n0 = (int)(col % K);
   const int G = HQ / H;
-  float sum[8], cmp[8];
+  float sum[VW], cmp[VW];
 #pragma unroll
-  for (int v = 0; v < 8; ++v) sum[v] = cmp[v] = 0.f;
+  for (int v = 0; v < VW; ++v) sum[v] = cmp[v] = 0.f;
 #pragma unroll 1
   for (int r0 = 0; r0 < kChunk; r0 += kInFlightOps) {
-    float dl[kInFlightOps][8];
+    float dl[kInFlightOps][VW];
 #pragma unroll
     for (int r = 0; r < kInFlightOps; ++r) {
       const bool in = r0 + r < n;
@@ -374,29 +402,29 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
       const long pr = start + len - 1 - lr;  // reverse scan order
       const long off = pr * C + col;
       const long arow = start + ((pr - start) / BA) * BA;
-      float pv[8], rv[8], a[8], qq[8], kk[8], dkv[8];
-      load8(P + off, pv);
-      load8(P + arow * C + col, rv);
-      load8(dq32 + off, a);
-      load8(q + off, qq);
-      load8(k + (pr * H + hh / G) * K + n0, kk);
-      load8(dkh32 + off, dkv);
-      float o[8];
+      float pv[VW], rv[VW], a[VW], qq[VW], kk[VW], dkv[VW];
+      loadw<VW>(P + off, pv);
+      loadw<VW>(P + arow * C + col, rv);
+      loadw<VW>(dq32 + off, a);
+      loadw<VW>(q + off, qq);
+      loadw<VW>(k + (pr * H + hh / G) * K + n0, kk);
+      loadw<VW>(dkh32 + off, dkv);
+      float o[VW];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
+      for (int v = 0; v < VW; ++v) {
         a[v] *= scale * exp2f(pv[v] - floorf(rv[v]));
         o[v] = qq[v] * a[v] - kk[v] * dkv[v];
         dl[r][v] = in ? o[v] : 0.f;
       }
       if (in) {
-        store8(dq + off, a);
-        store8(dq32 + off, o);
+        storew<VW>(dq + off, a);
+        storew<VW>(dq32 + off, o);
       }
     }
 #pragma unroll
     for (int r = 0; r < kInFlightOps; ++r) {
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
+      for (int v = 0; v < VW; ++v) {
         const float yk = dl[r][v] - cmp[v];
         const float tk = sum[v] + yk;
         cmp[v] = (tk - sum[v]) - yk;
@@ -406,7 +434,7 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
   }
   float* dst = scratch + chunk_row(start, len, kc, true) * C + col;
 #pragma unroll
-  for (int v = 0; v < 8; ++v) dst[v] = sum[v];
+  for (int v = 0; v < VW; ++v) dst[v] = sum[v];
 }
 
 template <typename Tin, typename Tout, bool kReverse, int VEC>
@@ -462,9 +490,10 @@ int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const _
   if (seqs.n == 0 || C == 0) return WALL_OK;
   if (C % 8 != 0) return WALL_ERR_UNSUPPORTED;
   const long groups = (C / 8 + kThreadsScan - 1) / kThreadsScan;
+  const long wgroups = (C / kWalkOps + kThreadsScan - 1) / kThreadsScan;
   const long chunks = seqs.cu ? (seqs.rows + kChunk - 1) / kChunk + seqs.n
                               : (long)seqs.n * ((seqs.T + kChunk - 1) / kChunk);
-  if (groups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  if (wgroups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
   if (chunks == 0) return WALL_OK;
   const dim3 grid((unsigned)chunks, (unsigned)groups);
   timing_mark(T_PREFIX, stream);
@@ -474,8 +503,9 @@ int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const _
                                                               nullptr);
   timing_mark(T_PREFIX, stream);
   timing_mark(T_OPERANDS, stream);
-  chunk_scan_operands_kernel<<<grid, kThreadsScan, 0, stream>>>(g, q, k, scratch, P, C, seqs, HQ,
-                                                                H, K, qh, kh, anchors);
+  chunk_scan_operands_kernel<kWalkOps>
+      <<<dim3((unsigned)chunks, (unsigned)wgroups), kThreadsScan, 0, stream>>>(
+          g, q, k, scratch, P, C, seqs, HQ, H, K, qh, kh, anchors);
   timing_mark(T_OPERANDS, stream);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
@@ -486,13 +516,14 @@ int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const fl
   const long C = (long)HQ * K;
   if (seqs.n == 0 || C == 0) return WALL_OK;
   if (C % 8 != 0) return WALL_ERR_UNSUPPORTED;
-  const long groups = (C / 8 + kThreadsScan - 1) / kThreadsScan;
+  const long wgroups = (C / kWalkDl + kThreadsScan - 1) / kThreadsScan;
   const long chunks = seqs.cu ? (seqs.rows + kChunk - 1) / kChunk + seqs.n
                               : (long)seqs.n * ((seqs.T + kChunk - 1) / kChunk);
-  if (groups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
+  if (wgroups > 65535 || chunks > 0x7fffffffL || seqs.n > 65535) return WALL_ERR_UNSUPPORTED;
   if (chunks == 0) return WALL_OK;
-  finalize_dl_kernel<<<dim3((unsigned)chunks, (unsigned)groups), kThreadsScan, 0, stream>>>(
-      q, k, P, dq32, dkh32, dkh32, dq, C, seqs, HQ, H, K, scale);
+  finalize_dl_kernel<kWalkDl>
+      <<<dim3((unsigned)chunks, (unsigned)wgroups), kThreadsScan, 0, stream>>>(
+          q, k, P, dq32, dkh32, dkh32, dq, C, seqs, HQ, H, K, scale);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

@@ -182,6 +182,9 @@ def test_empty_and_single_row():
         s = I.spec(2, T=T, B=1)
         x = _to(I.training_inputs(s))
         P, o, lse, grads = _run_gpu(x)
+        # the fused prefix forward (autograd path) on the same rows
+        og, lg, Pg = api.wall_attn_fwd_gate(x["q"], x["k"], x["v"], x["g"], x["scale"])
+        assert torch.equal(og, o) and torch.equal(Pg, P)
         assert o.shape == (1, T, s.HQ, s.V)
         if T == 1:
             # one visible key: o = v of the same row, dq = dk = dg = 0
@@ -227,7 +230,7 @@ def test_dq_from_stored_ds_matches_recompute(K):
         assert e < 1e-2, (name, e)
 
 
-@pytest.mark.parametrize("case", ["cfg2", "cfg4_reduced", "fp32_options"])
+@pytest.mark.parametrize("case", ["cfg2", "cfg4_reduced", "fp32_options", "varlen_ragged"])
 def test_fwd_gate_equals_prefix_then_forward(case):
     """wall_attn_fwd_gate fuses the prefix scan into the forward's operand
     pass: P must be bit for bit wall_prefix_cumsum's, o and lse bit for bit
@@ -237,10 +240,15 @@ def test_fwd_gate_equals_prefix_then_forward(case):
         s = I.spec(2)
     elif case == "cfg4_reduced":
         s = I.spec(4, len_lo=64, len_hi=600, window=128)
-    else:
+    elif case == "fp32_options":
         s = I.spec(4, dtype=torch.float32, K=64, V=64, HQ=4, H=2, window=100, len_lo=1,
                    len_hi=300)
-    x = _to(I.training_inputs(s))
+    else:
+        # empty and one-row sequences, chunk (32) and anchor-block (128)
+        # boundaries falling inside sequences
+        s = I.spec(4, K=64, V=64, HQ=4, H=2, n_seq=6, g_scalar=False, sink=False, window=0)
+    lengths = [0, 1, 33, 0, 130, 257] if case == "varlen_ragged" else None
+    x = _to(I.training_inputs(s, lengths=lengths))
     q, k, v, g, cu = x["q"], x["k"], x["v"], x["g"], x["cu_seqlens"]
     kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=x["window_size"],
               cu_seqlens=cu)
