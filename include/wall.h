@@ -145,7 +145,12 @@ int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* 
                        const int32_t* cu_seqlens, int n_seq, float* P, void* o, float* lse,
                        void* workspace, size_t workspace_bytes, wall_stream_t stream);
 
-/* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs. */
+/* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs.  For
+ * dense batches (n_seq == 0) on the bf16 tensor-core path it includes room
+ * for every dS tile of the causal problem, bf16 128 x 128 per (batch row,
+ * head, query block I, key block J <= I), B*HQ*nb(nb+1)/2 * 32 KB with
+ * nb = ceil(T/128), when that is at most 8 GiB (1.09 GB at B=1, T=8192,
+ * HQ=16); the dq pass then reads those tiles instead of recomputing them. */
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                int has_g_scalar, int n_seq);
 
@@ -161,9 +166,9 @@ size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, in
  * per query head, dL_t = q_t (.) dq_t - k_t (.) dk^(h)_t with the key-side
  * term -K_j (.) dK_j, then dg = the reverse cumulative sum of dL within each
  * sequence.  dk^(h), dv^(h) are summed over each GQA group.
- * fwd_workspace: NULL, or the workspace of the wall_attn_fwd call that
- * produced o and lse, with the same q, k, P, shapes and options and left
- * unchanged since.  On the bf16 tensor-core path the anchored operands that
+ * fwd_workspace: NULL, or the workspace of the wall_attn_fwd (or
+ * wall_attn_fwd_gate) call that produced o and lse, with the same q, k, P,
+ * shapes and options and left unchanged since.  On the bf16 tensor-core path the anchored operands that
  * call prepared in it are then read instead of recomputed; it is only read.
  * Elsewhere it is ignored.
  */
