@@ -106,22 +106,27 @@ struct BSmem {
 };
 static_assert(BSmem<128>::kAlloc <= 227 * 1024, "shared memory");
 
+// barrier slots, laid out from the query-stage count
+constexpr int kQStages = BSmem<128>::kStages;
+static_assert(BSmem<64>::kStages == kQStages, "one query-stage count");
 enum BBar {
   KV_FULL = 0,
-  Q_FULL = 1,     // +stage (3), TMA
-  Q_READY = 4,    // +stage (3), 2 producer warps
-  Q_EMPTY = 7,    // +stage (3), tcgen05.commit after dK(t)
-  O_FULL = 10,    // TMA
-  O_EMPTY = 11,   // tcgen05.commit after dV(t)
-  S_FULL = 12,
-  DP_FULL = 13,
-  P_READY = 14,   // 8 softmax warps
-  DS_READY = 15,  // 8 softmax warps
-  MM_DONE = 16,
-  MMA_DONE = 17,
-  COL_READY = 18,  // 4 warps of the second half: column sums in shared memory
-  EPI_STAGED = 19, // 8 softmax warps: dK, dV staged in shared memory
+  Q_FULL = 1,                       // + stage, TMA
+  Q_READY = Q_FULL + kQStages,      // + stage, 2 producer warps
+  Q_EMPTY = Q_READY + kQStages,     // + stage, tcgen05.commit after dK(t)
+  O_FULL = Q_EMPTY + kQStages,      // TMA
+  O_EMPTY = O_FULL + 1,             // tcgen05.commit after dV(t)
+  S_FULL = O_EMPTY + 1,
+  DP_FULL = S_FULL + 1,
+  P_READY = DP_FULL + 1,            // 8 softmax warps
+  DS_READY = P_READY + 1,           // 8 softmax warps
+  MM_DONE = DS_READY + 1,
+  MMA_DONE = MM_DONE + 1,
+  COL_READY = MMA_DONE + 1,         // 4 warps of the second half: column sums in shared memory
+  EPI_STAGED = COL_READY + 1,       // 8 softmax warps: dK, dV staged in shared memory
+  kNumBBars = EPI_STAGED + 1,
 };
+static_assert(kNumBBars <= BSmem<128>::kBars, "barrier slots");
 
 // TMEM columns (lanes = keys): S^T [0,128), dP^T [128,256), dV [256,384),
 // dK [384,512).  The softmax half h (queries 64h..64h+63) writes its P^T

@@ -97,19 +97,23 @@ struct Smem {
   static constexpr int kAlloc = kBytes + 1024;    // slack for 1 KB alignment
 };
 
+// barrier slots, laid out from the stage counts (so a change of kKS or kVS
+// cannot make two barriers share a slot)
 enum Bar {
   B_QFULL = 0,
-  B_KFULL = 1,    // +stage (3)
-  B_KREADY = 4,   // +stage (3), 2 rescale warps
-  B_KEMPTY = 7,   // +stage (3)
-  B_VFULL = 10,   // +stage (2)
-  B_VEMPTY = 12,  // +stage (2)
-  B_SFULL = 14,   // +S buffer (2)
-  B_PFULL = 16,   // +group (2), 4 warps each
-  B_PVDONE = 18,  // +group (2): O_group holds every PV issued so far
-  B_XCHG = 20,    // epilogue exchange of m, l between the groups (8 warps)
-  B_MMADONE = 21,
+  B_KFULL = 1,                  // + key stage
+  B_KREADY = B_KFULL + kKS,     // + key stage, 2 rescale warps
+  B_KEMPTY = B_KREADY + kKS,    // + key stage
+  B_VFULL = B_KEMPTY + kKS,     // + value stage
+  B_VEMPTY = B_VFULL + kVS,     // + value stage
+  B_SFULL = B_VEMPTY + kVS,     // + S buffer (2)
+  B_PFULL = B_SFULL + 2,        // + group (2), 4 warps each
+  B_PVDONE = B_PFULL + 2,       // + group (2): O_group holds every PV issued so far
+  B_XCHG = B_PVDONE + 2,        // epilogue exchange of m, l between the groups (8 warps)
+  B_MMADONE = B_XCHG + 1,
+  kNumBars = B_MMADONE + 1,
 };
+static_assert(kNumBars <= Smem<128, false>::kBars, "barrier slots");
 
 // bounded wait that also gives up once another role has given up
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* status,
