@@ -220,6 +220,13 @@ def test_workspace_sizes(lib):
     nb = (T + 127) // 128
     ds = al(B * HQ * nb * (nb + 1) // 2 * 128 * 128 * 2)
     assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc + ds
+    # beyond 8 GiB of tiles (B=1, T=65536, HQ=16: 68.9 GB) none are kept
+    Tb = 65536
+    big = lib.wall_attn_bwd_workspace(0, 1, Tb, 4, HQ * 2, K, V, 0, 0)
+    simtb = al(4 * Tb * HQ * 2) + 2 * al(4 * Tb * HQ * 2 * K) + al(4 * Tb * HQ * 2 * V) + \
+        2 * al(4 * Tb * HQ * 2)
+    tcb = 2 * al(2 * Tb * HQ * 2 * K) + al(4 * (Tb // 128) * HQ * 2 * K)
+    assert big == simtb + tcb
     # varlen packing (B == 1, n_seq > 0): no stored tiles, dq recomputes them
     simt1 = al(4 * T * HQ) + 2 * al(4 * T * HQ * K) + al(4 * T * HQ * V) + 2 * al(4 * T * HQ)
     tc1 = 2 * al(2 * T * HQ * K) + al(4 * ((T + 127) // 128 + 3) * HQ * K)
