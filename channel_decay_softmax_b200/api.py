@@ -317,7 +317,7 @@ def timing_read():
     """Per-stage {name: (launches, total_ms)} since the last read or enable;
     synchronizes on the recorded events and clears the totals."""
     import ctypes
-    n = 12
+    n = len(TIMING_SLOTS)
     names = (ctypes.c_char_p * n)()
     launches = (ctypes.c_int * n)()
     ms = (ctypes.c_double * n)()
