@@ -32,7 +32,9 @@
  *   - Pointers are device pointers, 16-byte aligned.  The caller allocates
  *     and owns every buffer, including workspaces whose sizes the *_workspace
  *     calls return; the library allocates no device memory and keeps no
- *     state between calls except one device status word (wall_get_status).
+ *     state between calls except one device status word (wall_get_status),
+ *     the fixed scratch array of wall_attn_decode_noalloc and the events of
+ *     the per-stage timing aid.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  Arguments are checked on the host before any launch;
  *     on a bad argument nothing is launched and the call returns an error.
