@@ -538,6 +538,59 @@ def workload_name():
             f"g=-0.05|N| (prefix scan + forward + backward incl. dg)")
 
 
+def assemble_line(args, world, tr, dec, peaks):
+    """The JSON line of our arm (without the cpu_baseline leg): headline,
+    per-stage table, the dominant kernel's roofline, clocks, e2e, decode.
+    `tr["stages"]` maps stage names to (launches, total ms) as
+    api.timing_read returns them."""
+    # per-stage device time from the library's events; the dominant stage's
+    # roofline uses its algorithmic FLOPs per launch over its average launch
+    # time (timed inside the timed region), against the sustained bf16 peak
+    # since it runs inside a long step
+    peak = peaks["bf16_tflops_sustained"]
+    stage_rows = {}
+    for name, (n, ms) in tr["stages"].items():
+        if n == 0:
+            continue
+        row = {"launches": n, "ms_per_launch": ms / n}
+        if name in STAGE_FWD_MULT:
+            fl = STAGE_FWD_MULT[name] * tr["fwd_flops"]
+            row["algorithmic_tflop"] = fl / 1e12
+            row["tflops"] = fl / (ms / n * 1e-3) / 1e12
+        stage_rows[name] = row
+    dom = ROOF_STAGE
+    d = stage_rows[dom]
+    roof = {"kernel": "bwd_tc_kernel (key-block dK, dV; also stores the dS tiles)",
+            "bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
+            "frac": d["tflops"] / peak,
+            "traffic": BWD_KEY_TRAFFIC_BYTES if dom == "bwd_keyblock" else None,
+            "peak_source": f"bf16_tflops_sustained of {peaks['source']} peaks",
+            "ms_per_launch": d["ms_per_launch"],
+            "timed": "CUDA events around this kernel only, on its launch stream, over the "
+                     "timed region",
+            "algorithmic": "%.3g FLOP per launch = %g x the forward's 2*N*(K+V) summed "
+                           "over (b,h)" % (d["algorithmic_tflop"] * 1e12, STAGE_FWD_MULT[dom])}
+    line = {"metric": METRIC, "value": tr["value"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tr["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_name(),
+                       "l2": "per-step working set ~0.45 GB > 126 MB L2 (no flush)",
+                       "parallelism": f"replicas x{world}"},
+            "frac_bf16_peak": tr["value"] / world / peaks["bf16_tflops_sustained"],
+            "fwd_tflops": tr["fwd_tflops"], "bwd_tflops": tr["bwd_tflops"],
+            "roofline": roof, "stages": stage_rows, "gpu_launches": tr["launches"],
+            "peaks": {k: peaks[k] for k in ("hbm_gbs", "bf16_tflops",
+                                             "bf16_tflops_sustained", "source")}}
+    if tr.get("clocks"):
+        line["clocks"] = tr["clocks"]
+    if "e2e" in tr:
+        line["e2e"] = tr["e2e"]
+    if dec is not None:
+        line["decode"] = dec
+    return line
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -568,53 +621,7 @@ def main(argv=None):
         dec = bench_decode(args, rank, peaks)
     barrier(world)
     if rank == 0:
-        s = tr["spec"]
-        # per-stage device time from the library's events over the timed
-        # steps; the dominant stage's roofline uses its algorithmic FLOPs per
-        # launch over its average launch time, against the sustained bf16
-        # peak since it runs inside a long step
-        peak = peaks["bf16_tflops_sustained"]
-        stage_rows = {}
-        for name, (n, ms) in tr["stages"].items():
-            if n == 0:
-                continue
-            row = {"launches": n, "ms_per_launch": ms / n}
-            if name in STAGE_FWD_MULT:
-                fl = STAGE_FWD_MULT[name] * tr["fwd_flops"]
-                row["algorithmic_tflop"] = fl / 1e12
-                row["tflops"] = fl / (ms / n * 1e-3) / 1e12
-            stage_rows[name] = row
-        dom = ROOF_STAGE
-        d = stage_rows[dom]
-        roof = {"kernel": "bwd_tc_kernel (key-block dK, dV; also stores the dS tiles)",
-                "bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
-                "frac": d["tflops"] / peak,
-                "traffic": BWD_KEY_TRAFFIC_BYTES if dom == "bwd_keyblock" else None,
-                "peak_source": f"bf16_tflops_sustained of {peaks['source']} peaks",
-                "ms_per_launch": d["ms_per_launch"],
-                "timed": "CUDA events around this kernel only, on its launch stream, over the "
-                         "timed region",
-                "algorithmic": "%.3g FLOP per launch = %g x the forward's 2*N*(K+V) summed "
-                               "over (b,h)" % (d["algorithmic_tflop"] * 1e12,
-                                               STAGE_FWD_MULT[dom])}
-        line = {"metric": METRIC, "value": tr["value"], "unit": "TFLOP/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": tr["ms"],
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": workload_name(),
-                           "l2": "per-step working set ~0.45 GB > 126 MB L2 (no flush)",
-                           "parallelism": f"replicas x{world}"},
-                "frac_bf16_peak": tr["value"] / world / peaks["bf16_tflops_sustained"],
-                "fwd_tflops": tr["fwd_tflops"], "bwd_tflops": tr["bwd_tflops"],
-                "roofline": roof, "stages": stage_rows, "gpu_launches": tr["launches"],
-                "peaks": {k: peaks[k] for k in ("hbm_gbs", "bf16_tflops",
-                                                 "bf16_tflops_sustained", "source")}}
-        if tr.get("clocks"):
-            line["clocks"] = tr["clocks"]
-        if "e2e" in tr:
-            line["e2e"] = tr["e2e"]
-        if dec is not None:
-            line["decode"] = dec
+        line = assemble_line(args, world, tr, dec, peaks)
         if world == 1 and not args.no_cpu:
             # about 10-15 s of host work (the cost grows with the square of
             # the sampled rows)
