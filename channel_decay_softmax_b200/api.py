@@ -31,7 +31,66 @@ def _n_seq(cu_seqlens, B):
         raise ValueError("cu_seqlens requires B == 1")
     if cu_seqlens.dtype != torch.int32:
         raise ValueError("cu_seqlens must be int32")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be 1-D [n_seq + 1]")
     return cu_seqlens.numel() - 1
+
+
+# The library receives bare pointers and sizes: a tensor of the wrong dtype
+# or shape would make a kernel read or write past its buffer.  These checks
+# run before any call into the library.
+
+def _io_dtype(q, *others):
+    """q's dtype (bf16 or fp32), shared by every tensor in ``others``."""
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"unsupported dtype {q.dtype}; use bfloat16 or float32")
+    for t in others:
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError(f"inputs must share one dtype: {q.dtype} and {t.dtype}")
+    return q.dtype
+
+
+def _expect(name, t, shape, dtype=None):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _opt_f32(name, t, shape):
+    """An optional fp32 argument (g_scalar, sink_bias): shape-checked, then
+    made contiguous fp32."""
+    if t is None:
+        return None
+    _expect(name, t, shape)
+    return t.contiguous().float()
+
+
+def _same_device(ref, *ts):
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"all tensors must be on {ref.device}, got one on {t.device}")
+
+
+def _check_cache(q, v, p, k_tilde, r_cache, C, T_kv, Tq):
+    """Shapes of a decode call against the cache: q and p [B,Tq,HQ,K],
+    v [B,Tcap,H,V], r_cache [B,ceil(Tcap/C),HQ,K] fp32, 1 <= Tq <= T_kv <= Tcap."""
+    if k_tilde.dim() != 4 or v.dim() != 4:
+        raise ValueError("k_tilde must be [B,Tcap,HQ,K] and v [B,Tcap,H,V]")
+    B, Tcap, HQ, K = k_tilde.shape
+    _io_dtype(k_tilde, q, v)
+    if v.shape[0] != B or v.shape[1] != Tcap or HQ % v.shape[2] != 0:
+        raise ValueError("v must be [B,Tcap,H,V] with the cache's B, Tcap and HQ % H == 0")
+    if C < 1:
+        raise ValueError("cache_chunk_size must be positive")
+    if not 1 <= Tq <= T_kv <= Tcap:
+        raise ValueError(f"need 1 <= Tq ({Tq}) <= T_kv ({T_kv}) <= capacity ({Tcap})")
+    _expect("q", q, (B, Tq, HQ, K))
+    _expect("p", p, (B, Tq, HQ, K), torch.float32)
+    _expect("r_cache", r_cache, (B, -(-Tcap // C), HQ, K), torch.float32)
+    _same_device(k_tilde, q, v, p, r_cache)
 
 
 def _ws(nbytes, device):
@@ -41,14 +100,18 @@ def _ws(nbytes, device):
 def prefix_cumsum(g, cu_seqlens=None, carry_in=None, return_carry=False):
     """P = cumsum_t(g) / ln 2 per sequence (fp32), with an optional carried-in
     prefix [n_seq or B, HQ, K]; README "Decode" builds P this way."""
+    if g.dim() != 4:
+        raise ValueError("g must be [B, T, HQ, K]")
+    _io_dtype(g)
     g = g.contiguous()
     B, T, HQ, K = g.shape
-    P = torch.empty(g.shape, dtype=torch.float32, device=g.device)
     nseq = _n_seq(cu_seqlens, B)
     ns = nseq if cu_seqlens is not None else B
+    cin = _opt_f32("carry_in", carry_in, (ns, HQ, K))
+    _same_device(g, cu_seqlens, cin)
+    P = torch.empty(g.shape, dtype=torch.float32, device=g.device)
     carry_out = torch.empty((ns, HQ, K), dtype=torch.float32, device=g.device) \
         if return_carry else None
-    cin = carry_in.contiguous().float() if carry_in is not None else None
     L.wall_prefix_cumsum(g, P, B, T, HQ, K, cu_seqlens, nseq, cin, carry_out)
     return (P, carry_out) if return_carry else P
 
@@ -60,6 +123,11 @@ def wall_attn_fwd(q, k, v, P, scale=None, g_scalar=None, sink_bias=None, window_
     operands, which wall_attn_bwd can reuse (its fwd_workspace)."""
     B, T, H, HQ, K, V = _shape_checks(q, k, v, P)
     nseq = _n_seq(cu_seqlens, B)
+    _io_dtype(q, k, v)
+    _expect("P", P, q.shape, torch.float32)
+    g_scalar = _opt_f32("g_scalar", g_scalar, (B, T, HQ))
+    sink_bias = _opt_f32("sink_bias", sink_bias, (HQ,))
+    _same_device(q, k, v, P, g_scalar, sink_bias, cu_seqlens)
     o = torch.empty((B, T, HQ, V), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, T, HQ), dtype=torch.float32, device=q.device)
     ws = _ws(L.wall_attn_fwd_workspace(q.dtype, B, T, H, HQ, K, V, g_scalar is not None, nseq),
@@ -79,6 +147,10 @@ def wall_attn_fwd_gate(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, wi
     g = g.contiguous()
     B, T, H, HQ, K, V = _shape_checks(q, k, v, g)
     nseq = _n_seq(cu_seqlens, B)
+    _io_dtype(q, k, v, g)
+    g_scalar = _opt_f32("g_scalar", g_scalar, (B, T, HQ))
+    sink_bias = _opt_f32("sink_bias", sink_bias, (HQ,))
+    _same_device(q, k, v, g, g_scalar, sink_bias, cu_seqlens)
     o = torch.empty((B, T, HQ, V), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, T, HQ), dtype=torch.float32, device=q.device)
     P = torch.empty((B, T, HQ, K), dtype=torch.float32, device=q.device)
@@ -96,6 +168,22 @@ def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=N
     for the same inputs, whose anchored operands are then reused."""
     B, T, H, HQ, K, V = _shape_checks(q, k, v, P)
     nseq = _n_seq(cu_seqlens, B)
+    _io_dtype(q, k, v, dO, o)
+    _expect("P", P, q.shape, torch.float32)
+    _expect("dO", dO, (B, T, HQ, V))
+    _expect("o", o, (B, T, HQ, V))
+    _expect("lse", lse, (B, T, HQ), torch.float32)
+    g_scalar = _opt_f32("g_scalar", g_scalar, (B, T, HQ))
+    sink_bias = _opt_f32("sink_bias", sink_bias, (HQ,))
+    _same_device(q, k, v, P, dO, o, lse, g_scalar, sink_bias, cu_seqlens, fwd_workspace)
+    if fwd_workspace is not None:
+        # the forward's operands are read from it: it must hold at least the
+        # forward workspace of this problem
+        need = L.wall_attn_fwd_workspace(q.dtype, B, T, H, HQ, K, V, g_scalar is not None, nseq)
+        have = fwd_workspace.numel() * fwd_workspace.element_size()
+        if not fwd_workspace.is_contiguous() or have < need:
+            raise ValueError(f"fwd_workspace holds {have} bytes; this problem's forward "
+                             f"workspace needs {need}")
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
@@ -151,12 +239,21 @@ def wall_attn(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size
 def build_wall_kv_cache(k, P, chunk_size=64, capacity=None, HQ=None):
     """Pre-rescaled decode cache (README "Decode"): k_tilde [B,Tcap,HQ,K] in
     k's dtype and r_cache [B,ceil(Tcap/C),HQ,K] fp32, Tcap = capacity or T."""
+    if k.dim() != 4 or P.dim() != 4:
+        raise ValueError("k must be [B,T,H,K] and P [B,T,HQ,K]")
+    _io_dtype(k)
     k = k.contiguous()
     P = P.contiguous()
     B, T, H, K = k.shape
     HQ = P.shape[2]
+    _expect("P", P, (B, T, HQ, K), torch.float32)
+    if HQ % H != 0:
+        raise ValueError("HQ must be a multiple of H")
+    _same_device(k, P)
     Tcap = capacity or T
     C = int(chunk_size)
+    if Tcap < T or C < 1:
+        raise ValueError("need capacity >= T and chunk_size >= 1")
     k_tilde = torch.empty((B, Tcap, HQ, K), dtype=k.dtype, device=k.device)
     r_cache = torch.empty((B, -(-Tcap // C), HQ, K), dtype=torch.float32, device=k.device)
     L.wall_build_kv_cache(k, P, B, T, H, HQ, K, C, 0, k_tilde, r_cache, Tcap)
@@ -167,16 +264,16 @@ def wall_attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias=None, scale=None,
                      cache_chunk_size=64, T_kv=None):
     """One decode step (README "Decode"); returns (o [B,1,HQ,V], lse
     [B,1,HQ]).  The first T_kv cache positions are read (default: all)."""
+    C = int(cache_chunk_size)
+    T_kv = k_tilde.shape[1] if T_kv is None else int(T_kv)
+    _check_cache(q, v, p_curr, k_tilde, r_cache, C, T_kv, 1)
     B, Tcap, HQ, K = k_tilde.shape
     H, V = v.shape[2], v.shape[3]
-    T_kv = Tcap if T_kv is None else int(T_kv)
-    if v.shape[1] != Tcap:
-        raise ValueError("v and k_tilde must have the same capacity")
+    sk = _opt_f32("sink_bias", sink_bias, (HQ,))
+    _same_device(k_tilde, sk)
     o = torch.empty((B, 1, HQ, V), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, 1, HQ), dtype=torch.float32, device=q.device)
-    C = int(cache_chunk_size)
     ws = _ws(L.wall_attn_decode_workspace(B, T_kv, H, HQ, V, C), q.device)
-    sk = sink_bias.contiguous().float() if sink_bias is not None else None
     L.wall_attn_decode(q.contiguous(), v, p_curr.contiguous(), k_tilde, r_cache, sk, scale or 0.0,
                        C, B, T_kv, Tcap, H, HQ, K, V, o, lse, ws)
     return o, lse
@@ -189,18 +286,20 @@ def wall_attn_decode_chunk(q, v, p, k_tilde, r_cache, sink_bias=None, scale=None
     the last Tq of the first T_kv cached positions (default: all), each
     attending causally to the cache up to its own position.  Returns
     (o [B,Tq,HQ,V], lse [B,Tq,HQ])."""
+    C = int(cache_chunk_size)
+    T_kv = k_tilde.shape[1] if T_kv is None else int(T_kv)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, Tq, HQ, K]")
+    Tq = q.shape[1]
+    _check_cache(q, v, p, k_tilde, r_cache, C, T_kv, Tq)
     B, Tcap, HQ, K = k_tilde.shape
     H, V = v.shape[2], v.shape[3]
-    Tq = q.shape[1]
-    T_kv = Tcap if T_kv is None else int(T_kv)
-    if v.shape[1] != Tcap:
-        raise ValueError("v and k_tilde must have the same capacity")
+    sk = _opt_f32("sink_bias", sink_bias, (HQ,))
+    _same_device(k_tilde, sk)
     o = torch.empty((B, Tq, HQ, V), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, Tq, HQ), dtype=torch.float32, device=q.device)
-    C = int(cache_chunk_size)
     ws = _ws(L.wall_attn_decode_chunk_workspace(L.dtype_code(q.dtype), B, Tq, T_kv, H, HQ, K, V,
                                                 C), q.device)
-    sk = sink_bias.contiguous().float() if sink_bias is not None else None
     L.wall_attn_decode_chunk(q.contiguous(), v, p.contiguous(), k_tilde, r_cache, sk,
                              scale or 0.0, C, B, Tq, T_kv, Tcap, H, HQ, K, V, o, lse, ws)
     return o, lse
@@ -220,6 +319,8 @@ class WallDecodeCache:
 
     def __init__(self, B, H, HQ, K, V, capacity, chunk_size=64, dtype=torch.bfloat16,
                  device="cuda", scale=None, sink_bias=None):
+        if HQ % H != 0 or capacity < 1 or chunk_size < 1:
+            raise ValueError("need HQ % H == 0, capacity >= 1 and chunk_size >= 1")
         self.B, self.H, self.HQ, self.K, self.V = B, H, HQ, K, V
         self.cap, self.C, self.scale, self.dtype = capacity, chunk_size, scale, dtype
         self.k_tilde = torch.empty((B, capacity, HQ, K), dtype=dtype, device=device)
@@ -227,7 +328,7 @@ class WallDecodeCache:
         self.r_cache = torch.empty((B, -(-capacity // chunk_size), HQ, K), dtype=torch.float32,
                                    device=device)
         self.carry = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
-        self.sink = sink_bias.contiguous().float() if sink_bias is not None else None
+        self.sink = _opt_f32("sink_bias", sink_bias, (HQ,))
         self.length = 0
         self.ws = _ws(L.wall_attn_decode_workspace(B, capacity, H, HQ, V, chunk_size), device)
         self.fused = (dtype == torch.bfloat16 and K in (64, 128) and V in (64, 128)
@@ -241,8 +342,9 @@ class WallDecodeCache:
     def append(self, k, v, g):
         """Appends Tn tokens: k [B,Tn,H,K], v [B,Tn,H,V], g [B,Tn,HQ,K];
         returns their prefix P [B,Tn,HQ,K]."""
+        Tn = self._check_tokens(k, v, g)
         k, v, g = k.contiguous(), v.contiguous(), g.contiguous()
-        B, Tn = k.shape[:2]
+        B = self.B
         t0 = self.length
         if t0 + Tn > self.cap:
             raise ValueError("decode cache capacity exceeded")
@@ -256,6 +358,19 @@ class WallDecodeCache:
         self.length = t0 + Tn
         return P
 
+    def _check_tokens(self, k, v, g, q=None):
+        """Shapes and dtype of Tn new tokens for this cache; returns Tn."""
+        if k.dim() != 4:
+            raise ValueError("k must be [B, Tn, H, K]")
+        Tn = k.shape[1]
+        B, H, HQ = self.B, self.H, self.HQ
+        _expect("k", k, (B, Tn, H, self.K), self.dtype)
+        _expect("v", v, (B, Tn, H, self.V), self.dtype)
+        _expect("g", g, (B, Tn, HQ, self.K), self.dtype)
+        _expect("q", q, (B, Tn, HQ, self.K), self.dtype)
+        _same_device(self.k_tilde, k, v, g, q)
+        return Tn
+
     def decode(self, q, p_curr):
         return wall_attn_decode(q, self.v, p_curr, self.k_tilde, self.r_cache, self.sink,
                                 self.scale, self.C, T_kv=self.length)
@@ -264,6 +379,7 @@ class WallDecodeCache:
         """Appends Tn tokens and attends all their queries at once (chunked
         prefill / multi-token decode): q [B,Tn,HQ,K], k [B,Tn,H,K],
         v [B,Tn,H,V], g [B,Tn,HQ,K]; returns (o [B,Tn,HQ,V], lse [B,Tn,HQ])."""
+        self._check_tokens(k, v, g, q)
         P = self.append(k, v, g)
         return wall_attn_decode_chunk(q, self.v, P, self.k_tilde, self.r_cache, self.sink,
                                       self.scale, self.C, T_kv=self.length)
@@ -274,6 +390,8 @@ class WallDecodeCache:
         takes the three-call path even where the fused step applies."""
         if fused is None:
             fused = self.fused
+        if self._check_tokens(k, v, g, q) != 1:
+            raise ValueError("step takes one token; use extend for several")
         if not fused:
             P = self.append(k, v, g)
             return self.decode(q, P[:, -1:])
