@@ -487,6 +487,96 @@ def bench_decode(args, rank, peaks):
     return out
 
 
+def config_fwd_flops(s: I.Spec, lengths) -> float:
+    """Algorithmic forward FLOPs of a (possibly packed) batch: 2 (K + V) per
+    visible (query, key) pair, summed over sequences and query heads."""
+    return 2.0 * sum(I.causal_pairs(int(n), s.window) for n in lengths) * s.HQ * (s.K + s.V)
+
+
+def bench_configs(args, world, rank):
+    """fwd+bwd TFLOP/s of the two other training workloads, L2 flushed before
+    every timed step (their working sets are near or below the 126 MB L2),
+    per step (events around it) and per kernel time (the library's stage
+    events, one rank's):
+    config 2 (B=2, T=1024, HQ=8, H=4, K=V=64) through the fused gate call
+    with the backward reusing its operands, config 4 (8 packed sequences of
+    512-4096 rows, HQ=16, H=2, K=V=128, g_scalar, sink with dsink, window
+    1024) through prefix scan, forward and backward.  Median over the timed
+    steps, max over ranks."""
+    from channel_decay_softmax_b200 import api
+
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+    for cfg in (2, 4):
+        ms, err, info = -1.0, None, {}
+        try:
+            s = I.spec(cfg, seed=rank_seed(cfg, rank))
+            x = I.training_inputs(s, device="cuda")
+            cu = x["cu_seqlens"]
+            lengths = (cu[1:] - cu[:-1]).tolist() if cu is not None else [x["T"]] * x["B"]
+            fwd = config_fwd_flops(s, lengths)
+            kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"],
+                      window_size=x["window_size"], cu_seqlens=cu)
+            q, k, v, g, dO = x["q"], x["k"], x["v"], x["g"], x["dO"]
+            if cfg == 2:
+                def step():
+                    o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, s.scale,
+                                                            return_workspace=True, **kw)
+                    api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, fwd_workspace=fws, **kw)
+                path = "fused gate forward + backward reusing its operands"
+            else:
+                def step():
+                    P = api.prefix_cumsum(g, cu)
+                    o, lse = api.wall_attn_fwd(q, k, v, P, s.scale, **kw)
+                    api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, want_dsink=True, **kw)
+                path = "prefix scan + forward + backward (with dsink)"
+            for _ in range(max(3, args.warmup)):
+                step()
+            n = min(max(args.steps, 10), 30)
+            evs = [(ev(), ev()) for _ in range(n)]
+            # the library's stage events give the device time of its own
+            # kernels; the events around each step also hold any time the
+            # GPU waits for the host to issue the step's launches
+            api.timing_enable(True)
+            try:
+                for a, b in evs:
+                    flush.zero_()
+                    a.record(stream)
+                    step()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                stages = api.timing_read()
+            finally:
+                api.timing_enable(False)
+            ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+            kernel_ms = sum(t for _, t in stages.values()) / n
+            info = dict(workload=f"{s.name}: B={x['B']} T={x['T']} HQ={s.HQ} H={s.H} "
+                                 f"K=V={s.K}" + (f", {len(lengths)} packed sequences"
+                                                 if cu is not None else "")
+                                 + (f", window {s.window}" if s.window else ""),
+                        path=path, fwd_bwd_flop=3.5 * fwd, timed_steps=n,
+                        kernel_ms_per_step=kernel_ms,
+                        l2="flushed (256 MB write) before every timed step")
+        except Exception as e:  # reported in the line; the headline stands
+            err = f"{type(e).__name__}: {e}"[:200]
+        ms = max_over_ranks(ms, world)
+        if err is None and ms > 0:
+            fl = info["fwd_bwd_flop"]
+            info.update(ms_per_step=ms, tflops=world * fl / (ms * 1e-3) / 1e12,
+                        kernel_tflops=fl / (info["kernel_ms_per_step"] * 1e-3) / 1e12)
+            out[f"config{cfg}"] = info
+        else:
+            out[f"config{cfg}"] = {"error": err or "failed on another rank"}
+    del flush
+    try:
+        torch.cuda.empty_cache()
+    except Exception:  # a failed config above may have left the context unusable
+        pass
+    return out
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline leg and the reference arm)
 
@@ -538,7 +628,7 @@ def workload_name():
             f"g=-0.05|N| (prefix scan + forward + backward incl. dg)")
 
 
-def assemble_line(args, world, tr, dec, peaks):
+def assemble_line(args, world, tr, dec, peaks, configs=None):
     """The JSON line of our arm (without the cpu_baseline leg): headline,
     per-stage table, the dominant kernel's roofline, clocks, e2e, decode.
     `tr["stages"]` maps stage names to (launches, total ms) as
@@ -588,6 +678,8 @@ def assemble_line(args, world, tr, dec, peaks):
         line["e2e"] = tr["e2e"]
     if dec is not None:
         line["decode"] = dec
+    if configs is not None:
+        line["configs"] = configs
     return line
 
 
@@ -604,6 +696,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -619,9 +712,10 @@ def main(argv=None):
     dec = None
     if not args.no_decode:
         dec = bench_decode(args, rank, peaks)
+    cfgs = None if args.no_configs else bench_configs(args, world, rank)
     barrier(world)
     if rank == 0:
-        line = assemble_line(args, world, tr, dec, peaks)
+        line = assemble_line(args, world, tr, dec, peaks, cfgs)
         if world == 1 and not args.no_cpu:
             # about 10-15 s of host work (the cost grows with the square of
             # the sampled rows)

@@ -68,3 +68,26 @@ def test_weak_scaling_counts_every_rank():
     assert abs(line4["value"] - 4 * line1["value"]) < 1e-6
     assert line4["config"]["parallelism"] == "replicas x4"
     assert "decode" not in line1
+
+
+def test_config_flops_count_visible_pairs():
+    s3 = bench.I.spec(3)
+    assert bench.config_fwd_flops(s3, [s3.T]) == bench.train_flops(s3)[0]
+    # config 4: windowed pairs of every packed sequence
+    s4 = bench.I.spec(4)
+    lengths = bench.I.varlen_lengths(s4)
+    W = s4.window
+    pairs = sum(min(n, W) * (min(n, W) + 1) // 2 + max(0, n - W) * W for n in lengths)
+    assert bench.config_fwd_flops(s4, lengths) == 2.0 * pairs * s4.HQ * (s4.K + s4.V)
+
+
+def test_line_carries_the_other_configs():
+    cfgs = {"config2": {"tflops": 400.0, "ms_per_step": 0.02},
+            "config4": {"error": "RuntimeError: x"}}
+    line = bench.assemble_line(argparse.Namespace(steps=10, warmup=3), 1, _tr(), None,
+                               dict(hbm_gbs=1.0, bf16_tflops=1.0, bf16_tflops_sustained=1.0,
+                                    source="fallback"), cfgs)
+    assert line["configs"] == cfgs
+    assert "configs" not in bench.assemble_line(
+        argparse.Namespace(steps=10, warmup=3), 1, _tr(), None,
+        dict(hbm_gbs=1.0, bf16_tflops=1.0, bf16_tflops_sustained=1.0, source="fallback"))
