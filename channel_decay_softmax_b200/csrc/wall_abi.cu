@@ -20,15 +20,19 @@ bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 bool ok_head_dim(int d) { return d >= 8 && d <= 128 && d % 8 == 0; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The status word's address on the current device (each device holds its
+// own copy of g_status).
 int* status_ptr() {
-  static int* p = nullptr;
-  if (!p) {
+  static int* p[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  if (!p[dev]) {
     int* q = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&q), g_status) != cudaSuccess)
       return nullptr;
-    p = q;
+    p[dev] = q;
   }
-  return p;
+  return p[dev];
 }
 
 // cu_seqlens must start at 0, never decrease and end at `rows`; a violation
@@ -189,6 +193,12 @@ ChunkWs chunk_ws_layout(int dtype, int B, int Tq, int T_kv, int H, int HQ, int K
 }  // namespace
 
 int* device_status() { return status_ptr(); }
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
 
 }  // namespace wall
 

@@ -707,13 +707,8 @@ int launch_dq_ds(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int
   if (!make_rows128_map(&tds, a.dS, tiles * 128, 128, 64) ||
       !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN))
     return WALL_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(bwd_dq_ds_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             QSmem<KD>::kAlloc) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_dq_ds_kernel<KD>, QSmem<KD>::kAlloc, attr)) return WALL_ERR_CUDA;
   DqParams p;
   p.anchors = ws.anchors;
   p.lse = a.lse;
@@ -741,13 +736,8 @@ int launch_dq(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* s
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BN) ||
       !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BM))
     return WALL_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(bwd_dq_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DSmem<KD>::kAlloc) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_dq_kernel<KD>, DSmem<KD>::kAlloc, attr)) return WALL_ERR_CUDA;
   DqParams p;
   p.anchors = ws.anchors;
   p.lse = a.lse;

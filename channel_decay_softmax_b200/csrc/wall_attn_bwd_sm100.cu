@@ -789,13 +789,8 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   if (a.dS && !make_rows128_map(&tds, a.dS, (long)pb.B * pb.HQ * ((long)nb * (nb + 1) / 2) * BK,
                                 32, 32))
     return WALL_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(bwd_tc_kernel<KD, kGS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             BSmem<KD>::kAlloc) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_tc_kernel<KD, kGS>, BSmem<KD>::kAlloc, attr)) return WALL_ERR_CUDA;
   BwdTcParams p;
   p.qh = static_cast<const __nv_bfloat16*>(ws.qh);
   p.anchors = ws.anchors;

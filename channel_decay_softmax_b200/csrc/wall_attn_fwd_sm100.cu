@@ -732,13 +732,9 @@ int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, in
       !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN) ||
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BN))
     return WALL_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(fwd_tc_kernel<KD, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<KD, false>::kAlloc) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(fwd_tc_kernel<KD, false>, Smem<KD, false>::kAlloc, attr))
+    return WALL_ERR_CUDA;
   FwdTcParams p;
   p.anchors = ws.anchors;
   p.GS = a.GS;
@@ -770,13 +766,9 @@ int launch_decode_chunk_tc(const FwdTcParams& p0, const void* k_tilde, const voi
       !make_cache_map(&tk, k_tilde, B, T_kv, Tcap, HQ, KD, BN) ||
       !make_cache_map(&tv, v, B, T_kv, Tcap, H, KD, BN))
     return WALL_ERR_CUDA;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(fwd_tc_kernel<KD, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<KD, true>::kAlloc) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(fwd_tc_kernel<KD, true>, Smem<KD, true>::kAlloc, attr))
+    return WALL_ERR_CUDA;
   dim3 grid(HQ, p0.n_blocks);
   fwd_tc_kernel<KD, true><<<grid, kThreads, Smem<KD, true>::kAlloc, stream>>>(tq, tk, tv, p0);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;

@@ -497,14 +497,8 @@ template <typename T, int KD, int VD>
 int launch_fwd(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(float) * (size_t)(BM * (KD + 1) + BN * (KD + 1) + BN * VD +
                                                BM * (BN + 1) + KD + BM + BN);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(fwd_simt_kernel<T, KD, VD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr_set = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(fwd_simt_kernel<T, KD, VD>, (int)smem, attr)) return WALL_ERR_CUDA;
   dim3 grid(pb.max_blocks64, pb.HQ);
   fwd_simt_kernel<T, KD, VD><<<grid, kThreads, smem, stream>>>(pb, a);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
@@ -517,17 +511,10 @@ int launch_bwd(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
   const size_t smem_dk = sizeof(float) * (size_t)(BN * (KD + 1) + BN * (VD + 1) +
                                                   BM * (KD + 1) + BM * (VD + 1) +
                                                   2 * BN * (BM + 1) + KD + 4 * BM);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(bwd_dq_simt_kernel<T, KD, VD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dkdv_simt_kernel<T, KD, VD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dk) !=
-            cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr_set = true;
-  }
+  static bool attr_dq[kMaxDevices] = {}, attr_dk[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_dq_simt_kernel<T, KD, VD>, (int)smem_dq, attr_dq) ||
+      !set_max_smem_once(bwd_dkdv_simt_kernel<T, KD, VD>, (int)smem_dk, attr_dk))
+    return WALL_ERR_CUDA;
   dim3 grid(pb.max_blocks64, pb.HQ);
   bwd_dq_simt_kernel<T, KD, VD><<<grid, kThreads, smem_dq, stream>>>(pb, a);
   if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;

@@ -722,13 +722,9 @@ int launch_decode_stream(const DecodeArgs& a, const StepArgs& st, __nv_bfloat16*
   if (stages > 4) stages = 4;
   if (stages < 2) return WALL_ERR_UNSUPPORTED;
   const int smem = stages * stage_bytes + tail + 1024;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(decode_stream_kernel<KD, VD, WPH, kStep>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-      return WALL_ERR_CUDA;
-    attr = true;
-  }
+  static bool attr[kMaxDevices] = {};
+  if (!set_max_smem_once(decode_stream_kernel<KD, VD, WPH, kStep>, 227 * 1024, attr))
+    return WALL_ERR_CUDA;
   const int n_items = a.B * a.H * a.splits;
   const int grid = n_items < 148 ? n_items : 148;
   const int warps = G * WPH + 1 + (kStep ? 1 : 0);  // consumers, TMA, finisher

@@ -19,15 +19,13 @@ constexpr size_t kScratchFloats = size_t(1) << 20;
 // Every GPU that loads the library holds this array until the process exits.
 __device__ __align__(256) float g_decode_scratch[kScratchFloats];
 
-constexpr int kMaxDevices = 64;
-
 // The array's device address on the current device.  In host code the name
 // g_decode_scratch is only a host-side stand-in, so the address is asked for
 // once per device, with that device current, and kept.
 float* scratch_on_current_device() {
   static float* addr[kMaxDevices] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return nullptr;

@@ -146,6 +146,28 @@ int decode_splits(int B, int T_kv, int H, int C);
 // the device status word kernels record bounded-wait timeouts in (wall_abi.cu)
 int* device_status();
 
+// Function attributes and symbol addresses belong to one device's context,
+// so one-time setup is kept per device: a process may drive the library on
+// several devices.
+constexpr int kMaxDevices = 64;
+// the calling thread's current device, or -1 (no device, or beyond kMaxDevices)
+int current_device();
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per device; `done` is the call site's own per-device flags.
+template <typename F>
+inline bool set_max_smem_once(F kernel, int bytes, bool (&done)[kMaxDevices]) {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
 int attn_decode(const void* q, const void* v, const float* p_curr, const void* k_tilde,
                 const float* r_cache, const float* sink, float scale, int C, int dtype, int B,
                 int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,

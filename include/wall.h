@@ -34,7 +34,13 @@
  *     calls return; the library allocates no device memory and keeps no
  *     state between calls except one device status word (wall_get_status),
  *     the fixed scratch array of wall_attn_decode_noalloc and the events of
- *     the per-stage timing aid.
+ *     the per-stage timing aid.  Calls run on the calling thread's current
+ *     device (cudaSetDevice); the status word and the scratch array exist
+ *     once per device, and per-device setup (kernel shared-memory limits,
+ *     symbol addresses) is done on a device's first call, for up to 64
+ *     devices in one process.  The timing aid times one device per process
+ *     (its events are created on the device current at a stage's first
+ *     timed launch).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  Arguments are checked on the host before any launch;
  *     on a bad argument nothing is launched and the call returns an error.
