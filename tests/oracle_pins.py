@@ -333,11 +333,43 @@ def pin_key_side_gate_grad(seed=13):
     return _ok("gate grad = q.dq - k.dk^(h), reverse cumsum", _err(dg, bw["dg"]), 1e-12)
 
 
+def pin_row_and_head_subsets(seed=14):
+    """The oracle's subset modes are bookkeeping only: a range of query rows
+    (with q holding just those rows' queries, as the decode and chunk parity
+    tests pass it, or the whole q) and a subset of (sequence, head) units
+    return the full computation's values there and NaN elsewhere, so parity
+    tests that use them compare against the full path the other pins fix."""
+    x = _inputs(seed, B=2, T=11, HQ=4, H=2, K=3, V=3, g_amp=0.3, decay=True, gs=True,
+                sink=True)
+    kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=7)
+    o, lse = wo.forward(x["q"], x["k"], x["v"], x["g"], **kw)
+    lo, hi = 6, 11
+    o_r, l_r = wo.forward(x["q"][:, lo:hi], x["k"], x["v"], x["g"], rows=(lo, hi),
+                          q_rows_only=True, **kw)
+    worst = max(_err(o_r[:, lo:hi], o[:, lo:hi]), _err(l_r[:, lo:hi], lse[:, lo:hi]))
+    o_w, l_w = wo.forward(x["q"], x["k"], x["v"], x["g"], rows=(2, 5), **kw)
+    worst = max(worst, _err(o_w[:, 2:5], o[:, 2:5]), _err(l_w[:, 2:5], lse[:, 2:5]))
+    untouched = (np.isnan(o_r[:, :lo]).all() and np.isnan(o_w[:, 5:]).all()
+                 and np.isnan(l_w[:, :2]).all())
+    # units: (sequence * HQ + head); here sequences are the batch rows
+    units = [0 * 4 + 1, 1 * 4 + 3]
+    o_u, _ = wo.forward(x["q"], x["k"], x["v"], x["g"], units=units, **kw)
+    bw = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], **kw)
+    bu = wo.backward(x["q"], x["k"], x["v"], x["g"], x["dO"], units=units, **kw)
+    for b, h in ((0, 1), (1, 3)):
+        worst = max(worst, _err(o_u[b, :, h], o[b, :, h]))
+        for key in ("dq", "dk_h", "dv_h", "dg", "dg_scalar"):
+            worst = max(worst, _err(bu[key][b, :, h], bw[key][b, :, h]))
+    untouched = untouched and np.isnan(o_u[0, :, 0]).all() and np.isnan(bu["dq"][1, :, 1]).all()
+    ok, detail = _ok("row and head subsets", worst, 1e-14)
+    return ok and untouched, detail + ("" if untouched else " (rows outside the subset written)")
+
+
 ALL_PINS = [pin_g_zero_textbook, pin_product_equals_prefix, pin_fox_scalar_gate,
             pin_channel_constant_gate, pin_window_sink_textbook, pin_gqa_repeat,
             pin_varlen_independent, pin_decode_row, pin_prefix_closed_form,
             pin_prefix_magnitude_long_context, pin_gradients_fd, pin_shift_invariance,
-            pin_key_side_gate_grad]
+            pin_key_side_gate_grad, pin_row_and_head_subsets]
 
 
 def run_all_pins():
