@@ -220,6 +220,7 @@ const char* wall_error_string(int code) {
 }
 
 int wall_get_status(wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return WALL_ERR_CUDA;
   int v = 0;
@@ -230,6 +231,7 @@ int wall_get_status(wall_stream_t stream) {
 }
 
 int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (limit_us < 1 || limit_us > 2000000) return WALL_ERR_INVALID_ARG;
   int* st = status_ptr();
   if (!st) return WALL_ERR_CUDA;
@@ -241,6 +243,7 @@ int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream) {
 int wall_prefix_cumsum(const void* g, int dtype, float* P, int B, int T, int HQ, int K,
                        const int32_t* cu_seqlens, int n_seq, const float* carry_in,
                        float* carry_out, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || T < 0 || HQ < 1 || K < 1) return WALL_ERR_INVALID_ARG;
   if (((long)HQ * K) % 8 != 0) return WALL_ERR_UNSUPPORTED;
@@ -279,6 +282,7 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
                   const float* sink_bias, int window_size, const int32_t* cu_seqlens, int n_seq,
                   void* o, float* lse, void* workspace, size_t workspace_bytes,
                   wall_stream_t stream) {
+  const TraceRange trace(__func__);
   AttnProblem pb;
   int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
   if (rc) return rc;
@@ -329,6 +333,7 @@ int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* 
                        const float* g_scalar, const float* sink_bias, int window_size,
                        const int32_t* cu_seqlens, int n_seq, float* P, void* o, float* lse,
                        void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   AttnProblem pb;
   int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
   if (rc) return rc;
@@ -390,6 +395,7 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
                   int window_size, const int32_t* cu_seqlens, int n_seq, void* dq, void* dk,
                   void* dv, void* dg, float* dg_scalar, float* dsink, void* workspace,
                   size_t workspace_bytes, const void* fwd_workspace, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   AttnProblem pb;
   int rc = make_problem(dtype, B, T, H, HQ, K, V, scale, window_size, cu_seqlens, n_seq, pb);
   if (rc) return rc;
@@ -474,6 +480,7 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
 int wall_build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ,
                         int K, int C, int t0, void* k_tilde, float* r_cache, int Tcap,
                         wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || Tn < 0 || H < 1 || HQ < 1 || HQ % H != 0 || C < 1 || t0 < 0 || Tcap < 0)
     return WALL_ERR_INVALID_ARG;
@@ -498,6 +505,7 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
                      const float* r_cache, const float* sink_bias, float scale, int C, int dtype,
                      int B, int T_kv, int Tcap, int H, int HQ, int K, int V, void* o, float* lse,
                      void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || T_kv < 1 || Tcap < T_kv || H < 1 || HQ < 1 || HQ % H != 0 || C < 1)
     return WALL_ERR_INVALID_ARG;
@@ -533,6 +541,7 @@ int wall_attn_decode_chunk(const void* q, const void* v, const float* p, const v
                            int dtype, int B, int Tq, int T_kv, int Tcap, int H, int HQ, int K,
                            int V, void* o, float* lse, void* workspace, size_t workspace_bytes,
                            wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || Tq < 0 || T_kv < 1 || Tq > T_kv || Tcap < T_kv || H < 1 || HQ < 1 ||
       HQ % H != 0 || C < 1)
@@ -577,6 +586,7 @@ int wall_decode_step(const void* q, const void* k, const void* v, const void* g,
                      const float* sink_bias, float scale, int C, int t, int B, int Tcap, int H,
                      int HQ, int K, int V, void* o, float* lse, void* workspace,
                      size_t workspace_bytes, wall_stream_t stream) {
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || t < 0 || Tcap < 1 || t >= Tcap || H < 1 || HQ < 1 || HQ % H != 0 || C < 1)
     return WALL_ERR_INVALID_ARG;

@@ -45,6 +45,7 @@ extern "C" int wall_attn_decode_noalloc(const void* q, const void* v, const floa
                                         int B, int T_kv, int Tcap, int H, int HQ, int K, int V,
                                         void* o, float* lse, wall_stream_t stream) {
   using namespace wall;
+  const TraceRange trace(__func__);
   if (dtype != WALL_BF16 && dtype != WALL_FP32) return WALL_ERR_INVALID_ARG;
   if (B < 0 || T_kv < 1 || Tcap < T_kv || H < 1 || HQ < 1 || HQ % H != 0 || C < 1)
     return WALL_ERR_INVALID_ARG;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <nvtx3/nvToolsExt.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -145,6 +146,16 @@ int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int 
 int decode_splits(int B, int T_kv, int H, int C);
 // the device status word kernels record bounded-wait timeouts in (wall_abi.cu)
 int* device_status();
+
+// An NVTX range named after the entry point it is opened in, so that a
+// profiler's timeline or kernel filter (ncu --nvtx) can pick out the
+// library's calls; with no tool attached the NVTX calls do nothing.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
 
 // Function attributes and symbol addresses belong to one device's context,
 // so one-time setup is kept per device: a process may drive the library on

@@ -50,6 +50,9 @@
  *     window_size <= 0 means no window; otherwise key j is visible from
  *     query i iff 0 <= i - j < window_size.
  *   - Empty problems (B == 0 or T == 0) are valid and launch nothing.
+ *   - Every call that launches work (and wall_get_status) opens an NVTX
+ *     range named after itself, for profiler timelines and ncu's --nvtx
+ *     filters; without a profiler attached the range costs nothing.
  */
 #ifndef WALL_H
 #define WALL_H

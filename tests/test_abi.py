@@ -256,3 +256,12 @@ def test_product_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "wall_oracle" not in src, f
+
+
+def test_library_errors_surface_as_wall_error(lib):
+    """A status code from the library reaches Python as WallError, with the
+    library's own description of it."""
+    with pytest.raises(L.WallError, match="invalid argument") as e:
+        L._check("wall_timing_enable_slots", lib.wall_timing_enable_slots(1 << 31))
+    assert e.value.code == L.WALL_ERR_INVALID_ARG
+    L._check("wall_timing_enable_slots", lib.wall_timing_enable_slots(0))
