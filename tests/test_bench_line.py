@@ -91,3 +91,16 @@ def test_line_carries_the_other_configs():
     assert "configs" not in bench.assemble_line(
         argparse.Namespace(steps=10, warmup=3), 1, _tr(), None,
         dict(hbm_gbs=1.0, bf16_tflops=1.0, bf16_tflops_sustained=1.0, source="fallback"))
+
+
+def test_decode_bytes_of_the_decode_workload():
+    """HBM bytes of one decode step at B=32, T_kv=32768, HQ=32, H=8,
+    K=V=128, C=64: k_tilde 8.590 GB + v 2.147 GB + r_cache 0.268 GB plus the
+    per-row q, p_curr, o and lse."""
+    s = bench.I.spec(5)
+    kt = 32 * 32768 * 32 * 128 * 2
+    v = 32 * 32768 * 8 * 128 * 2
+    rc = 32 * (32768 // 64) * 32 * 128 * 4
+    small = 32 * 32 * (128 * 2 + 128 * 4 + 128 * 2 + 4)
+    assert (kt, v, rc) == (8589934592, 2147483648, 268435456)
+    assert bench.decode_bytes(s, 32768) == kt + v + rc + small
