@@ -499,7 +499,8 @@ def bench_configs(args, world, rank):
     per step (events around it) and per kernel time (the library's stage
     events, one rank's):
     config 2 (B=2, T=1024, HQ=8, H=4, K=V=64) through the fused gate call
-    with the backward reusing its operands, config 4 (8 packed sequences of
+    with the backward reusing its operands, eagerly and replayed from a CUDA
+    graph (one rank's time), config 4 (8 packed sequences of
     512-4096 rows, HQ=16, H=2, K=V=128, g_scalar, sink with dsink, window
     1024) through prefix scan, forward and backward.  Median over the timed
     steps, max over ranks."""
@@ -552,13 +553,32 @@ def bench_configs(args, world, rank):
                 api.timing_enable(False)
             ms = statistics.median(a.elapsed_time(b) for a, b in evs)
             kernel_ms = sum(t for _, t in stages.values()) / n
+            graph = {}
+            if cfg == 2:
+                # the same step captured once in a CUDA graph and replayed:
+                # one launch per step instead of the host issuing eleven
+                try:
+                    sg = api.WallAttnStepGraph(q, k, v, g, dO, s.scale, **kw)
+                    gevs = [(ev(), ev()) for _ in range(n)]
+                    for a, b in gevs:
+                        flush.zero_()
+                        a.record(stream)
+                        sg.graph.replay()
+                        b.record(stream)
+                    torch.cuda.synchronize()
+                    gms = statistics.median(a.elapsed_time(b) for a, b in gevs)
+                    graph = dict(graph_ms_per_step=gms,
+                                 graph_tflops=3.5 * fwd / (gms * 1e-3) / 1e12)
+                    del sg
+                except Exception as e:  # reported; the eager numbers stand
+                    graph = {"graph_error": f"{type(e).__name__}: {e}"[:200]}
             info = dict(workload=f"{s.name}: B={x['B']} T={x['T']} HQ={s.HQ} H={s.H} "
                                  f"K=V={s.K}" + (f", {len(lengths)} packed sequences"
                                                  if cu is not None else "")
                                  + (f", window {s.window}" if s.window else ""),
                         path=path, fwd_bwd_flop=3.5 * fwd, timed_steps=n,
                         kernel_ms_per_step=kernel_ms,
-                        l2="flushed (256 MB write) before every timed step")
+                        l2="flushed (256 MB write) before every timed step", **graph)
         except Exception as e:  # reported in the line; the headline stands
             err = f"{type(e).__name__}: {e}"[:200]
         ms = max_over_ranks(ms, world)

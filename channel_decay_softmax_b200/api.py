@@ -236,6 +236,57 @@ def wall_attn(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, window_size
     return WallAttnFunction.apply(q, k, v, g, scale, g_scalar, sink_bias, window_size, cu_seqlens)
 
 
+class WallAttnStepGraph:
+    """One training step -- the fused prefix + forward and the backward
+    reusing its operands -- captured once in a CUDA graph for fixed shapes
+    and options, then replayed.  Small problems are bound by the host's
+    issue of the step's launches; a replay is one graph launch.
+
+    The inputs are copied into buffers the graph owns (``inputs``); replay()
+    copies any new inputs in, replays, and returns the graph's output
+    tensors (o, lse, dq, dk, dv, dg, dg_scalar, dsink), which the next replay
+    overwrites.
+    """
+
+    def __init__(self, q, k, v, g, dO, scale=None, g_scalar=None, sink_bias=None,
+                 window_size=None, cu_seqlens=None, want_dsink=False, warmup=2):
+        self.inputs = {n: t.detach().contiguous().clone()
+                       for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("dO", dO))}
+        self.scale, self.window, self.want_dsink = scale, window_size, want_dsink
+        self.gs = g_scalar.detach().contiguous().float().clone() if g_scalar is not None else None
+        self.sk = sink_bias.detach().contiguous().float().clone() if sink_bias is not None else None
+        self.cu = cu_seqlens.clone() if cu_seqlens is not None else None
+        # warm-up on a side stream (first-call setup happens outside the capture)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(max(1, warmup)):
+                self._step()
+        torch.cuda.current_stream().wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.outputs = self._step()
+
+    def _step(self):
+        x = self.inputs
+        o, lse, P, fws = wall_attn_fwd_gate(x["q"], x["k"], x["v"], x["g"], self.scale, self.gs,
+                                            self.sk, self.window, self.cu, return_workspace=True)
+        dq, dk, dv, dg, dgs, dsink = wall_attn_bwd(
+            x["dO"], x["q"], x["k"], x["v"], P, o, lse, self.scale, self.gs, self.sk,
+            self.window, self.cu, self.want_dsink and self.sk is not None, fws)
+        return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, dg=dg, dg_scalar=dgs, dsink=dsink)
+
+    def replay(self, **new_inputs):
+        """Copies the given inputs (any of q, k, v, g, dO) in and replays."""
+        for n, t in new_inputs.items():
+            if n not in self.inputs:
+                raise KeyError(f"unknown input {n}")
+            _expect(n, t, self.inputs[n].shape, self.inputs[n].dtype)
+            self.inputs[n].copy_(t)
+        self.graph.replay()
+        return self.outputs
+
+
 def build_wall_kv_cache(k, P, chunk_size=64, capacity=None, HQ=None):
     """Pre-rescaled decode cache (README "Decode"): k_tilde [B,Tcap,HQ,K] in
     k's dtype and r_cache [B,ceil(Tcap/C),HQ,K] fp32, Tcap = capacity or T."""
