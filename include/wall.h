@@ -50,6 +50,11 @@
  *     window_size <= 0 means no window; otherwise key j is visible from
  *     query i iff 0 <= i - j < window_size.
  *   - Empty problems (B == 0 or T == 0) are valid and launch nothing.
+ *   - No call allocates or synchronizes except wall_get_status and
+ *     wall_timing_read.  After an entry point's first call on a device
+ *     (which sets its kernels' shared-memory limits), its calls may be
+ *     captured in a CUDA graph and replayed; the timing aid must be off
+ *     during a capture.
  *   - Every call that launches work (and wall_get_status) opens an NVTX
  *     range named after itself, for profiler timelines and ncu's --nvtx
  *     filters; without a profiler attached the range costs nothing.
