@@ -173,3 +173,23 @@ def test_decode_cache_checks_new_tokens():
     with pytest.raises(ValueError):
         api.WallDecodeCache(B, H, HQ, K, V, capacity=64, device="cpu",
                             sink_bias=torch.zeros(HQ + 1))
+
+
+def test_readme_call_pattern_passes_the_checks():
+    """The calls exactly as the wall-attention-release README writes them
+    ("Usage", "Decode": positional and keyword names, a non-leaf g, an
+    expanded upstream gradient later) get through every check."""
+    import channel_decay_softmax_b200 as wa
+    B, T, H, HQ, K, V, C = 2, 64, 4, 8, 64, 64, 16
+    q = torch.randn(B, T, HQ, K, dtype=BF, requires_grad=True)
+    k = torch.randn(B, T, H, K, dtype=BF, requires_grad=True)
+    v = torch.randn(B, T, H, V, dtype=BF, requires_grad=True)
+    g = torch.randn(B, T, HQ, K, dtype=BF, requires_grad=True) * 0.02
+    _passes_checks(wa.wall_attn, q, k, v, g, scale=K ** -0.5)
+    P = torch.zeros(B, T, HQ, K)
+    _passes_checks(wa.build_wall_kv_cache, k.detach(), P, chunk_size=C)
+    k_tilde = torch.zeros(B, T, HQ, K, dtype=BF)
+    r_cache = torch.zeros(B, T // C, HQ, K)
+    _passes_checks(wa.wall_attn_decode, q=q.detach()[:, -1:], v=v.detach(), p_curr=P[:, -1:],
+                   k_tilde=k_tilde, r_cache=r_cache, sink_bias=None, scale=K ** -0.5,
+                   cache_chunk_size=C)
