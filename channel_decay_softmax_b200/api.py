@@ -478,6 +478,8 @@ def timing_enable_slots(names):
     """Times only the named stages (see TIMING_SLOTS); an empty list stops."""
     mask = 0
     for n in names:
+        if n not in TIMING_SLOTS:
+            raise ValueError(f"unknown stage {n!r}; the stages are {', '.join(TIMING_SLOTS)}")
         mask |= 1 << TIMING_SLOTS.index(n)
     L._check("wall_timing_enable_slots", L.lib().wall_timing_enable_slots(mask))
 

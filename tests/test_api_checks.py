@@ -193,3 +193,10 @@ def test_readme_call_pattern_passes_the_checks():
     _passes_checks(wa.wall_attn_decode, q=q.detach()[:, -1:], v=v.detach(), p_curr=P[:, -1:],
                    k_tilde=k_tilde, r_cache=r_cache, sink_bias=None, scale=K ** -0.5,
                    cache_chunk_size=C)
+
+
+def test_timing_slots_by_name():
+    api.timing_enable_slots(["bwd_keyblock", "fwd_tc"])
+    api.timing_enable_slots([])
+    with pytest.raises(ValueError, match="unknown stage 'bwd'"):
+        api.timing_enable_slots(["bwd"])
