@@ -200,3 +200,22 @@ def test_timing_slots_by_name():
     api.timing_enable_slots([])
     with pytest.raises(ValueError, match="unknown stage 'bwd'"):
         api.timing_enable_slots(["bwd"])
+
+
+def test_step_graph_replay_checks_new_inputs():
+    """WallAttnStepGraph.replay copies new inputs into the graph's buffers
+    only when they match them (the capture itself needs a GPU)."""
+    g = object.__new__(api.WallAttnStepGraph)
+    g.inputs = {"q": torch.zeros(1, 4, 2, 8, dtype=BF)}
+    replays = []
+    g.graph = type("G", (), {"replay": lambda self: replays.append(1)})()
+    g.outputs = {"o": None}
+    with pytest.raises(KeyError):
+        g.replay(x=torch.zeros(1))
+    with pytest.raises(ValueError):
+        g.replay(q=torch.zeros(1, 5, 2, 8, dtype=BF))
+    with pytest.raises(TypeError):
+        g.replay(q=torch.zeros(1, 4, 2, 8))
+    assert not replays
+    assert g.replay(q=torch.ones(1, 4, 2, 8, dtype=BF)) == {"o": None}
+    assert replays == [1] and float(g.inputs["q"].float().sum()) == 64.0
