@@ -13,9 +13,12 @@ step, the cache build and prefix scan GB/s, the 64-token streaming
 append loop, and the same 64 positions' queries as one chunk against the
 cache (multi-token decode / chunked prefill).
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
-the same workload on its own data (weak scaling, no collective on the data
-path); time is the max over ranks, value = all ranks' FLOPs / that time.
+Multi-GPU (one rank per GPU): every rank runs its own replica of the same
+workload on its own data (weak scaling, no collective on the data path);
+time is the max over ranks, value = all ranks' FLOPs / that time.  Launched
+under torchrun (WORLD_SIZE set) the ranks are torchrun's; `--gpus N` with
+N > 1 and no WORLD_SIZE starts the N ranks itself through
+torch.distributed.run, after checking that N devices are visible.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload, in the same metric.
@@ -54,6 +57,23 @@ ROOF_STAGE = "bwd_keyblock"
 TRAIN_CFG = 3
 DECODE_CFG = 5
 SM_COUNT = 148
+
+
+# a timed region whose median SM clock is within this fraction of the maximum
+# ran at the burst clock: its roofline takes the burst peak
+AT_MAX_CLOCK = 0.97
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, datasheet (for context only)
+
+
+def pick_peak(peaks, clocks):
+    """(peak TFLOP/s, name) for a kernel timed inside the bench's timed
+    region: the burst figure when that region ran at the maximum SM clock
+    (it is short next to the seconds-long power-capped loop the sustained
+    figure comes from), else the sustained one."""
+    if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and \
+            clocks["sm_mhz"] >= AT_MAX_CLOCK * clocks["sm_max_mhz"]:
+        return peaks["bf16_tflops"], "bf16_tflops (burst)"
+    return peaks["bf16_tflops_sustained"], "bf16_tflops_sustained"
 
 
 def load_peaks():
@@ -181,6 +201,30 @@ def dist_setup(backend="nccl", timeout_s=300):
     return world, rank, local
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(n: int, argv, impl: str) -> int:
+    """`--gpus N` (N > 1) outside torchrun: run this script as N ranks on
+    this node through torch.distributed.run (rendezvous on 127.0.0.1) and
+    return its exit status.  Our arm needs N visible devices and refuses to
+    start with fewer; the reference arm runs on the host cores."""
+    if impl != "reference":
+        have = torch.cuda.device_count()
+        if have < n:
+            print(f"bench.py: --gpus {n} needs {n} visible CUDA devices, found {have}",
+                  file=sys.stderr, flush=True)
+            return 2
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd).returncode
+
+
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -294,7 +338,9 @@ def bench_train_e2e(args, x, s, step_flops, world):
     timed region, as a training input pipeline does: on three streams, the
     upload of step i+1 and the download of step i-1 overlap the compute of
     step i (device inputs and pinned host outputs double-buffered, events
-    order each buffer's reuse)."""
+    order each buffer's reuse).  Events on each stream time its own work in
+    the timed steps, so the line shows which of the upload, the download and
+    the compute bounds the step."""
     from channel_decay_softmax_b200 import api
 
     names_in = ("q", "k", "v", "g", "dO")
@@ -309,20 +355,31 @@ def bench_train_e2e(args, x, s, step_flops, world):
     outputs_ready = [torch.cuda.Event(), torch.cuda.Event()]
     for e in inputs_free:
         e.record(s_comp)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    spans = {"h2d": [], "compute": [], "d2h": []}  # per timed step: (start, end) events
 
-    def step(i):
+    def step(i, timed=False):
         b = i % 2
         d = dev_in[b]
+        span = {n: (ev(), ev()) for n in spans} if timed else None
         with torch.cuda.stream(s_h2d):
             s_h2d.wait_event(inputs_free[b])
+            if timed:
+                span["h2d"][0].record(s_h2d)
             for n in names_in:
                 d[n].copy_(host_in[n], non_blocking=True)
+            if timed:
+                span["h2d"][1].record(s_h2d)
             inputs_ready[b].record(s_h2d)
         s_comp.wait_event(inputs_ready[b])
+        if timed:
+            span["compute"][0].record(s_comp)
         o, lse, P, fws = api.wall_attn_fwd_gate(d["q"], d["k"], d["v"], d["g"], s.scale,
                                                 return_workspace=True)
         dq, dk, dv, dg, _, _ = api.wall_attn_bwd(d["dO"], d["q"], d["k"], d["v"], P, o, lse,
                                                  s.scale, fwd_workspace=fws)
+        if timed:
+            span["compute"][1].record(s_comp)
         inputs_free[b].record(s_comp)
         outputs_ready[b].record(s_comp)
         outs = (dq, dk, dv, dg)
@@ -330,9 +387,16 @@ def bench_train_e2e(args, x, s, step_flops, world):
             host_out[b] = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
         with torch.cuda.stream(s_d2h):
             s_d2h.wait_event(outputs_ready[b])
+            if timed:
+                span["d2h"][0].record(s_d2h)
             for h, t in zip(host_out[b], outs):
                 t.record_stream(s_d2h)  # the allocator keeps it until the copy is done
                 h.copy_(t, non_blocking=True)
+            if timed:
+                span["d2h"][1].record(s_d2h)
+        if timed:
+            for n in spans:
+                spans[n].append(span[n])
 
     for i in range(args.warmup):
         step(i)
@@ -343,7 +407,7 @@ def bench_train_e2e(args, x, s, step_flops, world):
     t0.record(s_h2d)
     s_comp.wait_stream(s_h2d)
     for i in range(args.steps):
-        step(args.warmup + i)
+        step(args.warmup + i, timed=True)
     s_d2h.wait_stream(s_comp)
     t1.record(s_d2h)
     torch.cuda.synchronize()
@@ -351,8 +415,22 @@ def bench_train_e2e(args, x, s, step_flops, world):
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+    busy = {n: statistics.mean(a.elapsed_time(b) for a, b in spans[n]) for n in spans}
+    return e2e_record(world, step_flops, ms, h2d, d2h, busy)
+
+
+def e2e_record(world, step_flops, ms, h2d, d2h, busy):
+    """The e2e object: throughput through host buffers, bytes each way per
+    step, each stream's busy time per step (its own events) and the copy
+    bandwidths they imply, and the stream that bounds the step."""
+    limit = max(busy, key=busy.get)
     return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "h2d_ms_per_step": busy["h2d"], "d2h_ms_per_step": busy["d2h"],
+            "compute_ms_per_step": busy["compute"],
+            "h2d_gbs": h2d / (busy["h2d"] * 1e-3) / 1e9,
+            "d2h_gbs": d2h / (busy["d2h"] * 1e-3) / 1e9,
+            "limit": limit, "limit_share": busy[limit] / ms,
             "pipelined": "3 streams: upload of step i+1 and download of step i-1 overlap "
                          "step i; every step moves its own inputs and gradients"}
 
@@ -659,9 +737,9 @@ def assemble_line(args, world, tr, dec, peaks, configs=None):
     api.timing_read returns them."""
     # per-stage device time from the library's events; the dominant stage's
     # roofline uses its algorithmic FLOPs per launch over its average launch
-    # time (timed inside the timed region), against the sustained bf16 peak
-    # since it runs inside a long step
-    peak = peaks["bf16_tflops_sustained"]
+    # time (timed inside the timed region), against the measured burst bf16
+    # peak when that region ran at the maximum clock, else the sustained one
+    peak, peak_name = pick_peak(peaks, tr.get("clocks"))
     stage_rows = {}
     for name, (n, ms) in tr["stages"].items():
         if n == 0:
@@ -677,8 +755,12 @@ def assemble_line(args, world, tr, dec, peaks, configs=None):
     roof = {"kernel": "bwd_tc_kernel (key-block dK, dV; also stores the dS tiles)",
             "bound": "tensor", "achieved": d["tflops"], "peak": peak, "unit": "TFLOP/s",
             "frac": d["tflops"] / peak,
+            "frac_of_sustained": d["tflops"] / peaks["bf16_tflops_sustained"],
+            "frac_of_nominal": d["tflops"] / NOMINAL_BF16_TFLOPS,
             "traffic": BWD_KEY_TRAFFIC_BYTES if dom == "bwd_keyblock" else None,
-            "peak_source": f"bf16_tflops_sustained of {peaks['source']} peaks",
+            "peak_source": f"{peak_name} of {peaks['source']} peaks (timed region at "
+                           f"{(tr.get('clocks') or {}).get('sm_mhz')} MHz); nominal "
+                           f"{NOMINAL_BF16_TFLOPS:g} TFLOP/s dense bf16 for context",
             "ms_per_launch": d["ms_per_launch"],
             "timed": "CUDA events around this kernel only, on its launch stream, over the "
                      "timed region",
@@ -691,7 +773,10 @@ def assemble_line(args, world, tr, dec, peaks, configs=None):
             "config": {"workload": workload_name(),
                        "l2": "per-step working set ~0.45 GB > 126 MB L2 (no flush)",
                        "parallelism": f"replicas x{world}"},
-            "frac_bf16_peak": tr["value"] / world / peaks["bf16_tflops_sustained"],
+            "frac_bf16_peak": tr["value"] / world / peak,
+            "frac_bf16_peak_of": peak_name,
+            "frac_bf16_sustained": tr["value"] / world / peaks["bf16_tflops_sustained"],
+            "frac_bf16_nominal": tr["value"] / world / NOMINAL_BF16_TFLOPS,
             "fwd_tflops": tr["fwd_tflops"], "bwd_tflops": tr["bwd_tflops"],
             "roofline": roof, "stages": stage_rows, "gpu_launches": tr["launches"],
             "peaks": {k: peaks[k] for k in ("hbm_gbs", "bf16_tflops",
@@ -723,6 +808,11 @@ def main(argv=None):
     ap.add_argument("--no-configs", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv), args.impl)
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={os.environ['WORLD_SIZE']}; "
+              f"the ranks are torchrun's", file=sys.stderr, flush=True)
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

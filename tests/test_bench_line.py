@@ -45,8 +45,12 @@ def test_line_has_the_contract_keys():
     for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert key in roof, key
     assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
-    assert roof["peak"] == peaks["bf16_tflops_sustained"]
+    # the timed region ran at the maximum clock: the burst peak applies
+    assert roof["peak"] == peaks["bf16_tflops"]
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-12
+    assert abs(line["frac_bf16_peak"] - line["value"] / peaks["bf16_tflops"]) < 1e-12
+    assert abs(roof["frac_of_sustained"] - roof["achieved"] / 1394.4) < 1e-12
+    assert abs(line["frac_bf16_nominal"] - line["value"] / 2250.0) < 1e-12
     # the key block does 2 x the forward's FLOPs per launch
     fwd_flops = _tr()["fwd_flops"]
     assert abs(roof["achieved"] - 2 * fwd_flops / (0.654e-3) / 1e12) < 1e-6
@@ -104,3 +108,23 @@ def test_decode_bytes_of_the_decode_workload():
     small = 32 * 32 * (128 * 2 + 128 * 4 + 128 * 2 + 4)
     assert (kt, v, rc) == (8589934592, 2147483648, 268435456)
     assert bench.decode_bytes(s, 32768) == kt + v + rc + small
+
+
+def test_sustained_peak_below_the_maximum_clock():
+    """A timed region whose median SM clock sat below the maximum (the power
+    cap holding it down) takes the sustained peak."""
+    args = argparse.Namespace(steps=100, warmup=3)
+    peaks = dict(hbm_gbs=6549.4, bf16_tflops=1657.1, bf16_tflops_sustained=1394.4,
+                 sm_max_mhz=1965.0, source="measured")
+    tr = _tr()
+    tr["clocks"] = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    line = bench.assemble_line(args, 1, tr, None, peaks)
+    assert line["roofline"]["peak"] == peaks["bf16_tflops_sustained"]
+    assert line["frac_bf16_peak_of"] == "bf16_tflops_sustained"
+
+
+def test_e2e_names_the_bounding_stream():
+    r = bench.e2e_record(1, 9.6e11, 4.79, 117440512, 83886080,
+                         {"h2d": 4.5, "compute": 1.4, "d2h": 3.2})
+    assert r["limit"] == "h2d" and abs(r["h2d_gbs"] - 117440512 / 4.5e-3 / 1e9) < 1e-9
+    assert abs(r["value"] - 9.6e11 / 4.79e-3 / 1e12) < 1e-9
