@@ -576,12 +576,12 @@ def bench_configs(args, world, rank):
     every timed step (their working sets are near or below the 126 MB L2),
     per step (events around it) and per kernel time (the library's stage
     events, one rank's):
-    config 2 (B=2, T=1024, HQ=8, H=4, K=V=64) through the fused gate call
-    with the backward reusing its operands, eagerly and replayed from a CUDA
-    graph (one rank's time), config 4 (8 packed sequences of
+    config 2 (B=2, T=1024, HQ=8, H=4, K=V=64), eagerly and replayed from a
+    CUDA graph (one rank's time), and config 4 (8 packed sequences of
     512-4096 rows, HQ=16, H=2, K=V=128, g_scalar, sink with dsink, window
-    1024) through prefix scan, forward and backward.  Median over the timed
-    steps, max over ranks."""
+    1024), both through the fused gate call with the backward reusing its
+    operands (the autograd function's path).  Median over the timed steps,
+    max over ranks; config 4 also reports its per-stage kernel times."""
     from channel_decay_softmax_b200 import api
 
     stream = torch.cuda.current_stream()
@@ -599,18 +599,15 @@ def bench_configs(args, world, rank):
             kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"],
                       window_size=x["window_size"], cu_seqlens=cu)
             q, k, v, g, dO = x["q"], x["k"], x["v"], x["g"], x["dO"]
-            if cfg == 2:
-                def step():
-                    o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, s.scale,
-                                                            return_workspace=True, **kw)
-                    api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, fwd_workspace=fws, **kw)
-                path = "fused gate forward + backward reusing its operands"
-            else:
-                def step():
-                    P = api.prefix_cumsum(g, cu)
-                    o, lse = api.wall_attn_fwd(q, k, v, P, s.scale, **kw)
-                    api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, want_dsink=True, **kw)
-                path = "prefix scan + forward + backward (with dsink)"
+            want_dsink = x["sink_bias"] is not None
+
+            def step():
+                o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, s.scale,
+                                                        return_workspace=True, **kw)
+                api.wall_attn_bwd(dO, q, k, v, P, o, lse, s.scale, fwd_workspace=fws,
+                                  want_dsink=want_dsink, **kw)
+            path = "fused gate forward + backward reusing its operands" + \
+                (" (with dsink)" if want_dsink else "")
             for _ in range(max(3, args.warmup)):
                 step()
             n = min(max(args.steps, 10), 30)
@@ -660,6 +657,7 @@ def bench_configs(args, world, rank):
                                  + (f", window {s.window}" if s.window else ""),
                         path=path, fwd_bwd_flop=3.5 * fwd, timed_steps=n,
                         kernel_ms_per_step=kernel_ms,
+                        stage_ms_per_step={name: t / n for name, (c, t) in stages.items() if c},
                         l2="flushed (256 MB write) before every timed step", **graph)
         except Exception as e:  # reported in the line; the headline stands
             err = f"{type(e).__name__}: {e}"[:200]

@@ -13,7 +13,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libwall.so")
 
-WALL_OK, WALL_ERR_INVALID_ARG, WALL_ERR_UNSUPPORTED, WALL_ERR_CUDA, WALL_ERR_TIMEOUT = range(5)
+(WALL_OK, WALL_ERR_INVALID_ARG, WALL_ERR_UNSUPPORTED, WALL_ERR_CUDA, WALL_ERR_TIMEOUT,
+ WALL_ERR_RANGE) = range(6)
 WALL_BF16, WALL_FP32 = 0, 1
 
 EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn_fwd_workspace",
@@ -22,7 +23,8 @@ EXPORTS = ["wall_version", "wall_error_string", "wall_prefix_cumsum", "wall_attn
            "wall_selftest_wait_timeout", "wall_attn_decode_noalloc", "wall_timing_enable",
            "wall_timing_read", "wall_decode_step_workspace", "wall_decode_step",
            "wall_attn_decode_chunk_workspace", "wall_attn_decode_chunk",
-           "wall_attn_fwd_gate_workspace", "wall_attn_fwd_gate", "wall_timing_enable_slots"]
+           "wall_attn_fwd_gate_workspace", "wall_attn_fwd_gate", "wall_timing_enable_slots",
+           "wall_attn_bwd_workspace_min"]
 
 _lib = None
 
@@ -55,7 +57,9 @@ def lib():
         L.wall_attn_fwd.argtypes = [vp, vp, vp, fp, i, i, i, i, i, i, i, f, fp, fp, i, ip, i, vp,
                                     fp, vp, sz, vp]
         L.wall_attn_bwd_workspace.restype = sz
-        L.wall_attn_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.wall_attn_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i, i, i]
+        L.wall_attn_bwd_workspace_min.restype = sz
+        L.wall_attn_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i, i]
         L.wall_attn_bwd.restype = i
         L.wall_attn_bwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, i, i, f, fp, fp,
                                     i, ip, i, vp, vp, vp, vp, fp, fp, vp, sz, vp, vp]
@@ -165,9 +169,15 @@ def wall_attn_fwd(q, k, v, P, B, T, H, HQ, K, V, scale, g_scalar, sink_bias, win
         _p(workspace), ws_bytes, _stream(stream)))
 
 
-def wall_attn_bwd_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> int:
+def wall_attn_bwd_workspace(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0,
+                            window_size=0) -> int:
     return lib().wall_attn_bwd_workspace(dtype_code(dtype), B, T, H, HQ, K, V,
-                                         int(bool(has_g_scalar)), n_seq)
+                                         int(bool(has_g_scalar)), n_seq, int(window_size or 0))
+
+
+def wall_attn_bwd_workspace_min(dtype, B, T, H, HQ, K, V, has_g_scalar, n_seq=0) -> int:
+    return lib().wall_attn_bwd_workspace_min(dtype_code(dtype), B, T, H, HQ, K, V,
+                                             int(bool(has_g_scalar)), n_seq)
 
 
 def wall_attn_bwd(dO, q, k, v, P, o, lse, B, T, H, HQ, K, V, scale, g_scalar, sink_bias,

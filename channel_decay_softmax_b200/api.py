@@ -162,10 +162,13 @@ def wall_attn_fwd_gate(q, k, v, g, scale=None, g_scalar=None, sink_bias=None, wi
 
 
 def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=None,
-                  window_size=None, cu_seqlens=None, want_dsink=False, fwd_workspace=None):
+                  window_size=None, cu_seqlens=None, want_dsink=False, fwd_workspace=None,
+                  store_ds=True):
     """Backward; returns dq, dk, dv, dg, dg_scalar (or None), dsink (or None).
     fwd_workspace: the workspace returned by wall_attn_fwd(..., return_workspace=True)
-    for the same inputs, whose anchored operands are then reused."""
+    for the same inputs, whose anchored operands are then reused.  store_ds=False
+    gives the library the smaller workspace without the dS tiles: its dq pass
+    then recomputes them (less memory, more time)."""
     B, T, H, HQ, K, V = _shape_checks(q, k, v, P)
     nseq = _n_seq(cu_seqlens, B)
     _io_dtype(q, k, v, dO, o)
@@ -191,8 +194,13 @@ def wall_attn_bwd(dO, q, k, v, P, o, lse, scale=None, g_scalar=None, sink_bias=N
     dgs = torch.empty_like(g_scalar) if g_scalar is not None else None
     dsink = torch.empty((HQ,), dtype=torch.float32, device=q.device) \
         if (want_dsink and sink_bias is not None) else None
-    ws = _ws(L.wall_attn_bwd_workspace(q.dtype, B, T, H, HQ, K, V, g_scalar is not None, nseq),
-             q.device)
+    if store_ds:
+        nbytes = L.wall_attn_bwd_workspace(q.dtype, B, T, H, HQ, K, V, g_scalar is not None,
+                                           nseq, window_size or 0)
+    else:
+        nbytes = L.wall_attn_bwd_workspace_min(q.dtype, B, T, H, HQ, K, V, g_scalar is not None,
+                                               nseq)
+    ws = _ws(nbytes, q.device)
     L.wall_attn_bwd(dO.contiguous(), q, k, v, P, o, lse, B, T, H, HQ, K, V, scale or 0.0,
                     g_scalar, sink_bias, window_size or 0, cu_seqlens, nseq, dq, dk, dv, dg, dgs,
                     dsink, ws, fwd_workspace)
@@ -471,7 +479,7 @@ def timing_enable(on=True):
 
 TIMING_SLOTS = ("prefix_scan", "operands", "fwd_tc", "bwd_pre", "bwd_keyblock", "bwd_dq",
                 "bwd_finalize", "reverse_scan", "decode", "cache_build", "decode_step",
-                "decode_chunk")
+                "decode_chunk", "exact_units")
 
 
 def timing_enable_slots(names):

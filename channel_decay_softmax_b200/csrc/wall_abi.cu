@@ -86,8 +86,9 @@ int make_problem(int dtype, int B, int T, int H, int HQ, int K, int V, float sca
   pb.seqs.rows = pb.rows;
   pb.extra_blocks = cu_seqlens ? n_seq : 0;
   long nb = cu_seqlens ? (T + 63L) / 64 + n_seq : (long)B * ((T + 63L) / 64);
-  if (nb > 0x7fffffffL) return WALL_ERR_UNSUPPORTED;
+  if (nb > 0x7fffffffL || nb * HQ > 0x7fffffffL) return WALL_ERR_UNSUPPORTED;
   pb.max_blocks64 = (int)nb;
+  pb.units = nullptr;
   if (HQ > 65535) return WALL_ERR_UNSUPPORTED;
   return WALL_OK;
 }
@@ -96,9 +97,15 @@ struct FwdWs {
   size_t gs;       // inclusive prefix of g_scalar [rows, HQ]
   size_t qh, kh;   // anchored operands [rows, HQ, K] bf16 (tensor-core path)
   size_t anchors;  // [n_blocks128, HQ, K] fp32
+  size_t units;    // [n_seq * HQ + 1] int: units beyond the anchored range
   int n_blocks128;
   size_t total;
 };
+// sequences the workspace serves: B, or the cu_seqlens count (extra_blocks)
+size_t unit_flags_bytes(const AttnProblem& pb) {
+  return align256(sizeof(int) *
+                  ((size_t)(pb.extra_blocks > 0 ? pb.extra_blocks : pb.B) * pb.HQ + 1));
+}
 int blocks128(const AttnProblem& pb) {
   long nb = pb.extra_blocks > 0 ? (pb.T + 127L) / 128 + pb.extra_blocks
                                 : (long)pb.B * ((pb.T + 127L) / 128);
@@ -109,13 +116,14 @@ FwdWs fwd_ws_layout(const AttnProblem& pb, int has_gs) {
   size_t off = 0;
   w.gs = off;
   off += has_gs ? align256(sizeof(float) * pb.rows * pb.HQ) : 0;
-  w.qh = w.kh = w.anchors = off;
+  w.qh = w.kh = w.anchors = w.units = off;
   w.n_blocks128 = 0;
   if (fwd_tc_supported(pb)) {
     w.n_blocks128 = blocks128(pb);
     w.qh = off;      off += align256((size_t)2 * pb.rows * pb.HQ * pb.K);
     w.kh = off;      off += align256((size_t)2 * pb.rows * pb.HQ * pb.K);
     w.anchors = off; off += align256(sizeof(float) * (size_t)w.n_blocks128 * pb.HQ * pb.K);
+    w.units = off;   off += unit_flags_bytes(pb);
   }
   w.total = off;
   return w;
@@ -126,11 +134,11 @@ FwdWs fwd_ws_layout(const AttnProblem& pb, int has_gs) {
 constexpr size_t kMaxDsBytes = size_t(8) << 30;
 
 struct BwdWs {
-  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, qh, kh, anchors, dS, total;
+  size_t D, dq32, dkh32, dvh32, dgs_row, dgs_col, gs, qh, kh, anchors, units, dS, total;
   bool has_ds;
   int n_blocks128;
 };
-BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
+BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs, bool want_ds = true) {
   const long rows = pb.rows;
   const int HQ = pb.HQ, K = pb.K, V = pb.V;
   BwdWs w;
@@ -142,20 +150,23 @@ BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs) {
   w.dgs_row = off; off += align256(sizeof(float) * rows * HQ);
   w.dgs_col = off; off += align256(sizeof(float) * rows * HQ);
   w.gs = off;      off += has_gs ? align256(sizeof(float) * rows * HQ) : 0;
-  w.qh = w.kh = w.anchors = off;
+  w.qh = w.kh = w.anchors = w.units = off;
   w.n_blocks128 = 0;
   if (fwd_tc_supported(pb)) {
     w.n_blocks128 = blocks128(pb);
     w.qh = off;      off += align256((size_t)2 * rows * HQ * K);
     w.kh = off;      off += align256((size_t)2 * rows * HQ * K);
     w.anchors = off; off += align256(sizeof(float) * (size_t)w.n_blocks128 * HQ * K);
+    w.units = off;   off += unit_flags_bytes(pb);
   }
   w.dS = off;
   w.has_ds = false;
-  if (fwd_tc_supported(pb) && pb.extra_blocks == 0) {
-    // dS^T tiles (bf16, 128 x 128) of every (batch row, head, I, J <= I)
-    const size_t nb = (size_t)(pb.T + 127) / 128;
-    const size_t bytes = (size_t)pb.B * HQ * (nb * (nb + 1) / 2) * 128 * 128 * 2;
+  if (fwd_tc_supported(pb) && want_ds) {
+    // dS^T tiles (bf16, 128 x 128) of every (sequence, head, I, visible J),
+    // packed in the banded layout of DsLayout
+    const DsLayout lay = DsLayout::of_window(pb.window);
+    const size_t bytes = (size_t)DsLayout::total(lay, pb.rows, pb.T, pb.B, HQ, pb.extra_blocks) *
+                         128 * 128 * 2;
     if (bytes > 0 && bytes <= kMaxDsBytes) {
       w.has_ds = true;
       off += align256(bytes);
@@ -215,6 +226,7 @@ const char* wall_error_string(int code) {
     case WALL_ERR_UNSUPPORTED: return "unsupported dtype or size";
     case WALL_ERR_CUDA: return "CUDA error";
     case WALL_ERR_TIMEOUT: return "device wait timed out";
+    case WALL_ERR_RANGE: return "gate prefix outside the decode cache's anchored range";
     default: return "unknown status";
   }
 }
@@ -311,6 +323,7 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
     tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
     tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
     tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+    tw.units = reinterpret_cast<int*>(at(workspace, w.units));
     tw.n_blocks128 = w.n_blocks128;
     return attn_fwd_tc(pb, a, tw, status_ptr(), s);
   }
@@ -371,22 +384,32 @@ int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* 
   tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
   tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
   tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+  tw.units = reinterpret_cast<int*>(at(workspace, w.units));
   tw.n_blocks128 = w.n_blocks128;
   rc = scan_prefix_operands(static_cast<const __nv_bfloat16*>(g),
                             static_cast<const __nv_bfloat16*>(q),
                             static_cast<const __nv_bfloat16*>(k), P,
                             reinterpret_cast<float*>(at(workspace, w.total)), HQ, H, K, pb.seqs,
-                            tw.qh, tw.kh, tw.anchors, s);
+                            tw.qh, tw.kh, tw.anchors, tw.units, s);
   if (rc) return rc;
   return attn_fwd_tc(pb, a, tw, status_ptr(), s, /*prepared=*/true);
 }
 
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
-                               int has_g_scalar, int n_seq) {
+                               int has_g_scalar, int n_seq, int window_size) {
+  AttnProblem pb;
+  if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, window_size, nullptr, 0, pb) != WALL_OK)
+    return 0;
+  if (n_seq > 0 && B == 1) pb.extra_blocks = n_seq;
+  return bwd_ws_layout(pb, has_g_scalar).total;
+}
+
+size_t wall_attn_bwd_workspace_min(int dtype, int B, int T, int H, int HQ, int K, int V,
+                                   int has_g_scalar, int n_seq) {
   AttnProblem pb;
   if (make_problem(dtype, B, T, H, HQ, K, V, 0.f, 0, nullptr, 0, pb) != WALL_OK) return 0;
   if (n_seq > 0 && B == 1) pb.extra_blocks = n_seq;
-  return bwd_ws_layout(pb, has_g_scalar).total;
+  return bwd_ws_layout(pb, has_g_scalar, /*want_ds=*/false).total;
 }
 
 int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, const float* P,
@@ -412,7 +435,9 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   if (!ok_ptr(dO) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o) ||
       !ok_ptr(lse) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) || !ok_ptr(dg))
     return WALL_ERR_INVALID_ARG;
+  // the dS tiles if the workspace holds them, else the dq pass recomputes
   BwdWs w = bwd_ws_layout(pb, g_scalar != nullptr);
+  if (workspace_bytes < w.total) w = bwd_ws_layout(pb, g_scalar != nullptr, false);
   if (workspace == nullptr || workspace_bytes < w.total || !aligned16(workspace))
     return WALL_ERR_INVALID_ARG;
   if (cu_seqlens) {
@@ -429,9 +454,8 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   a.dvh32 = reinterpret_cast<float*>(at(workspace, w.dvh32));
   a.dgs_row = reinterpret_cast<float*>(at(workspace, w.dgs_row));
   a.dgs_col = reinterpret_cast<float*>(at(workspace, w.dgs_col));
-  // dq from stored dS tiles: dense causal without a window, tensor-core path
-  a.dS = (w.has_ds && pb.window == 0)
-             ? reinterpret_cast<__nv_bfloat16*>(at(workspace, w.dS)) : nullptr;
+  // dq from the stored dS tiles (tensor-core path, tiles within their cap)
+  a.dS = w.has_ds ? reinterpret_cast<__nv_bfloat16*>(at(workspace, w.dS)) : nullptr;
   a.GS = nullptr;
   if (g_scalar) {
     float* gs = reinterpret_cast<float*>(at(workspace, w.gs));
@@ -444,15 +468,17 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
     tw.qh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.qh));
     tw.kh = reinterpret_cast<__nv_bfloat16*>(at(workspace, w.kh));
     tw.anchors = reinterpret_cast<float*>(at(workspace, w.anchors));
+    tw.units = reinterpret_cast<int*>(at(workspace, w.units));
     tw.n_blocks128 = w.n_blocks128;
     const bool reuse = fwd_workspace != nullptr;
     if (reuse) {
-      // the forward's anchored operands, in its own workspace layout
+      // the forward's anchored operands and unit flags, in its own layout
       const FwdWs fw = fwd_ws_layout(pb, g_scalar != nullptr);
       void* fws = const_cast<void*>(fwd_workspace);
       tw.qh = reinterpret_cast<__nv_bfloat16*>(at(fws, fw.qh));
       tw.kh = reinterpret_cast<__nv_bfloat16*>(at(fws, fw.kh));
       tw.anchors = reinterpret_cast<float*>(at(fws, fw.anchors));
+      tw.units = reinterpret_cast<int*>(at(fws, fw.units));
     }
     // dg as well: dL's reverse scan starts inside the finalize pass
     rc = attn_bwd_tc(pb, a, tw, !reuse, dq, dk, dv, dg, status_ptr(), s);

@@ -448,8 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dq from the dS tiles the key-block kernel stored (dense causal problems
-// without a window): for the CTA's query block I and every key tile J <= I,
+// dq from the dS tiles the key-block kernel stored: for the CTA's query
+// block I and every key tile J it sees (J <= I, within the window),
 //   dQa += dS_IJ Kt_J,   Kt_J = Kh_J (.) 2^(R_I - R_J)  (exact, in place)
 // one contraction per tile instead of four (S, dP and this one recomputed,
 // and the exponentials); HBM carries the dS tiles, L2 keeps Kh.
@@ -498,7 +498,7 @@ enum QBar {
 template <int KD>
 __global__ void __launch_bounds__(kDsThreads, 1)
     bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_ds,
-                     const __grid_constant__ CUtensorMap tm_k, DqParams p, int ds_nb) {
+                     const __grid_constant__ CUtensorMap tm_k, DqParams p, DsLayout ds_lay) {
   using Lay = QSmem<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -521,9 +521,9 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   const int L = p.seqs.len(seq);
   const int i0 = blk * BM;
   const int ni = min(BM, L - i0);
-  const int nT = blk + 1;  // key tiles 0 .. I
-  const long tile0 =
-      ((long)seq * HQ + h) * ((long)ds_nb * (ds_nb + 1) / 2) + (long)blk * (blk + 1) / 2;
+  const int jlo = ds_lay.jlo(blk);  // key tiles jlo .. I
+  const int nT = blk - jlo + 1;
+  const long tile0 = ds_lay.pair_base(p.seqs, HQ, seq, h) + ds_lay.rowstart(blk);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDSS; ++s) {
@@ -580,9 +580,10 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         mbar_expect_tx(bar(K_FULL3 + st), Lay::kKT + K * 4);
         for (int b = 0; b < K / 64; ++b)
           tma_load_3d(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k, bar(K_FULL3 + st),
-                      b * 64, h, (int)(s0 + (long)t * BN));
-        bulk_load(sbase + Lay::oRJ + st * K * 4, p.anchors + ((long)(blk_off + t) * HQ + h) * K,
-                  K * 4, bar(K_FULL3 + st));
+                      b * 64, h, (int)(s0 + (long)(jlo + t) * BN));
+        bulk_load(sbase + Lay::oRJ + st * K * 4,
+                  p.anchors + ((long)(blk_off + jlo + t) * HQ + h) * K, K * 4,
+                  bar(K_FULL3 + st));
         issued = t + 1;
       }
       for (int t = max(0, issued - kKS3); t < issued; ++t)
@@ -701,8 +702,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 template <int KD>
 int launch_dq_ds(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                  cudaStream_t stream) {
-  const int nb = (pb.T + BM - 1) / BM;
-  const long tiles = (long)pb.B * pb.HQ * ((long)nb * (nb + 1) / 2);
+  const DsLayout lay = DsLayout::of_window(pb.window);
+  const long tiles = DsLayout::total(lay, pb.rows, pb.T, pb.B, pb.HQ, pb.extra_blocks);
   CUtensorMap tds, tk;
   if (!make_rows128_map(&tds, a.dS, tiles * 128, 128, 64) ||
       !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN))
@@ -723,7 +724,7 @@ int launch_dq_ds(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int
   p.n_blocks = ws.n_blocks128;
   p.status = status;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  bwd_dq_ds_kernel<KD><<<grid, kDsThreads, QSmem<KD>::kAlloc, stream>>>(tds, tk, p, nb);
+  bwd_dq_ds_kernel<KD><<<grid, kDsThreads, QSmem<KD>::kAlloc, stream>>>(tds, tk, p, lay);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
@@ -761,7 +762,7 @@ int launch_dq(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* s
 int attn_bwd_dq_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, int* status,
                    cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
-  if (a.dS) {  // the key-block kernel stored dS (dense causal, no window)
+  if (a.dS) {  // the key-block kernel stored its dS tiles
     return pb.K == 128 ? launch_dq_ds<128>(pb, a, ws, status, stream)
                        : launch_dq_ds<64>(pb, a, ws, status, stream);
   }

@@ -11,10 +11,12 @@
 //   dV_J  += P^T dO_I               (P^T from TMEM)
 //   dKa_J += dS^T Qt_I              (dS^T from TMEM); dk_j = scale 2^(R_J - P_j) dKa_j
 // dq comes from a separate query-block kernel (wall_attn_bwd_dq_sm100.cu), so
-// no fp32 atomics are needed.  For dense causal problems without a window
-// this kernel also stores every dS tile it forms (bf16, as the dK MMA reads
-// it), and the dq kernel is then one contraction dQa = dS Kt per tile instead
-// of recomputing S, P, dP and dS.
+// no fp32 atomics are needed.  Unless the tiles would exceed their workspace
+// cap this kernel also stores every dS tile it forms (bf16, as the dK MMA
+// reads it; packed per (sequence, head) in the banded layout DsLayout
+// describes, which covers varlen packing and windows), and the dq kernel is
+// then one contraction dQa = dS Kt per tile instead of recomputing S, P, dP
+// and dS.
 // The gate gradient needs dk per query head before the GQA sum; it is fused
 // into the finalize kernel as dL = q (.) dq - k (.) dk^(h) (blog, fast
 // training section 2: the key-side term is -K_j (.) dK_j), followed by the
@@ -69,11 +71,11 @@ struct BwdTcParams {
   float* dkh32;             // [rows, HQ, K]
   float* dvh32;             // [rows, HQ, V]
   float* dgs_col;           // [rows, HQ] or nullptr
-  // dS^T tiles for the dq kernel, or nullptr: tile (b, h, I, J), J <= I, at
-  // ((b * HQ + h) * nb(nb+1)/2 + I(I+1)/2 + J) * 128 * 128, rows = keys,
-  // 128 queries per row (dense sequences of nb 128-row blocks, no window)
+  // dS^T tiles for the dq kernel, or nullptr: tile (s, h, I, J) at row
+  // (ds_lay.pair_base(s, h) + ds_lay.rowstart(I) + J - ds_lay.jlo(I)) * 128,
+  // rows = keys, 128 queries per row
   __nv_bfloat16* dS;
-  int ds_nb;
+  DsLayout ds_lay;
   Seqs seqs;
   int HQ, H;
   float scale, scale_log2;
@@ -441,13 +443,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gs_j = (kGS && key_ok) ? p.GS[(s0 + jj) * HQ + h] * kLog2e : 0.f;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     const uint32_t scol = kColS + half * 64, dcol = kColDP + half * 64;
-    // the stored dS tile (I0, J), I0 = J: tile
-    // (b * HQ + h) * nb(nb+1)/2 + I(I+1)/2 + J, rows = keys, 128 queries each;
-    // this warp's 32 keys x 32 queries go through its staging block
+    // the stored dS tile (I, J = blk) of every query tile I this key block
+    // meets, rows = keys, 128 queries each; this warp's 32 keys x 32 queries
+    // go through its staging block
     const bool store_ds = p.dS != nullptr;
-    long ds_tile = store_ds ? ((long)seq * HQ + h) * ((long)p.ds_nb * (p.ds_nb + 1) / 2) +
-                                  (long)I0 * (I0 + 1) / 2 + blk
-                            : 0;
+    const long ds_base = store_ds ? p.ds_lay.pair_base(p.seqs, HQ, seq, h) : 0;
+    auto ds_tile_of = [&](int I) {
+      return ds_base + p.ds_lay.rowstart(I) + blk - p.ds_lay.jlo(I);
+    };
+    long ds_tile = store_ds ? ds_tile_of(I0) : 0;
     uint8_t* stg = smem + Lay::oStg + (warp - 4) * Lay::kStg;
     float colsum = 0.f;
     bool ok = true;
@@ -580,8 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit();
           }
         }
-        // tile (I + 1, J) follows tile (I, J) after the I + 1 tiles of row I
-        ds_tile += I0 + t + 1;
+        ds_tile = ds_tile_of(I0 + t + 1);
       }
     }
     // the stored tiles are complete before the CTA can exit
@@ -693,12 +696,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // D_i = dO_i . o_i; row part of the scalar-gate gradient, sum_j dS_ij =
-// D_i exp(sink - lse_i) (0 without a sink); dsink_h = -sum_i of the same.
+// D_i exp(sink - lse_i) (0 without a sink).
 __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
                                const __nv_bfloat16* __restrict__ o, const float* __restrict__ lse,
                                const float* __restrict__ sink, long rows, int HQ, int V,
-                               float* __restrict__ D, float* __restrict__ dgs_row,
-                               float* __restrict__ dsink) {
+                               float* __restrict__ D, float* __restrict__ dgs_row) {
   const int lanes = 8;  // 8 threads per (row, head), 8 channels each per step
   const long nrh = rows * HQ;
   const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -721,8 +723,31 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
     const int h = (int)(e % HQ);
     const float ps = sink ? exp2f((sink[h] - lse[e]) * kLog2e) : 0.f;
     if (dgs_row) dgs_row[e] = acc * ps;
-    if (dsink && sink) atomicAdd(&dsink[h], -acc * ps);
   }
+}
+
+// dsink_h = -sum_i exp(sink_h - lse_i) D_i (the sink's logit has a zero value
+// row), summed in a fixed order: one CTA per head, a strided sum per thread
+// and a tree in shared memory, so that repeated calls agree bit for bit.
+__global__ void __launch_bounds__(256)
+    sink_grad_kernel(const float* __restrict__ D, const float* __restrict__ lse,
+                     const float* __restrict__ sink, long rows, int HQ,
+                     float* __restrict__ dsink) {
+  __shared__ float part[256];
+  const int h = blockIdx.x;
+  const float s2 = sink[h] * kLog2e;
+  float acc = 0.f;
+  for (long t = threadIdx.x; t < rows; t += 256) {
+    const long e = t * HQ + h;
+    acc -= exp2f(s2 - lse[e] * kLog2e) * D[e];
+  }
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) dsink[h] = part[0];
 }
 
 // dk, dv = sums of the per-query-head dk^(h), dv^(h) over each GQA group;
@@ -785,8 +810,10 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
       !make_tile_map(&to, a.dO, pb.rows, pb.HQ, KD, BQ))
     return WALL_ERR_CUDA;
   memset(&tds, 0, sizeof(tds));  // unused without stored dS tiles
-  const int nb = (pb.T + BQ - 1) / BQ;
-  if (a.dS && !make_rows128_map(&tds, a.dS, (long)pb.B * pb.HQ * ((long)nb * (nb + 1) / 2) * BK,
+  const DsLayout lay = DsLayout::of_window(pb.window);
+  if (a.dS && !make_rows128_map(&tds, a.dS,
+                                DsLayout::total(lay, pb.rows, pb.T, pb.B, pb.HQ,
+                                                pb.extra_blocks) * BK,
                                 32, 32))
     return WALL_ERR_CUDA;
   static bool attr[kMaxDevices] = {};
@@ -802,7 +829,7 @@ int launch_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, in
   p.dvh32 = a.dvh32;
   p.dgs_col = a.GS ? a.dgs_col : nullptr;
   p.dS = a.dS;
-  p.ds_nb = (pb.T + BQ - 1) / BQ;
+  p.ds_lay = lay;
   p.seqs = pb.seqs;
   p.HQ = pb.HQ;
   p.H = pb.H;
@@ -841,8 +868,12 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
     const int blocks = (int)((threads + 255) / 256);
     bwd_pre_kernel<<<blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o), a.lse,
-        a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr, a.dsink);
+        a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr);
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+    if (a.dsink && a.sink) {
+      sink_grad_kernel<<<pb.HQ, 256, 0, stream>>>(a.D, a.lse, a.sink, pb.rows, pb.HQ, a.dsink);
+      if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+    }
   }
   timing_mark(T_BWD_PRE, stream);
   timing_mark(T_BWD_KEY, stream);
@@ -850,8 +881,20 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
                    : launch_bwd_tc_gs<64>(pb, a, ws, status, stream);
   timing_mark(T_BWD_KEY, stream);
   if (rc) return rc;
-  // dk, dv group sums and the scalar-gate parts need only the key-block
-  // kernel; they run before dL overwrites dk^(h)'s chunk rows with its sums
+  timing_mark(T_BWD_DQ, stream);
+  rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
+  timing_mark(T_BWD_DQ, stream);
+  if (rc) return rc;
+  // the units beyond the anchored range, again on CUDA cores: dk^(h),
+  // dv^(h), their column sums and the final dq, over what the tensor-core
+  // kernels wrote for them (one launch that only reads the flags when none
+  // is set)
+  timing_mark(T_EXACT, stream);
+  rc = attn_bwd_simt_units(pb, a, ws.units, stream);
+  timing_mark(T_EXACT, stream);
+  if (rc) return rc;
+  // dk, dv group sums and the scalar-gate parts; they run before dL
+  // overwrites dk^(h)'s chunk rows with its sums
   timing_mark(T_BWD_FIN, stream);
   {
     dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
@@ -862,17 +905,13 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
   }
   timing_mark(T_BWD_FIN, stream);
-  timing_mark(T_BWD_DQ, stream);
-  rc = attn_bwd_dq_tc(pb, a, ws, status, stream);
-  timing_mark(T_BWD_DQ, stream);
-  if (rc) return rc;
   // dq, dL and dL's chunk sums in one pass, then the reverse scan's
   // carries and chunk scans give dg
   timing_mark(T_BWD_FIN, stream);
   rc = finalize_dq_dl_sums(static_cast<const __nv_bfloat16*>(a.q),
                            static_cast<const __nv_bfloat16*>(a.k), a.P, a.dq32, a.dkh32,
                            static_cast<__nv_bfloat16*>(dq), pb.HQ, pb.H, pb.K, pb.scale,
-                           pb.seqs, stream);
+                           pb.seqs, ws.units, stream);
   timing_mark(T_BWD_FIN, stream);
   if (rc) return rc;
   timing_mark(T_REV_SCAN, stream);

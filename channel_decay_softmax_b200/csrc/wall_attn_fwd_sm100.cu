@@ -669,14 +669,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// preparation: anchored operands Qh, Kh (per query head) and block anchors
+// preparation: anchored operands Qh, Kh (per query head) and block anchors.
+// An anchored exponent |P - R| beyond kAnchorRange (a channel whose gate
+// sums past 2^kAnchorRange inside one block) flags its (sequence, head) unit
+// in `units`, which the SIMT kernels then recompute, or records
+// WALL_ERR_RANGE in `status` (the chunk call, which has no such fallback).
 
 __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
                                        const __nv_bfloat16* __restrict__ k,
                                        const float* __restrict__ P, Seqs seqs, int HQ, int H,
                                        int K, __nv_bfloat16* __restrict__ qh,
                                        __nv_bfloat16* __restrict__ khat,
-                                       float* __restrict__ anchors) {
+                                       float* __restrict__ anchors, int* __restrict__ units,
+                                       int* status) {
   const int s = blockIdx.y;
   __shared__ int s_blk_off;
   if (threadIdx.x == 0) {
@@ -705,16 +710,27 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
     float pv[8], rv[8], x[8], y[8];
     load8(P + (row * HQ + hh) * K + g8 * 8, pv);
     load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
+    bool wide = false;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) rv[c] = floorf(rv[c]);
+    for (int c = 0; c < 8; ++c) {
+      rv[c] = floorf(rv[c]);
+      wide |= fabsf(pv[c] - rv[c]) > kAnchorRange;
+    }
+    if (wide) {
+      if (units) {
+        set_flag(units + (long)s * HQ + hh);
+        set_flag(units + (long)seqs.n * HQ);  // some unit is flagged
+      }
+      record_status(status, WALL_ERR_RANGE);
+    }
     load8(q + (row * HQ + hh) * K + g8 * 8, x);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(pv[c] - rv[c]);
+    for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(pv[c] - rv[c]));
     store8(qh + (row * HQ + hh) * K + g8 * 8, y);
     if (k != nullptr) {  // without keys: the query operand and anchors only
       load8(k + (row * H + hh / G) * K + g8 * 8, x);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) y[c] = x[c] * exp2f(rv[c] - pv[c]);
+      for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(rv[c] - pv[c]));
       store8(khat + (row * HQ + hh) * K + g8 * 8, y);
     }
     if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, rv);
@@ -783,12 +799,15 @@ bool fwd_tc_supported(const AttnProblem& pb) {
 int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
                           const TcFwdWs& ws, cudaStream_t stream) {
   if (pb.rows == 0 || pb.seqs.n == 0) return WALL_OK;
+  if (cudaMemsetAsync(ws.units, 0, sizeof(int) * ((size_t)pb.seqs.n * pb.HQ + 1), stream) !=
+      cudaSuccess)
+    return WALL_ERR_CUDA;
   // enough CTAs to keep every SM streaming, split over the sequences
   const int per_seq = (148 * 8 + pb.seqs.n - 1) / pb.seqs.n;
   dim3 grid(per_seq < 1 ? 1 : per_seq, pb.seqs.n);
   anchor_operands_kernel<<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), P, pb.seqs,
-      pb.HQ, pb.H, pb.K, ws.qh, ws.kh, ws.anchors);
+      pb.HQ, pb.H, pb.K, ws.qh, ws.kh, ws.anchors, ws.units, nullptr);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
@@ -811,7 +830,8 @@ int attn_decode_chunk_tc(const void* q, const void* v, const float* p, const voi
   // block's first row), as the training forward prepares its queries
   const int per_seq = (148 * 8 + B - 1) / B;
   anchor_operands_kernel<<<dim3(per_seq < 1 ? 1 : per_seq, B), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), nullptr, p, seqs, HQ, H, K, qh, nullptr, anchors);
+      static_cast<const __nv_bfloat16*>(q), nullptr, p, seqs, HQ, H, K, qh, nullptr, anchors,
+      nullptr, status);
   if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
   FwdTcParams pr;
   pr.anchors = anchors;
@@ -848,6 +868,12 @@ int attn_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, int*
   rc = pb.K == 128 ? launch_fwd_tc<128>(pb, a, ws, status, stream)
                    : launch_fwd_tc<64>(pb, a, ws, status, stream);
   timing_mark(T_FWD, stream);
+  if (rc) return rc;
+  // the units the anchored operands cannot represent, again on CUDA cores
+  // (a persistent grid that only reads the flags when none is set)
+  timing_mark(T_EXACT, stream);
+  rc = attn_fwd_simt_units(pb, a, ws.units, stream);
+  timing_mark(T_EXACT, stream);
   return rc;
 }
 

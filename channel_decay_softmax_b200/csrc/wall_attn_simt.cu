@@ -3,18 +3,24 @@
 // This path computes with fp32 products throughout (no tensor cores), which
 // is what fp32 inputs need to meet a 1e-5 error bound; it also carries every
 // option (GQA, g_scalar, sink, window, varlen) for any head size up to 128.
+// The same kernels, given a mask of (sequence, head) units, recompute the
+// units the tensor-core path cannot represent (see wall_attn_fwd_sm100.cu).
 //
 // Per tile the decay exp2(P_i - P_j) (blog "Wall Attention", factorised
 // form with base-2 prefix) is split with one anchor R per CTA (blog, fast
-// training: per-block anchor, exp2(P_i - P_j) = exp2(P_i - R) exp2(R - P_j)):
+// training: per-block anchor, exp2(P_i - P_j) = exp2(P_i - R) exp2(R - P_j)),
+// placed on the CTA block's boundary that faces the streamed operand:
 //   forward / dq:  R = P at the CTA's first query row; the query tile is
 //                  rescaled once by exp2(P_i - R), each key tile by
 //                  exp2(R - P_j) as it is loaded.
-//   dk / dv:       R = P at the CTA's first key row; the roles swap.
-// With R inside the CTA's own block the factor on the CTA's fixed operand is
-// bounded by one block's accumulated gate, and the factor on the streamed
-// operand only shrinks towards zero for decaying gates (where the exact
-// contribution is equally negligible).
+//   dk / dv:       R = P at the CTA's last key row; the roles swap.
+// Off the diagonal tile the anchor then lies between every key and every
+// query, so for a decaying gate both factors are at most 1 (about 2 with
+// rounding): they can only underflow, and only where the exact product is
+// below 2^-126 as well, however strong the decay.  The diagonal tile pairs
+// rows of the CTA's own block, where one factor grows by the block's whole
+// accumulated gate; when that exceeds 2^kSpanExact on some channel the CTA
+// evaluates its diagonal tile pair by pair, exp2(P_in - P_jn) per channel.
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
@@ -24,6 +30,8 @@ namespace {
 constexpr int BM = 64;
 constexpr int BN = 64;
 constexpr int kThreads = 256;
+// anchored factors beyond 2^+-kSpanExact switch the diagonal tile to pairs
+constexpr float kSpanExact = 60.f;
 
 struct TileGeom {
   int seq, blk;
@@ -48,23 +56,53 @@ __device__ __forceinline__ bool visible(int i, int j, int window) {
   return j <= i && (window <= 0 || i - j < window);
 }
 
+// Work item -> (sequence, 64-row block, query head).  The kernels run a
+// persistent grid over items; with a unit mask only the items of flagged
+// (sequence, head) units are taken.  `reverse` hands out the last blocks of
+// the flat order first (the longest query blocks of a causal problem).
+__device__ __forceinline__ bool simt_item(const AttnProblem& pb, int item, bool reverse,
+                                          int& seq, int& blk, int& h) {
+  h = item % pb.HQ;
+  const int b = item / pb.HQ;
+  if (!seq_block(pb.seqs, BM, reverse ? pb.max_blocks64 - 1 - b : b, seq, blk)) return false;
+  return pb.units == nullptr || pb.units[(long)seq * pb.HQ + h] != 0;
+}
+
+// dst[r][n] = src[row0+r, src_head, n] * exp2(sign * (P[row0+r, h, n] - R[n]))
+// for sign = +1 or -1, or the raw element for sign = 0.  Returns true (in this
+// thread) when some loaded |P - R| exceeds kSpanExact.
 template <typename T, int KD>
-__device__ __forceinline__ void load_rows_anchored(float* dst, const T* src, const float* P,
+__device__ __forceinline__ bool load_rows_anchored(float* dst, const T* src, const float* P,
                                                    const float* R, long row0, int nrows,
                                                    int nmax, int src_heads, int src_head,
-                                                   int HQ, int h, int K, float sign) {
-  // dst[r][n] = src[row0+r, src_head, n] * exp2(sign * (P[row0+r, h, n] - R[n]))
+                                                   int HQ, int h, int K, int sign) {
+  bool wide = false;
   for (int e = threadIdx.x; e < nmax * KD; e += kThreads) {
     const int r = e / KD, n = e % KD;
     float val = 0.f;
     if (r < nrows && n < K) {
       const long row = row0 + r;
-      const float x = to_f32(src[(row * src_heads + src_head) * (long)K + n]);
-      const float p = P[(row * HQ + h) * (long)K + n];
-      val = x * exp2f(sign * (p - R[n]));
+      val = to_f32(src[(row * src_heads + src_head) * (long)K + n]);
+      if (sign != 0) {
+        const float d = P[(row * HQ + h) * (long)K + n] - R[n];
+        wide |= fabsf(d) > kSpanExact;
+        val *= exp2f(sign > 0 ? d : -d);
+      }
     }
     dst[r * (KD + 1) + n] = val;
   }
+  return wide;
+}
+
+// sum_n x_n y_n 2^(pa_n - pb_n) over the K channels of two rows, x from
+// shared memory (stride 1) and y, pa, pb from global memory: one pair of the
+// diagonal tile evaluated without an anchor.
+template <typename T>
+__device__ __forceinline__ float exact_dot(const float* xs, const T* y, const float* pa,
+                                           const float* pb, int K) {
+  float acc = 0.f;
+  for (int n = 0; n < K; ++n) acc += xs[n] * to_f32(y[n]) * exp2f(pa[n] - pb[n]);
+  return acc;
 }
 
 template <typename T, int VD, int PAD>
@@ -82,8 +120,8 @@ __device__ __forceinline__ void load_rows_plain(float* dst, const T* src, long r
 // forward
 
 template <typename T, int KD, int VD>
-__global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdArgs a) {
-  extern __shared__ float sm[];
+__device__ __forceinline__ void fwd_simt_block(const AttnProblem& pb, const FwdArgs& a, float* sm,
+                                               int seq, int blk, int h) {
   float* qt = sm;                      // [BM][KD+1]
   float* kt = qt + BM * (KD + 1);      // [BN][KD+1]
   float* vs = kt + BN * (KD + 1);      // [BN][VD]
@@ -92,10 +130,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
   float* gsq = R + KD;                 // [BM]
   float* gsk = gsq + BM;               // [BN]
 
-  const int h = blockIdx.y;
   const int kh = h / (pb.HQ / pb.H);
-  int seq, blk;
-  if (!seq_block(pb.seqs, BM, blockIdx.x, seq, blk)) return;
   const long s0 = pb.seqs.start(seq);
   const int L = pb.seqs.len(seq);
   const int i0 = blk * BM;
@@ -108,9 +143,11 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
   for (int n = threadIdx.x; n < KD; n += kThreads)
     R[n] = n < K ? a.P[((s0 + i0) * HQ + h) * (long)K + n] : 0.f;
   __syncthreads();
-  load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K, 1.f);
+  const bool wide = load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K, 1);
   for (int r = threadIdx.x; r < BM; r += kThreads)
     gsq[r] = (a.GS && r < ni) ? a.GS[(s0 + i0 + r) * HQ + h] : 0.f;
+  // every thread's flag reaches the whole CTA (this also orders the loads)
+  const bool exact = __syncthreads_or(wide) != 0;
 
   const int row = threadIdx.x / 4, sub = threadIdx.x % 4;
   float m = -INFINITY, l = 0.f;
@@ -121,11 +158,15 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
   const int jlast = i0 + ni - 1;
   const int jfirst = pb.window > 0 ? max(0, i0 - pb.window + 1) : 0;
   const float sl2 = pb.scale * kLog2e;
+  const long qrow = (s0 + i0 + min(row, ni - 1)) * HQ + h;
   for (int jb = jfirst / BN; jb <= jlast / BN; ++jb) {
     const int j0 = jb * BN;
     const int nj = min(BN, L - j0);
+    // the diagonal tile of a wide block: raw keys, pair-by-pair decay
+    const bool pairwise = exact && j0 == i0;
     __syncthreads();
-    load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K, -1.f);
+    load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K,
+                              pairwise ? 0 : -1);
     load_rows_plain<T, VD, 0>(vs, v, s0 + j0, nj, BN, pb.H, kh, V);
     for (int r = threadIdx.x; r < BN; r += kThreads)
       gsk[r] = (a.GS && r < nj) ? a.GS[(s0 + j0 + r) * HQ + h] : 0.f;
@@ -134,10 +175,19 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
     float sc[BN / 4];
 #pragma unroll
     for (int jj = 0; jj < BN / 4; ++jj) sc[jj] = 0.f;
-    for (int n = 0; n < KD; ++n) {
-      const float qv = qt[row * (KD + 1) + n];
+    if (!pairwise) {
+      for (int n = 0; n < KD; ++n) {
+        const float qv = qt[row * (KD + 1) + n];
 #pragma unroll
-      for (int jj = 0; jj < BN / 4; ++jj) sc[jj] += qv * kt[(sub + 4 * jj) * (KD + 1) + n];
+        for (int jj = 0; jj < BN / 4; ++jj) sc[jj] += qv * kt[(sub + 4 * jj) * (KD + 1) + n];
+      }
+    } else {
+#pragma unroll 1
+      for (int jj = 0; jj < BN / 4; ++jj) {
+        const int jl = min(sub + 4 * jj, nj - 1);
+        sc[jj] = exact_dot(kt + jl * (KD + 1), q + qrow * K, a.P + qrow * K,
+                           a.P + ((s0 + j0 + jl) * HQ + h) * (long)K, K);
+      }
     }
     const int i = i0 + row;
     float mt = -INFINITY;
@@ -193,12 +243,34 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
   }
 }
 
-// ---------------------------------------------------------------------------
-// backward, query side: D_i, dq, row part of the scalar-gate gradient, dsink
+// With a unit mask, nothing to do unless some unit is flagged: the mask's
+// last word (after the n_seq * HQ unit words) is set with any of them.
+__device__ __forceinline__ bool no_flagged_units(const AttnProblem& pb) {
+  return pb.units != nullptr &&
+         !__syncthreads_or(threadIdx.x == 0 && pb.units[(long)pb.seqs.n * pb.HQ] != 0);
+}
 
 template <typename T, int KD, int VD>
-__global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, BwdArgs a) {
+__global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdArgs a) {
   extern __shared__ float sm[];
+  if (no_flagged_units(pb)) return;
+  const int n_items = pb.max_blocks64 * pb.HQ;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int seq, blk, h;
+    if (!simt_item(pb, item, true, seq, blk, h)) continue;  // uniform in the CTA
+    __syncthreads();  // the previous item's shared-memory reads are done
+    fwd_simt_block<T, KD, VD>(pb, a, sm, seq, blk, h);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// backward, query side: D_i, dq, row part of the scalar-gate gradient, dsink
+// (with a unit mask: dq only; D, the row part and dsink come from the
+// tensor-core path's own pass)
+
+template <typename T, int KD, int VD>
+__device__ __forceinline__ void bwd_dq_simt_block(const AttnProblem& pb, const BwdArgs& a,
+                                                  float* sm, int seq, int blk, int h) {
   float* qt = sm;                      // [BM][KD+1]
   float* kt = qt + BM * (KD + 1);      // [BN][KD+1]
   float* vs = kt + BN * (KD + 1);      // [BN][VD+1]
@@ -210,10 +282,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
   float* lse2 = gsk + BN;              // [BM]
   float* Dv = lse2 + BM;               // [BM]
 
-  const int h = blockIdx.y;
+  const bool own_rows = pb.units == nullptr;
   const int kh = h / (pb.HQ / pb.H);
-  int seq, blk;
-  if (!seq_block(pb.seqs, BM, blockIdx.x, seq, blk)) return;
   const long s0 = pb.seqs.start(seq);
   const int L = pb.seqs.len(seq);
   const int i0 = blk * BM;
@@ -228,13 +298,13 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
   for (int n = threadIdx.x; n < KD; n += kThreads)
     R[n] = n < K ? a.P[((s0 + i0) * HQ + h) * (long)K + n] : 0.f;
   __syncthreads();
-  load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K, 1.f);
+  const bool wide = load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K, 1);
   load_rows_plain<T, VD, 1>(dOs, dO, s0 + i0, ni, BM, HQ, h, V);
   for (int r = threadIdx.x; r < BM; r += kThreads) {
     gsq[r] = (a.GS && r < ni) ? a.GS[(s0 + i0 + r) * HQ + h] : 0.f;
     lse2[r] = r < ni ? a.lse[(s0 + i0 + r) * HQ + h] * kLog2e : 0.f;
   }
-  __syncthreads();
+  const bool exact = __syncthreads_or(wide) != 0;
   const int row = threadIdx.x / 4, sub = threadIdx.x % 4;
   {  // D_i = dO_i . o_i
     float d = 0.f;
@@ -244,10 +314,10 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
     d = warp4_sum(d);
     if (sub == 0) {
       Dv[row] = d;
-      if (row < ni) a.D[(s0 + i0 + row) * HQ + h] = d;
+      if (own_rows && row < ni) a.D[(s0 + i0 + row) * HQ + h] = d;
     }
     // dsink_h = -sum_i exp(sink_h - lse_i) D_i (the sink's value row is zero)
-    if (a.sink && a.dsink) {
+    if (own_rows && a.sink && a.dsink) {
       float contrib = (sub == 0 && row < ni) ? -exp2f(a.sink[h] * kLog2e - lse2[row]) * d : 0.f;
       for (int off = 16; off > 0; off >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, off);
       if ((threadIdx.x & 31) == 0) atomicAdd(&a.dsink[h], contrib);
@@ -258,16 +328,22 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
   float dqa[KD / 4];
 #pragma unroll
   for (int c = 0; c < KD / 4; ++c) dqa[c] = 0.f;
+  float dqe[KD / 4];  // the diagonal tile's pairwise terms of a wide block
+#pragma unroll
+  for (int c = 0; c < KD / 4; ++c) dqe[c] = 0.f;
   double rowsum = 0.0;  // fp64: the scalar-gate gradient sums many cancelling terms
   const float Di = Dv[row];
   const int jlast = i0 + ni - 1;
   const int jfirst = pb.window > 0 ? max(0, i0 - pb.window + 1) : 0;
   const float sl2 = pb.scale * kLog2e;
+  const long qrow = (s0 + i0 + min(row, ni - 1)) * HQ + h;
   for (int jb = jfirst / BN; jb <= jlast / BN; ++jb) {
     const int j0 = jb * BN;
     const int nj = min(BN, L - j0);
+    const bool pairwise = exact && j0 == i0;
     __syncthreads();
-    load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K, -1.f);
+    load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K,
+                              pairwise ? 0 : -1);
     load_rows_plain<T, VD, 1>(vs, v, s0 + j0, nj, BN, pb.H, kh, V);
     for (int r = threadIdx.x; r < BN; r += kThreads)
       gsk[r] = (a.GS && r < nj) ? a.GS[(s0 + j0 + r) * HQ + h] : 0.f;
@@ -275,10 +351,19 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
     float sc[BN / 4], dp[BN / 4];
 #pragma unroll
     for (int jj = 0; jj < BN / 4; ++jj) sc[jj] = dp[jj] = 0.f;
-    for (int n = 0; n < KD; ++n) {
-      const float qv = qt[row * (KD + 1) + n];
+    if (!pairwise) {
+      for (int n = 0; n < KD; ++n) {
+        const float qv = qt[row * (KD + 1) + n];
 #pragma unroll
-      for (int jj = 0; jj < BN / 4; ++jj) sc[jj] += qv * kt[(sub + 4 * jj) * (KD + 1) + n];
+        for (int jj = 0; jj < BN / 4; ++jj) sc[jj] += qv * kt[(sub + 4 * jj) * (KD + 1) + n];
+      }
+    } else {
+#pragma unroll 1
+      for (int jj = 0; jj < BN / 4; ++jj) {
+        const int jl = min(sub + 4 * jj, nj - 1);
+        sc[jj] = exact_dot(kt + jl * (KD + 1), q + qrow * K, a.P + qrow * K,
+                           a.P + ((s0 + j0 + jl) * HQ + h) * (long)K, K);
+      }
     }
     for (int c = 0; c < VD; ++c) {
       const float dv_ = dOs[row * (VD + 1) + c];
@@ -300,25 +385,51 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
       Ss[row * (BN + 1) + jl] = ds;
     }
     __syncwarp();
-    for (int j = 0; j < BN; ++j) {
-      const float ds = Ss[row * (BN + 1) + j];
+    if (!pairwise) {
+      for (int j = 0; j < BN; ++j) {
+        const float ds = Ss[row * (BN + 1) + j];
 #pragma unroll
-      for (int c = 0; c < KD / 4; ++c) dqa[c] += ds * kt[j * (KD + 1) + sub + 4 * c];
+        for (int c = 0; c < KD / 4; ++c) dqa[c] += ds * kt[j * (KD + 1) + sub + 4 * c];
+      }
+    } else {
+      // dq_in += dS_ij k_jn 2^(P_in - P_jn), pair by pair
+      for (int j = 0; j < nj; ++j) {
+        const float ds = Ss[row * (BN + 1) + j];
+        if (ds == 0.f) continue;
+        const float* pj = a.P + ((s0 + j0 + j) * HQ + h) * (long)K;
+#pragma unroll
+        for (int c = 0; c < KD / 4; ++c) {
+          const int n = sub + 4 * c;
+          if (n < K)
+            dqe[c] += ds * kt[j * (KD + 1) + n] * exp2f(a.P[qrow * K + n] - pj[n]);
+        }
+      }
     }
   }
   rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 1);
   rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 2);
   if (row < ni) {
-    const long qrow = (s0 + i0 + row) * HQ + h;
 #pragma unroll
     for (int c = 0; c < KD / 4; ++c) {
       const int n = sub + 4 * c;
       if (n < K) {
         const float f = exp2f(a.P[qrow * K + n] - R[n]);
-        a.dq32[qrow * K + n] = pb.scale * f * dqa[c];
+        a.dq32[qrow * K + n] = pb.scale * (f * dqa[c] + dqe[c]);
       }
     }
-    if (sub == 0) a.dgs_row[qrow] = (float)rowsum;
+    if (own_rows && sub == 0) a.dgs_row[qrow] = (float)rowsum;
+  }
+}
+
+template <typename T, int KD, int VD>
+__global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, BwdArgs a) {
+  extern __shared__ float sm[];
+  const int n_items = pb.max_blocks64 * pb.HQ;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int seq, blk, h;
+    if (!simt_item(pb, item, true, seq, blk, h)) continue;  // uniform in the CTA
+    __syncthreads();
+    bwd_dq_simt_block<T, KD, VD>(pb, a, sm, seq, blk, h);
   }
 }
 
@@ -327,8 +438,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_simt_kernel(AttnProblem pb, B
 // scalar-gate gradient
 
 template <typename T, int KD, int VD>
-__global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb, BwdArgs a) {
-  extern __shared__ float sm[];
+__device__ __forceinline__ void bwd_dkdv_simt_block(const AttnProblem& pb, const BwdArgs& a,
+                                                    float* sm, int seq, int blk, int h) {
   float* kt = sm;                      // [BN][KD+1]
   float* vs = kt + BN * (KD + 1);      // [BN][VD+1]
   float* qt = vs + BN * (VD + 1);      // [BM][KD+1]
@@ -341,10 +452,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
   float* lse2 = gsk + BN;              // [BM]
   float* Dv = lse2 + BM;               // [BM]
 
-  const int h = blockIdx.y;
   const int kh = h / (pb.HQ / pb.H);
-  int seq, blk;
-  if (!seq_block(pb.seqs, BN, blockIdx.x, seq, blk)) return;
   const long s0 = pb.seqs.start(seq);
   const int L = pb.seqs.len(seq);
   const int j0 = blk * BN;
@@ -355,18 +463,23 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
   const T* v = static_cast<const T*>(a.v);
   const T* dO = static_cast<const T*>(a.dO);
 
+  // the anchor at the block's last key row: every later query lies past it
   for (int n = threadIdx.x; n < KD; n += kThreads)
-    R[n] = n < K ? a.P[((s0 + j0) * HQ + h) * (long)K + n] : 0.f;
+    R[n] = n < K ? a.P[((s0 + j0 + nj - 1) * HQ + h) * (long)K + n] : 0.f;
   __syncthreads();
-  load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K, -1.f);
+  const bool wide =
+      load_rows_anchored<T, KD>(kt, k, a.P, R, s0 + j0, nj, BN, pb.H, kh, HQ, h, K, -1);
   load_rows_plain<T, VD, 1>(vs, v, s0 + j0, nj, BN, pb.H, kh, V);
   for (int r = threadIdx.x; r < BN; r += kThreads)
     gsk[r] = (a.GS && r < nj) ? a.GS[(s0 + j0 + r) * HQ + h] : 0.f;
+  const bool exact = __syncthreads_or(wide) != 0;
 
   const int jr = threadIdx.x / 4, sub = threadIdx.x % 4;
-  float dka[KD / 4], dva[VD / 4];
+  const long krow = (s0 + j0 + min(jr, nj - 1)) * HQ + h;
+  const T* kraw = k + ((s0 + j0 + min(jr, nj - 1)) * pb.H + kh) * (long)K;
+  float dka[KD / 4], dva[VD / 4], dke[KD / 4];
 #pragma unroll
-  for (int c = 0; c < KD / 4; ++c) dka[c] = 0.f;
+  for (int c = 0; c < KD / 4; ++c) dka[c] = dke[c] = 0.f;
 #pragma unroll
   for (int c = 0; c < VD / 4; ++c) dva[c] = 0.f;
   double colsum = 0.0;  // fp64, as the row sums
@@ -376,8 +489,10 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
   for (int ib = j0 / BM; ib <= ilast / BM; ++ib) {
     const int i0 = ib * BM;
     const int ni = min(BM, L - i0);
+    const bool pairwise = exact && i0 == j0;
     __syncthreads();
-    load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K, 1.f);
+    load_rows_anchored<T, KD>(qt, q, a.P, R, s0 + i0, ni, BM, HQ, h, HQ, h, K,
+                              pairwise ? 0 : 1);
     load_rows_plain<T, VD, 1>(dOs, dO, s0 + i0, ni, BM, HQ, h, V);
     for (int r = threadIdx.x; r < BM; r += kThreads) {
       const bool in = r < ni;
@@ -389,10 +504,19 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
     float sc[BM / 4], dp[BM / 4];
 #pragma unroll
     for (int ii = 0; ii < BM / 4; ++ii) sc[ii] = dp[ii] = 0.f;
-    for (int n = 0; n < KD; ++n) {
-      const float kv_ = kt[jr * (KD + 1) + n];
+    if (!pairwise) {
+      for (int n = 0; n < KD; ++n) {
+        const float kv_ = kt[jr * (KD + 1) + n];
 #pragma unroll
-      for (int ii = 0; ii < BM / 4; ++ii) sc[ii] += kv_ * qt[(sub + 4 * ii) * (KD + 1) + n];
+        for (int ii = 0; ii < BM / 4; ++ii) sc[ii] += kv_ * qt[(sub + 4 * ii) * (KD + 1) + n];
+      }
+    } else {
+#pragma unroll 1
+      for (int ii = 0; ii < BM / 4; ++ii) {
+        const int il = min(sub + 4 * ii, ni - 1);
+        sc[ii] = exact_dot(qt + il * (KD + 1), kraw,
+                           a.P + ((s0 + i0 + il) * HQ + h) * (long)K, a.P + krow * K, K);
+      }
     }
     for (int c = 0; c < VD; ++c) {
       const float vv = vs[jr * (VD + 1) + c];
@@ -415,25 +539,41 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
       dSs[jr * (BM + 1) + il] = ds;
     }
     __syncwarp();
-    for (int i = 0; i < BM; ++i) {
-      const float p = Ps[jr * (BM + 1) + i];
-      const float ds = dSs[jr * (BM + 1) + i];
+    if (!pairwise) {
+      for (int i = 0; i < BM; ++i) {
+        const float p = Ps[jr * (BM + 1) + i];
+        const float ds = dSs[jr * (BM + 1) + i];
 #pragma unroll
-      for (int c = 0; c < VD / 4; ++c) dva[c] += p * dOs[i * (VD + 1) + sub + 4 * c];
+        for (int c = 0; c < VD / 4; ++c) dva[c] += p * dOs[i * (VD + 1) + sub + 4 * c];
 #pragma unroll
-      for (int c = 0; c < KD / 4; ++c) dka[c] += ds * qt[i * (KD + 1) + sub + 4 * c];
+        for (int c = 0; c < KD / 4; ++c) dka[c] += ds * qt[i * (KD + 1) + sub + 4 * c];
+      }
+    } else {
+      // dk_jn += dS_ij q_in 2^(P_in - P_jn), pair by pair
+      for (int i = 0; i < ni; ++i) {
+        const float p = Ps[jr * (BM + 1) + i];
+        const float ds = dSs[jr * (BM + 1) + i];
+#pragma unroll
+        for (int c = 0; c < VD / 4; ++c) dva[c] += p * dOs[i * (VD + 1) + sub + 4 * c];
+        if (ds == 0.f) continue;
+        const float* pi = a.P + ((s0 + i0 + i) * HQ + h) * (long)K;
+#pragma unroll
+        for (int c = 0; c < KD / 4; ++c) {
+          const int n = sub + 4 * c;
+          if (n < K) dke[c] += ds * qt[i * (KD + 1) + n] * exp2f(pi[n] - a.P[krow * K + n]);
+        }
+      }
     }
   }
   colsum += __shfl_xor_sync(0xffffffffu, colsum, 1);
   colsum += __shfl_xor_sync(0xffffffffu, colsum, 2);
   if (jr < nj) {
-    const long krow = (s0 + j0 + jr) * HQ + h;
 #pragma unroll
     for (int c = 0; c < KD / 4; ++c) {
       const int n = sub + 4 * c;
       if (n < K) {
         const float f = exp2f(R[n] - a.P[krow * K + n]);
-        a.dkh32[krow * K + n] = pb.scale * f * dka[c];
+        a.dkh32[krow * K + n] = pb.scale * (f * dka[c] + dke[c]);
       }
     }
 #pragma unroll
@@ -443,6 +583,39 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb,
     }
     // the logit carries -GS_j for key j
     if (sub == 0) a.dgs_col[krow] = (float)-colsum;
+  }
+}
+
+template <typename T, int KD, int VD>
+__global__ void __launch_bounds__(kThreads) bwd_dkdv_simt_kernel(AttnProblem pb, BwdArgs a) {
+  extern __shared__ float sm[];
+  const int n_items = pb.max_blocks64 * pb.HQ;
+  // the first key blocks of a causal problem see the most query tiles
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int seq, blk, h;
+    if (!simt_item(pb, item, false, seq, blk, h)) continue;  // uniform in the CTA
+    __syncthreads();
+    bwd_dkdv_simt_block<T, KD, VD>(pb, a, sm, seq, blk, h);
+  }
+}
+
+// The masked units' whole backward in one launch: the key-side items (dk^(h),
+// dv^(h), column sums) and the query-side items (dq), which read nothing the
+// other writes.
+template <typename T, int KD, int VD>
+__global__ void __launch_bounds__(kThreads) bwd_units_simt_kernel(AttnProblem pb, BwdArgs a) {
+  extern __shared__ float sm[];
+  if (no_flagged_units(pb)) return;
+  const int n1 = pb.max_blocks64 * pb.HQ;
+  for (int item = blockIdx.x; item < 2 * n1; item += gridDim.x) {
+    int seq, blk, h;
+    const bool key_side = item < n1;
+    if (!simt_item(pb, key_side ? item : item - n1, !key_side, seq, blk, h)) continue;
+    __syncthreads();
+    if (key_side)
+      bwd_dkdv_simt_block<T, KD, VD>(pb, a, sm, seq, blk, h);
+    else
+      bwd_dq_simt_block<T, KD, VD>(pb, a, sm, seq, blk, h);
   }
 }
 
@@ -493,65 +666,134 @@ __global__ void bwd_reduce_kernel(AttnProblem pb, BwdArgs a, T* dq, T* dk, T* dv
   }
 }
 
+// A persistent grid: every SM holds as many CTAs as its shared memory allows
+// (cached per device and kernel), never more CTAs than work items.
+template <typename F>
+int persistent_grid(F kernel, size_t smem, int n_items, int (&bps)[kMaxDevices]) {
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  if (bps[dev] == 0) {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, smem) != cudaSuccess)
+      return -1;
+    bps[dev] = b < 1 ? 1 : b;
+  }
+  const long g = 148L * bps[dev];
+  return (int)(n_items < g ? n_items : g);
+}
+
 template <typename T, int KD, int VD>
 int launch_fwd(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(float) * (size_t)(BM * (KD + 1) + BN * (KD + 1) + BN * VD +
                                                BM * (BN + 1) + KD + BM + BN);
   static bool attr[kMaxDevices] = {};
+  static int bps[kMaxDevices] = {};
   if (!set_max_smem_once(fwd_simt_kernel<T, KD, VD>, (int)smem, attr)) return WALL_ERR_CUDA;
-  dim3 grid(pb.max_blocks64, pb.HQ);
+  const int grid = persistent_grid(fwd_simt_kernel<T, KD, VD>, smem, pb.max_blocks64 * pb.HQ, bps);
+  if (grid < 0) return WALL_ERR_CUDA;
   fwd_simt_kernel<T, KD, VD><<<grid, kThreads, smem, stream>>>(pb, a);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
 template <typename T, int KD, int VD>
-int launch_bwd(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
+int launch_bwd_dq(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
+  const size_t smem = sizeof(float) * (size_t)(2 * BM * (KD + 1) + BN * (VD + 1) +
+                                               BM * (VD + 1) + BM * (BN + 1) + KD + 4 * BM);
+  static bool attr[kMaxDevices] = {};
+  static int bps[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_dq_simt_kernel<T, KD, VD>, (int)smem, attr)) return WALL_ERR_CUDA;
+  const int grid =
+      persistent_grid(bwd_dq_simt_kernel<T, KD, VD>, smem, pb.max_blocks64 * pb.HQ, bps);
+  if (grid < 0) return WALL_ERR_CUDA;
+  bwd_dq_simt_kernel<T, KD, VD><<<grid, kThreads, smem, stream>>>(pb, a);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+template <typename T, int KD, int VD>
+int launch_bwd_dkdv(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
+  const size_t smem = sizeof(float) * (size_t)(BN * (KD + 1) + BN * (VD + 1) + BM * (KD + 1) +
+                                               BM * (VD + 1) + 2 * BN * (BM + 1) + KD + 4 * BM);
+  static bool attr[kMaxDevices] = {};
+  static int bps[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_dkdv_simt_kernel<T, KD, VD>, (int)smem, attr)) return WALL_ERR_CUDA;
+  const int grid =
+      persistent_grid(bwd_dkdv_simt_kernel<T, KD, VD>, smem, pb.max_blocks64 * pb.HQ, bps);
+  if (grid < 0) return WALL_ERR_CUDA;
+  bwd_dkdv_simt_kernel<T, KD, VD><<<grid, kThreads, smem, stream>>>(pb, a);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
+template <typename T, int KD, int VD>
+int launch_bwd_units(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
   const size_t smem_dq = sizeof(float) * (size_t)(2 * BM * (KD + 1) + BN * (VD + 1) +
                                                   BM * (VD + 1) + BM * (BN + 1) + KD + 4 * BM);
   const size_t smem_dk = sizeof(float) * (size_t)(BN * (KD + 1) + BN * (VD + 1) +
                                                   BM * (KD + 1) + BM * (VD + 1) +
                                                   2 * BN * (BM + 1) + KD + 4 * BM);
-  static bool attr_dq[kMaxDevices] = {}, attr_dk[kMaxDevices] = {};
-  if (!set_max_smem_once(bwd_dq_simt_kernel<T, KD, VD>, (int)smem_dq, attr_dq) ||
-      !set_max_smem_once(bwd_dkdv_simt_kernel<T, KD, VD>, (int)smem_dk, attr_dk))
-    return WALL_ERR_CUDA;
-  dim3 grid(pb.max_blocks64, pb.HQ);
-  bwd_dq_simt_kernel<T, KD, VD><<<grid, kThreads, smem_dq, stream>>>(pb, a);
-  if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
-  bwd_dkdv_simt_kernel<T, KD, VD><<<grid, kThreads, smem_dk, stream>>>(pb, a);
+  const size_t smem = smem_dq > smem_dk ? smem_dq : smem_dk;
+  static bool attr[kMaxDevices] = {};
+  static int bps[kMaxDevices] = {};
+  if (!set_max_smem_once(bwd_units_simt_kernel<T, KD, VD>, (int)smem, attr)) return WALL_ERR_CUDA;
+  const int grid =
+      persistent_grid(bwd_units_simt_kernel<T, KD, VD>, smem, 2 * pb.max_blocks64 * pb.HQ, bps);
+  if (grid < 0) return WALL_ERR_CUDA;
+  bwd_units_simt_kernel<T, KD, VD><<<grid, kThreads, smem, stream>>>(pb, a);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
-template <typename T>
-int fwd_dispatch(const AttnProblem& pb, const FwdArgs& a, cudaStream_t s) {
-  const bool k64 = pb.K <= 64, v64 = pb.V <= 64;
-  if (k64 && v64) return launch_fwd<T, 64, 64>(pb, a, s);
-  if (k64) return launch_fwd<T, 64, 128>(pb, a, s);
-  if (v64) return launch_fwd<T, 128, 64>(pb, a, s);
-  return launch_fwd<T, 128, 128>(pb, a, s);
-}
+// the kernel template for the problem's head sizes (64 or 128 columns)
+#define WALL_SIMT_DISPATCH(LAUNCH, T, pb, ...)                            \
+  ((pb).K <= 64 ? ((pb).V <= 64 ? LAUNCH<T, 64, 64>(pb, __VA_ARGS__)     \
+                                : LAUNCH<T, 64, 128>(pb, __VA_ARGS__))   \
+                : ((pb).V <= 64 ? LAUNCH<T, 128, 64>(pb, __VA_ARGS__)    \
+                                : LAUNCH<T, 128, 128>(pb, __VA_ARGS__)))
 
-template <typename T>
-int bwd_dispatch(const AttnProblem& pb, const BwdArgs& a, cudaStream_t s) {
-  const bool k64 = pb.K <= 64, v64 = pb.V <= 64;
-  if (k64 && v64) return launch_bwd<T, 64, 64>(pb, a, s);
-  if (k64) return launch_bwd<T, 64, 128>(pb, a, s);
-  if (v64) return launch_bwd<T, 128, 64>(pb, a, s);
-  return launch_bwd<T, 128, 128>(pb, a, s);
+int fwd_any(const AttnProblem& pb, const FwdArgs& a, cudaStream_t s) {
+  return pb.dtype == WALL_BF16 ? WALL_SIMT_DISPATCH(launch_fwd, __nv_bfloat16, pb, a, s)
+                               : WALL_SIMT_DISPATCH(launch_fwd, float, pb, a, s);
 }
+int bwd_dq_any(const AttnProblem& pb, const BwdArgs& a, cudaStream_t s) {
+  return pb.dtype == WALL_BF16 ? WALL_SIMT_DISPATCH(launch_bwd_dq, __nv_bfloat16, pb, a, s)
+                               : WALL_SIMT_DISPATCH(launch_bwd_dq, float, pb, a, s);
+}
+int bwd_dkdv_any(const AttnProblem& pb, const BwdArgs& a, cudaStream_t s) {
+  return pb.dtype == WALL_BF16 ? WALL_SIMT_DISPATCH(launch_bwd_dkdv, __nv_bfloat16, pb, a, s)
+                               : WALL_SIMT_DISPATCH(launch_bwd_dkdv, float, pb, a, s);
+}
+int bwd_units_any(const AttnProblem& pb, const BwdArgs& a, cudaStream_t s) {
+  return pb.dtype == WALL_BF16 ? WALL_SIMT_DISPATCH(launch_bwd_units, __nv_bfloat16, pb, a, s)
+                               : WALL_SIMT_DISPATCH(launch_bwd_units, float, pb, a, s);
+}
+#undef WALL_SIMT_DISPATCH
 
 }  // namespace
 
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream) {
   if (pb.max_blocks64 == 0) return WALL_OK;
-  return pb.dtype == WALL_BF16 ? fwd_dispatch<__nv_bfloat16>(pb, a, stream)
-                               : fwd_dispatch<float>(pb, a, stream);
+  return fwd_any(pb, a, stream);
 }
 
 int attn_bwd_simt(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
   if (pb.max_blocks64 == 0) return WALL_OK;
-  return pb.dtype == WALL_BF16 ? bwd_dispatch<__nv_bfloat16>(pb, a, stream)
-                               : bwd_dispatch<float>(pb, a, stream);
+  // dkdv reads the D the dq kernel writes
+  const int rc = bwd_dq_any(pb, a, stream);
+  return rc ? rc : bwd_dkdv_any(pb, a, stream);
+}
+
+int attn_fwd_simt_units(const AttnProblem& pb, const FwdArgs& a, const int* units,
+                        cudaStream_t stream) {
+  if (pb.max_blocks64 == 0) return WALL_OK;
+  AttnProblem p = pb;
+  p.units = units;
+  return fwd_any(p, a, stream);
+}
+
+int attn_bwd_simt_units(const AttnProblem& pb, const BwdArgs& a, const int* units,
+                        cudaStream_t stream) {
+  if (pb.max_blocks64 == 0) return WALL_OK;
+  AttnProblem p = pb;
+  p.units = units;
+  return bwd_units_any(p, a, stream);
 }
 
 int attn_bwd_reduce(const AttnProblem& pb, const BwdArgs& a, void* dq, void* dk, void* dv,

@@ -38,6 +38,21 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// The anchored operands of a unit beyond the anchored range are recomputed
+// elsewhere, but the tensor-core kernels still read them (a key tile that
+// runs past its sequence reads the next one's rows, with zero weight):
+// clamped into the finite bf16 range, 0 times such a value stays 0.  Inside
+// the range the clamp never acts.
+__device__ __forceinline__ float saturate_bf16(float x) {
+  return fminf(fmaxf(x, -3.3895313892515355e38f), 3.3895313892515355e38f);
+}
+
+// Sets a flag word that many threads may find set: the word is read first,
+// so once it is set the threads that see it cost a load, not an atomic.
+__device__ __forceinline__ void set_flag(int* f) {
+  if (*reinterpret_cast<volatile int*>(f) == 0) atomicOr(f, 1);
+}
+
 // ---------------------------------------------------------------------------
 // element conversion
 
@@ -130,5 +145,49 @@ __device__ __forceinline__ bool seq_block(const Seqs& S, int bs, int flat, int& 
 }
 
 inline int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+// Where the tensor-core backward keeps its dS tiles (128 x 128, bf16).  A
+// query block I of a sequence sees key blocks J in [jlo(I), I]: every block
+// before it without a window, else the wb blocks a window of W keys reaches
+// back, wb = ceil((W - 1) / 128).  A (sequence, head) stores its tiles row by
+// row, tile (I, J) at rowstart(I) + J - jlo(I); the (sequence, head) pairs
+// follow each other sequence-major: pair (s, h) starts at
+// HQ * (tiles of the sequences before s) + h * tiles(nb(s)).
+struct DsLayout {
+  int wb;  // key blocks reached back beyond the query block; 1 << 28: no window
+  __host__ __device__ static DsLayout of_window(int window) {
+    DsLayout d;
+    d.wb = window > 0 ? (window - 1 + 127) / 128 : (1 << 28);
+    return d;
+  }
+  __host__ __device__ int jlo(int I) const { return I > wb ? I - wb : 0; }
+  // tiles of the query blocks before I: sum over I' < I of min(I', wb) + 1
+  __host__ __device__ long rowstart(int I) const {
+    const long i = I, w = wb;
+    return i <= w + 1 ? i * (i + 1) / 2 : (w + 1) * (w + 2) / 2 + (i - w - 1) * (w + 1);
+  }
+  __host__ __device__ long tiles(int nb) const { return rowstart(nb); }
+  // first tile of (sequence s, head h)
+  __device__ long pair_base(const Seqs& seqs, int HQ, int s, int h) const {
+    long before = 0;
+    int nb;
+    if (!seqs.cu) {
+      nb = (seqs.T + 127) / 128;
+      before = (long)s * tiles(nb);
+    } else {
+      for (int x = 0; x < s; ++x) before += tiles((seqs.len(x) + 127) / 128);
+      nb = (seqs.len(s) + 127) / 128;
+    }
+    return before * HQ + (long)h * tiles(nb);
+  }
+  // tiles of a whole problem: dense (B sequences of T rows), or a bound for
+  // n_seq packed sequences of `rows` rows in all (a sequence's tiles grow
+  // faster than its blocks, so one sequence holding every block is the most)
+  __host__ static long total(const DsLayout& d, long rows, int T, int B, int HQ,
+                             int n_seq_varlen) {
+    if (n_seq_varlen > 0) return (long)HQ * d.tiles((int)((rows + 127) / 128) + n_seq_varlen);
+    return (long)B * HQ * d.tiles((T + 127) / 128);
+  }
+};
 
 }  // namespace wall

@@ -28,10 +28,14 @@ namespace {
 using namespace sm100;
 using T_bf16 = __nv_bfloat16;
 
+// k_tilde = k * 2^(R_c - P) and r_cache = P at chunk starts (README
+// "Decode").  A chunk whose gate sums past 2^kAnchorRange from its first row
+// leaves k_tilde outside the range the decode reads it in: that records
+// WALL_ERR_RANGE in `status` (the layout has no other place for the row).
 template <typename T>
 __global__ void cache_kernel(const T* __restrict__ k, const float* __restrict__ P, int B, int Tn,
                              int H, int HQ, int K, int C, int t0, T* __restrict__ kt,
-                             float* __restrict__ rc, int Tcap) {
+                             float* __restrict__ rc, int Tcap, int* status) {
   const int G = HQ / H;
   const int NC = (Tcap + C - 1) / C;
   const int kgroups = K / 8;
@@ -53,8 +57,13 @@ __global__ void cache_kernel(const T* __restrict__ k, const float* __restrict__ 
     else
       load8(P + ((b * Tn + (cstart - t0)) * HQ + h) * K + n0, Rv);
     load8(k + ((b * Tn + tt) * H + h / G) * K + n0, kv);
+    bool wide = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = kv[i] * exp2f(Rv[i] - pv[i]);
+    for (int i = 0; i < 8; ++i) {
+      out[i] = kv[i] * exp2f(Rv[i] - pv[i]);
+      wide |= fabsf(Rv[i] - pv[i]) > kAnchorRange;
+    }
+    if (wide) record_status(status, WALL_ERR_RANGE);
     store8(kt + ((b * Tcap + t) * HQ + h) * K + n0, out);
     if (t == cstart) store8(rc + ((b * NC + c) * HQ + h) * K + n0, pv);
   }
@@ -241,14 +250,17 @@ constexpr int kDecTile = 32;
 //   own score = scale * q . k_new: the decay factor of a key at the query's
 //               own position is exp2(P_t - P_t) = 1, so no anchor enters
 //   appends   = r_cache[t/C] = P_t when t starts a chunk, k_tilde row t =
-//               k_new * exp2(R - P_t) rounded as the cache build rounds it,
-//               value row t, carry = P_t
+//               k_new * exp2(R - P_t) rounded as the cache build rounds it
+//               (and, as the cache build does, WALL_ERR_RANGE in the status
+//               word when |R - P_t| exceeds kAnchorRange), value row t,
+//               carry = P_t
 // Every split of this head read the carry and the chunk anchors before it
 // arrived, so the carry may be overwritten in place; row t and chunk t/C
 // (when t starts it) are outside the keys any split reads.
 template <int KD, int VD>
 __device__ __forceinline__ void step_merge_append(const DecodeArgs& a, const StepArgs& st, int b,
-                                                  int h, int kh, int g, int lane, float sl2) {
+                                                  int h, int kh, int g, int lane, float sl2,
+                                                  int* status) {
   constexpr int VPL = VD / 32, QPL = KD / 32;
   const long bh = (long)b * a.HQ + h;
   if (lane == 0) st.count[bh] = 0u;  // every split of this call has arrived
@@ -344,12 +356,15 @@ __device__ __forceinline__ void step_merge_append(const DecodeArgs& a, const Ste
   // append the token
   T_bf16* krow = static_cast<T_bf16*>(st.kt) + (((long)b * a.Tcap + t) * a.HQ + h) * KD + lane * QPL;
   float* crow = st.carry + bh * KD + lane * QPL;
+  bool wide = false;
 #pragma unroll
   for (int i = 0; i < QPL; ++i) {
     krow[i] = from_f32<T_bf16>(kx[i] * exp2f(R[i] - pv[i]));
+    wide |= fabsf(R[i] - pv[i]) > kAnchorRange;
     if (starts) rrow[i] = pv[i];
     crow[i] = pv[i];
   }
+  if (wide) record_status(status, WALL_ERR_RANGE);
   if (g == 0) {
     T_bf16* vrow = static_cast<T_bf16*>(st.vc) + (((long)b * a.Tcap + t) * a.H + kh) * VD + lane * VPL;
 #pragma unroll
@@ -454,10 +469,24 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
     long seq = 0;
     int n_it = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++n_it) {
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_it) {
       int b, kh, s;
       item_of(it, b, kh, s);
       const int h = kh * G + g;
+      if (!ok) {
+        // an earlier wait of this warp gave up (the status word says so):
+        // no more waits; the plain decode marks this item's partial empty,
+        // so its merge never reads what an earlier call left in the
+        // workspace
+        if constexpr (!kStep) {
+          if (par == 0 && lane == 0) {
+            const long part = ((long)b * a.HQ + h) * a.splits + s;
+            a.ws_ml[part * 2] = -INFINITY;
+            a.ws_ml[part * 2 + 1] = 0.f;
+          }
+        }
+        continue;
+      }
       const long k0 = (long)s * kps, k1 = min((long)a.T_kv, k0 + kps);
       const long qoff = ((long)b * a.HQ + h) * KD;
       float qv[QPL], pv[QPL];
@@ -574,8 +603,8 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
         const bool got = n_it == 0 || mbar_wait(xempty(g), (uint32_t)((n_it - 1) & 1), status);
 #pragma unroll
         for (int i = 0; i < VPL; ++i) xs[i] = acc[i];
-        xs[VPL] = m;
-        xs[VPL + 1] = l;
+        xs[VPL] = ok ? m : -INFINITY;  // a partial missing tiles counts as empty
+        xs[VPL + 1] = ok ? l : 0.f;
         __syncwarp();
         if (lane == 0 && got) mbar_arrive(xfull(g));
         continue;
@@ -614,12 +643,14 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(pfull(g));
       } else {
+        // a split that gave up on a wait is written as empty (max -inf, sum
+        // 0): the merge then skips it instead of mixing in missing tiles
         const long part = ((long)b * a.HQ + h) * a.splits + s;
 #pragma unroll
         for (int i = 0; i < VPL; ++i) a.ws_o[part * VD + lane * VPL + i] = acc[i];
         if (lane == 0) {
-          a.ws_ml[part * 2] = m;
-          a.ws_ml[part * 2 + 1] = l;
+          a.ws_ml[part * 2] = ok ? m : -INFINITY;
+          a.ws_ml[part * 2 + 1] = ok ? l : 0.f;
         }
       }
     }
@@ -661,7 +692,8 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
       if (last != 0u) {
         __threadfence();  // the other splits' partials after their arrivals
         for (int g = 0; g < G; ++g)
-          if ((last >> g) & 1u) step_merge_append<KD, VD>(a, st, b, kh * G + g, kh, g, lane, sl2);
+          if ((last >> g) & 1u)
+            step_merge_append<KD, VD>(a, st, b, kh * G + g, kh, g, lane, sl2, status);
       }
     }
   }
@@ -807,12 +839,12 @@ int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int 
   if (dtype == WALL_BF16)
     cache_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(k), P, B, Tn, H, HQ, K, C, t0,
-        static_cast<__nv_bfloat16*>(k_tilde), r_cache, Tcap);
+        static_cast<__nv_bfloat16*>(k_tilde), r_cache, Tcap, device_status());
   else
     cache_kernel<float><<<blocks, threads, 0, stream>>>(static_cast<const float*>(k), P, B, Tn,
                                                         H, HQ, K, C, t0,
                                                         static_cast<float*>(k_tilde), r_cache,
-                                                        Tcap);
+                                                        Tcap, device_status());
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

@@ -62,8 +62,9 @@ extern "C" int wall_attn_decode_noalloc(const void* q, const void* v, const floa
   if ((size_t)B * HQ * S * (V + 2) > kScratchFloats) return WALL_ERR_UNSUPPORTED;
   float* scratch = scratch_on_current_device();
   if (scratch == nullptr) return WALL_ERR_CUDA;
-  // every split writes its whole partial (o, max, sum), so nothing left in the
-  // scratch by an earlier call is read and nothing needs clearing
+  // every split writes its whole partial (o, max, sum), or an empty one if a
+  // bounded wait gave up, so nothing left in the scratch by an earlier call
+  // is read and nothing needs clearing
   const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)K);
   return attn_decode(q, v, p_curr, k_tilde, r_cache, sink_bias, sc, C, dtype, B, T_kv, Tcap, H, HQ,
                      K, V, o, lse, scratch, S, reinterpret_cast<cudaStream_t>(stream));

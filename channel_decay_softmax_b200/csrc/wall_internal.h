@@ -18,6 +18,7 @@ void timing_mark(int slot, cudaStream_t stream);
 enum TimingSlot {
   T_PREFIX = 0, T_OPERANDS = 1, T_FWD = 2, T_BWD_PRE = 3, T_BWD_KEY = 4, T_BWD_DQ = 5,
   T_BWD_FIN = 6, T_REV_SCAN = 7, T_DECODE = 8, T_CACHE = 9, T_STEP = 10, T_CHUNK = 11,
+  T_EXACT = 12,
 };
 
 // ---- scans (wall_scan.cu) ----
@@ -30,13 +31,14 @@ int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaSt
 // for the chunk carries, not P
 int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const __nv_bfloat16* k,
                          float* P, float* scratch, int HQ, int H, int K, const Seqs& seqs,
-                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors,
+                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors, int* units,
                          cudaStream_t stream);
 // the tensor-core backward's dq finalize fused with pass 1 of dL's reverse
-// scan: dq (bf16), dL over dq32, chunk sums of dL into dkh32's chunk rows
+// scan: dq (bf16), dL over dq32, chunk sums of dL into dkh32's chunk rows;
+// dq32 of the units flagged in `units` already holds the final dq
 int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* P,
                         float* dq32, float* dkh32, __nv_bfloat16* dq, int HQ, int H, int K,
-                        float scale, const Seqs& seqs, cudaStream_t stream);
+                        float scale, const Seqs& seqs, const int* units, cudaStream_t stream);
 // passes 2 and 3 of the reverse scan, the chunk sums already in scratch
 int scan_reverse_from_sums(const float* x, void* y, int out_dtype, float* scratch, long C,
                            const Seqs& seqs, cudaStream_t stream);
@@ -53,6 +55,9 @@ struct AttnProblem {
   long rows;         // B*T
   int max_blocks64;  // upper bound on 64-row blocks over all sequences
   int extra_blocks;  // varlen: sequences (each may add one partial block), else 0
+  // SIMT kernels only: nullptr, or [n_seq, HQ] flags; then only the flagged
+  // (sequence, head) units are computed
+  const int* units;
 };
 
 struct FwdArgs {
@@ -90,7 +95,17 @@ struct TcFwdWs {
   __nv_bfloat16* kh;   // [rows, HQ, K]  k * 2^(R_block - P)
   float* anchors;      // [n_blocks128, HQ, K]  P at each 128-row block start
   int n_blocks128;     // upper bound on 128-row blocks over all sequences
+  // [n_seq * HQ + 1]: nonzero for a (sequence, head) unit some of whose
+  // anchored exponents |P - R_block| exceed kAnchorRange, and in the last
+  // word if any unit is; the operand pass sets them, the SIMT kernels
+  // recompute those units
+  int* units;
 };
+// Anchored exponents of the tensor-core operands stay within +-kAnchorRange:
+// Qh, Kh and every per-tile rescaled key then stay normal bf16 numbers for
+// inputs up to 2^20 in magnitude, and the products the MMAs form are exact
+// to bf16 rounding.
+constexpr float kAnchorRange = 100.f;
 bool fwd_tc_supported(const AttnProblem& pb);
 int attn_prepare_operands(const AttnProblem& pb, const void* q, const void* k, const float* P,
                           const TcFwdWs& ws, cudaStream_t stream);
@@ -136,6 +151,15 @@ int attn_decode_chunk_split(const void* q, const void* v, const float* p, const 
 // ---- SIMT fp32 attention (wall_attn_simt.cu) ----
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);
 int attn_bwd_simt(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream);
+// the same kernels over the (sequence, head) units flagged in `units`
+// [n_seq * HQ + 1] only (the last word: some unit is flagged): o and lse;
+// dk^(h), dv^(h) and the column part of the scalar-gate gradient, and dq
+// (final, fp32) into dq32, in one launch.  D, the row part and dsink are
+// left to the tensor-core path's own pass.
+int attn_fwd_simt_units(const AttnProblem& pb, const FwdArgs& a, const int* units,
+                        cudaStream_t stream);
+int attn_bwd_simt_units(const AttnProblem& pb, const BwdArgs& a, const int* units,
+                        cudaStream_t stream);
 // dq, dk, dv outputs and dL (in place of dq32) from the per-head fp32 grads
 int attn_bwd_reduce(const AttnProblem& pb, const BwdArgs& a, void* dq, void* dk, void* dv,
                     cudaStream_t stream);

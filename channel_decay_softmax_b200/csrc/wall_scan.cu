@@ -48,7 +48,12 @@ __device__ __forceinline__ void loadv(const T* p, float* out, int vec) {
 // pass 1: per (sequence, chunk, column group) compensated column sums
 template <typename Tin, int VEC, bool kReverse>
 __global__ void __launch_bounds__(kThreadsScan)
-    chunk_sum_kernel(const Tin* __restrict__ x, float* __restrict__ scratch, long C, Seqs seqs) {
+    chunk_sum_kernel(const Tin* __restrict__ x, float* __restrict__ scratch, long C, Seqs seqs,
+                     int* __restrict__ zero = nullptr, int n_zero = 0) {
+  // words a later pass of the same call sets (the fused operand pass's unit
+  // flags), cleared here so that no separate launch is needed
+  if (zero && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int z = threadIdx.x; z < n_zero; z += blockDim.x) zero[z] = 0;
   int s, k;
   if (!seq_block(seqs, kChunk, (int)blockIdx.x, s, k)) return;
   const long start = seqs.start(s);
@@ -260,7 +265,8 @@ __device__ __forceinline__ void storew(float* p, const float* in) {
 // writing P, and for each row
 //   Qh = q * 2^(P - R),  Kh = k * 2^(R - P),  R = floor(P at the row's
 //   128-row block start)   (the anchors, written at the block start row)
-// as the forward's preparation kernel forms them.  R of a block whose start
+// as the forward's preparation kernel forms them, flagging the (sequence,
+// head) units with an exponent |P - R| beyond kAnchorRange as it does.  R of a block whose start
 // lies in an earlier chunk is that row's prefix, rebuilt from its chunk's
 // carry: the scan's first step is carry + g, then one fused rounding.
 // The carries come from a scratch that is not P, so no thread reads a carry
@@ -278,7 +284,8 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
                                const __nv_bfloat16* __restrict__ k,
                                const float* __restrict__ scratch, float* __restrict__ P, long C,
                                Seqs seqs, int HQ, int H, int K, __nv_bfloat16* __restrict__ qh,
-                               __nv_bfloat16* __restrict__ kh, float* __restrict__ anchors) {
+                               __nv_bfloat16* __restrict__ kh, float* __restrict__ anchors,
+                               int* __restrict__ units) {
   constexpr int BA = 128;  // anchor block rows of the tensor-core kernels
   __shared__ int s_blk_off;
   int s, kc;
@@ -321,6 +328,7 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
       cmp[v] = 0.f;
     }
   }
+  bool wide = false;  // some exponent of this thread's rows beyond kAnchorRange
 #pragma unroll
   for (int r0 = 0; r0 < kChunk; r0 += kInFlightOps) {
     float a[kInFlightOps][VW], qa[kInFlightOps][VW], ka[kInFlightOps][VW];
@@ -347,17 +355,25 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
       }
       if (r < n) {
         storew<VW>(P + pr * C + col, o);
-        float y[VW];
+        float e[VW], y[VW];
 #pragma unroll
-        for (int v = 0; v < VW; ++v) y[v] = qa[rr][v] * exp2f(o[v] - R[v]);
+        for (int v = 0; v < VW; ++v) {
+          e[v] = o[v] - R[v];
+          wide |= fabsf(e[v]) > kAnchorRange;
+          y[v] = saturate_bf16(qa[rr][v] * exp2f(e[v]));
+        }
         storew<VW>(qh + pr * C + col, y);
 #pragma unroll
-        for (int v = 0; v < VW; ++v) y[v] = ka[rr][v] * exp2f(R[v] - o[v]);
+        for (int v = 0; v < VW; ++v) y[v] = saturate_bf16(ka[rr][v] * exp2f(-e[v]));
         storew<VW>(kh + pr * C + col, y);
         if (lr == lb)
           storew<VW>(anchors + ((long)(s_blk_off + lr / BA) * HQ + hh) * K + n0, R);
       }
     }
+  }
+  if (wide) {
+    set_flag(units + (long)s * HQ + hh);
+    set_flag(units + (long)seqs.n * HQ);  // some unit is flagged
   }
 }
 
@@ -370,13 +386,15 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
 // and the chunk's compensated sum of dL in the order chunk_sum_kernel adds
 // it, into the chunk row of `scratch` (dk^(h) itself: this thread has read
 // that row's dk^(h) by then, and no other thread reads this chunk's rows).
+// For a (sequence, head) unit flagged in `units` the SIMT kernels have
+// written the final dq into dq32, so its factor is not applied.
 template <int VW>
 __global__ void __launch_bounds__(kThreadsScan, 4)
     finalize_dl_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const float* __restrict__ P, float* __restrict__ dq32,
                        const float* __restrict__ dkh32, float* __restrict__ scratch,
                        __nv_bfloat16* __restrict__ dq, long C, Seqs seqs, int HQ, int H, int K,
-                       float scale) {
+                       float scale, const int* __restrict__ units) {
   constexpr int BA = 128;
   int s, kc;
   if (!seq_block(seqs, kChunk, (int)blockIdx.x, s, kc)) return;
@@ -389,6 +407,7 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
   const int n = (int)min((long)kChunk, len - lr0);
   const int hh = (int)(col / K), n0 = (int)(col % K);
   const int G = HQ / H;
+  const bool final_dq = units[(long)s * HQ + hh] != 0;
   float sum[VW], cmp[VW];
 #pragma unroll
   for (int v = 0; v < VW; ++v) sum[v] = cmp[v] = 0.f;
@@ -412,7 +431,7 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
       float o[VW];
 #pragma unroll
       for (int v = 0; v < VW; ++v) {
-        a[v] *= scale * exp2f(pv[v] - floorf(rv[v]));
+        if (!final_dq) a[v] *= scale * exp2f(pv[v] - floorf(rv[v]));
         o[v] = qq[v] * a[v] - kk[v] * dkv[v];
         dl[r][v] = in ? o[v] : 0.f;
       }
@@ -484,7 +503,7 @@ int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seq
 
 int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const __nv_bfloat16* k,
                          float* P, float* scratch, int HQ, int H, int K, const Seqs& seqs,
-                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors,
+                         __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors, int* units,
                          cudaStream_t stream) {
   const long C = (long)HQ * K;
   if (seqs.n == 0 || C == 0) return WALL_OK;
@@ -497,7 +516,8 @@ int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const _
   if (chunks == 0) return WALL_OK;
   const dim3 grid((unsigned)chunks, (unsigned)groups);
   timing_mark(T_PREFIX, stream);
-  chunk_sum_kernel<__nv_bfloat16, 8, false><<<grid, kThreadsScan, 0, stream>>>(g, scratch, C, seqs);
+  chunk_sum_kernel<__nv_bfloat16, 8, false><<<grid, kThreadsScan, 0, stream>>>(
+      g, scratch, C, seqs, units, seqs.n * HQ + 1);
   const dim3 cgrid((unsigned)((C + 31) / 32), (unsigned)seqs.n);
   carry_kernel<false><<<cgrid, 32 * kCarryParts, 0, stream>>>(scratch, C, seqs, kInvLn2, nullptr,
                                                               nullptr);
@@ -505,14 +525,14 @@ int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const _
   timing_mark(T_OPERANDS, stream);
   chunk_scan_operands_kernel<kWalkOps>
       <<<dim3((unsigned)chunks, (unsigned)wgroups), kThreadsScan, 0, stream>>>(
-          g, q, k, scratch, P, C, seqs, HQ, H, K, qh, kh, anchors);
+          g, q, k, scratch, P, C, seqs, HQ, H, K, qh, kh, anchors, units);
   timing_mark(T_OPERANDS, stream);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
 int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* P,
                         float* dq32, float* dkh32, __nv_bfloat16* dq, int HQ, int H, int K,
-                        float scale, const Seqs& seqs, cudaStream_t stream) {
+                        float scale, const Seqs& seqs, const int* units, cudaStream_t stream) {
   const long C = (long)HQ * K;
   if (seqs.n == 0 || C == 0) return WALL_OK;
   if (C % 8 != 0) return WALL_ERR_UNSUPPORTED;
@@ -523,7 +543,7 @@ int finalize_dq_dl_sums(const __nv_bfloat16* q, const __nv_bfloat16* k, const fl
   if (chunks == 0) return WALL_OK;
   finalize_dl_kernel<kWalkDl>
       <<<dim3((unsigned)chunks, (unsigned)wgroups), kThreadsScan, 0, stream>>>(
-          q, k, P, dq32, dkh32, dkh32, dq, C, seqs, HQ, H, K, scale);
+          q, k, P, dq32, dkh32, dkh32, dq, C, seqs, HQ, H, K, scale, units);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

@@ -24,7 +24,7 @@ Slot g_slot[WALL_TIMING_SLOTS];
 const char* const kNames[WALL_TIMING_SLOTS] = {
     "prefix_scan", "operands", "fwd_tc", "bwd_pre", "bwd_keyblock",
     "bwd_dq", "bwd_finalize", "reverse_scan", "decode", "cache_build",
-    "decode_step", "decode_chunk"};
+    "decode_step", "decode_chunk", "exact_units"};
 
 }  // namespace
 

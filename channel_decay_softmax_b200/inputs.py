@@ -22,6 +22,14 @@ Values are drawn in fp32 from a torch Generator seeded 1000 + config and
 then cast to the config's dtype; both the CUDA path and the oracle consume
 the cast values.  The upstream gradient dO is N(0, 1) (the README example
 back-propagates o.sum(), i.e. dO = 1; a random dO is the stronger test).
+
+Strongly decaying channels (``g_strong``, any config): a fast-forgetting
+channel of a trained gate, the blog's "dynamic" channels, is not in the
+pages' workloads; this recipe adds it.  For query head h and channel n the
+channel class is (h * K + n) % 8; class c < len(g_strong) gets the per-step
+log-gate -g_strong[c] * |1 + 0.1 N| (so -3 forgets 95 % per step), the
+others keep the config's distribution.  ``strong_heads`` > 0 limits the
+strong channels to the first that many query heads.
 """
 from __future__ import annotations
 
@@ -50,6 +58,8 @@ class Spec:
     window: int = 0
     chunk: int = 64             # decode-cache chunk size
     seed: int = 0
+    g_strong: tuple = ()        # per-step decay of the strong channel classes
+    strong_heads: int = 0       # > 0: strong channels in heads [0, strong_heads) only
 
     @property
     def G(self) -> int:
@@ -96,9 +106,18 @@ def cu_seqlens_of(lengths) -> torch.Tensor:
 
 def _gate(gen, shape, s: Spec, device) -> torch.Tensor:
     x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
-    if s.g_kind == "decay":
-        return -s.g_amp * x.abs()
-    return s.g_amp * x
+    g = -s.g_amp * x.abs() if s.g_kind == "decay" else s.g_amp * x
+    if s.g_strong:
+        HQ, K = shape[-2], shape[-1]
+        cls = (torch.arange(HQ, device=device)[:, None] * K +
+               torch.arange(K, device=device)[None, :]) % 8
+        if s.strong_heads > 0:
+            cls[s.strong_heads:] = 8
+        jitter = (1.0 + 0.1 * torch.randn(shape, generator=gen, device=device,
+                                          dtype=torch.float32)).abs()
+        for c, a in enumerate(s.g_strong):
+            g = torch.where(cls == c, -float(a) * jitter, g)
+    return g
 
 
 def training_inputs(s: Spec, device="cpu", lengths=None) -> dict:

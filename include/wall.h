@@ -77,6 +77,8 @@ typedef struct CUstream_st* wall_stream_t; /* same type as cudaStream_t */
 #define WALL_ERR_UNSUPPORTED 2 /* dtype or head size not built */
 #define WALL_ERR_CUDA 3        /* a CUDA launch or copy failed */
 #define WALL_ERR_TIMEOUT 4     /* a kernel's bounded wait expired (from wall_get_status) */
+#define WALL_ERR_RANGE 5       /* a gate prefix left the decode cache's anchored range
+                                  (from wall_get_status; see wall_build_kv_cache) */
 
 /* dtypes */
 #define WALL_BF16 0
@@ -161,14 +163,28 @@ int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* 
                        const int32_t* cu_seqlens, int n_seq, float* P, void* o, float* lse,
                        void* workspace, size_t workspace_bytes, wall_stream_t stream);
 
-/* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs.  For
- * dense batches (n_seq == 0) on the bf16 tensor-core path it includes room
- * for every dS tile of the causal problem, bf16 128 x 128 per (batch row,
- * head, query block I, key block J <= I), B*HQ*nb(nb+1)/2 * 32 KB with
- * nb = ceil(T/128), when that is at most 8 GiB (1.09 GB at B=1, T=8192,
- * HQ=16); the dq pass then reads those tiles instead of recomputing them. */
+/* wall_attn_bwd_workspace -- bytes of workspace wall_attn_bwd needs for a
+ * problem with this window (window_size <= 0: none; a call with a window
+ * fits a workspace sized for a wider one or none).  On the bf16 tensor-core
+ * path it includes room for every dS tile the backward forms, bf16 128 x 128
+ * per (sequence, head, query block I, visible key block J), when that is at
+ * most 8 GiB; the dq pass then reads those tiles instead of recomputing them.
+ * Dense: B*HQ*nb(nb+1)/2 tiles without a window, nb = ceil(T/128) (1.09 GB
+ * at B=1, T=8192, HQ=16); a window of W keys keeps ceil((W-1)/128) + 1 key
+ * blocks per query block; varlen packing (n_seq > 0) reserves the tiles of
+ * one sequence holding every row plus n_seq partial blocks (a bound, since
+ * the lengths are on the device). */
 size_t wall_attn_bwd_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
-                               int has_g_scalar, int n_seq);
+                               int has_g_scalar, int n_seq, int window_size);
+
+/* wall_attn_bwd_workspace_min -- the least workspace wall_attn_bwd accepts:
+ * without room for the dS tiles (window-independent).  Given a workspace
+ * smaller than wall_attn_bwd_workspace's size but at least this one, the
+ * backward keeps no dS tiles and its dq pass recomputes S, P, dP and dS on
+ * the tensor cores (for callers short of memory; the results agree to bf16
+ * rounding). */
+size_t wall_attn_bwd_workspace_min(int dtype, int B, int T, int H, int HQ, int K, int V,
+                                   int has_g_scalar, int n_seq);
 
 /*
  * wall_attn_bwd -- gradients of a scalar loss through wall_attn_fwd (README
@@ -254,7 +270,10 @@ int wall_attn_decode(const void* q, const void* v, const float* p_curr, const vo
  * array's device address (cudaGetSymbolAddress) with that device current, so
  * make that first call before any stream capture.  All calls share the one
  * array and each call overwrites every partial it reads, so nothing needs
- * clearing; calls that overlap on the GPU (concurrent streams) race on it.
+ * clearing (after a device timeout, which wall_get_status reports, the splits
+ * that gave up are written as empty partials, so no earlier call's values are
+ * merged either); calls that overlap on the GPU (concurrent streams) race on
+ * it.
  */
 int wall_attn_decode_noalloc(const void* q, const void* v, const float* p_curr,
                              const void* k_tilde, const float* r_cache, const float* sink_bias,
@@ -390,10 +409,12 @@ int wall_selftest_wait_timeout(int limit_us, wall_stream_t stream);
  *   9 cache_build     wall_build_kv_cache
  *  10 decode_step     wall_decode_step (one launch per token)
  *  11 decode_chunk    wall_attn_decode_chunk (operands and attention)
+ *  12 exact_units     the CUDA-core recomputation of (sequence, head) units
+ *                     beyond the anchored operands' range (fwd and bwd)
  * wall_timing_enable(1) starts recording (and clears the totals);
  * wall_timing_enable(0) stops.  Not thread-safe: one host thread at a time.
  */
-#define WALL_TIMING_SLOTS 12
+#define WALL_TIMING_SLOTS 13
 int wall_timing_enable(int on);
 
 /*

@@ -36,6 +36,7 @@ int main(void) {
       (any_fn)wall_attn_decode_chunk, (any_fn)wall_get_status,
       (any_fn)wall_selftest_wait_timeout, (any_fn)wall_timing_enable,
       (any_fn)wall_timing_enable_slots,   (any_fn)wall_timing_read,
+      (any_fn)wall_attn_bwd_workspace_min,
   };
   for (size_t i = 0; i < sizeof(fns) / sizeof(fns[0]); ++i) CHECK(fns[i] != NULL);
 
@@ -52,7 +53,9 @@ int main(void) {
   CHECK(wall_attn_fwd(fake, fake, fake, ffake, WALL_BF16, 1, 0, 2, 4, 64, 64, 0.f, NULL, NULL,
                       0, NULL, 0, fake, ffake, fake, 0, NULL) == WALL_OK);
   CHECK(wall_attn_fwd_workspace(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0) > 0);
-  CHECK(wall_attn_bwd_workspace(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0) >
+  CHECK(wall_attn_bwd_workspace_min(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0) <
+        wall_attn_bwd_workspace(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0, 0));
+  CHECK(wall_attn_bwd_workspace(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0, 0) >
         wall_attn_fwd_workspace(WALL_BF16, 1, 8192, 4, 16, 128, 128, 0, 0));
   /* decode: the current token's key must be cached (T_kv >= 1) */
   CHECK(wall_attn_decode(fake, fake, ffake, fake, ffake, NULL, 0.f, 64, WALL_BF16, 1, 0, 10, 2,

@@ -365,11 +365,56 @@ def pin_row_and_head_subsets(seed=14):
     return ok and untouched, detail + ("" if untouched else " (rows outside the subset written)")
 
 
+def pin_strong_decay(seed=15):
+    """Strongly decaying channels.  (a) With every channel's gate at -60 per
+    step (a decay factor of e^-60 across one step) the decayed dot product of
+    any earlier key vanishes, so each row's logits are scale q_i . k_i on the
+    diagonal and 0 for every earlier key (not minus infinity): a textbook
+    softmax over that logit matrix, written here with numpy matrices, gives
+    o, lse and dq, dk, dv (the gradients flow through the diagonal logits
+    only).  (b) A mix of channels at -0.5, -1 and -3 per step over 48 rows
+    (2^-200 and below between distant rows): the product form and the
+    prefix form agree."""
+    x = _inputs(seed, B=1, T=9, HQ=2, H=1, K=3, V=2)
+    g = np.full_like(x["g"], -60.0)
+    bw = wo.backward(x["q"], x["k"], x["v"], g, x["dO"])
+    T, HQ = 9, 2
+    sc = 3 ** -0.5
+    worst = 0.0
+    for h in range(HQ):
+        q, k, v, dO = x["q"][0, :, h], x["k"][0, :, 0], x["v"][0, :, 0], x["dO"][0, :, h]
+        S = np.where(np.tri(T, dtype=bool), 0.0, -np.inf)
+        S[np.arange(T), np.arange(T)] = sc * np.sum(q * k, axis=1)
+        m = S.max(1, keepdims=True)
+        A = np.exp(S - m)
+        A /= A.sum(1, keepdims=True)
+        o = A @ v
+        lse = (m + np.log(np.exp(S - m).sum(1, keepdims=True)))[:, 0]
+        D = np.sum(dO * o, axis=1)
+        dSd = np.diag(A) * (np.sum(dO * v, axis=1) - D)   # dS on the diagonal
+        worst = max(worst, _err(bw["o"][0, :, h], o), _err(bw["lse"][0, :, h], lse),
+                    _err(bw["dq"][0, :, h], sc * dSd[:, None] * k),
+                    _err(bw["dk_h"][0, :, h], sc * dSd[:, None] * q),
+                    _err(bw["dv_h"][0, :, h], A.T @ dO))
+    r = _rng(seed + 1)
+    x = _inputs(seed + 2, B=1, T=48, HQ=2, H=1, K=4, V=3, g_amp=0.05)
+    gm = x["g"].copy()
+    for n, a in enumerate((0.5, 1.0, 3.0)):
+        gm[..., n] = -a * np.abs(1.0 + 0.1 * r.standard_normal(gm[..., n].shape))
+    o1, l1 = wo.forward(x["q"], x["k"], x["v"], gm, form="product")
+    o2, l2 = wo.forward(x["q"], x["k"], x["v"], gm, form="prefix")
+    b1 = wo.backward(x["q"], x["k"], x["v"], gm, x["dO"], form="product")
+    b2 = wo.backward(x["q"], x["k"], x["v"], gm, x["dO"], form="prefix")
+    worst = max(worst, _err(o1, o2), _err(l1, l2),
+                *(_err(b1[key], b2[key]) for key in ("dq", "dk", "dv", "dg")))
+    return _ok("strong decay: limit closed form, product vs prefix", worst, 1e-11)
+
+
 ALL_PINS = [pin_g_zero_textbook, pin_product_equals_prefix, pin_fox_scalar_gate,
             pin_channel_constant_gate, pin_window_sink_textbook, pin_gqa_repeat,
             pin_varlen_independent, pin_decode_row, pin_prefix_closed_form,
             pin_prefix_magnitude_long_context, pin_gradients_fd, pin_shift_invariance,
-            pin_key_side_gate_grad, pin_row_and_head_subsets]
+            pin_key_side_gate_grad, pin_row_and_head_subsets, pin_strong_decay]
 
 
 def run_all_pins():

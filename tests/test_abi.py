@@ -8,6 +8,7 @@ import re
 import pytest
 
 from channel_decay_softmax_b200 import _lib as L
+from channel_decay_softmax_b200 import api
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "wall.h")
@@ -190,7 +191,9 @@ def test_fwd_gate_workspace_and_checks(lib):
 def test_timing_slot_mask(lib):
     # host-only: the mask selects slots; bits past the slot count are refused
     assert lib.wall_timing_enable_slots(1 << 4) == L.WALL_OK
-    assert lib.wall_timing_enable_slots(1 << 12) == L.WALL_ERR_INVALID_ARG
+    n = len(api.TIMING_SLOTS)
+    assert lib.wall_timing_enable_slots(1 << (n - 1)) == L.WALL_OK
+    assert lib.wall_timing_enable_slots(1 << n) == L.WALL_ERR_INVALID_ARG
     assert lib.wall_timing_enable_slots(0) == L.WALL_OK
     assert lib.wall_timing_enable(0) == L.WALL_OK
 
@@ -205,36 +208,52 @@ def test_prefix_rejects_bad_arguments(lib):
 
 def test_workspace_sizes(lib):
     # backward: D, dq, dk^(h), dv^(h), two scalar-gate parts (+ its prefix);
-    # the bf16 tensor-core path adds the anchored operands q^, k^ (bf16) and
-    # the 128-row block anchors (fp32)
+    # the bf16 tensor-core path adds the anchored operands q^, k^ (bf16),
+    # the 128-row block anchors (fp32) and one int flag per (sequence, head)
     B, T, HQ, K, V = 2, 100, 8, 64, 64
     rows = B * T
     al = lambda x: (x + 255) // 256 * 256
     simt = al(4 * rows * HQ) + 2 * al(4 * rows * HQ * K) + al(4 * rows * HQ * V) + \
         2 * al(4 * rows * HQ)
     nblk = B * ((T + 127) // 128)
-    tc = 2 * al(2 * rows * HQ * K) + al(4 * nblk * HQ * K)
-    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 0, 0) == simt        # fp32
-    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 1, 0) == simt + al(4 * rows * HQ)
+    tc = 2 * al(2 * rows * HQ * K) + al(4 * nblk * HQ * K) + al(4 * B * HQ)
+
+    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 0, 0, 0) == simt        # fp32
+    assert lib.wall_attn_bwd_workspace(1, B, T, 4, HQ, K, V, 1, 0, 0) == simt + al(4 * rows * HQ)
     # bf16 dense: the stored dS tiles (bf16 128 x 128) of every (b, h, I, J <= I)
     nb = (T + 127) // 128
     ds = al(B * HQ * nb * (nb + 1) // 2 * 128 * 128 * 2)
-    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc + ds
+    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, K, V, 0, 0, 0) == simt + tc + ds
+    # the least workspace: no dS tiles (the dq pass then recomputes them)
+    assert lib.wall_attn_bwd_workspace_min(0, B, T, 4, HQ, K, V, 0, 0) == simt + tc
     # beyond 8 GiB of tiles (B=1, T=65536, HQ=16: 68.9 GB) none are kept
     Tb = 65536
-    big = lib.wall_attn_bwd_workspace(0, 1, Tb, 4, HQ * 2, K, V, 0, 0)
+    big = lib.wall_attn_bwd_workspace(0, 1, Tb, 4, HQ * 2, K, V, 0, 0, 0)
     simtb = al(4 * Tb * HQ * 2) + 2 * al(4 * Tb * HQ * 2 * K) + al(4 * Tb * HQ * 2 * V) + \
         2 * al(4 * Tb * HQ * 2)
-    tcb = 2 * al(2 * Tb * HQ * 2 * K) + al(4 * (Tb // 128) * HQ * 2 * K)
+    tcb = 2 * al(2 * Tb * HQ * 2 * K) + al(4 * (Tb // 128) * HQ * 2 * K) + al(4 * HQ * 2)
     assert big == simtb + tcb
-    # varlen packing (B == 1, n_seq > 0): no stored tiles, dq recomputes them
+    # varlen packing (B == 1, n_seq > 0): the lengths are on the device, so
+    # the tiles of one sequence holding every block (ceil(T/128) + n_seq)
     simt1 = al(4 * T * HQ) + 2 * al(4 * T * HQ * K) + al(4 * T * HQ * V) + 2 * al(4 * T * HQ)
-    tc1 = 2 * al(2 * T * HQ * K) + al(4 * ((T + 127) // 128 + 3) * HQ * K)
-    assert lib.wall_attn_bwd_workspace(0, 1, T, 4, HQ, K, V, 0, 3) == simt1 + tc1
-    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, 32, 32, 0, 0) == \
+    tc1 = 2 * al(2 * T * HQ * K) + al(4 * ((T + 127) // 128 + 3) * HQ * K) + al(4 * 3 * HQ)
+    nbv = (T + 127) // 128 + 3
+    ds1 = al(HQ * nbv * (nbv + 1) // 2 * 128 * 128 * 2)
+    assert lib.wall_attn_bwd_workspace(0, 1, T, 4, HQ, K, V, 0, 3, 0) == simt1 + tc1 + ds1
+    # a window of 256 keys: a query block keeps itself and ceil(255/128) = 2
+    # earlier key blocks: 1 + 2 + 3 + 3 + ... over nb = 8 blocks = 21 tiles
+    Tw = 1000
+    rw = B * Tw
+    simtw = al(4 * rw * HQ) + 2 * al(4 * rw * HQ * K) + al(4 * rw * HQ * V) + 2 * al(4 * rw * HQ)
+    tcw = 2 * al(2 * rw * HQ * K) + al(4 * B * 8 * HQ * K) + al(4 * B * HQ)
+    assert lib.wall_attn_bwd_workspace(0, B, Tw, 4, HQ, K, V, 0, 0, 256) == \
+        simtw + tcw + al(B * HQ * 21 * 128 * 128 * 2)
+    assert lib.wall_attn_bwd_workspace(0, B, Tw, 4, HQ, K, V, 0, 0, 0) == \
+        simtw + tcw + al(B * HQ * 36 * 128 * 128 * 2)
+    assert lib.wall_attn_bwd_workspace(0, B, T, 4, HQ, 32, 32, 0, 0, 0) == \
         al(4 * rows * HQ) + 2 * al(4 * rows * HQ * 32) + al(4 * rows * HQ * 32) + \
         2 * al(4 * rows * HQ)                                                     # SIMT bf16
-    assert lib.wall_attn_bwd_workspace(0, B, T, 3, HQ, K, V, 0, 0) == 0           # bad shape
+    assert lib.wall_attn_bwd_workspace(0, B, T, 3, HQ, K, V, 0, 0, 0) == 0           # bad shape
     assert lib.wall_attn_fwd_workspace(1, B, T, 4, HQ, K, V, 0, 0) == 0           # fp32, no opts
     assert lib.wall_attn_fwd_workspace(0, B, T, 4, HQ, K, V, 0, 0) == tc
     assert lib.wall_attn_decode_workspace(32, 32768, 8, 32, 128, 64) > 0

@@ -109,9 +109,13 @@ def test_both_configs_timed_per_step_kernel_and_graph(monkeypatch):
     assert c2["graph_ms_per_step"] == 0.5 and "graph_tflops" in c2
     assert "graph_ms_per_step" not in c4
     assert "packed sequences" in c4["workload"] and "window 1024" in c4["workload"]
-    # config 2 through the gate call reusing its workspace; config 4 through
-    # prefix + forward + backward with dsink
-    assert ("bwd", False, True) in calls and ("bwd", True, False) in calls
+    # both through the gate call, the backward reusing its workspace; config 4
+    # (packed sequences, with a sink) asks for dsink
+    assert ("bwd", False, True) in calls and ("bwd", True, True) in calls
+    assert any(c[0] == "fwd_gate" and c[2] for c in calls)  # packed sequences
+    assert not any(c[0] in ("prefix", "fwd") for c in calls)
+    for name, row in c4["stage_ms_per_step"].items():
+        assert row > 0, name
     assert any(c[0] == "replay" for c in calls)
 
 

@@ -27,9 +27,7 @@ def _same(got, want, what):
     for n, w in want.items():
         if w is None:
             assert got[n] is None, (what, n)
-        elif n == "dsink":  # a sum of atomics: the order may differ
-            assert torch.allclose(got[n], w, rtol=1e-5, atol=1e-6), (what, n)
-        else:
+        else:  # every output, dsink included, is summed in a fixed order
             assert torch.equal(got[n], w), (what, n)
 
 

@@ -209,22 +209,39 @@ def test_backward_reuses_forward_operands_bit_exactly():
         assert torch.equal(ta, tb), name
 
 
-@pytest.mark.parametrize("K", [64, 128])
-def test_dq_from_stored_ds_matches_recompute(K):
-    """Dense causal bf16 problems store the key-block kernel's dS tiles and
-    take dq as one contraction per tile; a window longer than the sequence
-    (the same attention) sends dq through the recomputing query-block kernel
-    instead.  Both match the oracle, with the scalar gate and sink, and agree
-    with each other to bf16 rounding."""
-    T = 700
-    s = I.spec(2, T=T, K=K, V=K, g_scalar=True, sink=True)
-    x_cpu = I.training_inputs(s)
-    _check_all(s, x_cpu, what=f"stored dS K={K}")
-    s_w = I.spec(2, T=T, K=K, V=K, g_scalar=True, sink=True, window=T + 1)
-    x_w = dict(x_cpu, window_size=T + 1)
-    _check_all(s_w, x_w, what=f"recompute K={K}")
-    _, _, _, ga = _run_gpu(_to(x_cpu))
-    _, _, _, gb = _run_gpu(_to(x_w))
+def _run_gpu_recompute(x):
+    """_run_gpu with the smaller backward workspace: no dS tiles, so the dq
+    pass recomputes S, P, dP and dS"""
+    q, k, v, g = x["q"], x["k"], x["v"], x["g"]
+    cu = x["cu_seqlens"]
+    P = api.prefix_cumsum(g, cu)
+    o, lse = api.wall_attn_fwd(q, k, v, P, x["scale"], x["g_scalar"], x["sink_bias"],
+                               x["window_size"], cu)
+    grads = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], x["g_scalar"],
+                              x["sink_bias"], x["window_size"], cu, store_ds=False)
+    torch.cuda.synchronize()
+    return P, o, lse, grads
+
+
+@pytest.mark.parametrize("case", ["dense_K64", "dense_K128", "varlen_window_K128"])
+def test_dq_from_stored_ds_matches_recompute(case):
+    """The key-block kernel stores its dS tiles (banded per (sequence, head)
+    for varlen packing and windows) and dq is one contraction per tile; the
+    smaller workspace without the tiles sends dq through the recomputing
+    query-block kernel instead.  Both match the oracle, with the scalar gate
+    and sink, and agree with each other to bf16 rounding."""
+    if case.startswith("dense"):
+        K = 64 if case.endswith("64") else 128
+        s = I.spec(2, T=700, K=K, V=K, g_scalar=True, sink=True)
+        lengths = None
+    else:
+        s = I.spec(4, K=128, V=128, HQ=8, H=2, n_seq=5, window=300)
+        lengths = [700, 1, 130, 0, 517]
+    x_cpu = I.training_inputs(s, lengths=lengths)
+    _check_all(s, x_cpu, what=f"stored dS {case}")
+    x = _to(x_cpu)
+    _, _, _, ga = _run_gpu(x)
+    _, _, _, gb = _run_gpu_recompute(x)
     for name, ta, tb in zip(("dq", "dk", "dv", "dg"), ga[:4], gb[:4]):
         e = float((ta.float() - tb.float()).norm() / tb.float().norm())
         assert e < 1e-2, (name, e)
@@ -265,3 +282,76 @@ def test_fwd_gate_equals_prefix_then_forward(case):
     torch.cuda.synchronize()
     for name, ta, tb in zip(("dq", "dk", "dv", "dg"), a[:4], b[:4]):
         assert torch.equal(ta, tb), name
+
+
+def _compare_units(s, xc, o, lse, grads, units, what):
+    """o, lse and the gradients of the given (sequence * HQ + head) units
+    against the oracle, element by element."""
+    ref = wo.backward(xc["q"], xc["k"], xc["v"], xc["g"], xc["dO"], units=units,
+                      **_oracle_kw(xc))
+    heads = sorted({u % s.HQ for u in units})
+    mask = np.zeros(o.shape[:3], dtype=bool)
+    mask[:, :, heads] = True
+    dq, dk, dv, dg, dgs, dsink = grads
+    kmask = np.zeros(dk.shape[:3], dtype=bool)
+    kmask[:, :, sorted({h // s.G for h in heads})] = True
+    assert_fwd(s.dtype, o, ref["o"], lse, ref["lse"], mask, what)
+    assert_grad(s.dtype, "dq", dq, ref["dq"], mask, what)
+    assert_grad(s.dtype, "dk", dk, ref["dk"], kmask, what)
+    assert_grad(s.dtype, "dv", dv, ref["dv"], kmask, what)
+    assert_grad(s.dtype, "dg", dg, ref["dg"], mask, what)
+    if dgs is not None:
+        assert_grad(s.dtype, "dg_scalar", dgs, ref["dg_scalar"], mask, what,
+                    relative_to_max=True)
+
+
+@pytest.mark.slow
+def test_cfg3_headline_call_sequence_full_size_sampled():
+    """The benchmark's own call sequence at T = 8192 on its inputs:
+    wall_attn_fwd_gate (prefix scan fused into the operand pass), then
+    wall_attn_bwd given the gate call's workspace.  One GQA group (4 query
+    heads) against the oracle, element by element."""
+    s = I.spec(3)
+    xc = I.training_inputs(s)
+    x = _to(xc)
+    o, lse, P, ws = api.wall_attn_fwd_gate(x["q"], x["k"], x["v"], x["g"], s.scale,
+                                           return_workspace=True)
+    grads = api.wall_attn_bwd(x["dO"], x["q"], x["k"], x["v"], P, o, lse, s.scale,
+                              fwd_workspace=ws)
+    torch.cuda.synchronize()
+    _compare_units(s, xc, o, lse, grads, [4, 5, 6, 7], "headline sequence T=8192")
+
+
+def _autograd_cfg4(s, xc, units, what):
+    x = _to(xc)
+    q, k, v, g = (x[n].clone().requires_grad_(True) for n in ("q", "k", "v", "g"))
+    gs = x["g_scalar"].clone().requires_grad_(True)
+    sk = x["sink_bias"].clone().requires_grad_(True)
+    o = api.wall_attn(q, k, v, g, scale=s.scale, g_scalar=gs, sink_bias=sk,
+                      window_size=x["window_size"], cu_seqlens=x["cu_seqlens"])
+    o.backward(x["dO"])
+    torch.cuda.synchronize()
+    # lse is not an autograd output: compare it from a forward call
+    _, lse = api.wall_attn_fwd(x["q"], x["k"], x["v"], api.prefix_cumsum(x["g"], x["cu_seqlens"]),
+                               s.scale, x["g_scalar"], x["sink_bias"], x["window_size"],
+                               x["cu_seqlens"])
+    _compare_units(s, xc, o.detach(), lse,
+                   (q.grad, k.grad, v.grad, g.grad, gs.grad, None), units, what)
+    if units is None or len(units) == s.HQ * s.n_seq:
+        ref = wo.backward(xc["q"], xc["k"], xc["v"], xc["g"], xc["dO"], **_oracle_kw(xc))
+        assert_grad(s.dtype, "dsink", sk.grad, ref["dsink"], None, what, relative_to_max=True)
+
+
+def test_cfg4_through_autograd_reduced():
+    """Config 4's options through the autograd function (the README's call
+    pattern), every unit, dsink included."""
+    s = I.spec(4, len_lo=64, len_hi=600, window=128)
+    units = [seq * s.HQ + h for seq in range(s.n_seq) for h in range(s.HQ)]
+    _autograd_cfg4(s, I.training_inputs(s), units, "cfg4 autograd reduced")
+
+
+@pytest.mark.slow
+def test_cfg4_through_autograd_full_size_sampled():
+    s = I.spec(4)
+    units = [seq * s.HQ + h for seq in range(s.n_seq) for h in (0, 1, 2, 3, 4, 5, 6, 7)]
+    _autograd_cfg4(s, I.training_inputs(s), units, "cfg4 autograd full")
