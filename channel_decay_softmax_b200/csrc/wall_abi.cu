@@ -178,6 +178,15 @@ BwdWs bwd_ws_layout(const AttnProblem& pb, int has_gs, bool want_ds = true) {
 
 inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
+// The fused prefix pass's chunk carries: one fp32 row of HQ*K per 32-row
+// chunk of every sequence (a bound for varlen packing: each sequence may add
+// one partial chunk).
+size_t gate_scratch_bytes(const AttnProblem& pb) {
+  const long chunks = pb.extra_blocks > 0 ? (pb.rows + 31) / 32 + pb.extra_blocks
+                                          : (long)pb.B * ((pb.T + 31) / 32);
+  return align256(sizeof(float) * (size_t)chunks * pb.HQ * pb.K);
+}
+
 // wall_attn_decode_chunk's workspace: the anchored queries and their block
 // anchors (tensor-core path) or the split partials (split path)
 struct ChunkWs {
@@ -338,7 +347,7 @@ size_t wall_attn_fwd_gate_workspace(int dtype, int B, int T, int H, int HQ, int 
   const FwdWs w = fwd_ws_layout(pb, has_g_scalar);
   // the forward's own layout first (wall_attn_bwd may reuse it), then the
   // chunk carries of the fused prefix pass
-  return w.total + (fwd_tc_supported(pb) ? align256(sizeof(float) * pb.rows * HQ * K) : 0);
+  return w.total + (fwd_tc_supported(pb) ? gate_scratch_bytes(pb) : 0);
 }
 
 int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* g, int dtype,
@@ -356,7 +365,7 @@ int wall_attn_fwd_gate(const void* q, const void* k, const void* v, const void* 
   if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(lse)) return WALL_ERR_INVALID_ARG;
   const FwdWs w = fwd_ws_layout(pb, g_scalar != nullptr);
   const bool tc = fwd_tc_supported(pb);
-  const size_t need = w.total + (tc ? align256(sizeof(float) * pb.rows * HQ * K) : 0);
+  const size_t need = w.total + (tc ? gate_scratch_bytes(pb) : 0);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
     return WALL_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

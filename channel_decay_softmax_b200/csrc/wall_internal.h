@@ -27,8 +27,8 @@ int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seq
 int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream);
 // the forward prefix fused with the tensor-core operand preparation: P (as
 // scan_prefix_log2 forms it, bit for bit), Qh, Kh and the 128-row block
-// anchors (as attn_prepare_operands forms them); scratch: fp32 [rows, HQ*K]
-// for the chunk carries, not P
+// anchors (as attn_prepare_operands forms them); scratch: fp32 [chunks, HQ*K]
+// for the chunk carries (one row per 32-row chunk of every sequence), not P
 int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const __nv_bfloat16* k,
                          float* P, float* scratch, int HQ, int H, int K, const Seqs& seqs,
                          __nv_bfloat16* qh, __nv_bfloat16* kh, float* anchors, int* units,

@@ -36,6 +36,15 @@ __device__ __forceinline__ long chunk_row(long start, long len, int k, bool reve
   return reverse ? start + len - 1 - (long)k * kChunk : start + (long)k * kChunk;
 }
 
+// Chunks of the sequences before s: the first slot of sequence s in a
+// compact [chunks, C] scratch (one row per chunk, in seq_block's order).
+__device__ __forceinline__ long chunks_before(const Seqs& seqs, int s) {
+  if (!seqs.cu) return (long)s * ((seqs.T + kChunk - 1) / kChunk);
+  long n = 0;
+  for (int x = 0; x < s; ++x) n += (seqs.len(x) + kChunk - 1) / kChunk;
+  return n;
+}
+
 template <typename T>
 __device__ __forceinline__ void loadv(const T* p, float* out, int vec) {
   if (vec == 8) {
@@ -49,7 +58,7 @@ __device__ __forceinline__ void loadv(const T* p, float* out, int vec) {
 template <typename Tin, int VEC, bool kReverse>
 __global__ void __launch_bounds__(kThreadsScan)
     chunk_sum_kernel(const Tin* __restrict__ x, float* __restrict__ scratch, long C, Seqs seqs,
-                     int* __restrict__ zero = nullptr, int n_zero = 0) {
+                     int* __restrict__ zero = nullptr, int n_zero = 0, bool compact = false) {
   // words a later pass of the same call sets (the fused operand pass's unit
   // flags), cleared here so that no separate launch is needed
   if (zero && blockIdx.x == 0 && blockIdx.y == 0)
@@ -90,7 +99,8 @@ __global__ void __launch_bounds__(kThreadsScan)
       }
     }
   }
-  float* dst = scratch + chunk_row(start, len, k, kReverse) * C + col;
+  // the flat chunk index is blockIdx.x: the compact slot
+  float* dst = scratch + (compact ? (long)blockIdx.x : chunk_row(start, len, k, kReverse)) * C + col;
 #pragma unroll
   for (int v = 0; v < VEC; ++v) dst[v] = sum[v];
 }
@@ -104,7 +114,8 @@ constexpr int kCarryBatch = 32;
 template <bool kReverse>
 __global__ void __launch_bounds__(32 * kCarryParts)
     carry_kernel(float* __restrict__ scratch, long C, Seqs seqs, float mul,
-                 const float* __restrict__ carry_in, float* __restrict__ carry_out) {
+                 const float* __restrict__ carry_in, float* __restrict__ carry_out,
+                 bool compact = false) {
   __shared__ double part_sum[kCarryParts][32];
   const int s = blockIdx.y;
   const int lane = threadIdx.x % 32, part = threadIdx.x / 32;
@@ -114,6 +125,10 @@ __global__ void __launch_bounds__(32 * kCarryParts)
   const long len = seqs.len(s);
   const int nchunk = (int)((len + kChunk - 1) / kChunk);
   const int per = (nchunk + kCarryParts - 1) / kCarryParts;
+  const long base = compact ? chunks_before(seqs, s) : 0;
+  auto slot = [&](int k) {
+    return compact ? base + k : chunk_row(start, len, k, kReverse);
+  };
   const int k0 = min(nchunk, part * per), k1 = min(nchunk, k0 + per);
   // range total
   double tot = 0.0;
@@ -121,7 +136,7 @@ __global__ void __launch_bounds__(32 * kCarryParts)
     float v[kCarryBatch];
 #pragma unroll
     for (int x = 0; x < kCarryBatch; ++x)
-      v[x] = (valid && kb + x < k1) ? scratch[chunk_row(start, len, kb + x, kReverse) * C + col]
+      v[x] = (valid && kb + x < k1) ? scratch[slot(kb + x) * C + col]
                                      : 0.f;
 #pragma unroll
     for (int x = 0; x < kCarryBatch; ++x) tot += (double)v[x];
@@ -140,11 +155,11 @@ __global__ void __launch_bounds__(32 * kCarryParts)
     float v[kCarryBatch];
 #pragma unroll
     for (int x = 0; x < kCarryBatch; ++x)
-      v[x] = (valid && kb + x < k1) ? scratch[chunk_row(start, len, kb + x, kReverse) * C + col]
+      v[x] = (valid && kb + x < k1) ? scratch[slot(kb + x) * C + col]
                                      : 0.f;
 #pragma unroll
     for (int x = 0; x < kCarryBatch; ++x) {
-      if (valid && kb + x < k1) scratch[chunk_row(start, len, kb + x, kReverse) * C + col] = (float)run;
+      if (valid && kb + x < k1) scratch[slot(kb + x) * C + col] = (float)run;
       run += (double)v[x];
     }
   }
@@ -270,7 +285,7 @@ __device__ __forceinline__ void storew(float* p, const float* in) {
 // lies in an earlier chunk is that row's prefix, rebuilt from its chunk's
 // carry: the scan's first step is carry + g, then one fused rounding.
 // The carries come from a scratch that is not P, so no thread reads a carry
-// another one has overwritten.  A thread walks its chunk's rows in order, so
+// another one has overwritten; it is compact, one row per 32-row chunk.  A thread walks its chunk's rows in order, so
 // the walkers are latency-bound: 4 columns per thread instead of 8 doubles
 // the threads in flight here (0.048 -> 0.039 ms at T = 8192); the dL walker
 // below is faster with 8 (0.046 against 0.053 ms).
@@ -309,11 +324,12 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
   const int n = (int)min((long)kChunk, len - lr0);
   const int hh = (int)(col / K), n0 = (int)(col % K);
   const int G = HQ / H;
-  // R: the anchor of the 128-row block this chunk lies in
+  // R: the anchor of the 128-row block this chunk lies in (the scratch is
+  // compact: one row per chunk, chunk kc of this sequence at blockIdx.x)
   const long lb = (lr0 / BA) * BA;
   float R[VW];
   {
-    const float* cb = scratch + chunk_row(start, len, (int)(lb / kChunk), false) * C + col;
+    const float* cb = scratch + ((long)blockIdx.x - kc + lb / kChunk) * C + col;
     float gb[VW];
     loadw<VW>(g + (start + lb) * C + col, gb);
 #pragma unroll
@@ -321,7 +337,7 @@ __global__ void __launch_bounds__(kThreadsScan, 4)
   }
   float acc[VW], cmp[VW];
   {
-    const float* c = scratch + chunk_row(start, len, kc, false) * C + col;
+    const float* c = scratch + (long)blockIdx.x * C + col;
 #pragma unroll
     for (int v = 0; v < VW; ++v) {
       acc[v] = c[v];
@@ -517,10 +533,10 @@ int scan_prefix_operands(const __nv_bfloat16* g, const __nv_bfloat16* q, const _
   const dim3 grid((unsigned)chunks, (unsigned)groups);
   timing_mark(T_PREFIX, stream);
   chunk_sum_kernel<__nv_bfloat16, 8, false><<<grid, kThreadsScan, 0, stream>>>(
-      g, scratch, C, seqs, units, seqs.n * HQ + 1);
+      g, scratch, C, seqs, units, seqs.n * HQ + 1, /*compact=*/true);
   const dim3 cgrid((unsigned)((C + 31) / 32), (unsigned)seqs.n);
   carry_kernel<false><<<cgrid, 32 * kCarryParts, 0, stream>>>(scratch, C, seqs, kInvLn2, nullptr,
-                                                              nullptr);
+                                                              nullptr, /*compact=*/true);
   timing_mark(T_PREFIX, stream);
   timing_mark(T_OPERANDS, stream);
   chunk_scan_operands_kernel<kWalkOps>

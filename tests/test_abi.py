@@ -169,9 +169,13 @@ def test_fwd_gate_workspace_and_checks(lib):
     al = lambda x: (x + 255) // 256 * 256
     B, T, H, HQ, K, V = 2, 100, 4, 8, 64, 64
     fwd = lib.wall_attn_fwd_workspace(0, B, T, H, HQ, K, V, 0, 0)
-    # the forward's layout, then the prefix scan's chunk carries [B*T, HQ*K] fp32
+    # the forward's layout, then the prefix scan's chunk carries: one fp32 row
+    # of HQ*K per 32-row chunk, [B*ceil(T/32), HQ*K]
     assert lib.wall_attn_fwd_gate_workspace(0, B, T, H, HQ, K, V, 0, 0) == \
-        fwd + al(4 * B * T * HQ * K)
+        fwd + al(4 * B * -(-T // 32) * HQ * K)
+    # varlen (n_seq sequences packed in B*T = 100 rows): each may add a chunk
+    assert lib.wall_attn_fwd_gate_workspace(0, 1, T, H, HQ, K, V, 0, 3) == \
+        lib.wall_attn_fwd_workspace(0, 1, T, H, HQ, K, V, 0, 3) + al(4 * (-(-T // 32) + 3) * HQ * K)
     # fp32 (SIMT path): no anchored operands, no carries
     assert lib.wall_attn_fwd_gate_workspace(1, B, T, H, HQ, K, V, 0, 0) == \
         lib.wall_attn_fwd_workspace(1, B, T, H, HQ, K, V, 0, 0)
