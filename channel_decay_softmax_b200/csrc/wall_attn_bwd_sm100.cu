@@ -46,6 +46,8 @@
 
 #include <string.h>
 
+#include <algorithm>
+
 #include <type_traits>
 
 #include "sm100_ptx.cuh"
@@ -727,8 +729,46 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
 }
 
 // dsink_h = -sum_i exp(sink_h - lse_i) D_i (the sink's logit has a zero value
-// row), summed in a fixed order: one CTA per head, a strided sum per thread
-// and a tree in shared memory, so that repeated calls agree bit for bit.
+// row), summed in a fixed order so that repeated calls agree bit for bit.
+// Two passes: CTA b sums rows [b R, (b + 1) R) per head (thread t takes head
+// t % HQ and every (256 / HQ)-th row, so a warp reads consecutive words),
+// then one thread per head adds the CTAs' partials in CTA order.
+__global__ void __launch_bounds__(256)
+    sink_partial_kernel(const float* __restrict__ D, const float* __restrict__ lse,
+                        const float* __restrict__ sink, long rows, int HQ, long rows_per_cta,
+                        float* __restrict__ part) {
+  __shared__ float acc_s[256];
+  const int per = 256 / HQ;  // threads per head
+  const int t = threadIdx.x, h = t % HQ, k = t / HQ;
+  float acc = 0.f;
+  if (k < per) {
+    const float s2 = sink[h] * kLog2e;
+    const long r0 = (long)blockIdx.x * rows_per_cta;
+    const long r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
+    for (long r = r0 + k; r < r1; r += per) {
+      const long e = r * HQ + h;
+      acc -= exp2f(s2 - lse[e] * kLog2e) * D[e];
+    }
+  }
+  acc_s[t] = acc;
+  __syncthreads();
+  if (t < HQ) {
+    float sum = 0.f;
+    for (int x = 0; x < per; ++x) sum += acc_s[t + x * HQ];
+    part[(long)blockIdx.x * HQ + t] = sum;
+  }
+}
+
+__global__ void sink_final_kernel(const float* __restrict__ part, int nb, int HQ,
+                                  float* __restrict__ dsink) {
+  for (int h = threadIdx.x; h < HQ; h += blockDim.x) {
+    float sum = 0.f;
+    for (int b = 0; b < nb; ++b) sum += part[(long)b * HQ + h];
+    dsink[h] = sum;
+  }
+}
+
+// The one-CTA-per-head form of the same sum, for more than 256 heads.
 __global__ void __launch_bounds__(256)
     sink_grad_kernel(const float* __restrict__ D, const float* __restrict__ lse,
                      const float* __restrict__ sink, long rows, int HQ,
@@ -852,6 +892,21 @@ int launch_bwd_tc_gs(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws,
 
 }  // namespace
 
+int sink_grad(const float* D, const float* lse, const float* sink, long rows, int HQ,
+              float* scratch, float* dsink, cudaStream_t stream) {
+  if (rows <= 0 || HQ <= 0) return WALL_OK;
+  if (HQ <= 256) {
+    const long nb = std::min<long>((rows + 63) / 64, 4 * 148);
+    const long per_cta = (rows + nb - 1) / nb;
+    sink_partial_kernel<<<(unsigned)nb, 256, 0, stream>>>(D, lse, sink, rows, HQ, per_cta,
+                                                           scratch);
+    sink_final_kernel<<<1, 256, 0, stream>>>(scratch, (int)nb, HQ, dsink);
+  } else {
+    sink_grad_kernel<<<HQ, 256, 0, stream>>>(D, lse, sink, rows, HQ, dsink);
+  }
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
 int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool prepare, void* dq,
                 void* dk, void* dv, void* dg, int* status, cudaStream_t stream) {
   if (pb.rows == 0 || ws.n_blocks128 == 0) return WALL_OK;
@@ -870,9 +925,10 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
         static_cast<const __nv_bfloat16*>(a.dO), static_cast<const __nv_bfloat16*>(a.o), a.lse,
         a.sink, pb.rows, pb.HQ, pb.V, a.D, a.GS ? a.dgs_row : nullptr);
     if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+    // the partials go through dq32, which the dq kernels overwrite later
     if (a.dsink && a.sink) {
-      sink_grad_kernel<<<pb.HQ, 256, 0, stream>>>(a.D, a.lse, a.sink, pb.rows, pb.HQ, a.dsink);
-      if (cudaGetLastError() != cudaSuccess) return WALL_ERR_CUDA;
+      rc = sink_grad(a.D, a.lse, a.sink, pb.rows, pb.HQ, a.dq32, a.dsink, stream);
+      if (rc) return rc;
     }
   }
   timing_mark(T_BWD_PRE, stream);

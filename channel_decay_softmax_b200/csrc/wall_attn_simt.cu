@@ -264,9 +264,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(AttnProblem pb, FwdA
 }
 
 // ---------------------------------------------------------------------------
-// backward, query side: D_i, dq, row part of the scalar-gate gradient, dsink
-// (with a unit mask: dq only; D, the row part and dsink come from the
-// tensor-core path's own pass)
+// backward, query side: D_i, dq, row part of the scalar-gate gradient (dsink
+// follows from D in sink_grad; with a unit mask: dq only, D and the row part
+// come from the tensor-core path's own pass)
 
 template <typename T, int KD, int VD>
 __device__ __forceinline__ void bwd_dq_simt_block(const AttnProblem& pb, const BwdArgs& a,
@@ -315,12 +315,6 @@ __device__ __forceinline__ void bwd_dq_simt_block(const AttnProblem& pb, const B
     if (sub == 0) {
       Dv[row] = d;
       if (own_rows && row < ni) a.D[(s0 + i0 + row) * HQ + h] = d;
-    }
-    // dsink_h = -sum_i exp(sink_h - lse_i) D_i (the sink's value row is zero)
-    if (own_rows && a.sink && a.dsink) {
-      float contrib = (sub == 0 && row < ni) ? -exp2f(a.sink[h] * kLog2e - lse2[row]) * d : 0.f;
-      for (int off = 16; off > 0; off >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, off);
-      if ((threadIdx.x & 31) == 0) atomicAdd(&a.dsink[h], contrib);
     }
   }
   __syncthreads();
@@ -775,8 +769,11 @@ int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream) 
 
 int attn_bwd_simt(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream) {
   if (pb.max_blocks64 == 0) return WALL_OK;
-  // dkdv reads the D the dq kernel writes
-  const int rc = bwd_dq_any(pb, a, stream);
+  // dkdv and dsink read the D the dq kernel writes; dsink's partials go
+  // through dkh32 before the dkdv kernel writes it
+  int rc = bwd_dq_any(pb, a, stream);
+  if (!rc && a.sink && a.dsink) rc = sink_grad(a.D, a.lse, a.sink, pb.rows, pb.HQ, a.dkh32,
+                                               a.dsink, stream);
   return rc ? rc : bwd_dkdv_any(pb, a, stream);
 }
 

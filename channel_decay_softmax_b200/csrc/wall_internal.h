@@ -148,6 +148,12 @@ int attn_decode_chunk_split(const void* q, const void* v, const float* p, const 
                             int V, void* o, float* lse, float* ws, int splits,
                             cudaStream_t stream);
 
+// dsink_h = -sum_i exp(sink_h - lse_i) D_i in a fixed order (bit-reproducible),
+// from D and lse [rows, HQ]; scratch holds min(ceil(rows / 64), 592) * HQ
+// floats until the launches complete (wall_attn_bwd_sm100.cu)
+int sink_grad(const float* D, const float* lse, const float* sink, long rows, int HQ,
+              float* scratch, float* dsink, cudaStream_t stream);
+
 // ---- SIMT fp32 attention (wall_attn_simt.cu) ----
 int attn_fwd_simt(const AttnProblem& pb, const FwdArgs& a, cudaStream_t stream);
 int attn_bwd_simt(const AttnProblem& pb, const BwdArgs& a, cudaStream_t stream);
