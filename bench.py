@@ -108,9 +108,14 @@ def decode_bytes(s: I.Spec, T_kv: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms; start()
+    """nvidia-smi clocks and throttle reasons sampled every 20 ms; start()
     returns once the first sample is in, mark() brackets the timed region and
-    only samples stamped inside it (plus one interval after) are kept."""
+    only samples stamped inside it (plus one interval after) are kept.  A
+    timed region shorter than the interval may hold none: then the last
+    sample before it and the first after it (each within 250 ms) stand in,
+    and the record says so ("in_window": 0)."""
+
+    INTERVAL_MS = 20
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -127,7 +132,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -156,24 +161,32 @@ class ClockSampler:
         rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
         os.unlink(self.file.name)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        sm, smax, reasons = [], 0.0, set()
+        parsed = []  # (stamp, sm MHz, max MHz, reasons)
         for r in rows:
             try:
                 stamp = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                if self.t0 is not None and not (self.t0 <= stamp <= (self.t1 or stamp) + 0.06):
-                    continue
-                sm.append(float(r[2]))
-                smax = max(smax, float(r[3]))
-                for n, val in zip(names, r[6:10]):
-                    if "Active" in val and "Not" not in val:
-                        reasons.add(n)
+                why = {n for n, val in zip(names, r[6:10]) if "Active" in val and "Not" not in val}
+                parsed.append((stamp, float(r[2]), float(r[3]), why))
             except (ValueError, IndexError):
                 continue
-        if not sm:
+        chosen, in_window = parsed, len(parsed)
+        if self.t0 is not None:
+            t1 = self.t1 if self.t1 is not None else float("inf")
+            chosen = [x for x in parsed if self.t0 <= x[0] <= t1 + self.INTERVAL_MS * 1e-3]
+            in_window = len(chosen)
+            if not chosen:
+                before = [x for x in parsed if self.t0 - 0.25 <= x[0] < self.t0]
+                after = [x for x in parsed if t1 < x[0] <= t1 + 0.25]
+                chosen = before[-1:] + after[:1]
+        if not chosen:
             return None
+        sm = [x[1] for x in chosen]
+        smax = max(x[2] for x in chosen)
+        reasons = set().union(*(x[3] for x in chosen))
         busy = [x for x in sm if x > 0.5 * smax] or sm
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm),
+                "reasons": sorted(reasons), "samples": len(sm), "in_window": in_window,
+                "interval_ms": self.INTERVAL_MS,
                 "window_ms": (self.t1 - self.t0) * 1e3 if self.t0 and self.t1 else None}
 
 

@@ -153,7 +153,8 @@ __device__ __forceinline__ int cache_tile_chunks(const FwdTcParams& p, int j0, i
   return min(nc, (p.T_kv + p.C - 1) / p.C - c0);
 }
 
-template <int KD, bool kCache>
+// kGS: the problem has a scalar gate (never in the cache form)
+template <int KD, bool kCache, bool kGS>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, FwdTcParams p) {
@@ -189,6 +190,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int jb_hi = (pos0 + i0 + ni - 1) / BN;
   const int jb_lo = p.window > 0 ? max(0, i0 - p.window + 1) / BN : 0;
   const int nT = jb_hi - jb_lo + 1;
+  // Key tile t is block jb_lo + t, or with a scalar gate jb_hi - t: the
+  // diagonal first, then back in time.  The gate's bias GS_i - GS_j falls
+  // by the gate's whole sum over the distance (tens of units of log2 across
+  // a 1024-key window), so in ascending order every tile would raise the
+  // rows' running max past the one-pass softmax's bound; from the diagonal
+  // back, the first tiles set the max and the later ones stay under it.
+  constexpr bool rev = kGS;
+  auto jb_of = [&](int t) { return rev ? jb_hi - t : jb_lo + t; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -240,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kCache) {
           // k_tilde rows of batch row `seq` (zeros past T_kv) and the
           // anchors of the tile's cached chunks
-          const int j0 = (jb_lo + t) * BN;
+          const int j0 = jb_of(t) * BN;
           int c0;
           const int nc = cache_tile_chunks(p, j0, c0);
           mbar_expect_tx(bar(B_KFULL + st), Lay::kT + nc * K * 4);
@@ -252,11 +261,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                       K * 4, bar(B_KFULL + st));
         } else {
           mbar_expect_tx(bar(B_KFULL + st), Lay::kT + K * 4);
-          const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+          const int row = (int)(s0 + (long)jb_of(t) * BN);
           for (int b = 0; b < K / 64; ++b)
             tma_load_3d(sbase + Lay::oK + st * Lay::kT + b * (BN * 128), &tm_k,
                         bar(B_KFULL + st), b * 64, h, row);
-          bulk_load(rj_dst, p.anchors + ((long)(blk_off + jb_lo + t) * HQ + h) * K, K * 4,
+          bulk_load(rj_dst, p.anchors + ((long)(blk_off + jb_of(t)) * HQ + h) * K, K * 4,
                     bar(B_KFULL + st));
         }
         issued = t + 1;
@@ -276,9 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kCache) {
           for (int b = 0; b < V / 64; ++b)
             tma_load_4d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v,
-                        bar(B_VFULL + st), b * 64, kh, (jb_lo + t) * BN, seq);
+                        bar(B_VFULL + st), b * 64, kh, jb_of(t) * BN, seq);
         } else {
-          const int row = (int)(s0 + (long)(jb_lo + t) * BN);
+          const int row = (int)(s0 + (long)jb_of(t) * BN);
           for (int b = 0; b < V / 64; ++b)
             tma_load_3d(sbase + Lay::oV + st * Lay::kT + b * (BN * 128), &tm_v,
                         bar(B_VFULL + st), b * 64, kh, row);
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // k_tilde rounding itself); rows of a chunk that holds no cached
         // position are zeros and get factor 0
         int c0;
-        const int nvalid = cache_tile_chunks(p, (jb_lo + t) * BN, c0);
+        const int nvalid = cache_tile_chunks(p, jb_of(t) * BN, c0);
         const int crows = p.C >= BN ? BN : p.C;  // tile rows per chunk
         for (int x = 0; x * crows < BN; ++x) {
           __nv_bfloat162 f[4];
@@ -434,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = pos0 + qi;                  // its position among the keys
     const bool row_ok = r < ni;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const bool has_gs = p.GS != nullptr;
+    constexpr bool has_gs = kGS;
     const int win = p.window > 0 ? p.window : 0x7fffffff;
     const float gs_i = (has_gs && row_ok) ? p.GS[(s0 + qi) * HQ + h] * kLog2e : 0.f;
     const uint32_t s_addr = tmem + lane_base + grp * 128;
@@ -446,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // they only keep step with their group (S ready, P "written")
     const bool idle = kCache && !__any_sync(0xffffffffu, row_ok);
     for (int t = grp; t < nT; t += 2) {
-      const int j0 = (jb_lo + t) * BN;
+      const int j0 = jb_of(t) * BN;
       if (idle) {
         const bool got = wait_bar(bar(B_SFULL + grp), (t >> 1) & 1, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -468,15 +477,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       // logits (log2 domain) with the causal / window / sequence mask.  The
-      // common case -- a fully visible tile without a scalar gate -- is a
-      // plain multiply; the decision is warp-uniform and hoisted out of the
-      // element loops.
+      // common case -- a fully visible tile -- is a multiply (plus, with a
+      // scalar gate, the bias GS_i - GS_j, from this warp's copy of the key
+      // prefix); the decision is warp-uniform and hoisted out of the element
+      // loops.
       // (rows past a cache chunk's queries compute on finite stand-in
       // queries and are never stored, so they do not hold the warp back)
       const bool fast =
           __all_sync(0xffffffffu, (kCache && !row_ok) ||
                                       (row_ok && (j0 + BN - 1 <= i) && (j0 + BN <= L) &&
-                                       (i - j0 < win) && !has_gs));
+                                       (i - j0 < win)));
       const float sl2 = p.scale_log2;
       const float bias_i = has_gs ? gs_i : 0.f;
       bool done = false;
@@ -490,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (fast && __all_sync(0xffffffffu, m_use != -INFINITY)) {
         uint32_t pk1[64];
         float r0 = 0.f, r1 = 0.f;
+        const float off = kGS ? bias_i - m_use : -m_use;
 #pragma unroll
         for (int c = 0; c < BN; c += 64) {
           uint32_t sv[64];
@@ -497,12 +508,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_addr + c + 32, sv + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const float p0 = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_use));
-            const float p1 = exp2f(fmaf(__uint_as_float(sv[e + 1]), sl2, -m_use));
-            r0 += p0;
-            r1 += p1;
+          for (int e = 0; e < 64; e += 4) {
+            // with a scalar gate the key prefix, four keys per shared-memory
+            // load (a broadcast); without one, a single FMA per logit
+            float4 gk = make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (kGS) gk = *reinterpret_cast<const float4*>(gsk + c + e);
+            const float p0 = exp2f(fmaf(__uint_as_float(sv[e]), sl2, off - gk.x));
+            const float p1 = exp2f(fmaf(__uint_as_float(sv[e + 1]), sl2, off - gk.y));
+            const float p2 = exp2f(fmaf(__uint_as_float(sv[e + 2]), sl2, off - gk.z));
+            const float p3 = exp2f(fmaf(__uint_as_float(sv[e + 3]), sl2, off - gk.w));
+            r0 += p0 + p2;
+            r1 += p1 + p3;
             pk1[(c + e) / 2] = pack_bf16x2(p0, p1);
+            pk1[(c + e) / 2 + 1] = pack_bf16x2(p2, p3);
           }
         }
         if (!__any_sync(0xffffffffu, !(r0 + r1 <= kRescaleBound))) {
@@ -523,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_addr + c, sv);
           tmem_ld32(s_addr + c + 32, sv + 32);
           tmem_wait_ld();
-          if (fast) {
+          if (fast && !has_gs) {
 #pragma unroll
             for (int e = 0; e < 64; e += 4) {
               mx0 = fmaxf(mx0, __uint_as_float(sv[e]) * sl2);
@@ -531,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mx2 = fmaxf(mx2, __uint_as_float(sv[e + 2]) * sl2);
               mx3 = fmaxf(mx3, __uint_as_float(sv[e + 3]) * sl2);
             }
-          } else {
+          } else {  // masked, or with the scalar gate's bias
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
               const int j = j0 + c + e;
@@ -575,12 +593,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_addr + c, sv);
           tmem_wait_ld();
           float e32[32];
-          if (fast) {
+          if (fast && !has_gs) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               e32[e] = exp2f(fmaf(__uint_as_float(sv[e]), sl2, -m_eff));
             }
-          } else {
+          } else {  // masked, or with the scalar gate's bias
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int j = j0 + c + e;
@@ -748,8 +766,9 @@ int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, in
       !make_tile_map(&tk, ws.kh, pb.rows, pb.HQ, KD, BN) ||
       !make_tile_map(&tv, a.v, pb.rows, pb.H, KD, BN))
     return WALL_ERR_CUDA;
-  static bool attr[kMaxDevices] = {};
-  if (!set_max_smem_once(fwd_tc_kernel<KD, false>, Smem<KD, false>::kAlloc, attr))
+  static bool attr[2][kMaxDevices] = {};
+  if (!set_max_smem_once(fwd_tc_kernel<KD, false, false>, Smem<KD, false>::kAlloc, attr[0]) ||
+      !set_max_smem_once(fwd_tc_kernel<KD, false, true>, Smem<KD, false>::kAlloc, attr[1]))
     return WALL_ERR_CUDA;
   FwdTcParams p;
   p.anchors = ws.anchors;
@@ -766,7 +785,12 @@ int launch_fwd_tc(const AttnProblem& pb, const FwdArgs& a, const TcFwdWs& ws, in
   p.rc = nullptr;
   p.C = p.NC = p.t_off = p.T_kv = 0;
   dim3 grid(pb.HQ, ws.n_blocks128);
-  fwd_tc_kernel<KD, false><<<grid, kThreads, Smem<KD, false>::kAlloc, stream>>>(tq, tk, tv, p);
+  if (a.GS)
+    fwd_tc_kernel<KD, false, true><<<grid, kThreads, Smem<KD, false>::kAlloc, stream>>>(tq, tk, tv,
+                                                                                        p);
+  else
+    fwd_tc_kernel<KD, false, false><<<grid, kThreads, Smem<KD, false>::kAlloc, stream>>>(tq, tk, tv,
+                                                                                         p);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 
@@ -783,10 +807,11 @@ int launch_decode_chunk_tc(const FwdTcParams& p0, const void* k_tilde, const voi
       !make_cache_map(&tv, v, B, T_kv, Tcap, H, KD, BN))
     return WALL_ERR_CUDA;
   static bool attr[kMaxDevices] = {};
-  if (!set_max_smem_once(fwd_tc_kernel<KD, true>, Smem<KD, true>::kAlloc, attr))
+  if (!set_max_smem_once(fwd_tc_kernel<KD, true, false>, Smem<KD, true>::kAlloc, attr))
     return WALL_ERR_CUDA;
   dim3 grid(HQ, p0.n_blocks);
-  fwd_tc_kernel<KD, true><<<grid, kThreads, Smem<KD, true>::kAlloc, stream>>>(tq, tk, tv, p0);
+  fwd_tc_kernel<KD, true, false><<<grid, kThreads, Smem<KD, true>::kAlloc, stream>>>(tq, tk, tv,
+                                                                                      p0);
   return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
 }
 

@@ -138,7 +138,9 @@ int wall_attn_fwd(const void* q, const void* k, const void* v, const float* P, i
 
 /* wall_attn_fwd_gate_workspace -- bytes of workspace wall_attn_fwd_gate needs:
  * wall_attn_fwd_workspace's layout first, then the prefix scan's chunk
- * carries (fp32 [B*T, HQ*K]) on the tensor-core path. */
+ * carries on the tensor-core path: fp32, one row of HQ*K per 32-row chunk
+ * of every sequence (B * ceil(T / 32) rows dense; ceil(B*T / 32) + n_seq
+ * rows with cu_seqlens). */
 size_t wall_attn_fwd_gate_workspace(int dtype, int B, int T, int H, int HQ, int K, int V,
                                     int has_g_scalar, int n_seq);
 

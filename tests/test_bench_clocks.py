@@ -42,7 +42,28 @@ def test_clock_record_from_samples_inside_the_window(tmp_path, monkeypatch):
     assert rec["sm_mhz"] == 1965.0            # median of 1965 x3 : 1900 x1
     assert rec["reasons"] == ["sw_power_cap"]  # "Not Active" fields are not reasons
     assert 3 <= rec["samples"] <= 16
+    assert rec["in_window"] == rec["samples"]
     assert 450 <= rec["window_ms"] <= 3000
+
+
+def test_window_shorter_than_the_interval_takes_the_nearest_samples(tmp_path, monkeypatch):
+    """A timed region between two samples: the sample before it and the one
+    after it stand in, and the record says none fell inside."""
+    _fake_smi(tmp_path, monkeypatch)
+    c = bench.ClockSampler(0).start()
+    time.sleep(0.3)
+    # the stand-in prints every 50 ms: a 1 ms window right after a sample
+    # holds none
+    c.mark(True)
+    c.mark(False)
+    c.t0 = c.t1 = time.time() - 0.1
+    c.t1 += 0.001
+    time.sleep(0.2)
+    rec = c.stop()
+    assert rec is not None
+    assert rec["sm_max_mhz"] == 1965.0
+    assert 1 <= rec["samples"] <= 2
+    assert rec["in_window"] <= 1
 
 
 def test_no_nvidia_smi_gives_no_record(tmp_path, monkeypatch):
