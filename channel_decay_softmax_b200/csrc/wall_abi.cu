@@ -466,7 +466,11 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   // dq from the stored dS tiles (tensor-core path, tiles within their cap)
   a.dS = w.has_ds ? reinterpret_cast<__nv_bfloat16*>(at(workspace, w.dS)) : nullptr;
   a.GS = nullptr;
-  if (g_scalar) {
+  if (g_scalar && fwd_workspace != nullptr && fwd_tc_supported(pb)) {
+    // the forward formed the prefix of the same g_scalar in its workspace
+    a.GS = reinterpret_cast<float*>(
+        at(const_cast<void*>(fwd_workspace), fwd_ws_layout(pb, 1).gs));
+  } else if (g_scalar) {
     float* gs = reinterpret_cast<float*>(at(workspace, w.gs));
     rc = scan_prefix_plain(g_scalar, gs, HQ, pb.seqs, s);
     if (rc) return rc;

@@ -732,7 +732,7 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ dO,
 // row), summed in a fixed order so that repeated calls agree bit for bit.
 // Two passes: CTA b sums rows [b R, (b + 1) R) per head (thread t takes head
 // t % HQ and every (256 / HQ)-th row, so a warp reads consecutive words),
-// then one thread per head adds the CTAs' partials in CTA order.
+// then one warp per head adds the CTAs' partials in a fixed order.
 __global__ void __launch_bounds__(256)
     sink_partial_kernel(const float* __restrict__ D, const float* __restrict__ lse,
                         const float* __restrict__ sink, long rows, int HQ, long rows_per_cta,
@@ -759,13 +759,17 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// one warp per head: lane l adds partials l, l + 32, ... in order, then a
+// fixed shuffle tree
 __global__ void sink_final_kernel(const float* __restrict__ part, int nb, int HQ,
                                   float* __restrict__ dsink) {
-  for (int h = threadIdx.x; h < HQ; h += blockDim.x) {
-    float sum = 0.f;
-    for (int b = 0; b < nb; ++b) sum += part[(long)b * HQ + h];
-    dsink[h] = sum;
-  }
+  const int h = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32), lane = threadIdx.x % 32;
+  if (h >= HQ) return;
+  float sum = 0.f;
+  for (int b = lane; b < nb; b += 32) sum += part[(long)b * HQ + h];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane == 0) dsink[h] = sum;
 }
 
 // The one-CTA-per-head form of the same sum, for more than 256 heads.
@@ -900,7 +904,7 @@ int sink_grad(const float* D, const float* lse, const float* sink, long rows, in
     const long per_cta = (rows + nb - 1) / nb;
     sink_partial_kernel<<<(unsigned)nb, 256, 0, stream>>>(D, lse, sink, rows, HQ, per_cta,
                                                            scratch);
-    sink_final_kernel<<<1, 256, 0, stream>>>(scratch, (int)nb, HQ, dsink);
+    sink_final_kernel<<<(HQ * 32 + 255) / 256, 256, 0, stream>>>(scratch, (int)nb, HQ, dsink);
   } else {
     sink_grad_kernel<<<HQ, 256, 0, stream>>>(D, lse, sink, rows, HQ, dsink);
   }

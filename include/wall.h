@@ -202,7 +202,8 @@ size_t wall_attn_bwd_workspace_min(int dtype, int B, int T, int H, int HQ, int K
  * sequence.  dk^(h), dv^(h) are summed over each GQA group.
  * fwd_workspace: NULL, or the workspace of the wall_attn_fwd (or
  * wall_attn_fwd_gate) call that produced o and lse, with the same q, k, P,
- * shapes and options and left unchanged since.  On the bf16 tensor-core path the anchored operands that
+ * shapes and options and left unchanged since.  On the bf16 tensor-core
+ * path the anchored operands (and, with g_scalar, the gate's prefix) that
  * call prepared in it are then read instead of recomputed; it is only read.
  * Elsewhere it is ignored.
  */

@@ -209,6 +209,26 @@ def test_backward_reuses_forward_operands_bit_exactly():
         assert torch.equal(ta, tb), name
 
 
+def test_backward_reuses_forward_operands_bit_exactly_with_options():
+    """The same with every option (varlen, window, g_scalar, sink): given
+    the forward's workspace, the backward also reads the forward's prefix of
+    g_scalar instead of scanning it again, and dsink is a fixed-order sum, so
+    all six gradients match the recomputing call bit for bit."""
+    s = I.spec(4, len_lo=64, len_hi=600, window=128)
+    x = _to(I.training_inputs(s))
+    q, k, v, g = x["q"], x["k"], x["v"], x["g"]
+    kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=x["window_size"],
+              cu_seqlens=x["cu_seqlens"])
+    o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, x["scale"], return_workspace=True, **kw)
+    a = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], want_dsink=True, **kw)
+    b = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], fwd_workspace=fws,
+                          want_dsink=True, **kw)
+    torch.cuda.synchronize()
+    for name, ta, tb in zip(("dq", "dk", "dv", "dg", "dg_scalar", "dsink"), a, b):
+        assert ta is not None and tb is not None, name
+        assert torch.equal(ta, tb), name
+
+
 def _run_gpu_recompute(x):
     """_run_gpu with the smaller backward workspace: no dS tiles, so the dq
     pass recomputes S, P, dP and dS"""
