@@ -454,6 +454,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a chunk of fewer than 128 queries leaves whole warps without a row:
     // they only keep step with their group (S ready, P "written")
     const bool idle = kCache && !__any_sync(0xffffffffu, row_ok);
+    // the scalar gate's key prefix of the group's next tile, one load per
+    // lane and key quarter, issued a tile ahead so that its L2 latency
+    // overlaps the current tile instead of preceding the wait for S
+    float gnext[kGS ? BN / 32 : 1];
+    auto load_gs = [&](int t) {
+#pragma unroll
+      for (int x = 0; x < BN / 32; ++x) {
+        const int j = jb_of(t) * BN + lane + 32 * x;
+        gnext[x] = (t < nT && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
+      }
+    };
+    if constexpr (has_gs) load_gs(grp);
     for (int t = grp; t < nT; t += 2) {
       const int j0 = jb_of(t) * BN;
       if (idle) {
@@ -463,12 +475,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(B_PFULL + grp));
         continue;
       }
-      if (has_gs || t == grp) {
+      if constexpr (has_gs) {
         __syncwarp();
-        for (int c = lane; c < BN; c += 32) {
-          const int j = j0 + c;
-          gsk[c] = (has_gs && j < L) ? p.GS[(s0 + j) * HQ + h] * kLog2e : 0.f;
-        }
+#pragma unroll
+        for (int x = 0; x < BN / 32; ++x) gsk[lane + 32 * x] = gnext[x];
+        __syncwarp();
+        load_gs(t + 2);
+      } else if (t == grp) {
+        __syncwarp();
+        for (int c = lane; c < BN; c += 32) gsk[c] = 0.f;
         __syncwarp();
       }
       {
