@@ -505,6 +505,86 @@ int launch_scan(const Tin* x, Tout* y, float* scratch, long C, const Seqs& seqs,
                                                         carry_out, stream);
 }
 
+// Few columns (the scalar gate's scans, C = HQ): the three passes in one CTA
+// per sequence, one launch instead of three.  Thread (part p, group of four
+// columns) sums rows [p R, (p + 1) R) of its sequence in fp64; the parts'
+// sums get their exclusive carries by a fixed-order Hillis-Steele scan over
+// the parts in shared memory (fp64); each thread then scans its rows again
+// from its carry.  Used while every sequence fits one CTA (all rows <=
+// kSmallRows: at most kSmallRows / parts rows per thread).
+constexpr int kSmallThreads = 1024;
+constexpr long kSmallRows = 65536;
+constexpr int kSmallMaxC = 64;
+
+template <bool kReverse>
+__global__ void __launch_bounds__(kSmallThreads)
+    scan_small_kernel(const float* __restrict__ x, float* __restrict__ y, int C, Seqs seqs) {
+  extern __shared__ double sm_small[];  // two buffers of [parts][C]
+  const int s = blockIdx.x;
+  const long start = seqs.start(s), len = seqs.len(s);
+  const int ng = C / 4;                        // float4 groups per row
+  const int parts = kSmallThreads / ng;
+  const int tid = threadIdx.x, g = tid % ng, p = tid / ng;
+  const bool active = p < parts;
+  const long R = (len + parts - 1) / parts;
+  const long r0 = active ? min(len, (long)p * R) : len;
+  const long r1 = min(len, r0 + R);
+  auto row_of = [&](long r) { return kReverse ? start + len - 1 - r : start + r; };
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long r = r0; r < r1; ++r) {
+    const float4 v = *reinterpret_cast<const float4*>(x + row_of(r) * C + g * 4);
+    acc[0] += v.x;
+    acc[1] += v.y;
+    acc[2] += v.z;
+    acc[3] += v.w;
+  }
+  // inclusive scan of the parts' sums, per column, then shifted to exclusive
+  double* buf[2] = {sm_small, sm_small + (long)parts * C};
+  const long slot = (long)p * C + g * 4;
+  if (active)
+    for (int e = 0; e < 4; ++e) buf[0][slot + e] = acc[e];
+  __syncthreads();
+  int cur = 0;
+  for (int off = 1; off < parts; off <<= 1) {
+    if (active)
+      for (int e = 0; e < 4; ++e)
+        buf[cur ^ 1][slot + e] =
+            buf[cur][slot + e] + (p >= off ? buf[cur][slot - (long)off * C + e] : 0.0);
+    __syncthreads();
+    cur ^= 1;
+  }
+  if (!active || r0 >= r1) return;
+  double run[4];
+  for (int e = 0; e < 4; ++e) run[e] = p > 0 ? buf[cur][slot - C + e] : 0.0;
+  for (long r = r0; r < r1; ++r) {
+    const long pr = row_of(r);
+    const float4 v = *reinterpret_cast<const float4*>(x + pr * C + g * 4);
+    run[0] += v.x;
+    run[1] += v.y;
+    run[2] += v.z;
+    run[3] += v.w;
+    *reinterpret_cast<float4*>(y + pr * C + g * 4) =
+        make_float4((float)run[0], (float)run[1], (float)run[2], (float)run[3]);
+  }
+}
+
+// fp32 in and out, no carries, small C: the one-launch scan applies
+bool small_scan_ok(const float* x, const float* y, long C, const Seqs& seqs) {
+  return C >= 4 && C <= kSmallMaxC && C % 4 == 0 && seqs.rows <= kSmallRows &&
+         ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) % 16) == 0;
+}
+
+template <bool kReverse>
+int launch_small_scan(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream) {
+  const int parts = kSmallThreads / (int)(C / 4);
+  const size_t smem = 2 * sizeof(double) * (size_t)parts * C;
+  static bool attr[2][kMaxDevices] = {};
+  if (!set_max_smem_once(scan_small_kernel<kReverse>, (int)smem, attr[kReverse ? 1 : 0]))
+    return WALL_ERR_CUDA;
+  scan_small_kernel<kReverse><<<seqs.n, kSmallThreads, smem, stream>>>(x, y, (int)C, seqs);
+  return cudaGetLastError() == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;
+}
+
 }  // namespace
 
 int scan_prefix_log2(const void* g, int dtype, float* P, long C, const Seqs& seqs,
@@ -588,11 +668,16 @@ int scan_reverse_from_sums(const float* x, void* y, int out_dtype, float* scratc
 }
 
 int scan_prefix_plain(const float* x, float* y, long C, const Seqs& seqs, cudaStream_t stream) {
+  if (seqs.n == 0 || C == 0) return WALL_OK;
+  if (small_scan_ok(x, y, C, seqs)) return launch_small_scan<false>(x, y, C, seqs, stream);
   return launch_scan<float, float, false>(x, y, y, C, seqs, 1.f, nullptr, nullptr, stream);
 }
 
 int scan_reverse(const float* x, void* y, int out_dtype, float* scratch, long C, const Seqs& seqs,
                  cudaStream_t stream) {
+  if (seqs.n == 0 || C == 0) return WALL_OK;
+  if (out_dtype == WALL_FP32 && small_scan_ok(x, static_cast<float*>(y), C, seqs))
+    return launch_small_scan<true>(x, static_cast<float*>(y), C, seqs, stream);
   if (out_dtype == WALL_BF16)
     return launch_scan<float, __nv_bfloat16, true>(x, static_cast<__nv_bfloat16*>(y), scratch, C,
                                                    seqs, 1.f, nullptr, nullptr, stream);
