@@ -437,10 +437,12 @@ int wall_attn_bwd(const void* dO, const void* q, const void* k, const void* v, c
   if (!ok_opt(g_scalar) || !ok_opt(sink_bias) || !ok_opt(dg_scalar) || !ok_opt(dsink))
     return WALL_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dsink) {
-    if (cudaMemsetAsync(dsink, 0, sizeof(float) * HQ, s) != cudaSuccess) return WALL_ERR_CUDA;
+  if (pb.rows == 0) {
+    // nothing to sum: dsink is 0 (otherwise the backward writes all of it)
+    if (dsink && cudaMemsetAsync(dsink, 0, sizeof(float) * HQ, s) != cudaSuccess)
+      return WALL_ERR_CUDA;
+    return WALL_OK;
   }
-  if (pb.rows == 0) return WALL_OK;
   if (!ok_ptr(dO) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(P) || !ok_ptr(o) ||
       !ok_ptr(lse) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) || !ok_ptr(dg))
     return WALL_ERR_INVALID_ARG;
