@@ -327,13 +327,15 @@ def bench_train(args, world, rank, peaks):
     stages[ROOF_STAGE] = roof_stage[ROOF_STAGE]
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    # launches of this library inside one step: forward: prefix chunk sums
-    # and carries 2, chunk scans fused with the operand preparation 1,
-    # tcgen05 forward 1; backward (reusing the forward's operands): D/sink
-    # pre-pass 1, tcgen05 key-block (dK, dV, dS tiles) 1, dk/dv group sums 1,
-    # tcgen05 query-block dq 1, dq/dL finalize with dL's chunk sums 1,
-    # reverse-scan carries and chunk scans 2
-    launches_per_step = 11
+    # launches of this library inside one step (the ncu launch list in
+    # profiles/ shows the same 13): forward: prefix chunk sums and carries 2,
+    # chunk scans fused with the operand preparation 1, tcgen05 forward 1,
+    # the check for units past the anchored range 1; backward (reusing the
+    # forward's operands): D pre-pass 1, tcgen05 key-block (dK, dV, dS tiles)
+    # 1, tcgen05 query-block dq 1, the units check 1, dk/dv group sums 1,
+    # dq/dL finalize with dL's chunk sums 1, reverse-scan carries and chunk
+    # scans 2
+    launches_per_step = 13
     res = dict(ms=ms_max, value=weak_scaling_value(step_flops, ms_max, world) / 1e12,
                fwd_ms=fwd_ms, bwd_ms=bwd_ms,
                fwd_tflops=fwd_flops / (fwd_ms * 1e-3) / 1e12,
