@@ -589,6 +589,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         ds_tile = ds_tile_of(I0 + t + 1);
       }
     }
+    // The epilogue's rows of P and the block's anchors, loaded now so that
+    // their latency overlaps the last MMAs and the staging below.  Warp w
+    // takes rows w, w + 8, ...; lane = KD/32 consecutive channels;
+    // dk_j = scale 2^(R_J - P_j) dKa_j
+    constexpr int CPL = KD / 32;
+    const int c0 = lane * CPL;
+    float rjv[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) rjv[i] = anc[(long)blk * HQ * K + c0 + i];
+    constexpr int kRowsPerWarp = BK / 8;
+    float pj[kRowsPerWarp][CPL];
+#pragma unroll
+    for (int x = 0; x < kRowsPerWarp; ++x) {
+      const int rr = (warp - 4) + 8 * x;
+      const long krow = (s0 + j0 + (rr < nj ? rr : 0)) * HQ + h;
+      if constexpr (CPL == 4) {
+        const float4 a = *reinterpret_cast<const float4*>(p.P + krow * K + c0);
+        pj[x][0] = a.x; pj[x][1] = a.y; pj[x][2 % CPL] = a.z; pj[x][3 % CPL] = a.w;
+      } else {
+        const float2 a = *reinterpret_cast<const float2*>(p.P + krow * K + c0);
+        pj[x][0] = a.x; pj[x][1 % CPL] = a.y;
+      }
+    }
     // the stored tiles are complete before the CTA can exit
     if (store_ds && lane == 0) bulk_wait_all();
     // ---- dK, dV epilogue.  Thread = key row in TMEM, but a row per thread
@@ -623,28 +646,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(bar(EPI_STAGED));  // every warp arrives, even after an abort
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(EPI_STAGED), 0, p.status, abort_flag));
     if (ok) {
-      // warp w takes rows w, w + 8, ...; lane = KD/32 consecutive channels;
-      // dk_j = scale 2^(R_J - P_j) dKa_j
-      constexpr int CPL = KD / 32;
-      const int c0 = lane * CPL;
-      float rjv[CPL];
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) rjv[i] = anc[(long)blk * HQ * K + c0 + i];
-      // every P load of the warp's 16 rows in flight before the first use
-      constexpr int kRowsPerWarp = BK / 8;
-      float pj[kRowsPerWarp][CPL];
-#pragma unroll
-      for (int x = 0; x < kRowsPerWarp; ++x) {
-        const int rr = (warp - 4) + 8 * x;
-        const long krow = (s0 + j0 + (rr < nj ? rr : 0)) * HQ + h;
-        if constexpr (CPL == 4) {
-          const float4 a = *reinterpret_cast<const float4*>(p.P + krow * K + c0);
-          pj[x][0] = a.x; pj[x][1] = a.y; pj[x][2 % CPL] = a.z; pj[x][3 % CPL] = a.w;
-        } else {
-          const float2 a = *reinterpret_cast<const float2*>(p.P + krow * K + c0);
-          pj[x][0] = a.x; pj[x][1 % CPL] = a.y;
-        }
-      }
 #pragma unroll
       for (int x = 0; x < kRowsPerWarp; ++x) {
         const int rr = (warp - 4) + 8 * x;
