@@ -33,40 +33,49 @@ using T_bf16 = __nv_bfloat16;
 // leaves k_tilde outside the range the decode reads it in: that records
 // WALL_ERR_RANGE in `status` (the layout has no other place for the row).
 template <typename T>
-__global__ void cache_kernel(const T* __restrict__ k, const float* __restrict__ P, int B, int Tn,
-                             int H, int HQ, int K, int C, int t0, T* __restrict__ kt,
-                             float* __restrict__ rc, int Tcap, int* status) {
+__global__ void __launch_bounds__(256)
+    cache_kernel(const T* __restrict__ k, const float* __restrict__ P, int B, int Tn, int H,
+                 int HQ, int K, int C, int t0, T* __restrict__ kt, float* __restrict__ rc,
+                 int Tcap, int* status) {
+  // a CTA takes whole rows (b, t): the row's split into (head, 8 channels)
+  // groups needs only 32-bit arithmetic, and every group of the row shares
+  // the chunk start's anchors (L1 hits after the first)
   const int G = HQ / H;
   const int NC = (Tcap + C - 1) / C;
   const int kgroups = K / 8;
-  const long total = (long)B * Tn * HQ * kgroups;
-  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long)gridDim.x * blockDim.x) {
-    const int kg = (int)(e % kgroups);
-    const int h = (int)((e / kgroups) % HQ);
-    const long tt = (e / ((long)kgroups * HQ)) % Tn;
-    const long b = e / ((long)kgroups * HQ * Tn);
+  const int per_row = HQ * kgroups;
+  const long rows = (long)B * Tn;
+  bool wide = false;
+  for (long row = blockIdx.x; row < rows; row += gridDim.x) {
+    const long b = row / Tn;
+    const long tt = row - b * Tn;
     const long t = t0 + tt;
     const long c = t / C;
     const long cstart = c * C;
-    const int n0 = kg * 8;
-    float pv[8], Rv[8], kv[8], out[8];
-    load8(P + ((b * Tn + tt) * HQ + h) * K + n0, pv);
-    if (cstart < t0)
-      load8(rc + ((b * NC + c) * HQ + h) * K + n0, Rv);
-    else
-      load8(P + ((b * Tn + (cstart - t0)) * HQ + h) * K + n0, Rv);
-    load8(k + ((b * Tn + tt) * H + h / G) * K + n0, kv);
-    bool wide = false;
+    const float* prow = P + row * HQ * K;
+    const float* rrow = cstart < t0 ? rc + (b * NC + c) * HQ * K
+                                    : P + (b * Tn + (cstart - t0)) * HQ * K;
+    const T* krow = k + row * H * K;
+    T* ktrow = kt + (b * Tcap + t) * HQ * K;
+    float* rcrow = t == cstart ? rc + (b * NC + c) * HQ * K : nullptr;
+    for (int i = threadIdx.x; i < per_row; i += blockDim.x) {
+      const int h = i / kgroups;
+      const int n0 = (i - h * kgroups) * 8;
+      const int off = h * K + n0;
+      float pv[8], Rv[8], kv[8], out[8];
+      load8(prow + off, pv);
+      load8(rrow + off, Rv);
+      load8(krow + (h / G) * K + n0, kv);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      out[i] = kv[i] * exp2f(Rv[i] - pv[i]);
-      wide |= fabsf(Rv[i] - pv[i]) > kAnchorRange;
+      for (int e = 0; e < 8; ++e) {
+        out[e] = kv[e] * exp2f(Rv[e] - pv[e]);
+        wide |= fabsf(Rv[e] - pv[e]) > kAnchorRange;
+      }
+      store8(ktrow + off, out);
+      if (rcrow) store8(rcrow + off, pv);
     }
-    if (wide) record_status(status, WALL_ERR_RANGE);
-    store8(kt + ((b * Tcap + t) * HQ + h) * K + n0, out);
-    if (t == cstart) store8(rc + ((b * NC + c) * HQ + h) * K + n0, pv);
   }
+  if (wide) record_status(status, WALL_ERR_RANGE);
 }
 
 template <typename T>
@@ -831,11 +840,11 @@ DecodeArgs decode_args(const void* q, const void* v, const float* p_curr, const 
 
 int build_kv_cache(const void* k, const float* P, int dtype, int B, int Tn, int H, int HQ, int K,
                    int C, int t0, void* k_tilde, float* r_cache, int Tcap, cudaStream_t stream) {
-  const long total = (long)B * Tn * HQ * (K / 8);
-  if (total == 0) return WALL_OK;
+  const long rows = (long)B * Tn;
+  if (rows == 0 || HQ * (K / 8) == 0) return WALL_OK;
   const int threads = 256;
-  const long want = (total + threads - 1) / threads;
-  const int blocks = (int)(want < 148L * 64 ? want : 148L * 64);
+  // whole rows per CTA, eight CTAs per SM, the grid striding over the rest
+  const int blocks = (int)(rows < 148L * 8 * 4 ? rows : 148L * 8 * 4);
   if (dtype == WALL_BF16)
     cache_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(k), P, B, Tn, H, HQ, K, C, t0,

@@ -229,6 +229,36 @@ def test_backward_reuses_forward_operands_bit_exactly_with_options():
         assert torch.equal(ta, tb), name
 
 
+@pytest.mark.parametrize("case", ["cfg3_block", "options"])
+def test_repeated_calls_bit_identical(case):
+    """Two identical forward + backward calls give identical bits in every
+    output, dsink and dg_scalar included: the library has no float atomics
+    and fixes every summation order."""
+    if case == "cfg3_block":
+        s = I.spec(3, T=1024)
+    else:
+        s = I.spec(4, len_lo=64, len_hi=600, window=128)
+    x = _to(I.training_inputs(s))
+    q, k, v, g = x["q"], x["k"], x["v"], x["g"]
+    kw = dict(g_scalar=x["g_scalar"], sink_bias=x["sink_bias"], window_size=x["window_size"],
+              cu_seqlens=x["cu_seqlens"])
+    want_dsink = x["sink_bias"] is not None
+    runs = []
+    for _ in range(2):
+        o, lse, P, fws = api.wall_attn_fwd_gate(q, k, v, g, x["scale"], return_workspace=True,
+                                                **kw)
+        grads = api.wall_attn_bwd(x["dO"], q, k, v, P, o, lse, x["scale"], fwd_workspace=fws,
+                                  want_dsink=want_dsink, **kw)
+        runs.append((o, lse, P) + tuple(grads))
+    torch.cuda.synchronize()
+    names = ("o", "lse", "P", "dq", "dk", "dv", "dg", "dg_scalar", "dsink")
+    for name, a, b in zip(names, runs[0], runs[1]):
+        if a is None:
+            assert b is None, name
+            continue
+        assert torch.equal(a, b), name
+
+
 def _run_gpu_recompute(x):
     """_run_gpu with the smaller backward workspace: no dS tiles, so the dq
     pass recomputes S, P, dP and dS"""
