@@ -804,44 +804,39 @@ __global__ void bwd_finalize_kernel(Seqs seqs, int HQ, int H, int K, int V,
                                     const float* __restrict__ dvh32, float* __restrict__ dgs_row,
                                     const float* __restrict__ dgs_col, T* __restrict__ dk,
                                     T* __restrict__ dv) {
+  // CTAs take rows of the sequence, threads the row's (kv head, 8 channels)
+  // groups of dk then dv: 32-bit arithmetic only, and each group's G loads
+  // issued together
   const int s = blockIdx.y;
   const long s0 = seqs.start(s);
   const int L = seqs.len(s);
   const int G = HQ / H;
-  const long stride = (long)gridDim.x * blockDim.x;
-  const long tid0 = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int kg = K / 8;
-  const long nk = (long)L * H * kg;
-  for (long e = tid0; e < nk; e += stride) {
-    const int g8 = (int)(e % kg);
-    const int kv = (int)((e / kg) % H);
-    const int t = (int)(e / ((long)kg * H));
+  const int kg = K / 8, vg = V / 8;
+  const int per_k = H * kg, per_row = H * (kg + vg);
+  for (int t = blockIdx.x; t < L; t += gridDim.x) {
     const long row = s0 + t;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, x[8];
-    for (int g = 0; g < G; ++g) {
-      load8(dkh32 + (row * HQ + kv * G + g) * K + g8 * 8, x);
+    for (int i = threadIdx.x; i < per_row; i += blockDim.x) {
+      const bool is_k = i < per_k;
+      const int j = is_k ? i : i - per_k;
+      const int D = is_k ? K : V;
+      const int ng = is_k ? kg : vg;
+      const int kv = j / ng;
+      const int n0 = (j - kv * ng) * 8;
+      const float* src = (is_k ? dkh32 : dvh32) + (row * HQ + kv * G) * D + n0;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, x[8];
+#pragma unroll 4
+      for (int g = 0; g < G; ++g) {
+        load8(src + (long)g * D, x);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] += x[c];
+        for (int c = 0; c < 8; ++c) acc[c] += x[c];
+      }
+      store8((is_k ? dk : dv) + (row * H + kv) * D + n0, acc);
     }
-    store8(dk + (row * H + kv) * K + g8 * 8, acc);
-  }
-  const int vg = V / 8;
-  const long nv = (long)L * H * vg;
-  for (long e = tid0; e < nv; e += stride) {
-    const int g8 = (int)(e % vg);
-    const int kv = (int)((e / vg) % H);
-    const int t = (int)(e / ((long)vg * H));
-    const long row = s0 + t;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, x[8];
-    for (int g = 0; g < G; ++g) {
-      load8(dvh32 + (row * HQ + kv * G + g) * V + g8 * 8, x);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] += x[c];
-    }
-    store8(dv + (row * H + kv) * V + g8 * 8, acc);
   }
   if (dgs_row && dgs_col) {
-    for (long e = tid0; e < (long)L * HQ; e += stride) dgs_row[s0 * HQ + e] += dgs_col[s0 * HQ + e];
+    const long stride = (long)gridDim.x * blockDim.x;
+    for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < (long)L * HQ; e += stride)
+      dgs_row[s0 * HQ + e] += dgs_col[s0 * HQ + e];
   }
 }
 
@@ -958,8 +953,11 @@ int attn_bwd_tc(const AttnProblem& pb, const BwdArgs& a, const TcFwdWs& ws, bool
   // overwrites dk^(h)'s chunk rows with its sums
   timing_mark(T_BWD_FIN, stream);
   {
-    dim3 grid((148 * 8 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
-    bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+    // a row's groups per CTA (a multiple of 32 threads, at most 256)
+    const int per_row = pb.H * (pb.K / 8 + pb.V / 8);
+    const int threads = std::min(256, (per_row + 31) / 32 * 32);
+    dim3 grid((148 * 16 + pb.seqs.n - 1) / (pb.seqs.n < 1 ? 1 : pb.seqs.n), pb.seqs.n);
+    bwd_finalize_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
         pb.seqs, pb.HQ, pb.H, pb.K, pb.V, a.dkh32, a.dvh32, a.GS ? a.dgs_row : nullptr,
         a.GS ? a.dgs_col : nullptr, static_cast<__nv_bfloat16*>(dk),
         static_cast<__nv_bfloat16*>(dv));

@@ -731,42 +731,44 @@ __global__ void anchor_operands_kernel(const __nv_bfloat16* __restrict__ q,
   const int L = seqs.len(s);
   const int G = HQ / H;
   const int kg = K / 8;
-  const long total = (long)L * HQ * kg;
-  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long)gridDim.x * blockDim.x) {
-    const int g8 = (int)(e % kg);
-    const int hh = (int)((e / kg) % HQ);
-    const int t = (int)(e / ((long)kg * HQ));
-    const int b = t / BM;
-    const long row = s0 + t;
-    const long arow = s0 + (long)b * BM;
-    float pv[8], rv[8], x[8], y[8];
-    load8(P + (row * HQ + hh) * K + g8 * 8, pv);
-    load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
-    bool wide = false;
+  const int per_row = HQ * kg;
+  // CTAs take rows of the sequence, threads the row's (head, 8 channels)
+  // groups: 32-bit arithmetic only
+  for (int t = blockIdx.x; t < L; t += gridDim.x) {
+    for (int i = threadIdx.x; i < per_row; i += blockDim.x) {
+      const int hh = i / kg;
+      const int g8 = i - hh * kg;
+      const int b = t / BM;
+      const long row = s0 + t;
+      const long arow = s0 + (long)b * BM;
+      float pv[8], rv[8], x[8], y[8];
+      load8(P + (row * HQ + hh) * K + g8 * 8, pv);
+      load8(P + (arow * HQ + hh) * K + g8 * 8, rv);
+      bool wide = false;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      rv[c] = floorf(rv[c]);
-      wide |= fabsf(pv[c] - rv[c]) > kAnchorRange;
-    }
-    if (wide) {
-      if (units) {
-        set_flag(units + (long)s * HQ + hh);
-        set_flag(units + (long)seqs.n * HQ);  // some unit is flagged
+      for (int c = 0; c < 8; ++c) {
+        rv[c] = floorf(rv[c]);
+        wide |= fabsf(pv[c] - rv[c]) > kAnchorRange;
       }
-      record_status(status, WALL_ERR_RANGE);
-    }
-    load8(q + (row * HQ + hh) * K + g8 * 8, x);
+      if (wide) {
+        if (units) {
+          set_flag(units + (long)s * HQ + hh);
+          set_flag(units + (long)seqs.n * HQ);  // some unit is flagged
+        }
+        record_status(status, WALL_ERR_RANGE);
+      }
+      load8(q + (row * HQ + hh) * K + g8 * 8, x);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(pv[c] - rv[c]));
-    store8(qh + (row * HQ + hh) * K + g8 * 8, y);
-    if (k != nullptr) {  // without keys: the query operand and anchors only
-      load8(k + (row * H + hh / G) * K + g8 * 8, x);
+      for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(pv[c] - rv[c]));
+      store8(qh + (row * HQ + hh) * K + g8 * 8, y);
+      if (k != nullptr) {  // without keys: the query operand and anchors only
+        load8(k + (row * H + hh / G) * K + g8 * 8, x);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(rv[c] - pv[c]));
-      store8(khat + (row * HQ + hh) * K + g8 * 8, y);
+        for (int c = 0; c < 8; ++c) y[c] = saturate_bf16(x[c] * exp2f(rv[c] - pv[c]));
+        store8(khat + (row * HQ + hh) * K + g8 * 8, y);
+      }
+      if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, rv);
     }
-    if (t == b * BM) store8(anchors + ((long)(s_blk_off + b) * HQ + hh) * K + g8 * 8, rv);
   }
 }
 
