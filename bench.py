@@ -46,7 +46,7 @@ METRIC = "fwd+bwd TFLOP/s & % of BF16 peak at T=8192; decode GB/s vs HBM peak"
 # DRAM bytes (read + write) of one launch of the key-block backward kernel
 # (bwd_tc_kernel) on the T=8192 workload, from the ncu capture summarized in
 # profiles/; None once the kernel changed since that capture.
-BWD_KEY_TRAFFIC_BYTES = 371602688 + 1172543000
+BWD_KEY_TRAFFIC_BYTES = 370527488 + 1171600000
 # algorithmic FLOPs of each tensor-core stage per launch, as multiples of the
 # forward's 2*N*(K+V): the backward's five contractions are QK^T, dO V^T, dV,
 # dK (the key-block kernel) and dq (the query-block kernel, which also
