@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       const uint32_t bytes = (uint32_t)(oR + G * KD * 4);
-      long seq = 0;
+      int seq = 0;  // tiles of this CTA so far (32-bit: the ring's stage and phase)
       bool ok = true;
       for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
         int b, kh, s;
@@ -459,13 +459,13 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
                           kh * G + g, row);
           for (int bx = 0; bx < VD / 64; ++bx)
             tma_load_3d(sb + oV + bx * kKBox, &tm_v, full(st), bx * 64, kh, row);
-          const long c = j0 / a.C;
+          const int c = (int)j0 / a.C;
           bulk_load(sb + oR, a.rc + (((long)b * NC + c) * a.HQ + (long)kh * G) * KD, G * KD * 4,
                     full(st));
         }
       }
       // no copy may still be landing when the CTA exits
-      for (long q = seq > stages ? seq - stages : 0; q < seq; ++q)
+      for (int q = seq > stages ? seq - stages : 0; q < seq; ++q)
         mbar_wait(full((int)(q % stages)), (uint32_t)((q / stages) & 1), status);
     }
   } else if (warp < nw) {
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
     const float sl2 = a.scale * kLog2e;
     float* qt = qts + warp * KD;
     float* xs = xch + (g * 32 + lane) * (VPL + 2);
-    long seq = 0;
+    int seq = 0;  // tiles of this CTA so far
     int n_it = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_it) {
@@ -513,14 +513,14 @@ __global__ void __launch_bounds__(32 * (kStep ? 10 : 9), 1)
       for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
       long c_last = -1;
       for (long j0 = k0; ok && j0 < k1; j0 += kDecTile, ++seq) {
-        if ((((j0 - k0) / kDecTile) % WPH) != par) continue;  // the other warp's tile
+        if ((((int)(j0 - k0) / kDecTile) % WPH) != par) continue;  // the other warp's tile
         const int st = (int)(seq % stages);
         {
           const bool got = mbar_wait(full(st), (uint32_t)((seq / stages) & 1), status);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         }
         const uint8_t* sb = smem + st * stage_bytes;
-        const long c = j0 / a.C;
+        const int c = (int)j0 / a.C;
         if (c != c_last) {
           // the query scaled for this chunk: scale*log2e * q * 2^(p_curr - R_c)
           const float* R = reinterpret_cast<const float*>(sb + oR) + g * KD;
