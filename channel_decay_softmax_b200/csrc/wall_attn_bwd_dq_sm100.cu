@@ -552,8 +552,12 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
-      // the dS ring
+      // the dS ring.  Each stored tile is read once: evict_first, so that
+      // the 1 GB stream does not push out of L2 the key tiles that every
+      // query block of the head reads again (those load with evict_last;
+      // 0.218 against 0.237 ms at T = 8192, 1.09 GB of tiles)
       tma_prefetch_desc(&tm_ds);
+      const uint64_t pol_ds = l2_evict_first();
       int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t % kDSS;
@@ -562,8 +566,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         mbar_expect_tx(bar(D_FULL + st), Lay::kDsT);
         const int drow = (int)((tile0 + t) * 128);
         for (int b = 0; b < 2; ++b)
-          tma_load_2d(sbase + Lay::oDS + st * Lay::kDsT + b * (128 * 128), &tm_ds,
-                      bar(D_FULL + st), b * 64, drow);
+          tma_load_2d_hint(sbase + Lay::oDS + st * Lay::kDsT + b * (128 * 128), &tm_ds,
+                           bar(D_FULL + st), b * 64, drow, pol_ds);
         issued = t + 1;
       }
       // no copy may still be in flight when the CTA exits
@@ -572,6 +576,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     } else if (lane == 1) {
       // the key ring
       tma_prefetch_desc(&tm_k);
+      const uint64_t pol_k = l2_evict_last();
       int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t % kKS3;
@@ -579,8 +584,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
           break;
         mbar_expect_tx(bar(K_FULL3 + st), Lay::kKT + K * 4);
         for (int b = 0; b < K / 64; ++b)
-          tma_load_3d(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k, bar(K_FULL3 + st),
-                      b * 64, h, (int)(s0 + (long)(jlo + t) * BN));
+          tma_load_3d_hint(sbase + Lay::oK + st * Lay::kKT + b * (BN * 128), &tm_k,
+                           bar(K_FULL3 + st), b * 64, h, (int)(s0 + (long)(jlo + t) * BN), pol_k);
         bulk_load(sbase + Lay::oRJ + st * K * 4,
                   p.anchors + ((long)(blk_off + jlo + t) * HQ + h) * K, K * 4,
                   bar(K_FULL3 + st));
